@@ -1,0 +1,154 @@
+/*
+ * tok.h -- C ABI of the B200 Haar patcher and FSQ quantizer library (libtok.so).
+ *
+ * Four operations of a causal image/video tokenizer's data-parallel path:
+ *   tok_haar_fwd    two-level causal full-packet orthonormal Haar patcher
+ *   tok_haar_inv    its inverse (the unpatcher)
+ *   tok_fsq_encode  1x1 C->6 projection + FSQ bound/round + mixed-radix index
+ *   tok_fsq_decode  index -> normalized codes -> 1x1 6->C projection
+ *
+ * Conventions for every call:
+ *   - Pointers are DEVICE pointers (memory the GPU can address), owned by the
+ *     caller; the library allocates nothing and keeps no state between calls.
+ *   - Work is enqueued on `stream` (0 = the legacy default stream) and the
+ *     call returns without synchronizing.  Results are visible to later work
+ *     on the same stream.
+ *   - Tensors are dense and row-major with the last index fastest.
+ *   - Argument errors are detected on the host and returned before anything
+ *     is launched; an empty tensor (a zero extent) returns TOK_OK and touches
+ *     no memory (its pointers may then be NULL).  A launch failure returns
+ *     TOK_ERR_CUDA; tok_last_cuda_error() gives the CUDA error code.
+ *   - Inputs and outputs must not overlap (TOK_ERR_ALIAS).
+ *   - Pointers need natural alignment of their element type (TOK_ERR_ALIGN
+ *     otherwise).  16-byte-aligned buffers with suitable extents take the
+ *     vectorized kernels; other layouts take element-wise GPU kernels with
+ *     identical results.  There is no CPU path.
+ *
+ * Sources for the operations (page title, section):
+ *   [guide] "NVIDIA Cosmos Tokenizer 完全指南" (a guide to the Cosmos Tokenizer
+ *           README): 6.1 and 6.2 (encode API shapes), 7.1 (Haar patching),
+ *           7.2 (FSQ), 7.3 (causal time axis).
+ *   [card]  "nvidia/Cosmos-Tokenize1-CV8x8x8-720p" model card: Model
+ *           Architecture (2-level Haar, x4 in space and time; FSQ).
+ *   [notes] "Cosmos World Foundation Model Platform for Physical AI
+ *           (Cosmos-Predict1)" notes: model architecture, item 1 (FSQ levels
+ *           (8,8,8,5,5,5), vocabulary 64,000).
+ */
+#ifndef TOK_H
+#define TOK_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TOK_ABI_VERSION 1
+
+/* Number of FSQ codes: 8*8*8*5*5*5 ([guide] 7.2, [notes]). */
+#define TOK_FSQ_CODEBOOK 64000
+/* FSQ channels ([guide] 6.2: codes have 6 channels). */
+#define TOK_FSQ_DIM 6
+
+typedef enum {
+    TOK_OK = 0,
+    TOK_ERR_NULL = 1,  /* a required pointer is NULL */
+    TOK_ERR_SHAPE = 2, /* extents violate the operation's shape rule, or overflow */
+    TOK_ERR_ALIGN = 3, /* a pointer is not aligned to its element size */
+    TOK_ERR_DTYPE = 4, /* unknown tok_dtype */
+    TOK_ERR_ALIAS = 5, /* an input buffer overlaps an output buffer */
+    TOK_ERR_CUDA = 6   /* the kernel launch failed; see tok_last_cuda_error() */
+} tok_status;
+
+typedef enum {
+    TOK_F32 = 0,  /* IEEE binary32 */
+    TOK_BF16 = 1  /* bfloat16: fp32 accumulation inside, one round-to-nearest-even at the store */
+} tok_dtype;
+
+/* TOK_ABI_VERSION of the loaded library. */
+int tok_abi_version(void);
+
+/* Static, NUL-terminated name of a status code. */
+const char *tok_status_str(tok_status status);
+
+/* cudaError_t of the last launch that returned TOK_ERR_CUDA on this thread (0 if none). */
+int tok_last_cuda_error(void);
+
+/*
+ * tok_haar_fwd -- two-level causal full-packet Haar patcher.
+ * [guide] 7.1 (Patcher / Patcher3D, patch_size=4, patch_method="haar"),
+ * [guide] 6.1 and 7.3 (t = 1 + (T-1)/4), [card] Model Architecture.
+ *
+ *   x : [B, C, T, H, W] of `dt`           (input, not modified)
+ *   y : [B, 64C, T', H/4, W/4] of `dt`     T' = 1 + (T-1)/4, when T > 1
+ *       [B, 16C, 1,  H/4, W/4] of `dt`     when T == 1 (images: no time axis)
+ *
+ * Each level pairs samples along t, y and x into a low band (a+b)/sqrt(2) and
+ * a high band (a-b)/sqrt(2); on video, a copy of frame 0 is put in front of
+ * the time axis first.  Level 2 transforms all 8C (2D: 4C) first-level
+ * channels.  Output channel (8*s2 + s1)*C + c holds subband s1 of level 1
+ * refined by subband s2 of level 2, s = 4*bt + 2*by + bx (bit 1 = high band);
+ * on the 2D path (4*s2 + s1)*C + c with s = 2*by + bx.
+ * Shape rule: B, C >= 0; T == 1 or T % 4 == 1; H % 4 == 0; W % 4 == 0.
+ */
+tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                        int64_t W, cudaStream_t stream);
+
+/*
+ * tok_haar_inv -- the unpatcher, left inverse of tok_haar_fwd ([guide] 7.1:
+ * UnPatcher / UnPatcher3D; [card] Model Architecture: the decoder ends with
+ * the inverse wavelet transform).
+ *
+ *   y : coefficients laid out as tok_haar_fwd writes them (input)
+ *   x : [B, C, T, H, W] (output); T, H, W are the pixel-space extents.
+ *
+ * Level 2 is undone first, then level 1, each with a = (L+H)/sqrt(2),
+ * b = (L-H)/sqrt(2); after each level the first reconstructed frame (the
+ * replica of frame 0) is dropped.  Same shape rule as tok_haar_fwd.
+ */
+tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                        int64_t W, cudaStream_t stream);
+
+/*
+ * tok_fsq_encode -- fused 1x1 projection + FSQ quantization + index pack.
+ * [guide] 7.2 (bound with tanh, rounding, levels [8,8,8,5,5,5], implicit
+ * codebook of 64000, mixed-radix codes_to_indices), [guide] 6.2 (indices
+ * [B,t,h,w], codes [B,6,t,h,w]), [notes] model architecture item 1.
+ *
+ *   u     : [B, C, S] fp32 latent, S = t*h*w token positions (input)
+ *   w     : [6, C] fp32 projection, row-major (input, device memory)
+ *   idx   : [B, S] int32 indices in [0, 64000) (output)
+ *   codes : [B, 6, S] fp32 normalized codes q_i / floor(L_i/2), or NULL
+ *
+ * z_i = sum_c w[i][c] * u[c] is evaluated in fp32 as a chain of fused
+ * multiply-adds over c = 0..C-1 from 0.  Channel i (L levels) is quantized to
+ * q = round(tanh(z + shift)*half - off), half = (L-1)(1+1e-3)/2, off = 0.5
+ * for even L else 0, shift = atanh(off/half); the digit q + floor(L/2) of
+ * channel i has place value (1, 8, 64, 512, 2560, 12800)[i].  The kernel
+ * compares z against the exact fp32 decision thresholds of that function.
+ * Shape rule: B, S >= 0; 1 <= C <= 4096.
+ */
+tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, float *codes, int64_t B, int64_t C,
+                          int64_t S, cudaStream_t stream);
+
+/*
+ * tok_fsq_decode -- index unpack (indices_to_codes, [guide] 7.2) + 1x1 6->C
+ * projection with the transposed encode weight.
+ *
+ *   idx       : [B, S] int32 (input)
+ *   w         : [6, C] fp32 (input; the same matrix tok_fsq_encode takes)
+ *   out       : [B, C, S] fp32, out[c] = sum_i w[i][c] * zhat_i (output)
+ *   bad_count : device int32 counter or NULL.  Each index outside [0, 64000)
+ *               adds 1 (atomically) and its token's C outputs are NaN.
+ *               The caller zeroes it; the library only adds to it.
+ * Shape rule: B, S >= 0; 1 <= C <= 4096.
+ */
+tok_status tok_fsq_decode(const int32_t *idx, const float *w, float *out, int32_t *bad_count, int64_t B,
+                          int64_t C, int64_t S, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TOK_H */

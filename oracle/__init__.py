@@ -1,0 +1,186 @@
+"""CPU oracle for the Haar patcher and the FSQ quantizer.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference legs of ``bench.py`` may import this package.  The
+product (``haar_wavelet_patching_b200``) never imports it and has no CPU
+fallback.
+
+The arithmetic lives in plain C (``haar.c``, ``fsq.c``) in double precision;
+this module only marshals numpy arrays through ctypes.  Each C function cites
+the page and section it follows.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from .build import build as _build
+
+_lib = None
+
+FSQ_LEVELS = (8, 8, 8, 5, 5, 5)
+FSQ_CODEBOOK = 64000
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        # ORACLE_SO lets the mutation test load a copy of the oracle with a planted mistake.
+        path = os.environ.get("ORACLE_SO") or _build()
+        lib = ctypes.CDLL(path)
+        i64, dp, fp = ctypes.c_int64, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_float)
+        for name in ("oracle_haar_fwd", "oracle_haar_inv", "oracle_haar_fwd_blockform"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [dp, dp, i64, i64, i64, i64, i64]
+        lib.oracle_haar_level_fwd.restype = ctypes.c_int
+        lib.oracle_haar_level_fwd.argtypes = [dp, dp, i64, i64, i64, i64]
+        lib.oracle_haar_out_frames.restype = i64
+        lib.oracle_haar_out_frames.argtypes = [i64]
+        lib.oracle_fsq_levels.restype = ctypes.c_int
+        lib.oracle_fsq_levels.argtypes = [ctypes.c_int]
+        lib.oracle_fsq_basis.restype = i64
+        lib.oracle_fsq_basis.argtypes = [ctypes.c_int]
+        lib.oracle_fsq_bound.restype = ctypes.c_double
+        lib.oracle_fsq_bound.argtypes = [ctypes.c_double, ctypes.c_int]
+        lib.oracle_fsq_quantize.restype = ctypes.c_int
+        lib.oracle_fsq_quantize.argtypes = [ctypes.c_float, ctypes.c_int]
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_fsq_pack.restype = i64
+        lib.oracle_fsq_pack.argtypes = [ip]
+        lib.oracle_fsq_unpack.restype = None
+        lib.oracle_fsq_unpack.argtypes = [i64, ip]
+        i32p = ctypes.POINTER(ctypes.c_int32)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        lib.oracle_fsq_encode.restype = i64
+        lib.oracle_fsq_encode.argtypes = [fp, fp, i64, i64, i64, i32p, dp, u8p]
+        lib.oracle_fsq_decode.restype = i64
+        lib.oracle_fsq_decode.argtypes = [i32p, fp, i64, i64, i64, dp]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a, ctype):
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"{what}: oracle rejected the shape (code {rc})")
+
+
+def out_frames(T: int) -> int:
+    """Latent frames of the two-level patcher: 1 + (T-1)/4, or 1 for an image."""
+    return int(_load().oracle_haar_out_frames(T))
+
+
+def haar_out_shape(B, C, T, H, W):
+    if T == 1:
+        return (B, 16 * C, 1, H // 4, W // 4)
+    return (B, 64 * C, out_frames(T), H // 4, W // 4)
+
+
+def haar_fwd(x: np.ndarray) -> np.ndarray:
+    """Two-level causal full-packet Haar patcher, level by level, in double.
+
+    x: [B, C, T, H, W] (any real dtype; converted exactly to float64).
+    Returns y: [B, 64C, 1+(T-1)/4, H/4, W/4], or [B, 16C, 1, H/4, W/4] if T == 1.
+    """
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, C, T, H, W = x.shape
+    y = np.zeros(haar_out_shape(B, C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_fwd(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double), B, C, T, H, W),
+           "haar_fwd")
+    return y
+
+
+def haar_fwd_blockform(x: np.ndarray) -> np.ndarray:
+    """Same transform through its derived 4x4x4 Walsh-Hadamard block form (pins only)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, C, T, H, W = x.shape
+    y = np.zeros(haar_out_shape(B, C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_fwd_blockform(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double),
+                                             B, C, T, H, W), "haar_fwd_blockform")
+    return y
+
+
+def haar_inv(y: np.ndarray, T: int, H: int, W: int) -> np.ndarray:
+    """Two-level unpatcher; T, H, W are the pixel-space extents.  Returns [B, C, T, H, W]."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    B = y.shape[0]
+    C = y.shape[1] // (16 if T == 1 else 64)
+    if y.shape != haar_out_shape(B, C, T, H, W):
+        raise ValueError(f"haar_inv: coefficient shape {y.shape} does not match T,H,W={T},{H},{W}")
+    x = np.zeros((B, C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_inv(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), B, C, T, H, W),
+           "haar_inv")
+    return x
+
+
+def haar_level_fwd(x: np.ndarray) -> np.ndarray:
+    """One level: [C, T, H, W] -> [8C, (T+1)/2, H/2, W/2] (T odd > 1) or [4C, 1, H/2, W/2] (T == 1)."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    C, T, H, W = x.shape
+    shape = (4 * C, 1, H // 2, W // 2) if T == 1 else (8 * C, (T + 1) // 2, H // 2, W // 2)
+    y = np.zeros(shape, dtype=np.float64)
+    _check(_load().oracle_haar_level_fwd(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double), C, T, H, W),
+           "haar_level_fwd")
+    return y
+
+
+def fsq_basis():
+    return tuple(int(_load().oracle_fsq_basis(i)) for i in range(6))
+
+
+def fsq_bound(z: float, i: int) -> float:
+    return float(_load().oracle_fsq_bound(float(z), i))
+
+
+def fsq_quantize(z: float, i: int) -> int:
+    return int(_load().oracle_fsq_quantize(float(z), i))
+
+
+def fsq_pack(digits) -> int:
+    d = (ctypes.c_int * 6)(*[int(v) for v in digits])
+    return int(_load().oracle_fsq_pack(d))
+
+
+def fsq_unpack(idx: int):
+    d = (ctypes.c_int * 6)()
+    _load().oracle_fsq_unpack(int(idx), d)
+    return tuple(d)
+
+
+def fsq_encode(u: np.ndarray, w: np.ndarray):
+    """Projection C->6 (fp32 fmaf chain) + tanh bound + round + index pack.
+
+    u: [B, C, S] float32; w: [6, C] float32.
+    Returns (idx [B,S] int32, codes [B,6,S] float64, near [B,S] bool).
+    """
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    B, C, S = u.shape
+    if w.shape != (6, C):
+        raise ValueError(f"fsq_encode: weight shape {w.shape} != (6, {C})")
+    idx = np.zeros((B, S), dtype=np.int32)
+    codes = np.zeros((B, 6, S), dtype=np.float64)
+    near = np.zeros((B, S), dtype=np.uint8)
+    _load().oracle_fsq_encode(_ptr(u, ctypes.c_float), _ptr(w, ctypes.c_float), B, C, S,
+                              _ptr(idx, ctypes.c_int32), _ptr(codes, ctypes.c_double),
+                              _ptr(near, ctypes.c_uint8))
+    return idx, codes, near.astype(bool)
+
+
+def fsq_decode(idx: np.ndarray, w: np.ndarray):
+    """Index unpack -> normalized codes -> 6->C projection, in double.
+
+    idx: [B, S] int32; w: [6, C].  Returns (out [B, C, S] float64, n_bad).
+    """
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    B, S = idx.shape
+    C = w.shape[1]
+    out = np.zeros((B, C, S), dtype=np.float64)
+    bad = _load().oracle_fsq_decode(_ptr(idx, ctypes.c_int32), _ptr(w, ctypes.c_float), B, C, S,
+                                    _ptr(out, ctypes.c_double))
+    return out, int(bad)
