@@ -1,0 +1,421 @@
+"""Benchmark of the tokenizer hot path on B200: Haar patcher + unpatcher + FSQ encode + decode.
+
+One step = tok_haar_fwd and tok_haar_inv on a 121-frame 704x1280 bf16 clip
+([1,3,121,704,1280] -> [1,192,31,176,320] -> back), then tok_fsq_encode and
+tok_fsq_decode on the 64-clip latent grid of that geometry ([64,16,16*44*80]
+fp32, 16 -> 6 projection, levels (8,8,8,5,5,5)).  Inputs are seeded synthetic
+data resident in HBM; every input (654 MB clip, 231 MB latent) is larger than
+the 126 MB L2, so nothing is flushed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU, weak scaling)
+
+Rank 0 prints one JSON line.  ``value`` is algorithmic bytes moved per second
+(GB/s) summed over all ranks, timed on the device with CUDA events between
+barriers, max over ranks.  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload on the host cores instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Haar fwd/inv + FSQ enc/dec GB/s & Mvoxel/s at 121x704x1280 bf16; % HBM peak"
+CLIP = (1, 3, 121, 704, 1280)          # bf16 clip
+LATENT = (64, 16, 16 * 44 * 80)        # fp32 latent grid: 64 clips at 8x16x16 compression
+FALLBACK_HBM_GBS = 6650.0
+# Bounded sample for the CPU oracle: the first 33 frames of the clip, 8 of the 64 latent grids.
+CPU_SAMPLE_FRAMES = 33
+CPU_SAMPLE_GRIDS = 8
+
+
+def haar_bytes(shape, elem=2):
+    B, C, T, H, W = shape
+    tq = 1 if T == 1 else 1 + (T - 1) // 4
+    nx = B * C * T * H * W
+    ny = B * C * (16 if T == 1 else 64) * tq * (H // 4) * (W // 4)
+    return nx * elem, ny * elem
+
+
+def fsq_bytes(shape):
+    B, C, S = shape
+    return B * C * S * 4, B * S * 4
+
+
+def step_bytes(clip=CLIP, latent=LATENT):
+    hx, hy = haar_bytes(clip)
+    fu, fi = fsq_bytes(latent)
+    return {"haar_fwd": hx + hy, "haar_inv": hx + hy, "fsq_encode": fu + fi, "fsq_decode": fu + fi}
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "haar_wavelet_patching_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    digest = kernel_source_digest()
+    for ln in lines:
+        parts = [p.strip() for p in ln.strip().strip("|").split("|")]
+        if len(parts) >= 3 and parts[0] == kernel and parts[2] == digest:
+            try:
+                return float(parts[1])
+            except ValueError:
+                return None
+    return None
+
+
+def max_over_ranks(v: float, device) -> float:
+    """Max of a per-rank time over the default process group (any backend); v itself on one rank."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return v
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Weak scaling: every rank moves bytes_per_step per step; GB/s of the whole job over the slowest rank."""
+    return world * bytes_per_step * steps / (max_ms / 1e3) / 1e9
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append((time.time(), ln.strip()))
+
+    def stop(self, t0, t1):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait(timeout=5)
+        rows = [ln for ts, ln in self.lines if t0 - 0.15 <= ts <= t1 + 0.15] or [ln for _, ln in self.lines[-3:]]
+        mhz, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for r in rows:
+            f = [v.strip() for v in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                mhz.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(mhz)) if mhz else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+# ---------------------------------------------------------------------------
+# The CPU oracle on a bounded sample (cpu_baseline and --impl reference).
+# ---------------------------------------------------------------------------
+def oracle_sample_inputs(frames=CPU_SAMPLE_FRAMES, grids=CPU_SAMPLE_GRIDS):
+    import synth
+    clip = synth.smooth_field((1, 3, frames, 704, 1280), seed=3)  # the first frames of the benchmark clip
+    lat = synth.fsq_input(4)[:grids]
+    return synth.bf16_bits_to_f64(clip), lat, synth.fsq_weight()
+
+
+def oracle_step(x64, lat, w):
+    import oracle
+    y = oracle.haar_fwd(x64)
+    oracle.haar_inv(y, *x64.shape[2:])
+    idx, _, _ = oracle.fsq_encode(lat, w)
+    oracle.fsq_decode(idx, w)
+
+
+def oracle_sample_bytes(frames=CPU_SAMPLE_FRAMES, grids=CPU_SAMPLE_GRIDS):
+    b = step_bytes((1, 3, frames, 704, 1280), (grids,) + LATENT[1:])
+    return sum(b.values())
+
+
+def sample_text(frames, grids):
+    return (f"clip frames [0,{frames}) of [1,3,121,704,1280] bf16 (Haar fwd+inv) and {grids} of 64 latent "
+            f"grids (FSQ enc+dec); single-threaded C oracle in double")
+
+
+def cpu_baseline(reps=3):
+    x64, lat, w = oracle_sample_inputs()
+    oracle_step(x64, lat, w)  # load / warm
+    t = time.perf_counter()
+    for _ in range(reps):
+        oracle_step(x64, lat, w)
+    dt = (time.perf_counter() - t) / reps
+    return {"value": round(oracle_sample_bytes() / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"{sample_text(CPU_SAMPLE_FRAMES, CPU_SAMPLE_GRIDS)}; {reps} reps of {dt:.2f} s"}
+
+
+def reference_sample(steps, warmup, budget_s=150.0):
+    """Per-step sample (frames = 1 + 4m, grids) sized so steps + warmup oracle passes take about budget_s."""
+    x64, lat, w = oracle_sample_inputs(5, 1)
+    t = time.perf_counter()
+    oracle_step(x64, lat, w)
+    probe = time.perf_counter() - t
+    scale = budget_s / max(steps + warmup, 1) / max(probe, 1e-3)
+    m = int(max(1, min(30, scale)))          # latent frames beyond the first, up to the whole clip
+    grids = int(max(1, min(64, scale)))
+    return 1 + 4 * m, grids
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    frames, grids = reference_sample(args.steps, args.warmup)
+    x64, lat, w = oracle_sample_inputs(frames, grids)
+    for _ in range(args.warmup):
+        oracle_step(x64, lat, w)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(x64, lat, w)
+    dt = (time.perf_counter() - t) / max(args.steps, 1)
+    value = oracle_sample_bytes(frames, grids) / dt / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": "per step: " + sample_text(frames, grids)},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def workload_config():
+    return {"workload": "clip [1,3,121,704,1280] bf16 Haar fwd+inv; latent [64,16,16x44x80] fp32 FSQ enc+dec",
+            "clip": list(CLIP), "coeffs": [1, 192, 31, 176, 320], "latent": list(LATENT), "levels": [8, 8, 8, 5, 5, 5],
+            "fsq_codes_output": False, "l2": "no flush: every input is larger than the 126 MB L2",
+            "parallelism": "data-parallel replicas, one per GPU"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm.
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import haar_wavelet_patching_b200 as hwp
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream(dev)
+
+    # Inputs: seeded, generated on the host, pinned, copied once to HBM.
+    x_host = torch.from_numpy(synth.haar_input(3).view(np.int16)).view(torch.bfloat16).pin_memory()
+    u_host = torch.from_numpy(synth.fsq_input(4)).pin_memory()
+    w_dev = torch.from_numpy(synth.fsq_weight()).to(dev)
+    x = x_host.to(dev)
+    u = u_host.to(dev)
+    y = torch.empty(hwp.haar_coeff_shape(*CLIP), dtype=torch.bfloat16, device=dev)
+    xr = torch.empty_like(x)
+    idx = torch.empty(LATENT[0], LATENT[2], dtype=torch.int32, device=dev)
+    ur = torch.empty_like(u)
+    T, H, W = CLIP[2:]
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        hwp.tok_haar_fwd(x, y)
+        if ev is not None:
+            ev[1].record(stream)
+        hwp.tok_haar_inv(y, xr)
+        if ev is not None:
+            ev[2].record(stream)
+        hwp.tok_fsq_encode(u, w_dev, idx)
+        if ev is not None:
+            ev[3].record(stream)
+        hwp.tok_fsq_decode(idx, w_dev, ur)
+        if ev is not None:
+            ev[4].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(K)]
+    try:
+        gpu_id = f"GPU-{torch.cuda.get_device_properties(dev).uuid}"
+    except (AttributeError, RuntimeError):
+        gpu_id = str(local_rank)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for k in range(K):
+        step(evs[k])
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    clocks = sampler.stop(t0, t1)
+
+    total_ms = max_over_ranks(evs[0][0].elapsed_time(evs[K - 1][4]), dev)
+    names = ("haar_fwd", "haar_inv", "fsq_encode", "fsq_decode")
+    per = {n: float(np.mean([evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(K)])) for i, n in enumerate(names)}
+    ms_per_step = total_ms / K
+    sb = step_bytes()
+    bytes_step = sum(sb.values())
+    value = job_throughput(bytes_step, K, world, total_ms)
+
+    # End to end through the C ABI with host buffers: pinned H2D of the clip and latent, the four calls,
+    # D2H of the coefficients, the reconstruction, the indices and the decoded latent.
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    xr_host = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+    idx_host = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    ur_host = torch.empty(u.shape, dtype=u.dtype).pin_memory()
+    h2d = x_host.numel() * 2 + u_host.numel() * 4
+    d2h = y.numel() * 2 + xr.numel() * 2 + idx.numel() * 4 + ur.numel() * 4
+    Ke = max(3, min(K, 10))
+
+    def e2e_step():
+        x.copy_(x_host, non_blocking=True)
+        u.copy_(u_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+        xr_host.copy_(xr, non_blocking=True)
+        idx_host.copy_(idx, non_blocking=True)
+        ur_host.copy_(ur, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    barrier()
+
+    if rank != 0:
+        return 0
+    peak, peak_kind = measured_peak()
+    dom = max(("haar_fwd", "haar_inv"), key=lambda n: per[n])
+    achieved = sb[dom] / (per[dom] / 1e3) / 1e9
+    voxels = CLIP[0] * CLIP[2] * CLIP[3] * CLIP[4]
+    tokens = LATENT[0] * LATENT[2]
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_config(),
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1), "peak": peak,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6.65 TB/s", "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": recorded_traffic(dom), "algorithmic_bytes_per_launch": sb[dom]},
+        "per_kernel": {n: {"ms": round(per[n], 4), "GB/s": round(sb[n] / (per[n] / 1e3) / 1e9, 1),
+                           "frac_of_peak": round(sb[n] / (per[n] / 1e3) / 1e9 / peak, 4),
+                           "bytes": sb[n]} for n in names},
+        "mvoxel_per_s": {"haar_fwd": round(voxels / per["haar_fwd"] / 1e3, 1),
+                         "haar_inv": round(voxels / per["haar_inv"] / 1e3, 1)},
+        "mtoken_per_s": {"fsq_encode": round(tokens / per["fsq_encode"] / 1e3, 1),
+                         "fsq_decode": round(tokens / per["fsq_decode"] / 1e3, 1)},
+        "e2e": {"value": round(job_throughput(bytes_step, Ke, world, e2e_ms), 2), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": Ke,
+                "ms_per_step": round(e2e_ms / Ke, 3)},
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,216 @@
+"""B200 Haar patcher / unpatcher and FSQ quantizer: Python binding of libtok.so.
+
+The functions named like the C ABI (``tok_haar_fwd`` ...) marshal torch CUDA
+tensors into the C calls of ``include/tok.h`` and nothing else: every step of
+the computation runs in the library's sm_100a kernels.  There is no CPU path;
+a missing library or a CPU tensor raises.
+
+Convenience wrappers (``haar_fwd``, ``haar_inv``, ``fsq_encode``,
+``fsq_decode``) allocate outputs with torch and call the same entry points.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtok.so")
+
+TOK_OK, TOK_ERR_NULL, TOK_ERR_SHAPE, TOK_ERR_ALIGN, TOK_ERR_DTYPE, TOK_ERR_ALIAS, TOK_ERR_CUDA = range(7)
+TOK_F32, TOK_BF16 = 0, 1
+FSQ_CODEBOOK = 64000
+FSQ_DIM = 6
+
+# Every symbol include/tok.h declares.
+ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_haar_fwd", "tok_haar_inv",
+               "tok_fsq_encode", "tok_fsq_decode")
+
+_lib = None
+
+
+class TokError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        msg = lib().tok_status_str(status).decode()
+        if status == TOK_ERR_CUDA:
+            msg += f" (cudaError {lib().tok_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}")
+
+
+def lib():
+    """The loaded libtok.so; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m haar_wavelet_patching_b200.build` "
+                              "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+        L.tok_abi_version.restype = i32
+        L.tok_abi_version.argtypes = []
+        L.tok_status_str.restype = ctypes.c_char_p
+        L.tok_status_str.argtypes = [i32]
+        L.tok_last_cuda_error.restype = i32
+        L.tok_last_cuda_error.argtypes = []
+        for f in (L.tok_haar_fwd, L.tok_haar_inv):
+            f.restype = i32
+            f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
+        L.tok_fsq_encode.restype = i32
+        L.tok_fsq_encode.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+        L.tok_fsq_decode.restype = i32
+        L.tok_fsq_decode.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
+        _lib = L
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return TOK_F32
+    if t.dtype == torch.bfloat16:
+        return TOK_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: the patcher takes float32 or bfloat16")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _stream(t: torch.Tensor, stream):
+    if stream is None:
+        stream = torch.cuda.current_stream(t.device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(status, what):
+    if status != TOK_OK:
+        raise TokError(status, what)
+
+
+# ---------------------------------------------------------------------------
+# Shape rules (host logic).
+# ---------------------------------------------------------------------------
+def latent_frames(T: int) -> int:
+    """1 + (T-1)/4 latent frames for T = 1 + 4k video frames; 1 for an image."""
+    if T == 1:
+        return 1
+    if T < 1 or T % 4 != 1:
+        raise ValueError(f"T={T}: the causal two-level patcher needs T == 1 or T % 4 == 1")
+    return 1 + (T - 1) // 4
+
+
+def haar_coeff_shape(B, C, T, H, W):
+    if H % 4 or W % 4:
+        raise ValueError(f"H={H}, W={W} must be multiples of 4")
+    return (B, (16 if T == 1 else 64) * C, latent_frames(T), H // 4, W // 4)
+
+
+# ---------------------------------------------------------------------------
+# C-ABI calls.
+# ---------------------------------------------------------------------------
+def tok_haar_fwd(x: torch.Tensor, y: torch.Tensor, stream=None):
+    """x [B,C,T,H,W] -> y [B,64C,T',H/4,W/4] (T == 1: [B,16C,1,H/4,W/4]); same dtype."""
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5:
+        raise ValueError("x must be [B, C, T, H, W]")
+    if y.dtype != x.dtype:
+        raise TypeError("x and y must have the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != haar_coeff_shape(B, C, T, H, W):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {haar_coeff_shape(B, C, T, H, W)}")
+    _check(lib().tok_haar_fwd(_ptr(x), _ptr(y), _dtype_code(x), B, C, T, H, W, _stream(x, stream)), "tok_haar_fwd")
+    return y
+
+
+def tok_haar_inv(y: torch.Tensor, x: torch.Tensor, stream=None):
+    """Coefficients y -> x [B,C,T,H,W] (the output's shape gives T, H, W)."""
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5:
+        raise ValueError("x must be [B, C, T, H, W]")
+    if y.dtype != x.dtype:
+        raise TypeError("x and y must have the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != haar_coeff_shape(B, C, T, H, W):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {haar_coeff_shape(B, C, T, H, W)}")
+    _check(lib().tok_haar_inv(_ptr(y), _ptr(x), _dtype_code(x), B, C, T, H, W, _stream(x, stream)), "tok_haar_inv")
+    return x
+
+
+def _latent_dims(u: torch.Tensor):
+    if u.dim() < 2:
+        raise ValueError("latent must be [B, C, ...]")
+    B, C = u.shape[0], u.shape[1]
+    S = 1
+    for d in u.shape[2:]:
+        S *= d
+    return B, C, S
+
+
+def tok_fsq_encode(u: torch.Tensor, w: torch.Tensor, idx: torch.Tensor, codes: torch.Tensor = None, stream=None):
+    """u [B,C,...] fp32, w [6,C] fp32 -> idx [B,...] int32 (+ codes [B,6,...] fp32)."""
+    for t, n in ((u, "u"), (w, "w"), (idx, "idx"), (codes, "codes")):
+        _cuda(t, n)
+    B, C, S = _latent_dims(u)
+    if u.dtype != torch.float32 or w.dtype != torch.float32 or idx.dtype != torch.int32:
+        raise TypeError("u and w must be float32, idx int32")
+    if tuple(w.shape) != (FSQ_DIM, C):
+        raise ValueError(f"w must be [6, {C}]")
+    if idx.numel() != B * S or (codes is not None and (codes.numel() != B * FSQ_DIM * S or codes.dtype != torch.float32)):
+        raise ValueError("idx must hold B*S int32 and codes B*6*S float32")
+    _check(lib().tok_fsq_encode(_ptr(u), _ptr(w), _ptr(idx), _ptr(codes), B, C, S, _stream(u, stream)),
+           "tok_fsq_encode")
+    return idx, codes
+
+
+def tok_fsq_decode(idx: torch.Tensor, w: torch.Tensor, out: torch.Tensor, bad_count: torch.Tensor = None,
+                   stream=None):
+    """idx [B,...] int32, w [6,C] -> out [B,C,...] fp32; bad_count: optional 1-element int32 CUDA tensor."""
+    for t, n in ((idx, "idx"), (w, "w"), (out, "out"), (bad_count, "bad_count")):
+        _cuda(t, n)
+    B, C, S = _latent_dims(out)
+    if idx.dtype != torch.int32 or w.dtype != torch.float32 or out.dtype != torch.float32:
+        raise TypeError("idx must be int32, w and out float32")
+    if tuple(w.shape) != (FSQ_DIM, C) or idx.numel() != B * S:
+        raise ValueError(f"w must be [6, {C}] and idx hold B*S = {B * S} indices")
+    if bad_count is not None and (bad_count.dtype != torch.int32 or bad_count.numel() < 1):
+        raise ValueError("bad_count must be an int32 CUDA tensor")
+    _check(lib().tok_fsq_decode(_ptr(idx), _ptr(w), _ptr(out), _ptr(bad_count), B, C, S, _stream(idx, stream)),
+           "tok_fsq_decode")
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Allocating wrappers.
+# ---------------------------------------------------------------------------
+def haar_fwd(x: torch.Tensor, stream=None) -> torch.Tensor:
+    y = torch.empty(haar_coeff_shape(*x.shape), dtype=x.dtype, device=x.device)
+    return tok_haar_fwd(x, y, stream)
+
+
+def haar_inv(y: torch.Tensor, T: int, H: int, W: int, stream=None) -> torch.Tensor:
+    B = y.shape[0]
+    C = y.shape[1] // (16 if T == 1 else 64)
+    x = torch.empty((B, C, T, H, W), dtype=y.dtype, device=y.device)
+    return tok_haar_inv(y, x, stream)
+
+
+def fsq_encode(u: torch.Tensor, w: torch.Tensor, with_codes: bool = False, stream=None):
+    B = u.shape[0]
+    idx = torch.empty((B,) + tuple(u.shape[2:]), dtype=torch.int32, device=u.device)
+    codes = torch.empty((B, FSQ_DIM) + tuple(u.shape[2:]), dtype=torch.float32, device=u.device) if with_codes else None
+    tok_fsq_encode(u, w, idx, codes, stream)
+    return (idx, codes) if with_codes else idx
+
+
+def fsq_decode(idx: torch.Tensor, w: torch.Tensor, bad_count: torch.Tensor = None, stream=None) -> torch.Tensor:
+    out = torch.empty((idx.shape[0], w.shape[1]) + tuple(idx.shape[1:]), dtype=torch.float32, device=idx.device)
+    return tok_fsq_decode(idx, w, out, bad_count, stream)

@@ -1,0 +1,437 @@
+// Two-level causal full-packet Haar patcher and unpatcher for sm_100a.
+//
+// Sources: "NVIDIA Cosmos Tokenizer 完全指南", section 7.1 (Patcher, Patcher3D,
+// UnPatcher, UnPatcher3D; taps 1/sqrt(2); c -> 4c / 8c per level; frame 0
+// repeated; patch_size=4 = two levels), sections 6.1 and 7.3 (t = 1 + (T-1)/4);
+// "nvidia/Cosmos-Tokenize1-CV8x8x8-720p" model card, Model Architecture.
+//
+// Kernel design.  The two levels are not run as two passes: along one axis,
+// two full-packet levels on four samples are the 4-point Walsh-Hadamard
+// transform (coefficient k = 2*b2 + b1 equals (1/2) sum_n (-1)^popcount(k&n) x_n),
+// and the two frame-0 replicas compose into "output frame 0 reads four copies of
+// frame 0, output frame t' >= 1 reads frames 4t'-3 .. 4t'".  So every 4x4x4 block
+// of the clip maps to one value in each of 64C channel planes, with +-1
+// butterflies in fp32 and one exact scale by 1/8 (1/4 in 2D).  The
+// transform is its own inverse up to that scale, so the unpatcher runs the same
+// butterflies; its output frame 0 is sample 3 of window 0 (the replicas are
+// dropped level by level, which keeps the last copy).
+//
+// Memory: the path moves each input byte and each output byte once and does
+// ~7 flops per element, so it is bound by HBM.  A thread owns NB horizontally
+// adjacent blocks: it reads 16 (3D) or 4 (2D) input rows of 4*NB contiguous
+// elements (one or two 16-byte loads per row; a warp covers 512 contiguous
+// bytes per row) and writes NB contiguous elements to each of the 64C (16C)
+// channel planes (a warp covers 32*NB contiguous elements per plane).  All
+// arithmetic stays in registers; nothing is staged through shared memory.
+#include "tok_common.cuh"
+
+namespace tok {
+namespace {
+
+// One axis of the two-level transform, unnormalized, in place (natural order).
+__device__ __forceinline__ void haar4(float &a0, float &a1, float &a2, float &a3)
+{
+    const float l0 = a0 + a1, h0 = a0 - a1, l1 = a2 + a3, h1 = a2 - a3; // level 1
+    a0 = l0 + l1;                                                        // k = 0: low, low
+    a1 = h0 + h1;                                                        // k = 1: level-1 high
+    a2 = l0 - l1;                                                        // k = 2: level-2 high
+    a3 = h0 - h1;                                                        // k = 3: high, high
+}
+
+// Output channel group (in units of C) of the coefficient with per-axis index k.
+// s_l = 4*bt_l + 2*by_l + bx_l; channel group = 8*s2 + s1 (2D: 4*s2 + s1).
+__host__ __device__ constexpr int group3d(int kt, int ky, int kx)
+{
+    return 8 * (4 * (kt >> 1) + 2 * (ky >> 1) + (kx >> 1)) + (4 * (kt & 1) + 2 * (ky & 1) + (kx & 1));
+}
+__host__ __device__ constexpr int group2d(int ky, int kx)
+{
+    return 4 * (2 * (ky >> 1) + (kx >> 1)) + (2 * (ky & 1) + (kx & 1));
+}
+
+// Per-axis indices of channel group g (the inverse of group3d / group2d), so the
+// kernels can walk the channel planes in address order with one pointer.
+__host__ __device__ constexpr int kt_of(int g) { return 2 * ((g >> 3) >> 2) + ((g & 7) >> 2); }
+__host__ __device__ constexpr int ky_of(int g) { return 2 * (((g >> 3) >> 1) & 1) + (((g & 7) >> 1) & 1); }
+__host__ __device__ constexpr int kx_of(int g) { return 2 * ((g >> 3) & 1) + (g & 1); }
+__host__ __device__ constexpr int ky2_of(int g) { return 2 * ((g >> 2) >> 1) + ((g & 3) >> 1); }
+__host__ __device__ constexpr int kx2_of(int g) { return 2 * ((g >> 2) & 1) + (g & 1); }
+static_assert(group3d(kt_of(37), ky_of(37), kx_of(37)) == 37, "group3d inverse");
+static_assert(group2d(ky2_of(13), kx2_of(13)) == 13, "group2d inverse");
+
+constexpr int kThreads = 128;
+
+struct Geometry {
+    int64_t BC;      // B*C (plane pairs)
+    int64_t C;       // input channels
+    int64_t T, H, W; // pixel extents
+    int64_t Tq, h, w; // latent extents
+    int64_t wn;       // thread columns per row = w / NB
+};
+
+// ---------------------------------------------------------------------------
+// Forward, video: x [B,C,T,H,W] -> y [B,64C,Tq,h,w].
+// grid.x covers the (i, jn) items of one latent frame, grid.y the latent frame,
+// grid.z the (b, c) pair; y and z loop when the grid is capped.
+// ---------------------------------------------------------------------------
+template <typename T, int NB, bool VEC>
+__global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restrict__ x, T *__restrict__ y, Geometry g)
+{
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.wn)
+        return;
+    const int64_t i = item / g.wn;
+    const int64_t j0 = (item - i * g.wn) * NB;
+    const int64_t plane_in = g.H * g.W, plane_out = g.Tq * g.h * g.w;
+    const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y; // (b, c, t')
+    if (pair >= g.BC * g.Tq)
+        return;
+    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t b = bc / g.C, c = bc - b * g.C;
+    const T *xc = x + bc * g.T * plane_in + (4 * i) * g.W + 4 * j0;
+    T *yc = y + (b * 64 * g.C + c) * plane_out + i * g.w + j0;
+    {
+        {
+            float v[NB][4][4][4]; // [block][t][y][x]
+            if (tq == 0) {
+                // Output frame 0 reads frame 0 four times.
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    float row[4 * NB];
+                    Row<T, 4 * NB, VEC>::load(xc + r * g.W, row);
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int d = 0; d < 4; ++d) {
+                            const float s = row[4 * nb + d];
+                            v[nb][0][r][d] = s;
+                            v[nb][1][r][d] = s;
+                            v[nb][2][r][d] = s;
+                            v[nb][3][r][d] = s;
+                        }
+                }
+            } else {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        float row[4 * NB];
+                        Row<T, 4 * NB, VEC>::load(xc + (4 * tq - 3 + a) * plane_in + r * g.W, row);
+#pragma unroll
+                        for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                v[nb][a][r][d] = row[4 * nb + d];
+                    }
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        haar4(v[nb][a][r][0], v[nb][a][r][1], v[nb][a][r][2], v[nb][a][r][3]);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int d = 0; d < 4; ++d)
+                        haar4(v[nb][a][0][d], v[nb][a][1][d], v[nb][a][2][d], v[nb][a][3][d]);
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int d = 0; d < 4; ++d)
+                        haar4(v[nb][0][r][d], v[nb][1][r][d], v[nb][2][r][d], v[nb][3][r][d]);
+            }
+            T *yp = yc + tq * g.h * g.w;
+            const int64_t cstride = g.C * plane_out;
+#pragma unroll
+            for (int grp = 0; grp < 64; ++grp, yp += cstride) {
+                float o[NB];
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+                    o[nb] = v[nb][kt_of(grp)][ky_of(grp)][kx_of(grp)] * 0.125f;
+                Row<T, NB, VEC>::store(yp, o);
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Inverse, video: y [B,64C,Tq,h,w] -> x [B,C,T,H,W].
+// ---------------------------------------------------------------------------
+template <typename T, int NB, bool VEC>
+__global__ void __launch_bounds__(kThreads) haar3d_inv_kernel(const T *__restrict__ y, T *__restrict__ x, Geometry g)
+{
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.wn)
+        return;
+    const int64_t i = item / g.wn;
+    const int64_t j0 = (item - i * g.wn) * NB;
+    const int64_t plane_in = g.Tq * g.h * g.w, plane_out = g.H * g.W;
+    const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y; // (b, c, t')
+    if (pair >= g.BC * g.Tq)
+        return;
+    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t b = bc / g.C, c = bc - b * g.C;
+    const T *yc = y + (b * 64 * g.C + c) * plane_in + i * g.w + j0;
+    T *xc = x + bc * g.T * plane_out + (4 * i) * g.W + 4 * j0;
+    {
+        {
+            float v[NB][4][4][4]; // [block][kt][ky][kx] -> [block][t][y][x]
+            const T *yp = yc + tq * g.h * g.w;
+            const int64_t cstride = g.C * plane_in;
+#pragma unroll
+            for (int grp = 0; grp < 64; ++grp, yp += cstride) {
+                float in[NB];
+                Row<T, NB, VEC>::load(yp, in);
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+                    v[nb][kt_of(grp)][ky_of(grp)][kx_of(grp)] = in[nb];
+            }
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        haar4(v[nb][a][r][0], v[nb][a][r][1], v[nb][a][r][2], v[nb][a][r][3]);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int d = 0; d < 4; ++d)
+                        haar4(v[nb][a][0][d], v[nb][a][1][d], v[nb][a][2][d], v[nb][a][3][d]);
+#pragma unroll
+                for (int r = 0; r < 4; ++r)
+#pragma unroll
+                    for (int d = 0; d < 4; ++d)
+                        haar4(v[nb][0][r][d], v[nb][1][r][d], v[nb][2][r][d], v[nb][3][r][d]);
+            }
+            // Window 0 rebuilds frame 0 as its last sample; window t' >= 1 rebuilds frames 4t'-3 .. 4t'.
+            const int a_first = (tq == 0) ? 3 : 0;
+#pragma unroll
+            for (int a = 0; a < 4; ++a) {
+                if (a < a_first)
+                    continue;
+                const int64_t f = (tq == 0) ? 0 : 4 * tq - 3 + a;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    float row[4 * NB];
+#pragma unroll
+                    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            row[4 * nb + d] = v[nb][a][r][d] * 0.125f;
+                    Row<T, 4 * NB, VEC>::store(xc + f * plane_out + r * g.W, row);
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Image path (T == 1): x [B,C,1,H,W] <-> y [B,16C,1,h,w].
+// ---------------------------------------------------------------------------
+template <typename T, int NB, bool VEC>
+__global__ void __launch_bounds__(kThreads) haar2d_fwd_kernel(const T *__restrict__ x, T *__restrict__ y, Geometry g)
+{
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.wn)
+        return;
+    const int64_t i = item / g.wn;
+    const int64_t j0 = (item - i * g.wn) * NB;
+    const int64_t plane_out = g.h * g.w;
+    const int64_t bc = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if (bc >= g.BC)
+        return;
+    {
+        const int64_t b = bc / g.C, c = bc - b * g.C;
+        const T *xc = x + bc * g.H * g.W + (4 * i) * g.W + 4 * j0;
+        T *yc = y + (b * 16 * g.C + c) * plane_out + i * g.w + j0;
+        float v[NB][4][4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float row[4 * NB];
+            Row<T, 4 * NB, VEC>::load(xc + r * g.W, row);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int d = 0; d < 4; ++d)
+                    v[nb][r][d] = row[4 * nb + d];
+        }
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                haar4(v[nb][r][0], v[nb][r][1], v[nb][r][2], v[nb][r][3]);
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                haar4(v[nb][0][d], v[nb][1][d], v[nb][2][d], v[nb][3][d]);
+        }
+        T *yp = yc;
+        const int64_t cstride = g.C * plane_out;
+#pragma unroll
+        for (int grp = 0; grp < 16; ++grp, yp += cstride) {
+            float o[NB];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                o[nb] = v[nb][ky2_of(grp)][kx2_of(grp)] * 0.25f;
+            Row<T, NB, VEC>::store(yp, o);
+        }
+    }
+}
+
+template <typename T, int NB, bool VEC>
+__global__ void __launch_bounds__(kThreads) haar2d_inv_kernel(const T *__restrict__ y, T *__restrict__ x, Geometry g)
+{
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.wn)
+        return;
+    const int64_t i = item / g.wn;
+    const int64_t j0 = (item - i * g.wn) * NB;
+    const int64_t plane_in = g.h * g.w;
+    const int64_t bc = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if (bc >= g.BC)
+        return;
+    {
+        const int64_t b = bc / g.C, c = bc - b * g.C;
+        const T *yc = y + (b * 16 * g.C + c) * plane_in + i * g.w + j0;
+        T *xc = x + bc * g.H * g.W + (4 * i) * g.W + 4 * j0;
+        float v[NB][4][4];
+        const T *yp = yc;
+        const int64_t cstride = g.C * plane_in;
+#pragma unroll
+        for (int grp = 0; grp < 16; ++grp, yp += cstride) {
+            float in[NB];
+            Row<T, NB, VEC>::load(yp, in);
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+                v[nb][ky2_of(grp)][kx2_of(grp)] = in[nb];
+        }
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+                haar4(v[nb][r][0], v[nb][r][1], v[nb][r][2], v[nb][r][3]);
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                haar4(v[nb][0][d], v[nb][1][d], v[nb][2][d], v[nb][3][d]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            float row[4 * NB];
+#pragma unroll
+            for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                for (int d = 0; d < 4; ++d)
+                    row[4 * nb + d] = v[nb][r][d] * 0.25f;
+            Row<T, 4 * NB, VEC>::store(xc + r * g.W, row);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+constexpr int64_t kMaxGridYZ = 65535;
+
+template <typename T, int NB, bool VEC>
+tok_status launch3d(bool fwd, const void *in, void *out, Geometry g, cudaStream_t stream)
+{
+    g.wn = g.w / NB;
+    const int64_t gx = (g.h * g.wn + kThreads - 1) / kThreads;
+    if (gx > 0x7FFFFFFF)
+        return TOK_ERR_SHAPE;
+    const int64_t pairs = g.BC * g.Tq;
+    const unsigned gy = (unsigned)(pairs < kMaxGridYZ ? pairs : kMaxGridYZ);
+    const int64_t gz = (pairs + gy - 1) / gy;
+    if (gz > kMaxGridYZ)
+        return TOK_ERR_SHAPE;
+    const dim3 grid((unsigned)gx, gy, (unsigned)gz);
+    if (fwd)
+        haar3d_fwd_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    else
+        haar3d_inv_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    return launch_status();
+}
+
+template <typename T, int NB, bool VEC>
+tok_status launch2d(bool fwd, const void *in, void *out, Geometry g, cudaStream_t stream)
+{
+    g.wn = g.w / NB;
+    const int64_t gx = (g.h * g.wn + kThreads - 1) / kThreads;
+    if (gx > 0x7FFFFFFF)
+        return TOK_ERR_SHAPE;
+    const unsigned gy = (unsigned)(g.BC < kMaxGridYZ ? g.BC : kMaxGridYZ);
+    const int64_t gz = (g.BC + gy - 1) / gy;
+    if (gz > kMaxGridYZ)
+        return TOK_ERR_SHAPE;
+    const dim3 grid((unsigned)gx, gy, (unsigned)gz);
+    if (fwd)
+        haar2d_fwd_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    else
+        haar2d_inv_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    return launch_status();
+}
+
+tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                     int64_t W, cudaStream_t stream)
+{
+    if (dt != TOK_F32 && dt != TOK_BF16)
+        return TOK_ERR_DTYPE;
+    if (B < 0 || C < 0 || T < 1 || H < 0 || W < 0 || H % 4 || W % 4 || (T != 1 && T % 4 != 1))
+        return TOK_ERR_SHAPE;
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    Geometry g{};
+    g.C = C;
+    g.T = T;
+    g.H = H;
+    g.W = W;
+    g.Tq = T == 1 ? 1 : 1 + (T - 1) / 4;
+    g.h = H / 4;
+    g.w = W / 4;
+    int64_t nx, ny, bytes_x, bytes_y;
+    if (!prod_ok({B, C}, &g.BC) || !prod_ok({g.BC, T, H, W}, &nx) || !prod_ok({nx, es}, &bytes_x) ||
+        !prod_ok({g.BC, T == 1 ? 16 : 64, g.Tq, g.h, g.w}, &ny) || !prod_ok({ny, es}, &bytes_y))
+        return TOK_ERR_SHAPE;
+    if (nx == 0)
+        return TOK_OK;
+    if (!in || !out)
+        return TOK_ERR_NULL;
+    if (!aligned(in, es) || !aligned(out, es))
+        return TOK_ERR_ALIGN;
+    const int64_t bytes_in = fwd ? bytes_x : bytes_y, bytes_out = fwd ? bytes_y : bytes_x;
+    if (overlaps(in, bytes_in, out, bytes_out))
+        return TOK_ERR_ALIAS;
+
+    const bool a16 = aligned(in, 16) && aligned(out, 16);
+    if (T > 1) {
+        // Two adjacent blocks per thread: 8 input elements per row, pairs per plane.
+        const bool vec = a16 && W % 8 == 0;
+        if (dt == TOK_BF16)
+            return vec ? launch3d<__nv_bfloat16, 2, true>(fwd, in, out, g, stream)
+                       : launch3d<__nv_bfloat16, 1, false>(fwd, in, out, g, stream);
+        return vec ? launch3d<float, 2, true>(fwd, in, out, g, stream)
+                   : launch3d<float, 1, false>(fwd, in, out, g, stream);
+    }
+    // Image path: four adjacent blocks per thread: 16 input elements per row, quads per plane.
+    const bool vec = a16 && W % 16 == 0;
+    if (dt == TOK_BF16)
+        return vec ? launch2d<__nv_bfloat16, 4, true>(fwd, in, out, g, stream)
+                   : launch2d<__nv_bfloat16, 1, false>(fwd, in, out, g, stream);
+    return vec ? launch2d<float, 4, true>(fwd, in, out, g, stream) : launch2d<float, 1, false>(fwd, in, out, g, stream);
+}
+
+} // namespace
+} // namespace tok
+
+extern "C" tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                                   int64_t W, cudaStream_t stream)
+{
+    return tok::haar_call(true, x, y, dt, B, C, T, H, W, stream);
+}
+
+extern "C" tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                                   int64_t W, cudaStream_t stream)
+{
+    return tok::haar_call(false, y, x, dt, B, C, T, H, W, stream);
+}

@@ -46,6 +46,13 @@ extern "C" {
 
 #define TOK_ABI_VERSION 1
 
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define TOK_API __attribute__((visibility("default")))
+#else
+#define TOK_API
+#endif
+
 /* Number of FSQ codes: 8*8*8*5*5*5 ([guide] 7.2, [notes]). */
 #define TOK_FSQ_CODEBOOK 64000
 /* FSQ channels ([guide] 6.2: codes have 6 channels). */
@@ -67,13 +74,13 @@ typedef enum {
 } tok_dtype;
 
 /* TOK_ABI_VERSION of the loaded library. */
-int tok_abi_version(void);
+TOK_API int tok_abi_version(void);
 
 /* Static, NUL-terminated name of a status code. */
-const char *tok_status_str(tok_status status);
+TOK_API const char *tok_status_str(tok_status status);
 
 /* cudaError_t of the last launch that returned TOK_ERR_CUDA on this thread (0 if none). */
-int tok_last_cuda_error(void);
+TOK_API int tok_last_cuda_error(void);
 
 /*
  * tok_haar_fwd -- two-level causal full-packet Haar patcher.
@@ -92,7 +99,7 @@ int tok_last_cuda_error(void);
  * on the 2D path (4*s2 + s1)*C + c with s = 2*by + bx.
  * Shape rule: B, C >= 0; T == 1 or T % 4 == 1; H % 4 == 0; W % 4 == 0.
  */
-tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+TOK_API tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                         int64_t W, cudaStream_t stream);
 
 /*
@@ -107,7 +114,7 @@ tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t
  * b = (L-H)/sqrt(2); after each level the first reconstructed frame (the
  * replica of frame 0) is dropped.  Same shape rule as tok_haar_fwd.
  */
-tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+TOK_API tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                         int64_t W, cudaStream_t stream);
 
 /*
@@ -127,9 +134,9 @@ tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t
  * for even L else 0, shift = atanh(off/half); the digit q + floor(L/2) of
  * channel i has place value (1, 8, 64, 512, 2560, 12800)[i].  The kernel
  * compares z against the exact fp32 decision thresholds of that function.
- * Shape rule: B, S >= 0; 1 <= C <= 4096.
+ * Shape rule: B, S >= 0; 1 <= C <= 1024.
  */
-tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, float *codes, int64_t B, int64_t C,
+TOK_API tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, float *codes, int64_t B, int64_t C,
                           int64_t S, cudaStream_t stream);
 
 /*
@@ -142,9 +149,9 @@ tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, float *c
  *   bad_count : device int32 counter or NULL.  Each index outside [0, 64000)
  *               adds 1 (atomically) and its token's C outputs are NaN.
  *               The caller zeroes it; the library only adds to it.
- * Shape rule: B, S >= 0; 1 <= C <= 4096.
+ * Shape rule: B, S >= 0; 1 <= C <= 1024.
  */
-tok_status tok_fsq_decode(const int32_t *idx, const float *w, float *out, int32_t *bad_count, int64_t B,
+TOK_API tok_status tok_fsq_decode(const int32_t *idx, const float *w, float *out, int32_t *bad_count, int64_t B,
                           int64_t C, int64_t S, cudaStream_t stream);
 
 #ifdef __cplusplus

@@ -1,0 +1,115 @@
+"""libtok.so loads on a machine without a GPU, exports every symbol tok.h declares,
+and rejects bad arguments on the host before anything is launched.
+
+No call here reaches a kernel launch: each case fails validation (or is empty)
+first, so the tests run on CPU-only machines.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import haar_wavelet_patching_b200 as hwp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from haar_wavelet_patching_b200.build import build
+    build()
+    return hwp.lib()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(tok_\w+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert names, "no declarations found in include/*.h"
+    assert names == set(hwp.ABI_SYMBOLS)
+    for n in names:
+        assert hasattr(lib, n), f"libtok.so does not export {n}"
+
+
+def test_version_and_status_strings(lib):
+    assert lib.tok_abi_version() == 1
+    for code in range(7):
+        assert lib.tok_status_str(code).decode().startswith("TOK_")
+    assert lib.tok_last_cuda_error() == 0
+
+
+F = ctypes.c_void_p
+NULL = F(0)
+A = F(0x10000)      # stand-in device addresses: never dereferenced on these paths
+Bp = F(0x8000000)
+
+
+def fwd(lib, x, y, dt, B, C, T, H, W):
+    return lib.tok_haar_fwd(x, y, dt, B, C, T, H, W, NULL)
+
+
+def test_haar_shape_rules(lib):
+    assert fwd(lib, A, Bp, 0, 1, 3, 3, 64, 64) == hwp.TOK_ERR_SHAPE    # T % 4 != 1
+    assert fwd(lib, A, Bp, 0, 1, 3, 5, 62, 64) == hwp.TOK_ERR_SHAPE    # H % 4
+    assert fwd(lib, A, Bp, 0, 1, 3, 5, 64, 66) == hwp.TOK_ERR_SHAPE    # W % 4
+    assert fwd(lib, A, Bp, 0, -1, 3, 5, 64, 64) == hwp.TOK_ERR_SHAPE
+    assert fwd(lib, A, Bp, 0, 1, 3, 0, 64, 64) == hwp.TOK_ERR_SHAPE    # T >= 1
+    assert fwd(lib, A, Bp, 0, 1 << 40, 1 << 20, 5, 1 << 20, 1 << 20) == hwp.TOK_ERR_SHAPE  # overflow
+    assert fwd(lib, A, Bp, 7, 1, 3, 5, 64, 64) == hwp.TOK_ERR_DTYPE
+
+
+def test_haar_empty_is_ok_without_pointers(lib):
+    assert fwd(lib, NULL, NULL, 1, 0, 3, 5, 64, 64) == hwp.TOK_OK
+    assert fwd(lib, NULL, NULL, 1, 2, 0, 5, 64, 64) == hwp.TOK_OK
+    assert fwd(lib, NULL, NULL, 0, 2, 3, 1, 0, 64) == hwp.TOK_OK
+    assert lib.tok_haar_inv(NULL, NULL, 0, 0, 3, 5, 8, 8, NULL) == hwp.TOK_OK
+
+
+def test_haar_null_alignment_alias(lib):
+    assert fwd(lib, NULL, Bp, 1, 1, 3, 5, 64, 64) == hwp.TOK_ERR_NULL
+    assert fwd(lib, A, NULL, 1, 1, 3, 5, 64, 64) == hwp.TOK_ERR_NULL
+    assert fwd(lib, F(0x10001), Bp, 1, 1, 3, 5, 64, 64) == hwp.TOK_ERR_ALIGN   # bf16 needs 2 bytes
+    assert fwd(lib, F(0x10002), Bp, 0, 1, 3, 5, 64, 64) == hwp.TOK_ERR_ALIGN   # fp32 needs 4 bytes
+    assert fwd(lib, A, A, 1, 1, 3, 5, 64, 64) == hwp.TOK_ERR_ALIAS
+    # x occupies 3*5*64*64*2 = 122880 bytes; y starting inside it overlaps
+    assert fwd(lib, A, F(0x10000 + 122880 - 16), 1, 1, 3, 5, 64, 64) == hwp.TOK_ERR_ALIAS
+    assert lib.tok_haar_inv(A, F(0x10000 + 64), 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
+
+
+def test_fsq_argument_rules(lib):
+    enc, dec = lib.tok_fsq_encode, lib.tok_fsq_decode
+    assert enc(A, Bp, F(0x20000000), NULL, 1, 0, 16, NULL) == hwp.TOK_ERR_SHAPE       # C >= 1
+    assert enc(A, Bp, F(0x20000000), NULL, 1, 5000, 16, NULL) == hwp.TOK_ERR_SHAPE    # C <= 1024
+    assert enc(A, Bp, F(0x20000000), NULL, -1, 16, 16, NULL) == hwp.TOK_ERR_SHAPE
+    assert enc(NULL, NULL, NULL, NULL, 0, 16, 16, NULL) == hwp.TOK_OK                   # empty
+    assert enc(NULL, Bp, F(0x20000000), NULL, 1, 16, 16, NULL) == hwp.TOK_ERR_NULL
+    assert enc(A, Bp, F(0x20000002), NULL, 1, 16, 16, NULL) == hwp.TOK_ERR_ALIGN
+    assert enc(A, Bp, F(0x10000 + 64), NULL, 1, 16, 16, NULL) == hwp.TOK_ERR_ALIAS     # idx inside u
+    assert enc(A, Bp, F(0x20000000), F(0x20000000 + 16), 1, 16, 16, NULL) == hwp.TOK_ERR_ALIAS  # codes/idx
+    assert dec(A, Bp, NULL, NULL, 1, 16, 16, NULL) == hwp.TOK_ERR_NULL
+    assert dec(A, Bp, F(0x10000), NULL, 1, 16, 16, NULL) == hwp.TOK_ERR_ALIAS
+    assert dec(A, Bp, F(0x20000000), F(0x20000000 + 8), 1, 16, 16, NULL) == hwp.TOK_ERR_ALIAS  # counter in out
+    assert dec(NULL, NULL, NULL, NULL, 3, 16, 0, NULL) == hwp.TOK_OK
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 1, 5, 8, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        hwp.tok_haar_fwd(x, torch.zeros(1, 64, 2, 2, 2))
+
+
+def test_host_shape_logic():
+    assert hwp.haar_coeff_shape(1, 3, 121, 704, 1280) == (1, 192, 31, 176, 320)
+    assert hwp.haar_coeff_shape(16, 3, 1, 1024, 1024) == (16, 48, 1, 256, 256)
+    with pytest.raises(ValueError):
+        hwp.latent_frames(7)

@@ -1,0 +1,64 @@
+"""Host-side logic of bench.py: byte accounting, the max-over-ranks timing and the
+rank rules of the reference arm, run as two gloo ranks on the CPU."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def test_algorithmic_bytes_of_the_workload():
+    sb = bench.step_bytes()
+    # clip [1,3,121,704,1280] bf16 read + [1,192,31,176,320] bf16 written
+    assert sb["haar_fwd"] == 3 * 121 * 704 * 1280 * 2 + 192 * 31 * 176 * 320 * 2 == 1_324_646_400
+    assert sb["haar_inv"] == sb["haar_fwd"]
+    # 64 x 56320 tokens: 16 fp32 read + 1 int32 written = 68 bytes per token
+    assert sb["fsq_encode"] == 64 * 56320 * 68 == sb["fsq_decode"]
+
+
+def test_job_throughput_is_weak_scaling():
+    assert bench.job_throughput(10 ** 9, 10, 1, 1000.0) == pytest.approx(10.0)
+    assert bench.job_throughput(10 ** 9, 10, 4, 1000.0) == pytest.approx(40.0)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        m = bench.max_over_ranks(10.0 + rank, "cpu")
+
+        class A:
+            steps, warmup = 1, 0
+        # Ranks other than 0 leave the reference arm at once, without work.
+        rc = bench.run_reference(A, rank, world) if rank != 0 else 0
+        dist.barrier()
+        out[rank] = (m, rc)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo_two_ranks():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 11.0
+    assert res[1][1] == 0
+
+
+def test_single_process_max_is_identity():
+    assert bench.max_over_ranks(3.5, "cpu") == 3.5
