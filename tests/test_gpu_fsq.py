@@ -100,8 +100,8 @@ def test_thresholds_exactly_at_boundaries():
                 for _ in range(abs(k)):
                     v = np.nextafter(v, np.float32(np.inf if k > 0 else -np.inf))
                 zs.append(v)
-    zs += [np.float32(0.0), np.float32(-0.0), np.float32(np.inf), np.float32(-np.inf), np.float32(1e30),
-           np.float32(-1e30)]
+    # (no infinities: 0 * inf in the projection chain would be NaN, which has no code)
+    zs += [np.float32(0.0), np.float32(-0.0), np.float32(1e30), np.float32(-1e30)]
     zs = np.array(zs, np.float32)
     u = np.zeros((1, 6, zs.size), np.float32)
     for i in range(6):

@@ -148,9 +148,11 @@ def test_empty_is_noop():
 
 
 def test_bad_arguments_raise_before_launch():
-    x = torch.zeros(1, 1, 9, 16, 16, device="cuda")
+    buf = torch.zeros(8192, device="cuda")
+    x = buf[:2304].view(1, 1, 9, 16, 16)
+    y = buf[1024:1024 + 3072].view(1, 64, 3, 4, 4)  # overlaps x
     with pytest.raises(hwp.TokError, match="ALIAS"):
-        hwp.tok_haar_fwd(x, x.view(-1)[: 64 * 3 * 16].view(1, 64, 3, 4, 4))
+        hwp.tok_haar_fwd(x, y)
     with pytest.raises(ValueError):
         hwp.haar_fwd(torch.zeros(1, 1, 7, 16, 16, device="cuda"))
 
