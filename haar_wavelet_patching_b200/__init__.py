@@ -16,14 +16,15 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtok.so")
 
-TOK_OK, TOK_ERR_NULL, TOK_ERR_SHAPE, TOK_ERR_ALIGN, TOK_ERR_DTYPE, TOK_ERR_ALIAS, TOK_ERR_CUDA = range(7)
+(TOK_OK, TOK_ERR_NULL, TOK_ERR_SHAPE, TOK_ERR_ALIGN, TOK_ERR_DTYPE, TOK_ERR_ALIAS, TOK_ERR_CUDA,
+ TOK_ERR_TIMEOUT) = range(8)
 TOK_F32, TOK_BF16 = 0, 1
 FSQ_CODEBOOK = 64000
 FSQ_DIM = 6
 
 # Every symbol include/tok.h declares.
-ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_haar_fwd", "tok_haar_inv",
-               "tok_fsq_encode", "tok_fsq_decode")
+ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
+               "tok_haar_inv", "tok_fsq_encode", "tok_fsq_decode")
 
 _lib = None
 
@@ -52,6 +53,8 @@ def lib():
         L.tok_status_str.argtypes = [i32]
         L.tok_last_cuda_error.restype = i32
         L.tok_last_cuda_error.argtypes = []
+        L.tok_check_device.restype = i32
+        L.tok_check_device.argtypes = [vp]
         for f in (L.tok_haar_fwd, L.tok_haar_inv):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
@@ -117,6 +120,12 @@ def haar_coeff_shape(B, C, T, H, W):
 # ---------------------------------------------------------------------------
 # C-ABI calls.
 # ---------------------------------------------------------------------------
+def tok_check_device(device=None, stream=None):
+    """Synchronize the stream; raise TokError if a kernel stopped after a bounded wait ran out."""
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    _check(lib().tok_check_device(ctypes.c_void_p(stream.cuda_stream)), "tok_check_device")
+
 def tok_haar_fwd(x: torch.Tensor, y: torch.Tensor, stream=None):
     """x [B,C,T,H,W] -> y [B,64C,T',H/4,W/4] (T == 1: [B,16C,1,H/4,W/4]); same dtype."""
     _cuda(x, "x"), _cuda(y, "y")

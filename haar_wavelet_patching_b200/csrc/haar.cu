@@ -24,6 +24,7 @@
 // channel planes (a warp covers 32*NB contiguous elements per plane).  All
 // arithmetic stays in registers; nothing is staged through shared memory.
 #include "tok_common.cuh"
+#include "tok_internal.h"
 
 namespace tok {
 namespace {
@@ -403,6 +404,11 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
     if (overlaps(in, bytes_in, out, bytes_out))
         return TOK_ERR_ALIAS;
 
+    const HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w};
+    if (haar_tma_eligible(in, out, dt, dims))
+        return haar_tma_launch(fwd, in, out, dt, dims, stream);
+
+    // Register path: any 4-aligned W and element-aligned pointers.
     const bool a16 = aligned(in, 16) && aligned(out, 16);
     if (T > 1) {
         // Two adjacent blocks per thread: 8 input elements per row, pairs per plane.

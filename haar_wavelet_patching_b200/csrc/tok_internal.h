@@ -1,0 +1,28 @@
+// Declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "tok.h"
+
+namespace tok {
+
+// Extents of one Haar call: pixels [B, C, T, H, W], coefficients [B, G*C, Tq, h, w].
+struct HaarDims {
+    int64_t B, C, T, H, W;
+    int64_t Tq, h, w;
+};
+
+// The TMA path takes 16-byte-aligned tensors whose rows are multiples of 16 bytes.
+bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
+tok_status haar_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream);
+
+// Synchronizes `stream`, returns in *count the barrier-wait timeouts of this device's
+// kernels since the last call, and clears them.
+tok_status read_and_clear_timeouts(cudaStream_t stream, unsigned int *count);
+
+// Remembers a CUDA error for tok_last_cuda_error().
+void record_cuda_error(cudaError_t e);
+
+} // namespace tok

@@ -1,0 +1,66 @@
+"""Run one operation of the library on a random workload, for profiling and timing.
+
+    python -m haar_wavelet_patching_b200.run_case --op haar_inv --shape 1,3,33,704,1280 --dtype bf16 --iters 3
+    python -m haar_wavelet_patching_b200.run_case --op fsq_encode --shape 48,16,56320 --iters 3
+
+Inputs are random tensors made on the device by torch (their values do not
+change the kernels' work).  Prints the mean CUDA-event time per launch and the
+algorithmic GB/s.
+"""
+import argparse
+
+import torch
+
+import haar_wavelet_patching_b200 as hwp
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--op", required=True, choices=("haar_fwd", "haar_inv", "fsq_encode", "fsq_decode"))
+    ap.add_argument("--shape", required=True, help="B,C,T,H,W for haar ops; B,C,S for fsq ops")
+    ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--codes", action="store_true", help="fsq_encode: also write the codes")
+    a = ap.parse_args()
+    shape = tuple(int(v) for v in a.shape.split(","))
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
+
+    if a.op in ("haar_fwd", "haar_inv"):
+        B, C, T, H, W = shape
+        x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
+        y = torch.empty(hwp.haar_coeff_shape(*shape), dtype=dt, device=dev)
+        if a.op == "haar_inv":
+            y.copy_((torch.rand(y.shape, generator=g, device=dev) * 2 - 1).to(dt))
+            run = lambda: hwp.tok_haar_inv(y, x)  # noqa: E731
+        else:
+            run = lambda: hwp.tok_haar_fwd(x, y)  # noqa: E731
+        nbytes = (x.numel() + y.numel()) * x.element_size()
+    else:
+        B, C, S = shape
+        w = torch.randn(6, C, generator=g, device=dev) / C ** 0.5
+        u = torch.randn(shape, generator=g, device=dev)
+        idx = torch.randint(0, hwp.FSQ_CODEBOOK, (B, S), generator=g, device=dev, dtype=torch.int32)
+        codes = torch.empty(B, 6, S, device=dev) if a.codes else None
+        if a.op == "fsq_encode":
+            run = lambda: hwp.tok_fsq_encode(u, w, idx, codes)  # noqa: E731
+            nbytes = (u.numel() + idx.numel() + (codes.numel() if codes is not None else 0)) * 4
+        else:
+            run = lambda: hwp.tok_fsq_decode(idx, w, u)  # noqa: E731
+            nbytes = (u.numel() + idx.numel()) * 4
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.iters):
+        run()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / a.iters
+    print(f"{a.op} {shape} {a.dtype}: {ms * 1e3:.1f} us per launch, {nbytes / ms / 1e6:.1f} GB/s")
+
+
+if __name__ == "__main__":
+    main()

@@ -65,7 +65,8 @@ typedef enum {
     TOK_ERR_ALIGN = 3, /* a pointer is not aligned to its element size */
     TOK_ERR_DTYPE = 4, /* unknown tok_dtype */
     TOK_ERR_ALIAS = 5, /* an input buffer overlaps an output buffer */
-    TOK_ERR_CUDA = 6   /* the kernel launch failed; see tok_last_cuda_error() */
+    TOK_ERR_CUDA = 6,   /* a CUDA call or kernel launch failed; see tok_last_cuda_error() */
+    TOK_ERR_TIMEOUT = 7 /* reported by tok_check_device(): a kernel stopped after a bounded wait ran out */
 } tok_status;
 
 typedef enum {
@@ -79,8 +80,19 @@ TOK_API int tok_abi_version(void);
 /* Static, NUL-terminated name of a status code. */
 TOK_API const char *tok_status_str(tok_status status);
 
-/* cudaError_t of the last launch that returned TOK_ERR_CUDA on this thread (0 if none). */
+/* cudaError_t of the last call that returned TOK_ERR_CUDA on this thread (0 if none). */
 TOK_API int tok_last_cuda_error(void);
+
+/*
+ * tok_check_device -- synchronize `stream` and report whether any kernel of
+ * this library on the current device gave up a bounded wait since the last
+ * check (TOK_ERR_TIMEOUT; that call's output is incomplete), then clear the
+ * record.  The TMA-pipelined kernels wait on shared-memory barriers for their
+ * copies; a wait that runs out (never expected) ends the kernel instead of
+ * hanging the GPU.  Not part of the pages' method: an error channel for the
+ * asynchronous calls.  Returns TOK_OK, TOK_ERR_TIMEOUT or TOK_ERR_CUDA.
+ */
+TOK_API tok_status tok_check_device(cudaStream_t stream);
 
 /*
  * tok_haar_fwd -- two-level causal full-packet Haar patcher.

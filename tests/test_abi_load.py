@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.tok_abi_version() == 1
-    for code in range(7):
+    for code in range(8):
         assert lib.tok_status_str(code).decode().startswith("TOK_")
     assert lib.tok_last_cuda_error() == 0
 

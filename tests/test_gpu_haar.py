@@ -26,7 +26,7 @@ TOL_F32 = 1e-5
 
 def run_fwd(xd: torch.Tensor) -> torch.Tensor:
     y = hwp.haar_fwd(xd)
-    torch.cuda.synchronize()
+    hwp.tok_check_device()
     return y
 
 
@@ -59,7 +59,7 @@ def check_inv(y: torch.Tensor, T, H, W, label):
     y64 = to_f64(y)
     ref = oracle.haar_inv(y64, T, H, W)
     x = hwp.haar_inv(y, T, H, W)
-    torch.cuda.synchronize()
+    hwp.tok_check_device()
     got = to_f64(x)
     err = np.abs(got - ref)
     if y.dtype == torch.float32:
@@ -74,8 +74,15 @@ def check_inv(y: torch.Tensor, T, H, W, label):
 
 
 SMALL = [
-    # (shape, dtype, note)
+    # (shape, dtype, note).  TMA path: 16-byte-aligned tensors with W*elem/4 a multiple of 16 bytes
+    # (bf16: W % 32 == 0, fp32: W % 16 == 0); the others take the register kernels.
     ((1, 3, 9, 64, 64), synth.F32, "config 1"),
+    ((2, 3, 13, 40, 96), synth.BF16, "TMA bf16, partial tiles in x and y"),
+    ((1, 2, 9, 36, 80), synth.F32, "TMA fp32, partial tiles"),
+    ((2, 2, 17, 64, 544), synth.BF16, "TMA bf16, several tiles per row, ragged last"),
+    ((1, 1, 5, 4, 32), synth.BF16, "TMA bf16, one block row"),
+    ((3, 2, 1, 24, 160), synth.BF16, "TMA image path, partial tiles"),
+    ((2, 1, 1, 20, 48), synth.F32, "TMA image path fp32"),
     ((2, 3, 13, 64, 264), synth.F32, "vector path, 5 CTAs per frame, ragged tail"),
     ((2, 3, 13, 64, 264), synth.BF16, "vector path bf16"),
     ((1, 2, 9, 16, 44), synth.BF16, "W % 8 == 4: element-wise path"),
@@ -127,6 +134,25 @@ def test_misaligned_pointers_take_elementwise_path():
     hwp.tok_haar_inv(yo, xr[1:].view(shape))
     torch.cuda.synchronize()
     assert torch.equal(xr[1:].view(shape), hwp.haar_inv(yv, 9, 16, 64))
+
+
+@pytest.mark.parametrize("shape,dtype", [((2, 3, 13, 40, 96), torch.bfloat16), ((1, 2, 9, 36, 80), torch.float32),
+                                         ((3, 2, 1, 24, 160), torch.bfloat16)])
+def test_tma_and_register_paths_agree_bitwise(shape, dtype):
+    """The TMA kernels and the register kernels (taken for a misaligned view) give identical bits."""
+    x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
+    y_tma = hwp.haar_fwd(x)
+    buf = torch.empty(x.numel() + 1, dtype=dtype, device="cuda")
+    buf[1:].copy_(x.reshape(-1))
+    ybuf = torch.empty(y_tma.numel() + 1, dtype=dtype, device="cuda")
+    hwp.tok_haar_fwd(buf[1:].view(shape), ybuf[1:].view(y_tma.shape))
+    hwp.tok_check_device()
+    assert torch.equal(ybuf[1:].view(y_tma.shape), y_tma)
+    xr_tma = hwp.haar_inv(y_tma, *shape[2:])
+    xbuf = torch.empty_like(buf)
+    hwp.tok_haar_inv(ybuf[1:].view(y_tma.shape), xbuf[1:].view(shape))
+    hwp.tok_check_device()
+    assert torch.equal(xbuf[1:].view(shape), xr_tma)
 
 
 def test_constant_and_causal_structure_on_gpu():
