@@ -12,7 +12,7 @@ namespace tok {
 
 // Wait limit of one mbarrier wait, in polls (each poll may suspend the warp
 // for a while inside try_wait); about a second or more on a B200.
-constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr uint32_t kWaitPolls = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
