@@ -1,4 +1,4 @@
-// TMA-pipelined Haar patcher / unpatcher for sm_100a (the main path).
+// TMA-fed Haar patcher / unpatcher for sm_100a (the main path).
 //
 // Same transform as haar.cu (sources: "NVIDIA Cosmos Tokenizer 完全指南" 7.1, 6.1,
 // 7.3; "nvidia/Cosmos-Tokenize1-CV8x8x8-720p" model card, Model Architecture):
@@ -6,26 +6,31 @@
 // through the per-axis 4-point transform of the two full-packet levels, with the
 // two frame-0 replicas composed into "window 0 reads frame 0 four times".
 //
-// Design.  Work is cut into warp tiles of 64 horizontally adjacent blocks:
-// one block row of one (b, c, t') window on video (4 frames x 4 rows x 256
-// pixels <-> 64 planes x 64 coefficients), four block rows on images (4 x 16
-// rows of 256 pixels <-> 16 planes x 4 x 64); 4096 elements either way.  Every
-// warp of a persistent CTA runs its own pipeline, with no CTA-wide barrier:
-//   - lane 0 keeps NI TMA loads in flight into the warp's input buffers (a 3D
-//     box of pixels, or one 5D box holding all 64 coefficient planes); each
-//     completes on that buffer's mbarrier;
-//   - the lanes copy their values into registers, and lane 0 at once refills
-//     the buffer with the tile NI steps ahead;
-//   - the lanes transform, write the results to the warp's output buffer, and
-//     lane 0 issues one TMA store for the whole tile.
-// Each lane owns two horizontally adjacent blocks and keeps them in f32x2 pairs
-// (block j in .x, block j+1 in .y), so every butterfly is one packed sm_100
-// add or fused multiply-add.  TMA clips partial tiles at the tensor edges
-// (zero fill on load, nothing stored out of bounds), so any w and h work.
+// Design.  The path is HBM-bound, so what matters is keeping enough bytes in
+// flight while the SM computes.  Work is cut into warp tiles of 64 horizontally
+// adjacent blocks: one block row of one (b, c, t') window on video (4 frames x
+// 4 rows x 256 pixels <-> 64 planes x 64 coefficients), four block rows on
+// images; 4096 elements either way.  Each CTA is a single warp that walks its
+// tiles with a ring of NI shared-memory buffers:
+//   - lane 0 keeps NI TMA loads in flight (a 3D box of pixels, or one 5D box
+//     holding all 64 coefficient planes), each completing on its buffer's
+//     mbarrier, and refills a buffer as soon as the lanes have copied it into
+//     registers;
+//   - the lanes transform in registers and store straight to global memory
+//     (4 bytes per plane per lane on the forward: 128 contiguous bytes per warp
+//     per plane; 16 bytes per pixel row on the inverse), predicated at the
+//     tensor edges.
+// Several single-warp CTAs share an SM, so there is no CTA-wide barrier; while
+// one warp computes, the others' loads are in flight.  Each lane owns two
+// horizontally adjacent blocks and keeps them in f32x2 pairs (block j in .x,
+// block j+1 in .y), so every butterfly is one packed sm_100 add or fused
+// multiply-add.  TMA zero-fills loads past the tensor edges.
 //
 // Waits are bounded: a barrier that does not complete within kWaitPolls polls
 // makes the warp stop, drain what it issued and count a timeout that
 // tok_check_device() reports.  No cluster multicast is used.
+#include <cstring>
+
 #include "tma.cuh"
 #include "tok_common.cuh"
 #include "tok_internal.h"
@@ -37,20 +42,19 @@ static __device__ unsigned int g_wait_timeouts = 0;
 
 namespace {
 
-constexpr int kTileBlocks = 64;        // blocks across a warp tile (256 pixels)
-constexpr int kTileElems = 4096;       // elements of a warp tile, on either side
-constexpr int kSmemBudget = 192 * 1024; // shared memory per CTA
+constexpr int kTileBlocks = 64; // blocks across a warp tile (256 pixels)
+constexpr int kTileElems = 4096; // elements of a warp tile, on either side
 
 template <typename T> struct WarpPipe {
-    static constexpr int NI = sizeof(T) == 2 ? 3 : 2;              // input buffers per warp
+    static constexpr int NI = 3;                                 // input buffers (loads in flight)
     static constexpr int TILE_BYTES = kTileElems * sizeof(T);
-    static constexpr int WARP_BYTES = (NI + 1) * TILE_BYTES + 64;   // + output buffer + barriers
-    static constexpr int WARPS = kSmemBudget / WARP_BYTES;          // 6 (bf16) or 3 (fp32)
-    static constexpr int SMEM = WARPS * WARP_BYTES;
+    static constexpr int SMEM = NI * TILE_BYTES + 8 * NI;        // buffers + mbarriers
+    static constexpr int CTAS_PER_SM = (224 * 1024) / SMEM;      // 9 (bf16) or 4 (fp32)
 };
 
 struct TileGrid {
     int ntx, nty, Tq, C, T;
+    int64_t H, W, h, w;
     int64_t ntiles;
 };
 
@@ -118,15 +122,33 @@ template <> struct SRow<float> {
     static __device__ __forceinline__ void store_pair(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
 };
 
+// Global stores of results: two coefficients (blocks j, j+1) of one plane, or one
+// pixel row of 8 elements (4 of block j, 4 of block j+1).
+__device__ __forceinline__ void gstore_pair(__nv_bfloat16 *p, float2 v)
+{
+    *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(v.x, v.y);
+}
+__device__ __forceinline__ void gstore_pair(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
+__device__ __forceinline__ void gstore_row(__nv_bfloat16 *p, const float2 *v)
+{
+    *reinterpret_cast<uint4 *>(p) = make_uint4(pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x),
+                                               pack_bf16x2(v[0].y, v[1].y), pack_bf16x2(v[2].y, v[3].y));
+}
+__device__ __forceinline__ void gstore_row(float *p, const float2 *v)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(v[0].x, v[1].x, v[2].x, v[3].x);
+    *reinterpret_cast<float4 *>(p + 4) = make_float4(v[0].y, v[1].y, v[2].y, v[3].y);
+}
+
 // Video: one block row (tile rows = 1); images: four block rows, done one after another.
 template <bool VIDEO> struct TileRows {
     static constexpr int RW = VIDEO ? 1 : 4;
 };
 
 template <typename T, bool VIDEO, bool FWD>
-__global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
+__global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
-                    const __grid_constant__ CUtensorMap ymap, const TileGrid tg)
+                    const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
 {
     using P = WarpPipe<T>;
     constexpr int NI = P::NI, WT = kTileBlocks;
@@ -139,11 +161,9 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
     constexpr float SCALE = VIDEO ? 0.125f : 0.25f;
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned char *wbase = smem_raw + warp * (NI + 1) * TILE_BYTES;
-    T *in_buf = reinterpret_cast<T *>(wbase);
-    T *out_buf = reinterpret_cast<T *>(wbase + NI * TILE_BYTES);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + P::WARPS * (NI + 1) * TILE_BYTES) + warp * NI;
+    const int lane = threadIdx.x;
+    T *in_buf = reinterpret_cast<T *>(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + NI * TILE_BYTES);
 
     auto decode = [&](int64_t n, int &tx, int &ty, int &tq, int64_t &bc) {
         tx = (int)(n % tg.ntx);
@@ -154,7 +174,7 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
         bc = n / tg.Tq;
     };
 
-    // Lane 0: start the TMA load of tile n into input buffer s.
+    // Lane 0: start the TMA load of tile n into buffer s.
     auto issue_load = [&](int64_t n, int s) {
         int tx, ty, tq;
         int64_t bc;
@@ -175,21 +195,20 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
         }
     };
 
-    const int64_t nwarps = (int64_t)gridDim.x * P::WARPS;
-    const int64_t first = (int64_t)blockIdx.x * P::WARPS + warp;
+    const int64_t first = blockIdx.x, step = gridDim.x;
     int64_t issued = 0; // tiles whose load lane 0 has issued
     if (lane == 0) {
         for (int s = 0; s < NI; ++s)
             mbar_init(smem_addr(bars + s), 1);
         fence_barrier_init();
-        for (int s = 0; s < NI && first + s * nwarps < tg.ntiles; ++s, ++issued)
-            issue_load(first + s * nwarps, s);
+        for (int s = 0; s < NI && first + s * step < tg.ntiles; ++s, ++issued)
+            issue_load(first + s * step, s);
     }
     __syncwarp();
 
     int k = 0;
     bool failed = false;
-    for (int64_t n = first; n < tg.ntiles; n += nwarps, ++k) {
+    for (int64_t n = first; n < tg.ntiles; n += step, ++k) {
         const int s = k % NI;
         const bool ok = mbar_wait(smem_addr(bars + s), (uint32_t)(k / NI) & 1u);
         if (__any_sync(0xFFFFFFFFu, !ok)) {
@@ -200,6 +219,8 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
         int64_t bc;
         decode(n, tx, ty, tq, bc);
         const T *tin = in_buf + s * kTileElems;
+        const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
+        const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
 
 #pragma unroll
         for (int rw = 0; rw < RW; ++rw) {
@@ -228,7 +249,7 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int64_t nn = n + NI * nwarps;
+                    const int64_t nn = n + NI * step;
                     if (nn < tg.ntiles) {
                         issue_load(nn, s);
                         ++issued;
@@ -254,61 +275,46 @@ __global__ void __launch_bounds__(32 * WarpPipe<T>::WARPS, 1)
                         haar4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
             }
             const float2 scale = make_float2(SCALE, SCALE);
-#pragma unroll
-            for (int a = 0; a < NA; ++a)
-#pragma unroll
-                for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-                    for (int d = 0; d < 4; ++d)
-                        v[a][rr][d] = __fmul2_rn(v[a][rr][d], scale);
 
-            if (rw == 0) {
-                // The output buffer is free once the previous tile's store has read it.
-                if (lane == 0)
-                    bulk_wait_read<0>();
-                __syncwarp();
-            }
+            const int64_t row = (int64_t)ty * RW + rw; // block row
+            if (!col_ok || row >= tg.h)
+                continue;
             if constexpr (FWD) {
+                // y[b][g*C + c][tq][row][j0 .. j0+1]
+                const int64_t b = bc / tg.C, c = bc - b * tg.C;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w, cstride = (int64_t)tg.C * plane;
+                T *yp = out + (b * G * tg.C + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
+                for (int g = 0; g < G; ++g, yp += cstride) {
                     const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
-                    SRow<T>::store_pair(out_buf + (g * RW + rw) * WT + 2 * lane, p);
+                    gstore_pair(yp, __fmul2_rn(p, scale));
                 }
             } else {
+                // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only.
+                T *xb = out + (bc * tg.T) * tg.H * tg.W + (4 * row) * tg.W + 4 * j0;
 #pragma unroll
-                for (int a = 0; a < NA; ++a)
+                for (int a = 0; a < NA; ++a) {
+                    if (VIDEO && tq == 0 && a != 3)
+                        continue;
+                    const int64_t f = VIDEO ? (tq == 0 ? 0 : 4 * tq - 3 + a) : 0;
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr)
-                        SRow<T>::store(out_buf + (a * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                    for (int rr = 0; rr < 4; ++rr) {
+                        float2 o[4];
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            o[d] = __fmul2_rn(v[a][rr][d], scale);
+                        gstore_row(xb + f * tg.H * tg.W + rr * tg.W, o);
+                    }
+                }
             }
-        }
-        fence_proxy_async_smem(); // make this lane's results visible to the TMA engine
-        __syncwarp();
-
-        if (lane == 0) {
-            const uint32_t src = smem_addr(out_buf);
-            if constexpr (FWD) {
-                const int b = (int)(bc / tg.C), c = (int)(bc - (int64_t)b * tg.C);
-                tma_store_5d(&ymap, WT * tx, RW * ty, tq, c, G * b, src);
-            } else if (VIDEO && tq > 0) {
-                tma_store_3d(&xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), src);
-            } else {
-                // Window 0 keeps the last of its four frames (the others are the replicas); images have one.
-                tma_store_3d(&xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T),
-                             smem_addr(out_buf + (VIDEO ? 3 * FRAME : 0)));
-            }
-            bulk_commit();
         }
     }
 
-    if (lane == 0) {
-        if (failed) {
-            // Drain the loads this warp issued and did not consume, each wait again bounded.
-            for (int64_t it = k; it < issued; ++it)
-                mbar_wait(smem_addr(bars + (it % NI)), (uint32_t)(it / NI) & 1u);
-            atomicAdd(&g_wait_timeouts, 1u);
-        }
-        bulk_wait_all(); // stores must finish reading shared memory before the CTA exits
+    if (lane == 0 && failed) {
+        // Drain the loads this warp issued and did not consume, each wait again bounded.
+        for (int64_t it = k; it < issued; ++it)
+            mbar_wait(smem_addr(bars + (it % NI)), (uint32_t)(it / NI) & 1u);
+        atomicAdd(&g_wait_timeouts, 1u);
     }
     __syncwarp();
 }
@@ -322,23 +328,25 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
     constexpr int G = VIDEO ? 64 : 16, RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
-    const void *xp = FWD ? in : out, *yp = FWD ? out : in;
-
+    // Only the input side goes through TMA: pixels on the forward, coefficients on the inverse.
     CUtensorMap xm4, xm1, ym;
-    const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
-    const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
-    const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
-    const uint64_t ydims[5] = {(uint64_t)d.w, (uint64_t)d.h, (uint64_t)d.Tq, (uint64_t)d.C, (uint64_t)(G * d.B)};
-    const uint64_t plane = d.Tq * d.h * d.w * es;
-    const uint64_t ystr[4] = {d.w * es, d.h * d.w * es, plane, d.C * plane};
-    const uint32_t ybox[5] = {(uint32_t)WT, (uint32_t)RW, 1u, 1u, (uint32_t)G};
-    if (!encode_tensor_map(&xm1, dt, 3, xp, xdims, xstr, box1) || !encode_tensor_map(&ym, dt, 5, yp, ydims, ystr, ybox))
-        return TOK_ERR_SHAPE;
-    if (VIDEO) {
-        if (!encode_tensor_map(&xm4, dt, 3, xp, xdims, xstr, box4))
+    memset(&xm4, 0, sizeof xm4);
+    memset(&xm1, 0, sizeof xm1);
+    memset(&ym, 0, sizeof ym);
+    if (FWD) {
+        const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
+        const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
+        const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
+        if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
+            (VIDEO && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
             return TOK_ERR_SHAPE;
     } else {
-        xm4 = xm1;
+        const uint64_t ydims[5] = {(uint64_t)d.w, (uint64_t)d.h, (uint64_t)d.Tq, (uint64_t)d.C, (uint64_t)(G * d.B)};
+        const uint64_t plane = d.Tq * d.h * d.w * es;
+        const uint64_t ystr[4] = {d.w * es, d.h * d.w * es, plane, d.C * plane};
+        const uint32_t ybox[5] = {(uint32_t)WT, (uint32_t)RW, 1u, 1u, (uint32_t)G};
+        if (!encode_tensor_map(&ym, dt, 5, in, ydims, ystr, ybox))
+            return TOK_ERR_SHAPE;
     }
 
     TileGrid tg;
@@ -347,19 +355,22 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
     tg.Tq = (int)d.Tq;
     tg.C = (int)d.C;
     tg.T = (int)d.T;
+    tg.H = d.H;
+    tg.W = d.W;
+    tg.h = d.h;
+    tg.w = d.w;
     tg.ntiles = (int64_t)tg.ntx * tg.nty * d.Tq * d.B * d.C;
 
     // Per call: the attribute belongs to the current device.
-    cudaError_t attr_err =
+    const cudaError_t attr_err =
         cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
-    const int64_t ctas_needed = (tg.ntiles + P::WARPS - 1) / P::WARPS; // a warp per tile at most
-    const int64_t ctas = sm_count();
-    const unsigned grid = (unsigned)(ctas_needed < ctas ? ctas_needed : ctas);
-    haar_tma_kernel<T, VIDEO, FWD><<<grid, 32 * P::WARPS, P::SMEM, stream>>>(xm4, xm1, ym, tg);
+    const int64_t ctas = (int64_t)P::CTAS_PER_SM * sm_count();
+    const unsigned grid = (unsigned)(tg.ntiles < ctas ? tg.ntiles : ctas);
+    haar_tma_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
     return launch_status();
 }
 
