@@ -46,16 +46,28 @@ constexpr int kTileBlocks = 64; // blocks across a warp tile (256 pixels)
 constexpr int kTileElems = 4096; // elements of a warp tile, on either side
 
 template <typename T> struct WarpPipe {
-    static constexpr int NI = 3;                                 // input buffers (loads in flight)
+    static constexpr int NI = 2;                                 // input buffers (loads in flight)
     static constexpr int TILE_BYTES = kTileElems * sizeof(T);
     static constexpr int SMEM = NI * TILE_BYTES + 8 * NI;        // buffers + mbarriers
-    static constexpr int CTAS_PER_SM = (224 * 1024) / SMEM;      // 9 (bf16) or 4 (fp32)
+    static constexpr int CTAS_PER_SM = (208 * 1024) / SMEM;      // 12 (bf16) or 6 (fp32)
+};
+
+// Exact n / d for 32-bit n by a 64-bit multiply-high: with m = ceil(2^64 / d),
+// floor(n * m / 2^64) = floor(n / d) because n * (m - 2^64/d) / 2^64 < 2^-32 <= 1/d
+// cannot carry the fraction of n / d past the next integer.  d = 1 is kept apart.
+struct FastDiv {
+    uint32_t d;
+    uint64_t m;
+    FastDiv() = default;
+    explicit FastDiv(uint32_t div) : d(div), m(div > 1 ? ~0ull / div + 1 : 0) {}
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1 ? n : (uint32_t)__umul64hi(n, m); }
 };
 
 struct TileGrid {
-    int ntx, nty, Tq, C, T;
+    FastDiv ntx, nty, Tq, C;
+    int T;
     int64_t H, W, h, w;
-    int64_t ntiles;
+    uint32_t ntiles;
 };
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
@@ -165,17 +177,16 @@ __global__ void __launch_bounds__(32)
     T *in_buf = reinterpret_cast<T *>(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + NI * TILE_BYTES);
 
-    auto decode = [&](int64_t n, int &tx, int &ty, int &tq, int64_t &bc) {
-        tx = (int)(n % tg.ntx);
-        n /= tg.ntx;
-        ty = (int)(n % tg.nty);
-        n /= tg.nty;
-        tq = (int)(n % tg.Tq);
-        bc = n / tg.Tq;
+    auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
+        const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.Tq.div(q2);
+        tx = (int)(n - q1 * tg.ntx.d);
+        ty = (int)(q1 - q2 * tg.nty.d);
+        tq = (int)(q2 - q3 * tg.Tq.d);
+        bc = q3;
     };
 
     // Lane 0: start the TMA load of tile n into buffer s.
-    auto issue_load = [&](int64_t n, int s) {
+    auto issue_load = [&](uint32_t n, int s) {
         int tx, ty, tq;
         int64_t bc;
         decode(n, tx, ty, tq, bc);
@@ -189,14 +200,14 @@ __global__ void __launch_bounds__(32)
                 tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
             }
         } else {
-            const int b = (int)(bc / tg.C), c = (int)(bc - (int64_t)b * tg.C);
+            const int b = (int)tg.C.div((uint32_t)bc), c = (int)(bc - (int64_t)b * tg.C.d);
             mbar_expect_tx(bar, TILE_BYTES);
             tma_load_5d(dst, &ymap, WT * tx, RW * ty, tq, c, G * b, bar);
         }
     };
 
-    const int64_t first = blockIdx.x, step = gridDim.x;
-    int64_t issued = 0; // tiles whose load lane 0 has issued
+    const uint32_t first = blockIdx.x, step = gridDim.x;
+    uint32_t issued = 0; // tiles whose load lane 0 has issued
     if (lane == 0) {
         for (int s = 0; s < NI; ++s)
             mbar_init(smem_addr(bars + s), 1);
@@ -208,7 +219,7 @@ __global__ void __launch_bounds__(32)
 
     int k = 0;
     bool failed = false;
-    for (int64_t n = first; n < tg.ntiles; n += step, ++k) {
+    for (uint32_t n = first; n < tg.ntiles; n += step, ++k) {
         const int s = k % NI;
         const bool ok = mbar_wait(smem_addr(bars + s), (uint32_t)(k / NI) & 1u);
         if (__any_sync(0xFFFFFFFFu, !ok)) {
@@ -249,9 +260,9 @@ __global__ void __launch_bounds__(32)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    const int64_t nn = n + NI * step;
+                    const uint64_t nn = (uint64_t)n + NI * step;
                     if (nn < tg.ntiles) {
-                        issue_load(nn, s);
+                        issue_load((uint32_t)nn, s);
                         ++issued;
                     }
                 }
@@ -280,14 +291,16 @@ __global__ void __launch_bounds__(32)
             if (!col_ok || row >= tg.h)
                 continue;
             if constexpr (FWD) {
-                // y[b][g*C + c][tq][row][j0 .. j0+1]
-                const int64_t b = bc / tg.C, c = bc - b * tg.C;
-                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w, cstride = (int64_t)tg.C * plane;
-                T *yp = out + (b * G * tg.C + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart,
+                // a 32-bit stride (checked on the host), so each address is one wide multiply-add.
+                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                const int64_t plane = (int64_t)tg.Tq.d * tg.h * tg.w;
+                const uint32_t cstride = (uint32_t)(tg.C.d * plane);
+                T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
 #pragma unroll
-                for (int g = 0; g < G; ++g, yp += cstride) {
+                for (int g = 0; g < G; ++g) {
                     const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
-                    gstore_pair(yp, __fmul2_rn(p, scale));
+                    gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
                 }
             } else {
                 // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only.
@@ -312,8 +325,8 @@ __global__ void __launch_bounds__(32)
 
     if (lane == 0 && failed) {
         // Drain the loads this warp issued and did not consume, each wait again bounded.
-        for (int64_t it = k; it < issued; ++it)
-            mbar_wait(smem_addr(bars + (it % NI)), (uint32_t)(it / NI) & 1u);
+        for (uint32_t it = k; it < issued; ++it)
+            mbar_wait(smem_addr(bars + (it % NI)), (it / NI) & 1u);
         atomicAdd(&g_wait_timeouts, 1u);
     }
     __syncwarp();
@@ -349,17 +362,18 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
             return TOK_ERR_SHAPE;
     }
 
+    const int64_t ntx = (d.w + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
     TileGrid tg;
-    tg.ntx = (int)((d.w + WT - 1) / WT);
-    tg.nty = (int)((d.h + RW - 1) / RW);
-    tg.Tq = (int)d.Tq;
-    tg.C = (int)d.C;
+    tg.ntx = FastDiv((uint32_t)ntx);
+    tg.nty = FastDiv((uint32_t)nty);
+    tg.Tq = FastDiv((uint32_t)d.Tq);
+    tg.C = FastDiv((uint32_t)d.C);
     tg.T = (int)d.T;
     tg.H = d.H;
     tg.W = d.W;
     tg.h = d.h;
     tg.w = d.w;
-    tg.ntiles = (int64_t)tg.ntx * tg.nty * d.Tq * d.B * d.C;
+    tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err =
@@ -369,7 +383,7 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
         return TOK_ERR_CUDA;
     }
     const int64_t ctas = (int64_t)P::CTAS_PER_SM * sm_count();
-    const unsigned grid = (unsigned)(tg.ntiles < ctas ? tg.ntiles : ctas);
+    const unsigned grid = (unsigned)((int64_t)tg.ntiles < ctas ? tg.ntiles : ctas);
     haar_tma_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
     return launch_status();
 }
@@ -383,9 +397,11 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
         return false;
     if ((d.w * es) % 16 != 0) // row strides of both tensors must be multiples of 16 bytes
         return false;
-    // Coordinates are 32-bit: frames of the flattened [B*C*T] axis and the group axis must fit.
+    // Coordinates are 32-bit: frames of the flattened [B*C*T] axis and the group axis must fit,
+    // tiles are numbered in 32 bits, and the 64 planes of one channel lie within a 32-bit offset.
+    const int64_t ntiles = ((d.w + 63) / 64) * ((d.h + 3) / 4 + d.h) * d.Tq * d.B * d.C; // generous bound
     if (d.B * d.C * d.T >= (int64_t)1 << 31 || 64 * d.B >= (int64_t)1 << 31 || d.W >= (int64_t)1 << 31 ||
-        d.H >= (int64_t)1 << 31)
+        d.H >= (int64_t)1 << 31 || ntiles >= (int64_t)1 << 32 || 64 * d.C * d.Tq * d.h * d.w >= (int64_t)1 << 32)
         return false;
     return sm_count() > 0;
 }
