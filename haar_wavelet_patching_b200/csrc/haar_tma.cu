@@ -6,25 +6,26 @@
 // through the per-axis 4-point transform of the two full-packet levels, with the
 // two frame-0 replicas composed into "window 0 reads frame 0 four times".
 //
-// Design.  The path is HBM-bound, so what matters is keeping enough bytes in
-// flight while the SM computes.  Work is cut into warp tiles of 64 horizontally
-// adjacent blocks: one block row of one (b, c, t') window on video (4 frames x
-// 4 rows x 256 pixels <-> 64 planes x 64 coefficients), four block rows on
-// images; 4096 elements either way.  Each CTA is a single warp that walks its
-// tiles with a ring of NI shared-memory buffers:
-//   - lane 0 keeps NI TMA loads in flight (a 3D box of pixels, or one 5D box
-//     holding all 64 coefficient planes), each completing on its buffer's
-//     mbarrier, and refills a buffer as soon as the lanes have copied it into
-//     registers;
-//   - the lanes transform in registers and store straight to global memory
-//     (4 bytes per plane per lane on the forward: 128 contiguous bytes per warp
-//     per plane; 16 bytes per pixel row on the inverse), predicated at the
-//     tensor edges.
-// Several single-warp CTAs share an SM, so there is no CTA-wide barrier; while
-// one warp computes, the others' loads are in flight.  Each lane owns two
-// horizontally adjacent blocks and keeps them in f32x2 pairs (block j in .x,
-// block j+1 in .y), so every butterfly is one packed sm_100 add or fused
-// multiply-add.  TMA zero-fills loads past the tensor edges.
+// Design.  The path is HBM-bound, so what matters is how many bytes are in
+// flight and how compact the region of memory being touched at any moment is.
+// Work is cut into warp tiles of 64 horizontally adjacent blocks: one block row
+// of one (b, c, t') window on video (4 frames x 4 rows x 256 pixels <-> 64
+// planes x 64 coefficients), four block rows on images; 4096 elements either
+// way.  Each CTA is one warp that owns KT consecutive tiles:
+//   - lane 0 issues the KT TMA loads at once (a 3D box of pixels, or one 5D box
+//     holding all 64 coefficient planes), each completing on its own mbarrier;
+//   - the lanes take the tiles in order as they land, transform in registers
+//     and store straight to global memory (4 bytes per plane per lane on the
+//     forward: 128 contiguous bytes per warp per plane; 16 bytes per pixel row
+//     on the inverse), predicated at the tensor edges.
+// The grid is one-shot (a CTA per KT tiles, launched in tile order) rather than
+// persistent: CTAs retire and are replaced in order, so the live working set
+// stays a compact, moving window of the tensors, which measured better on
+// B200 than persistent CTAs striding over the whole tensor.  Several
+// single-warp CTAs share an SM; while one computes, the others' loads are in
+// flight.  Each lane owns two horizontally adjacent blocks and keeps them in
+// f32x2 pairs (block j in .x, block j+1 in .y), so every butterfly is one packed
+// sm_100 add or fused multiply-add.  TMA zero-fills loads past the tensor edges.
 //
 // Waits are bounded: a barrier that does not complete within kWaitPolls polls
 // makes the warp stop, drain what it issued and count a timeout that
@@ -45,11 +46,10 @@ namespace {
 constexpr int kTileBlocks = 64; // blocks across a warp tile (256 pixels)
 constexpr int kTileElems = 4096; // elements of a warp tile, on either side
 
-template <typename T> struct WarpPipe {
-    static constexpr int NI = 2;                                 // input buffers (loads in flight)
+template <typename T> struct WarpTiles {
+    static constexpr int KT = sizeof(T) == 2 ? 4 : 2;  // tiles per CTA, all loaded at once (32 KB)
     static constexpr int TILE_BYTES = kTileElems * sizeof(T);
-    static constexpr int SMEM = NI * TILE_BYTES + 8 * NI;        // buffers + mbarriers
-    static constexpr int CTAS_PER_SM = (208 * 1024) / SMEM;      // 12 (bf16) or 6 (fp32)
+    static constexpr int SMEM = KT * TILE_BYTES + 8 * KT; // buffers + mbarriers
 };
 
 // Exact n / d for 32-bit n by a 64-bit multiply-high: with m = ceil(2^64 / d),
@@ -162,8 +162,8 @@ __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
                     const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
 {
-    using P = WarpPipe<T>;
-    constexpr int NI = P::NI, WT = kTileBlocks;
+    using P = WarpTiles<T>;
+    constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
     constexpr int G = VIDEO ? 64 : 16;  // channel groups
     constexpr int NA = VIDEO ? 4 : 1;   // frames of a window
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(32)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int lane = threadIdx.x;
     T *in_buf = reinterpret_cast<T *>(smem_raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + NI * TILE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * TILE_BYTES);
 
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
         const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.Tq.div(q2);
@@ -185,50 +185,43 @@ __global__ void __launch_bounds__(32)
         bc = q3;
     };
 
-    // Lane 0: start the TMA load of tile n into buffer s.
-    auto issue_load = [&](uint32_t n, int s) {
-        int tx, ty, tq;
-        int64_t bc;
-        decode(n, tx, ty, tq, bc);
-        const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
-        if constexpr (FWD) {
-            if (VIDEO && tq > 0) {
-                mbar_expect_tx(bar, NA * FRAME_BYTES);
-                tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
-            } else {
-                mbar_expect_tx(bar, FRAME_BYTES);
-                tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
-            }
-        } else {
-            const int b = (int)tg.C.div((uint32_t)bc), c = (int)(bc - (int64_t)b * tg.C.d);
-            mbar_expect_tx(bar, TILE_BYTES);
-            tma_load_5d(dst, &ymap, WT * tx, RW * ty, tq, c, G * b, bar);
-        }
-    };
+    const uint32_t first = blockIdx.x * (uint32_t)KT;
+    const int count = (int)min((uint32_t)KT, tg.ntiles - first); // tiles of this CTA
 
-    const uint32_t first = blockIdx.x, step = gridDim.x;
-    uint32_t issued = 0; // tiles whose load lane 0 has issued
     if (lane == 0) {
-        for (int s = 0; s < NI; ++s)
+        for (int s = 0; s < KT; ++s)
             mbar_init(smem_addr(bars + s), 1);
         fence_barrier_init();
-        for (int s = 0; s < NI && first + s * step < tg.ntiles; ++s, ++issued)
-            issue_load(first + s * step, s);
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t bc;
+            decode(first + s, tx, ty, tq, bc);
+            const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
+            if constexpr (FWD) {
+                if (VIDEO && tq > 0) {
+                    mbar_expect_tx(bar, NA * FRAME_BYTES);
+                    tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
+                } else {
+                    mbar_expect_tx(bar, FRAME_BYTES);
+                    tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
+                }
+            } else {
+                const int b = (int)tg.C.div((uint32_t)bc), c = (int)(bc - (int64_t)b * tg.C.d);
+                mbar_expect_tx(bar, TILE_BYTES);
+                tma_load_5d(dst, &ymap, WT * tx, RW * ty, tq, c, G * b, bar);
+            }
+        }
     }
     __syncwarp();
 
-    int k = 0;
-    bool failed = false;
-    for (uint32_t n = first; n < tg.ntiles; n += step, ++k) {
-        const int s = k % NI;
-        const bool ok = mbar_wait(smem_addr(bars + s), (uint32_t)(k / NI) & 1u);
-        if (__any_sync(0xFFFFFFFFu, !ok)) {
-            failed = true;
+    int s = 0;
+    for (; s < count; ++s) {
+        const bool ok = mbar_wait(smem_addr(bars + s), 0u);
+        if (__any_sync(0xFFFFFFFFu, !ok))
             break;
-        }
         int tx, ty, tq;
         int64_t bc;
-        decode(n, tx, ty, tq, bc);
+        decode(first + s, tx, ty, tq, bc);
         const T *tin = in_buf + s * kTileElems;
         const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
         const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
@@ -252,19 +245,6 @@ __global__ void __launch_bounds__(32)
                         v[kt_of(g)][ky_of(g)][kx_of(g)] = p;
                     else
                         v[0][ky2_of(g)][kx2_of(g)] = p;
-                }
-            }
-            if (rw == RW - 1) {
-                // Every lane holds its inputs: hand the buffer back to the TMA engine and
-                // start the load NI tiles ahead right away.
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    const uint64_t nn = (uint64_t)n + NI * step;
-                    if (nn < tg.ntiles) {
-                        issue_load((uint32_t)nn, s);
-                        ++issued;
-                    }
                 }
             }
 
@@ -323,10 +303,10 @@ __global__ void __launch_bounds__(32)
         }
     }
 
-    if (lane == 0 && failed) {
-        // Drain the loads this warp issued and did not consume, each wait again bounded.
-        for (uint32_t it = k; it < issued; ++it)
-            mbar_wait(smem_addr(bars + (it % NI)), (it / NI) & 1u);
+    if (s < count && lane == 0) {
+        // A wait ran out: drain the loads still in flight (each wait again bounded), then report.
+        for (int r = s; r < count; ++r)
+            mbar_wait(smem_addr(bars + r), 0u);
         atomicAdd(&g_wait_timeouts, 1u);
     }
     __syncwarp();
@@ -337,7 +317,7 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    using P = WarpPipe<T>;
+    using P = WarpTiles<T>;
     constexpr int G = VIDEO ? 64 : 16, RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
@@ -382,8 +362,7 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
-    const int64_t ctas = (int64_t)P::CTAS_PER_SM * sm_count();
-    const unsigned grid = (unsigned)((int64_t)tg.ntiles < ctas ? tg.ntiles : ctas);
+    const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
     haar_tma_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
     return launch_status();
 }
