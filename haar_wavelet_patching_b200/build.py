@@ -44,7 +44,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    subprocess.run([nvcc, "-shared", "-cudart", "static", "-o", TARGET + ".tmp", *objs], check=True)
+    subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
+                    "-o", TARGET + ".tmp", *objs], check=True)
     os.replace(TARGET + ".tmp", TARGET)
     return TARGET
 

@@ -84,11 +84,13 @@ extern "C" int tok_last_cuda_error(void) { return tok::g_last_cuda_error; }
 
 extern "C" tok_status tok_check_device(cudaStream_t stream)
 {
-    unsigned int n = 0;
-    const tok_status st = tok::read_and_clear_timeouts(stream, &n);
+    unsigned int nh = 0, nf = 0;
+    tok_status st = tok::read_and_clear_haar_timeouts(stream, &nh);
+    if (st == TOK_OK)
+        st = tok::read_and_clear_fsq_timeouts(stream, &nf);
     if (st != TOK_OK)
         return st;
-    return n ? TOK_ERR_TIMEOUT : TOK_OK;
+    return (nh || nf) ? TOK_ERR_TIMEOUT : TOK_OK;
 }
 
 extern "C" const char *tok_status_str(tok_status status)

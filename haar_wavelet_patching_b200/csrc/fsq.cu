@@ -22,15 +22,31 @@
 //
 // Memory: encode reads 4C bytes and writes 4 bytes per token (plus 24 with
 // codes); decode reads 4 and writes 4C.  At C = 16 that is 68 bytes against
-// ~96 FMAs and 33 compares per token, under the HBM roofline.  A thread owns 4
+// ~96 FMAs and 33 compares per token, under the HBM roofline.
+//
+// Encode at C = 16 with 16-byte-aligned tensors (the main path): one-shot
+// single-warp CTAs, each owning two tiles of 128 consecutive tokens x 16
+// channel planes (8 KB); lane 0 issues both TMA loads at once, the lanes take
+// 4 tokens each and run the projection as packed f32x2 fused multiply-adds
+// (two tokens per instruction, each lane of the pair the same fp32 chain).  A
+// grid of small CTAs in token order keeps the working set a compact, moving
+// window, which measured well above a grid of large CTAs on B200.
+// Other shapes, and decode, use CTAs of 256 threads in which a thread owns 4
 // consecutive tokens of one batch item: one 16-byte load or store per channel
 // plane, 512 contiguous bytes per warp.  The weight lives in shared memory as
 // [c][8] (6 used), read with two broadcast vector loads per channel.
 #include <cmath>
+#include <cstring>
 
+#include "tma.cuh"
 #include "tok_common.cuh"
+#include "tok_internal.h"
 
 namespace tok {
+
+// FSQ kernels that gave up on a barrier wait since the last check.
+static __device__ unsigned int g_fsq_wait_timeouts = 0;
+
 namespace {
 
 constexpr int kThreads = 256;
@@ -183,6 +199,142 @@ __global__ void __launch_bounds__(kThreads)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Encode, TMA path (C = 16).
+// ---------------------------------------------------------------------------
+constexpr int kEncTokens = 128; // tokens per tile: 16 planes x 512 bytes = 8 KB
+constexpr int kEncKT = 2;       // tiles per CTA, loaded at once
+constexpr int kEncSmem = kEncKT * 16 * kEncTokens * 4 + 8 * kEncKT + 16 * 8 * 4;
+
+template <bool CODES>
+__global__ void __launch_bounds__(32)
+    fsq_encode_tma_kernel(const __grid_constant__ CUtensorMap umap, const float *__restrict__ w,
+                          int32_t *__restrict__ idx, float *__restrict__ codes, int64_t S, FastDiv ntx,
+                          uint32_t ntiles, Thresholds th)
+{
+    constexpr int TILE = 16 * kEncTokens;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    float *tiles = reinterpret_cast<float *>(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + kEncKT * TILE * 4);
+    float *ws = reinterpret_cast<float *>(smem_raw + kEncKT * TILE * 4 + 8 * kEncKT); // [16][8]
+    const int lane = threadIdx.x;
+    const uint32_t first = blockIdx.x * (uint32_t)kEncKT;
+    const int count = (int)min((uint32_t)kEncKT, ntiles - first);
+
+    if (lane == 0) {
+        for (int s = 0; s < kEncKT; ++s)
+            mbar_init(smem_addr(bars + s), 1);
+        fence_barrier_init();
+        for (int s = 0; s < count; ++s) {
+            const uint32_t n = first + s, b = ntx.div(n), tx = n - b * ntx.d;
+            const uint32_t bar = smem_addr(bars + s);
+            mbar_expect_tx(bar, TILE * 4);
+            tma_load_3d(smem_addr(tiles + s * TILE), &umap, (int)(tx * kEncTokens), 0, (int)b, bar);
+        }
+    }
+    for (int k = lane; k < 16 * 8; k += 32) {
+        const int c = k >> 3, i = k & 7;
+        ws[k] = (i < 6) ? w[i * 16 + c] : 0.0f;
+    }
+    __syncwarp();
+
+    int s = 0;
+    for (; s < count; ++s) {
+        const bool ok = mbar_wait(smem_addr(bars + s), 0u);
+        if (__any_sync(0xFFFFFFFFu, !ok))
+            break;
+        const uint32_t n = first + s, b = ntx.div(n), tx = n - b * ntx.d;
+        const float *tin = tiles + s * TILE;
+        // z[i][0] holds tokens (0, 1) of this lane, z[i][1] tokens (2, 3).
+        float2 z[6][2];
+#pragma unroll
+        for (int i = 0; i < 6; ++i)
+            z[i][0] = z[i][1] = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float4 q = *reinterpret_cast<const float4 *>(tin + c * kEncTokens + 4 * lane);
+            const float4 wa = *reinterpret_cast<const float4 *>(ws + c * 8);
+            const float2 wb = *reinterpret_cast<const float2 *>(ws + c * 8 + 4);
+            const float wc[6] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y};
+            const float2 u01 = make_float2(q.x, q.y), u23 = make_float2(q.z, q.w);
+#pragma unroll
+            for (int i = 0; i < 6; ++i) {
+                const float2 wi = make_float2(wc[i], wc[i]);
+                z[i][0] = __ffma2_rn(wi, u01, z[i][0]);
+                z[i][1] = __ffma2_rn(wi, u23, z[i][1]);
+            }
+        }
+        const int64_t t0 = (int64_t)tx * kEncTokens + 4 * lane;
+        if (t0 >= S) // S % 4 == 0: a lane's four tokens are all in range or all out
+            continue;
+        float id[4], zh[6][4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            float zt[6];
+#pragma unroll
+            for (int i = 0; i < 6; ++i) {
+                const float2 p = z[i][t >> 1];
+                zt[i] = (t & 1) ? p.y : p.x;
+            }
+            const int d0 = count_at_or_above(zt[0], th.t8), d1 = count_at_or_above(zt[1], th.t8);
+            const int d2 = count_at_or_above(zt[2], th.t8), d3 = count_at_or_above(zt[3], th.t5);
+            const int d4 = count_at_or_above(zt[4], th.t5), d5 = count_at_or_above(zt[5], th.t5);
+            id[t] = __int_as_float(d0 + 8 * d1 + 64 * d2 + 512 * d3 + 2560 * d4 + 12800 * d5);
+            if constexpr (CODES) {
+                zh[0][t] = (float)(d0 - 4) * 0.25f;
+                zh[1][t] = (float)(d1 - 4) * 0.25f;
+                zh[2][t] = (float)(d2 - 4) * 0.25f;
+                zh[3][t] = (float)(d3 - 2) * 0.5f;
+                zh[4][t] = (float)(d4 - 2) * 0.5f;
+                zh[5][t] = (float)(d5 - 2) * 0.5f;
+            }
+        }
+        *reinterpret_cast<float4 *>(idx + (int64_t)b * S + t0) = make_float4(id[0], id[1], id[2], id[3]);
+        if constexpr (CODES) {
+#pragma unroll
+            for (int i = 0; i < 6; ++i)
+                *reinterpret_cast<float4 *>(codes + ((int64_t)b * 6 + i) * S + t0) =
+                    make_float4(zh[i][0], zh[i][1], zh[i][2], zh[i][3]);
+        }
+    }
+
+    if (s < count && lane == 0) {
+        for (int r = s; r < count; ++r) // drain, each wait again bounded
+            mbar_wait(smem_addr(bars + r), 0u);
+        atomicAdd(&g_fsq_wait_timeouts, 1u);
+    }
+    __syncwarp();
+}
+
+// Launches the TMA encode, or returns false if the layout does not suit it.
+bool try_encode_tma(const float *u, const float *w, int32_t *idx, float *codes, int64_t B, int64_t C, int64_t S,
+                    cudaStream_t stream, tok_status *st)
+{
+    if (C != 16 || S % 4 != 0 || !aligned(u, 16) || !aligned(idx, 16) || (codes && !aligned(codes, 16)))
+        return false;
+    const int64_t ntx = (S + kEncTokens - 1) / kEncTokens, ntiles = ntx * B;
+    if (S >= ((int64_t)1 << 31) || B >= ((int64_t)1 << 31) || ntiles >= ((int64_t)1 << 32) || sm_count() <= 0)
+        return false;
+    CUtensorMap umap;
+    memset(&umap, 0, sizeof umap);
+    const uint64_t dims[3] = {(uint64_t)S, 16, (uint64_t)B}, strides[2] = {(uint64_t)S * 4, (uint64_t)S * 16 * 4};
+    const uint32_t box[3] = {(uint32_t)kEncTokens, 16, 1};
+    if (!encode_tensor_map(&umap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, u, dims, strides, box))
+        return false;
+    auto kern = codes ? fsq_encode_tma_kernel<true> : fsq_encode_tma_kernel<false>;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmem);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        *st = TOK_ERR_CUDA;
+        return true;
+    }
+    const unsigned grid = (unsigned)((ntiles + kEncKT - 1) / kEncKT);
+    kern<<<grid, 32, kEncSmem, stream>>>(umap, w, idx, codes, S, FastDiv((uint32_t)ntx), (uint32_t)ntiles,
+                                         thresholds());
+    *st = launch_status();
+    return true;
+}
+
 template <int CT, int TPT, bool VEC>
 __global__ void __launch_bounds__(kThreads)
     fsq_decode_kernel(const int32_t *__restrict__ idx, const float *__restrict__ w, float *__restrict__ out,
@@ -260,6 +412,26 @@ unsigned grid_for(int64_t n)
 }
 
 } // namespace
+
+tok_status read_and_clear_fsq_timeouts(cudaStream_t stream, unsigned int *count)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(count, g_fsq_wait_timeouts, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && *count)
+        e = cudaMemcpyToSymbolAsync(g_fsq_wait_timeouts, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice,
+                                    stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    return TOK_OK;
+}
+
 } // namespace tok
 
 extern "C" tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, float *codes, int64_t B, int64_t C,
@@ -282,6 +454,9 @@ extern "C" tok_status tok_fsq_encode(const float *u, const float *w, int32_t *id
     if (overlaps(u, bu, idx, bi) || overlaps(w, bw, idx, bi) ||
         (codes && (overlaps(u, bu, codes, bc) || overlaps(w, bw, codes, bc) || overlaps(idx, bi, codes, bc))))
         return TOK_ERR_ALIAS;
+    tok_status st = TOK_OK;
+    if (try_encode_tma(u, w, idx, codes, B, C, S, stream, &st))
+        return st;
     const bool vec = S % 4 == 0 && aligned(u, 16) && aligned(idx, 16) && (!codes || aligned(codes, 16));
     const size_t smem = (size_t)C * 8 * sizeof(float);
     const Thresholds &th = thresholds();

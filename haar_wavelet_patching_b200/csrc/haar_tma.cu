@@ -52,17 +52,6 @@ template <typename T> struct WarpTiles {
     static constexpr int SMEM = KT * TILE_BYTES + 8 * KT; // buffers + mbarriers
 };
 
-// Exact n / d for 32-bit n by a 64-bit multiply-high: with m = ceil(2^64 / d),
-// floor(n * m / 2^64) = floor(n / d) because n * (m - 2^64/d) / 2^64 < 2^-32 <= 1/d
-// cannot carry the fraction of n / d past the next integer.  d = 1 is kept apart.
-struct FastDiv {
-    uint32_t d;
-    uint64_t m;
-    FastDiv() = default;
-    explicit FastDiv(uint32_t div) : d(div), m(div > 1 ? ~0ull / div + 1 : 0) {}
-    __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1 ? n : (uint32_t)__umul64hi(n, m); }
-};
-
 struct TileGrid {
     FastDiv ntx, nty, Tq, C;
     int T;
@@ -400,7 +389,7 @@ tok_status haar_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, co
     return fwd ? launch<float, false, true>(in, out, d, stream) : launch<float, false, false>(in, out, d, stream);
 }
 
-tok_status read_and_clear_timeouts(cudaStream_t stream, unsigned int *count)
+tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)
 {
     unsigned int zero = 0;
     cudaError_t e = cudaMemcpyFromSymbolAsync(count, g_wait_timeouts, sizeof(unsigned int), 0,

@@ -95,6 +95,17 @@ template <int N> __device__ __forceinline__ void bulk_wait_read()
 // Wait until every committed bulk store has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
+// Exact n / d for 32-bit n by a 64-bit multiply-high: with m = ceil(2^64 / d),
+// floor(n * m / 2^64) = floor(n / d) because n * (m - 2^64/d) / 2^64 < 2^-32 <= 1/d
+// cannot carry the fraction of n / d past the next integer.  d = 1 is kept apart.
+struct FastDiv {
+    uint32_t d;
+    uint64_t m;
+    FastDiv() = default;
+    explicit FastDiv(uint32_t div) : d(div), m(div > 1 ? ~0ull / div + 1 : 0) {}
+    __device__ __forceinline__ uint32_t div(uint32_t n) const { return d == 1 ? n : (uint32_t)__umul64hi(n, m); }
+};
+
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------

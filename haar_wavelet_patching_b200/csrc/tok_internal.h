@@ -18,9 +18,10 @@ struct HaarDims {
 bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
 tok_status haar_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream);
 
-// Synchronizes `stream`, returns in *count the barrier-wait timeouts of this device's
-// kernels since the last call, and clears them.
-tok_status read_and_clear_timeouts(cudaStream_t stream, unsigned int *count);
+// Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
+// Haar (resp. FSQ) kernels since the last call, and clear them.
+tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count);
+tok_status read_and_clear_fsq_timeouts(cudaStream_t stream, unsigned int *count);
 
 // Remembers a CUDA error for tok_last_cuda_error().
 void record_cuda_error(cudaError_t e);

@@ -27,7 +27,7 @@ def encode_gpu(u_np, w_np, with_codes=True):
     u = torch.from_numpy(u_np).cuda()
     w = torch.from_numpy(w_np).cuda()
     idx, codes = hwp.fsq_encode(u, w, with_codes=True) if with_codes else (hwp.fsq_encode(u, w), None)
-    torch.cuda.synchronize()
+    hwp.tok_check_device()
     return idx.cpu().numpy(), (codes.cpu().numpy() if codes is not None else None)
 
 
@@ -76,9 +76,11 @@ def test_encode_decode_configs(cfg):
     check_decode(idx, w, f"config {cfg}")
 
 
-@pytest.mark.parametrize("B,C,S", [(3, 16, 4097), (2, 16, 1), (1, 3, 1000), (2, 40, 512), (1, 1, 8), (5, 6, 999)])
+@pytest.mark.parametrize("B,C,S", [(3, 16, 4100), (2, 16, 132), (1, 16, 128), (3, 16, 4097), (2, 16, 1), (1, 3, 1000),
+                                   (2, 40, 512), (1, 1, 8), (5, 6, 999)])
 def test_encode_decode_shapes(B, C, S):
-    """Ragged S (element-wise path), C != 16 (runtime channel count), tiny sizes."""
+    """C = 16 with S % 4 == 0 takes the TMA encode (ragged last tile when S % 128 != 0); odd S takes the
+    element-wise kernels; C != 16 the runtime-channel kernels; tiny sizes."""
     u = synth.normal((B, C, S), seed=B * 1000 + C * 10 + S, std=1.5)
     w = synth.fsq_weight(C, seed=C)
     idx, _, _ = check_encode(u, w, f"B={B} C={C} S={S}")
@@ -149,6 +151,19 @@ def test_decode_inverts_encode_on_centres():
     zhat = q / np.array([L // 2 for L in LEVELS])[:, None]
     np.testing.assert_array_equal(out.cpu().numpy()[0], zhat)
     np.testing.assert_array_equal(codes[0], zhat)
+
+
+def test_tma_and_register_encode_agree_bitwise():
+    """The TMA encode (aligned, C = 16) and the register encode (a misaligned view) give identical results."""
+    u = synth.fsq_input(2)
+    w = torch.from_numpy(synth.fsq_weight()).cuda()
+    ud = torch.from_numpy(u).cuda()
+    idx_tma, codes_tma = hwp.fsq_encode(ud, w, with_codes=True)
+    buf = torch.empty(ud.numel() + 1, device="cuda")
+    buf[1:].copy_(ud.reshape(-1))
+    idx_reg, codes_reg = hwp.fsq_encode(buf[1:].view(ud.shape), w, with_codes=True)
+    hwp.tok_check_device()
+    assert torch.equal(idx_tma, idx_reg) and torch.equal(codes_tma, codes_reg)
 
 
 def test_encode_without_codes_and_empty():
