@@ -16,6 +16,9 @@
 // butterflies; its output frame 0 is sample 3 of window 0 (the replicas are
 // dropped level by level, which keeps the last copy).
 //
+// This file holds the register kernels, taken when the TMA path of haar_tma.cu
+// cannot be (rows not a multiple of 16 bytes, or pointers not 16-byte aligned).
+//
 // Memory: the path moves each input byte and each output byte once and does
 // ~7 flops per element, so it is bound by HBM.  A thread owns NB horizontally
 // adjacent blocks: it reads 16 (3D) or 4 (2D) input rows of 4*NB contiguous
@@ -60,7 +63,7 @@ __host__ __device__ constexpr int kx2_of(int g) { return 2 * ((g >> 2) & 1) + (g
 static_assert(group3d(kt_of(37), ky_of(37), kx_of(37)) == 37, "group3d inverse");
 static_assert(group2d(ky2_of(13), kx2_of(13)) == 13, "group2d inverse");
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 64; // small CTAs: more resident warps per SM measured faster on B200
 
 struct Geometry {
     int64_t BC;      // B*C (plane pairs)

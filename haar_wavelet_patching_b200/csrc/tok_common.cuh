@@ -44,9 +44,9 @@ inline bool aligned(const void *p, uintptr_t n) { return ((uintptr_t)p % n) == 0
 tok_status launch_status();
 
 // ---------------------------------------------------------------------------
-// Device-side memory access.  Inputs are streamed once: loads bypass L1
-// allocation.  Outputs use plain stores (the next kernel of a pipeline may
-// find the tail of them in L2).
+// Device-side memory access.  ld_stream_* bypass L1 allocation (used by the
+// FSQ register kernels, where they measured faster).  Outputs use plain stores
+// (the next kernel of a pipeline may find the tail of them in L2).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint4 ld_stream_u4(const void *p)
 {
@@ -82,8 +82,9 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 }
 
 // N consecutive elements of type T <-> floats.  VEC: p is aligned to
-// min(16, N * sizeof(T)) bytes and the widest vector form is used; otherwise
-// element-wise accesses.
+// min(16, N * sizeof(T)) bytes and the widest vector form is used (plain
+// cached loads: measured faster than L1::no_allocate for these kernels);
+// otherwise element-wise accesses.
 template <typename T, int N, bool VEC> struct Row;
 
 template <int N, bool VEC> struct Row<float, N, VEC> {
@@ -92,14 +93,14 @@ template <int N, bool VEC> struct Row<float, N, VEC> {
         if constexpr (VEC && N % 4 == 0) {
 #pragma unroll
             for (int k = 0; k < N / 4; ++k) {
-                const uint4 r = ld_stream_u4(p + 4 * k);
+                const uint4 r = *reinterpret_cast<const uint4 *>(p + 4 * k);
                 v[4 * k + 0] = __uint_as_float(r.x);
                 v[4 * k + 1] = __uint_as_float(r.y);
                 v[4 * k + 2] = __uint_as_float(r.z);
                 v[4 * k + 3] = __uint_as_float(r.w);
             }
         } else if constexpr (VEC && N == 2) {
-            const uint2 r = ld_stream_u2(p);
+            const uint2 r = *reinterpret_cast<const uint2 *>(p);
             v[0] = __uint_as_float(r.x);
             v[1] = __uint_as_float(r.y);
         } else {
@@ -130,7 +131,7 @@ template <int N, bool VEC> struct Row<__nv_bfloat16, N, VEC> {
         if constexpr (VEC && N % 8 == 0) {
 #pragma unroll
             for (int k = 0; k < N / 8; ++k) {
-                const uint4 r = ld_stream_u4(p + 8 * k);
+                const uint4 r = *reinterpret_cast<const uint4 *>(p + 8 * k);
                 v[8 * k + 0] = bf16_lo(r.x);
                 v[8 * k + 1] = bf16_hi(r.x);
                 v[8 * k + 2] = bf16_lo(r.y);
@@ -141,13 +142,13 @@ template <int N, bool VEC> struct Row<__nv_bfloat16, N, VEC> {
                 v[8 * k + 7] = bf16_hi(r.w);
             }
         } else if constexpr (VEC && N == 4) {
-            const uint2 r = ld_stream_u2(p);
+            const uint2 r = *reinterpret_cast<const uint2 *>(p);
             v[0] = bf16_lo(r.x);
             v[1] = bf16_hi(r.x);
             v[2] = bf16_lo(r.y);
             v[3] = bf16_hi(r.y);
         } else if constexpr (VEC && N == 2) {
-            const uint32_t r = ld_stream_u1(p);
+            const uint32_t r = *reinterpret_cast<const uint32_t *>(p);
             v[0] = bf16_lo(r);
             v[1] = bf16_hi(r);
         } else {
