@@ -1,6 +1,6 @@
 """Shared helpers of the GPU parity tests: dtype plumbing and the tolerances.
 
-Tolerances (derived in the design notes from the arithmetic of the kernels):
+Tolerances (derived from the arithmetic of the kernels):
   fp32 Haar      max |gpu - oracle| <= 1e-5.
   bf16 Haar      |gpu - oracle| <= ulp_bf16(oracle) + E, where E bounds the fp32
                  accumulation error of the kernel's butterflies:
