@@ -24,7 +24,7 @@ FSQ_DIM = 6
 
 # Every symbol include/tok.h declares.
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
-               "tok_haar_inv", "tok_fsq_encode", "tok_fsq_decode")
+               "tok_haar_inv", "tok_haar_fwd_windows", "tok_haar_inv_windows", "tok_fsq_encode", "tok_fsq_decode")
 
 _lib = None
 
@@ -58,6 +58,9 @@ def lib():
         for f in (L.tok_haar_fwd, L.tok_haar_inv):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
+        for f in (L.tok_haar_fwd_windows, L.tok_haar_inv_windows):
+            f.restype = i32
+            f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, vp]
         L.tok_fsq_encode.restype = i32
         L.tok_fsq_encode.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
         L.tok_fsq_decode.restype = i32
@@ -126,6 +129,7 @@ def tok_check_device(device=None, stream=None):
         stream = torch.cuda.current_stream(device)
     _check(lib().tok_check_device(ctypes.c_void_p(stream.cuda_stream)), "tok_check_device")
 
+
 def tok_haar_fwd(x: torch.Tensor, y: torch.Tensor, stream=None):
     """x [B,C,T,H,W] -> y [B,64C,T',H/4,W/4] (T == 1: [B,16C,1,H/4,W/4]); same dtype."""
     _cuda(x, "x"), _cuda(y, "y")
@@ -151,6 +155,31 @@ def tok_haar_inv(y: torch.Tensor, x: torch.Tensor, stream=None):
     if tuple(y.shape) != haar_coeff_shape(B, C, T, H, W):
         raise ValueError(f"y has shape {tuple(y.shape)}, expected {haar_coeff_shape(B, C, T, H, W)}")
     _check(lib().tok_haar_inv(_ptr(y), _ptr(x), _dtype_code(x), B, C, T, H, W, _stream(x, stream)), "tok_haar_inv")
+    return x
+
+
+def _haar_windows(fwd, x, y, t_begin, t_end, stream):
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != haar_coeff_shape(B, C, T, H, W):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {haar_coeff_shape(B, C, T, H, W)}")
+    f = lib().tok_haar_fwd_windows if fwd else lib().tok_haar_inv_windows
+    src, dst = (x, y) if fwd else (y, x)
+    _check(f(_ptr(src), _ptr(dst), _dtype_code(x), B, C, T, H, W, int(t_begin), int(t_end), _stream(x, stream)),
+           "tok_haar_fwd_windows" if fwd else "tok_haar_inv_windows")
+
+
+def tok_haar_fwd_windows(x: torch.Tensor, y: torch.Tensor, t_begin: int, t_end: int, stream=None):
+    """Forward restricted to latent frames [t_begin, t_end) of the full tensors x, y."""
+    _haar_windows(True, x, y, t_begin, t_end, stream)
+    return y
+
+
+def tok_haar_inv_windows(y: torch.Tensor, x: torch.Tensor, t_begin: int, t_end: int, stream=None):
+    """Inverse restricted to latent frames [t_begin, t_end): writes only those windows' pixel frames."""
+    _haar_windows(False, x, y, t_begin, t_end, stream)
     return x
 
 

@@ -66,10 +66,11 @@ static_assert(group2d(ky2_of(13), kx2_of(13)) == 13, "group2d inverse");
 constexpr int kThreads = 64; // small CTAs: more resident warps per SM measured faster on B200
 
 struct Geometry {
-    int64_t BC;      // B*C (plane pairs)
-    int64_t C;       // input channels
-    int64_t T, H, W; // pixel extents
+    int64_t BC;       // B*C (plane pairs)
+    int64_t C;        // input channels
+    int64_t T, H, W;  // pixel extents
     int64_t Tq, h, w; // latent extents
+    int64_t tq0, nq;  // latent frames processed: [tq0, tq0 + nq)
     int64_t wn;       // thread columns per row = w / NB
 };
 
@@ -88,9 +89,9 @@ __global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restric
     const int64_t j0 = (item - i * g.wn) * NB;
     const int64_t plane_in = g.H * g.W, plane_out = g.Tq * g.h * g.w;
     const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y; // (b, c, t')
-    if (pair >= g.BC * g.Tq)
+    if (pair >= g.BC * g.nq)
         return;
-    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t bc = pair / g.nq, tq = g.tq0 + (pair - bc * g.nq);
     const int64_t b = bc / g.C, c = bc - b * g.C;
     const T *xc = x + bc * g.T * plane_in + (4 * i) * g.W + 4 * j0;
     T *yc = y + (b * 64 * g.C + c) * plane_out + i * g.w + j0;
@@ -173,9 +174,9 @@ __global__ void __launch_bounds__(kThreads) haar3d_inv_kernel(const T *__restric
     const int64_t j0 = (item - i * g.wn) * NB;
     const int64_t plane_in = g.Tq * g.h * g.w, plane_out = g.H * g.W;
     const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y; // (b, c, t')
-    if (pair >= g.BC * g.Tq)
+    if (pair >= g.BC * g.nq)
         return;
-    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t bc = pair / g.nq, tq = g.tq0 + (pair - bc * g.nq);
     const int64_t b = bc / g.C, c = bc - b * g.C;
     const T *yc = y + (b * 64 * g.C + c) * plane_in + i * g.w + j0;
     T *xc = x + bc * g.T * plane_out + (4 * i) * g.W + 4 * j0;
@@ -345,7 +346,7 @@ tok_status launch3d(bool fwd, const void *in, void *out, Geometry g, cudaStream_
     const int64_t gx = (g.h * g.wn + kThreads - 1) / kThreads;
     if (gx > 0x7FFFFFFF)
         return TOK_ERR_SHAPE;
-    const int64_t pairs = g.BC * g.Tq;
+    const int64_t pairs = g.BC * g.nq;
     const unsigned gy = (unsigned)(pairs < kMaxGridYZ ? pairs : kMaxGridYZ);
     const int64_t gz = (pairs + gy - 1) / gy;
     if (gz > kMaxGridYZ)
@@ -377,8 +378,9 @@ tok_status launch2d(bool fwd, const void *in, void *out, Geometry g, cudaStream_
     return launch_status();
 }
 
+// Latent frames [t_begin, t_end) of the full tensors; t_end < 0 means "through the last".
 tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
-                     int64_t W, cudaStream_t stream)
+                     int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream)
 {
     if (dt != TOK_F32 && dt != TOK_BF16)
         return TOK_ERR_DTYPE;
@@ -393,11 +395,17 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
     g.Tq = T == 1 ? 1 : 1 + (T - 1) / 4;
     g.h = H / 4;
     g.w = W / 4;
+    if (t_end < 0)
+        t_end = g.Tq;
+    if (t_begin < 0 || t_begin > t_end || t_end > g.Tq)
+        return TOK_ERR_SHAPE;
+    g.tq0 = t_begin;
+    g.nq = t_end - t_begin;
     int64_t nx, ny, bytes_x, bytes_y;
     if (!prod_ok({B, C}, &g.BC) || !prod_ok({g.BC, T, H, W}, &nx) || !prod_ok({nx, es}, &bytes_x) ||
         !prod_ok({g.BC, T == 1 ? 16 : 64, g.Tq, g.h, g.w}, &ny) || !prod_ok({ny, es}, &bytes_y))
         return TOK_ERR_SHAPE;
-    if (nx == 0)
+    if (nx == 0 || g.nq == 0)
         return TOK_OK;
     if (!in || !out)
         return TOK_ERR_NULL;
@@ -407,7 +415,7 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
     if (overlaps(in, bytes_in, out, bytes_out))
         return TOK_ERR_ALIAS;
 
-    const HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w};
+    const HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, g.tq0, g.nq};
     if (haar_tma_eligible(in, out, dt, dims))
         return haar_tma_launch(fwd, in, out, dt, dims, stream);
 
@@ -436,11 +444,27 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
 extern "C" tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                                    int64_t W, cudaStream_t stream)
 {
-    return tok::haar_call(true, x, y, dt, B, C, T, H, W, stream);
+    return tok::haar_call(true, x, y, dt, B, C, T, H, W, 0, -1, stream);
 }
 
 extern "C" tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                                    int64_t W, cudaStream_t stream)
 {
-    return tok::haar_call(false, y, x, dt, B, C, T, H, W, stream);
+    return tok::haar_call(false, y, x, dt, B, C, T, H, W, 0, -1, stream);
+}
+
+extern "C" tok_status tok_haar_fwd_windows(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream)
+{
+    if (t_end < 0)
+        return TOK_ERR_SHAPE;
+    return tok::haar_call(true, x, y, dt, B, C, T, H, W, t_begin, t_end, stream);
+}
+
+extern "C" tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream)
+{
+    if (t_end < 0)
+        return TOK_ERR_SHAPE;
+    return tok::haar_call(false, y, x, dt, B, C, T, H, W, t_begin, t_end, stream);
 }

@@ -53,8 +53,8 @@ template <typename T> struct WarpTiles {
 };
 
 struct TileGrid {
-    FastDiv ntx, nty, Tq, C;
-    int T;
+    FastDiv ntx, nty, nq, C; // tiles across, tile rows, latent frames processed, channels
+    int T, Tq, tq0;          // frames, latent frames of the tensor, first latent frame processed
     int64_t H, W, h, w;
     uint32_t ntiles;
 };
@@ -167,10 +167,10 @@ __global__ void __launch_bounds__(32)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * TILE_BYTES);
 
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
-        const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.Tq.div(q2);
+        const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
         tx = (int)(n - q1 * tg.ntx.d);
         ty = (int)(q1 - q2 * tg.nty.d);
-        tq = (int)(q2 - q3 * tg.Tq.d);
+        tq = tg.tq0 + (int)(q2 - q3 * tg.nq.d);
         bc = q3;
     };
 
@@ -263,7 +263,7 @@ __global__ void __launch_bounds__(32)
                 // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart,
                 // a 32-bit stride (checked on the host), so each address is one wide multiply-add.
                 const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
-                const int64_t plane = (int64_t)tg.Tq.d * tg.h * tg.w;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
                 const uint32_t cstride = (uint32_t)(tg.C.d * plane);
                 T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
 #pragma unroll
@@ -335,14 +335,16 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
     TileGrid tg;
     tg.ntx = FastDiv((uint32_t)ntx);
     tg.nty = FastDiv((uint32_t)nty);
-    tg.Tq = FastDiv((uint32_t)d.Tq);
+    tg.nq = FastDiv((uint32_t)d.nq);
     tg.C = FastDiv((uint32_t)d.C);
     tg.T = (int)d.T;
+    tg.Tq = (int)d.Tq;
+    tg.tq0 = (int)d.tq0;
     tg.H = d.H;
     tg.W = d.W;
     tg.h = d.h;
     tg.w = d.w;
-    tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
+    tg.ntiles = (uint32_t)(ntx * nty * d.nq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err =

@@ -8,10 +8,12 @@
 
 namespace tok {
 
-// Extents of one Haar call: pixels [B, C, T, H, W], coefficients [B, G*C, Tq, h, w].
+// Extents of one Haar call: pixels [B, C, T, H, W], coefficients [B, G*C, Tq, h, w];
+// the call processes latent frames [tq0, tq0 + nq).
 struct HaarDims {
     int64_t B, C, T, H, W;
     int64_t Tq, h, w;
+    int64_t tq0, nq;
 };
 
 // The TMA path takes 16-byte-aligned tensors whose rows are multiples of 16 bytes.

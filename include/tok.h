@@ -130,6 +130,25 @@ TOK_API tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B,
                         int64_t W, cudaStream_t stream);
 
 /*
+ * tok_haar_fwd_windows / tok_haar_inv_windows -- the same transforms restricted
+ * to latent frames [t_begin, t_end), 0 <= t_begin <= t_end <= T' (T' = 1 on
+ * images).  x and y are the full tensors with the extents above; only latent
+ * frames t' in the range are written (forward: y[:, :, t']; inverse: the pixel
+ * frames of window t', i.e. frame 0 for t' = 0 and frames 4t'-3 .. 4t'
+ * otherwise), and only the pixel frames those windows read are read.  Windows
+ * are independent (the causal structure of [guide] 7.1 and 7.3: output frame t'
+ * depends on input frames 4t'-3 .. 4t' only, and frame 0 on frame 0 only), so
+ * a clip can be transformed chunk by chunk as its frames arrive, and the chunks
+ * compose to exactly the full call's result.  An empty range returns TOK_OK;
+ * a range outside [0, T'] returns TOK_ERR_SHAPE.  Not on the pages' API: a
+ * streaming form of the same operation.
+ */
+TOK_API tok_status tok_haar_fwd_windows(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                        int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream);
+TOK_API tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                        int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream);
+
+/*
  * tok_fsq_encode -- fused 1x1 projection + FSQ quantization + index pack.
  * [guide] 7.2 (bound with tanh, rounding, levels [8,8,8,5,5,5], implicit
  * codebook of 64000, mixed-radix codes_to_indices), [guide] 6.2 (indices

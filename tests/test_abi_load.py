@@ -85,6 +85,19 @@ def test_haar_null_alignment_alias(lib):
     assert lib.tok_haar_inv(A, F(0x10000 + 64), 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
 
 
+def test_haar_window_rules(lib):
+    fw, iw = lib.tok_haar_fwd_windows, lib.tok_haar_inv_windows
+    # clip T = 9 -> 3 latent frames
+    assert fw(A, Bp, 1, 1, 3, 9, 64, 64, 2, 1, NULL) == hwp.TOK_ERR_SHAPE     # begin > end
+    assert fw(A, Bp, 1, 1, 3, 9, 64, 64, 0, 4, NULL) == hwp.TOK_ERR_SHAPE     # end > T'
+    assert fw(A, Bp, 1, 1, 3, 9, 64, 64, -1, 2, NULL) == hwp.TOK_ERR_SHAPE
+    assert fw(A, Bp, 1, 1, 3, 9, 64, 64, 0, -1, NULL) == hwp.TOK_ERR_SHAPE    # no open-ended range
+    assert fw(NULL, NULL, 1, 1, 3, 9, 64, 64, 2, 2, NULL) == hwp.TOK_OK       # empty range touches nothing
+    assert iw(NULL, NULL, 1, 1, 3, 9, 64, 64, 3, 3, NULL) == hwp.TOK_OK
+    assert fw(A, Bp, 1, 1, 3, 1, 64, 64, 0, 2, NULL) == hwp.TOK_ERR_SHAPE     # images have one latent frame
+    assert iw(A, A, 1, 1, 3, 9, 64, 64, 0, 1, NULL) == hwp.TOK_ERR_ALIAS
+
+
 def test_fsq_argument_rules(lib):
     enc, dec = lib.tok_fsq_encode, lib.tok_fsq_decode
     assert enc(A, Bp, F(0x20000000), NULL, 1, 0, 16, NULL) == hwp.TOK_ERR_SHAPE       # C >= 1

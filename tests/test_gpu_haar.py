@@ -155,6 +155,35 @@ def test_tma_and_register_paths_agree_bitwise(shape, dtype):
     assert torch.equal(xbuf[1:].view(shape), xr_tma)
 
 
+@pytest.mark.parametrize("shape,dtype,chunks", [
+    ((1, 3, 41, 64, 128), torch.bfloat16, [(0, 1), (1, 4), (4, 7), (7, 11)]),    # TMA path
+    ((2, 2, 29, 40, 72), torch.bfloat16, [(0, 3), (3, 8)]),                      # register path (W % 32 != 0)
+    ((1, 2, 21, 32, 64), torch.float32, [(0, 2), (2, 2), (2, 6)]),               # fp32, an empty chunk
+    ((2, 3, 1, 32, 64), torch.bfloat16, [(0, 1)]),                               # image: one window
+])
+def test_windows_compose_to_the_full_call(shape, dtype, chunks):
+    """Chunks of latent frames, processed separately, give exactly the full result; each chunk
+    writes only its own frames (everything else keeps a sentinel)."""
+    B, C, T, H, W = shape
+    x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
+    y_full = hwp.haar_fwd(x)
+    x_full = hwp.haar_inv(y_full, T, H, W)
+    y = torch.full_like(y_full, float("nan"))
+    xr = torch.full_like(x, float("nan"))
+    for a, b in chunks:
+        before = y.clone()
+        hwp.tok_haar_fwd_windows(x, y, a, b)
+        hwp.tok_check_device()
+        changed = (y != before) & ~(torch.isnan(y) & torch.isnan(before))
+        outside = torch.ones(y.shape[2], dtype=torch.bool, device="cuda")
+        outside[a:b] = False
+        assert not changed[:, :, outside].any(), f"forward chunk {(a, b)} wrote outside its frames"
+        hwp.tok_haar_inv_windows(y, xr, a, b)
+        hwp.tok_check_device()
+    assert torch.equal(y, y_full)
+    assert torch.equal(xr, x_full)
+
+
 def test_constant_and_causal_structure_on_gpu():
     C = 3
     x = torch.full((2, C, 9, 16, 32), 0.375, device="cuda")
