@@ -23,7 +23,9 @@
  *     channel with L levels, half = (L-1)(1+eps)/2, off = 0.5 for even L and
  *     0 for odd L, shift = atanh(off/half); v = tanh(z + shift)*half - off;
  *     q = round(v), ties to even.  eps = 1e-3.  This yields exactly L integers
- *     q in [-floor(L/2), ceil(L/2)-1] and maps z = 0 to q = 0.
+ *     q in [-floor(L/2), ceil(L/2)-1] and maps z = 0 to q = 0.  Parity
+ *     unpinned by the pages for eps and the even-level offset: they are pinned
+ *     only through their consequences (level counts, centre code, symmetry).
  *   - digit d = q + floor(L/2) in [0, L); index = sum_i d_i * basis_i with
  *     channel 0 least significant, basis = (1, 8, 64, 512, 2560, 12800);
  *     indices are 0-based, in [0, 64000).

@@ -24,7 +24,8 @@
  *     in space and in time; the decoder ends with the inverse transform.
  *
  * Readings where the pages are silent (each one is a convention shared with
- * the CUDA path, not something the pages pin):
+ * the CUDA path; parity unpinned by the pages for the first two -- any fixed
+ * sign or subband permutation would be equally valid):
  *   - high band of a pair (a, b) is (a - b)/sqrt(2), low band (a + b)/sqrt(2);
  *   - subband s = 4*bt + 2*by + bx (bit = 1 for the high band of that axis)
  *     is written to output channel s*C + c, so after two levels channel
