@@ -33,6 +33,10 @@ def _load():
             f = getattr(lib, name)
             f.restype = ctypes.c_int
             f.argtypes = [dp, dp, i64, i64, i64, i64, i64]
+        for name in ("oracle_haar_fwd_adjoint", "oracle_haar_inv_adjoint"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [dp, dp, i64, i64, i64, i64, i64]
         lib.oracle_haar_level_fwd.restype = ctypes.c_int
         lib.oracle_haar_level_fwd.argtypes = [dp, dp, i64, i64, i64, i64]
         lib.oracle_haar_out_frames.restype = i64
@@ -56,6 +60,12 @@ def _load():
         lib.oracle_fsq_encode.argtypes = [fp, fp, i64, i64, i64, i32p, dp, u8p]
         lib.oracle_fsq_decode.restype = i64
         lib.oracle_fsq_decode.argtypes = [i32p, fp, i64, i64, i64, dp]
+        lib.oracle_fsq_ste_slope.restype = ctypes.c_double
+        lib.oracle_fsq_ste_slope.argtypes = [ctypes.c_double, ctypes.c_int]
+        lib.oracle_fsq_encode_backward.restype = None
+        lib.oracle_fsq_encode_backward.argtypes = [fp, fp, fp, i64, i64, i64, dp, dp]
+        lib.oracle_fsq_decode_backward.restype = None
+        lib.oracle_fsq_decode_backward.argtypes = [i32p, fp, fp, i64, i64, i64, dp, dp]
         _lib = lib
     return _lib
 
@@ -115,6 +125,29 @@ def haar_inv(y: np.ndarray, T: int, H: int, W: int) -> np.ndarray:
     _check(_load().oracle_haar_inv(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), B, C, T, H, W),
            "haar_inv")
     return x
+
+
+def haar_fwd_adjoint(gy: np.ndarray, T: int, H: int, W: int) -> np.ndarray:
+    """Gradient of the patcher: coefficient-shaped gy -> pixel-shaped gx = M^T gy (video only)."""
+    gy = np.ascontiguousarray(gy, dtype=np.float64)
+    B = gy.shape[0]
+    C = gy.shape[1] // 64
+    if gy.shape != haar_out_shape(B, C, T, H, W):
+        raise ValueError("haar_fwd_adjoint: shape mismatch")
+    gx = np.zeros((B, C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_fwd_adjoint(_ptr(gy, ctypes.c_double), _ptr(gx, ctypes.c_double), B, C, T, H, W),
+           "haar_fwd_adjoint")
+    return gx
+
+
+def haar_inv_adjoint(gx: np.ndarray) -> np.ndarray:
+    """Gradient of the unpatcher: pixel-shaped gx -> coefficient-shaped gy (video only)."""
+    gx = np.ascontiguousarray(gx, dtype=np.float64)
+    B, C, T, H, W = gx.shape
+    gy = np.zeros(haar_out_shape(B, C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_inv_adjoint(_ptr(gx, ctypes.c_double), _ptr(gy, ctypes.c_double), B, C, T, H, W),
+           "haar_inv_adjoint")
+    return gy
 
 
 def haar_level_fwd(x: np.ndarray) -> np.ndarray:
@@ -184,3 +217,33 @@ def fsq_decode(idx: np.ndarray, w: np.ndarray):
     bad = _load().oracle_fsq_decode(_ptr(idx, ctypes.c_int32), _ptr(w, ctypes.c_float), B, C, S,
                                     _ptr(out, ctypes.c_double))
     return out, int(bad)
+
+
+def fsq_ste_slope(z: float, i: int) -> float:
+    return float(_load().oracle_fsq_ste_slope(float(z), i))
+
+
+def fsq_encode_backward(u: np.ndarray, w: np.ndarray, g: np.ndarray):
+    """Straight-through encode backward: (grad_u [B,C,S], grad_w [6,C]) in float64."""
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    B, C, S = u.shape
+    gu = np.zeros((B, C, S), dtype=np.float64)
+    gw = np.zeros((6, C), dtype=np.float64)
+    _load().oracle_fsq_encode_backward(_ptr(u, ctypes.c_float), _ptr(w, ctypes.c_float), _ptr(g, ctypes.c_float),
+                                       B, C, S, _ptr(gu, ctypes.c_double), _ptr(gw, ctypes.c_double))
+    return gu, gw
+
+
+def fsq_decode_backward(idx: np.ndarray, w: np.ndarray, g: np.ndarray):
+    """Decode backward: (grad_codes [B,6,S], grad_w [6,C]) in float64."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    B, C, S = g.shape
+    gc = np.zeros((B, 6, S), dtype=np.float64)
+    gw = np.zeros((6, C), dtype=np.float64)
+    _load().oracle_fsq_decode_backward(_ptr(idx, ctypes.c_int32), _ptr(w, ctypes.c_float), _ptr(g, ctypes.c_float),
+                                       B, C, S, _ptr(gc, ctypes.c_double), _ptr(gw, ctypes.c_double))
+    return gc, gw

@@ -164,3 +164,86 @@ int64_t oracle_fsq_decode(const int32_t *idx, const float *w, int64_t B, int64_t
         }
     return bad;
 }
+
+/*
+ * Straight-through derivative of the normalized code of channel i with respect
+ * to its pre-quantization value: round_ste passes the gradient through the
+ * rounding ([guide] section 7.2), so d zhat / d z = bound'(z) / floor(L/2) =
+ * half * sech^2(z + shift) / floor(L/2).  Evaluated in double.
+ */
+double oracle_fsq_ste_slope(double z, int i)
+{
+    const int L = FSQ_L[i];
+    const double half = (L - 1) * (1.0 + FSQ_EPS) / 2.0;
+    const double off = (L % 2 == 0) ? 0.5 : 0.0;
+    const double shift = atanh(off / half);
+    const double c = cosh(z + shift);
+    return half / (c * c) / (double)(L / 2);
+}
+
+/*
+ * Encode backward (straight-through).  u: [B][C][S] fp32, w: [6][C],
+ * g: [B][6][S] fp32 (gradient of the normalized codes).  With z the same fp32
+ * chain as the forward and t_i = g_i * slope_i(z_i):
+ *   grad_u[b][c][s] = sum_i w[i][c] t_i          (double)
+ *   grad_w[i][c]    = sum_{b,s} t_i u[b][c][s]   (double, over all tokens)
+ */
+void oracle_fsq_encode_backward(const float *u, const float *w, const float *g, int64_t B, int64_t C, int64_t S,
+                                double *grad_u, double *grad_w)
+{
+    for (int64_t k = 0; k < FSQ_DIM * C; ++k)
+        grad_w[k] = 0.0;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t s = 0; s < S; ++s) {
+            double t[FSQ_DIM];
+            for (int i = 0; i < FSQ_DIM; ++i) {
+                float z = 0.0f;
+                for (int64_t c = 0; c < C; ++c)
+                    z = fmaf(w[i * C + c], u[(b * C + c) * S + s], z);
+                t[i] = (double)g[(b * FSQ_DIM + i) * S + s] * oracle_fsq_ste_slope((double)z, i);
+            }
+            for (int64_t c = 0; c < C; ++c) {
+                const double uc = u[(b * C + c) * S + s];
+                double acc = 0.0;
+                for (int i = 0; i < FSQ_DIM; ++i) {
+                    acc += (double)w[i * C + c] * t[i];
+                    grad_w[i * C + c] += t[i] * uc;
+                }
+                grad_u[(b * C + c) * S + s] = acc;
+            }
+        }
+}
+
+/*
+ * Decode backward.  idx: [B][S], w: [6][C], g: [B][C][S] fp32 (gradient of the
+ * decoded latent).  With zhat the normalized code of each token:
+ *   grad_codes[b][i][s] = sum_c w[i][c] g[b][c][s]      (double)
+ *   grad_w[i][c]        = sum_{b,s} zhat_i g[b][c][s]   (double)
+ * Tokens with an invalid index contribute nothing and get zero code gradients.
+ */
+void oracle_fsq_decode_backward(const int32_t *idx, const float *w, const float *g, int64_t B, int64_t C, int64_t S,
+                                double *grad_codes, double *grad_w)
+{
+    for (int64_t k = 0; k < FSQ_DIM * C; ++k)
+        grad_w[k] = 0.0;
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t s = 0; s < S; ++s) {
+            const int64_t id = idx[b * S + s];
+            const int valid = id >= 0 && id < FSQ_CODEBOOK;
+            int digits[FSQ_DIM];
+            double zhat[FSQ_DIM];
+            if (valid)
+                oracle_fsq_unpack(id, digits);
+            for (int i = 0; i < FSQ_DIM; ++i) {
+                const int half_width = FSQ_L[i] / 2;
+                zhat[i] = valid ? (double)(digits[i] - half_width) / (double)half_width : 0.0;
+                double acc = 0.0;
+                for (int64_t c = 0; c < C; ++c) {
+                    const double gc = g[(b * C + c) * S + s];
+                    acc += (double)w[i * C + c] * gc;
+                    grad_w[i * C + c] += zhat[i] * gc;
+                }
+                grad_codes[(b * FSQ_DIM + i) * S + s] = valid ? acc : 0.0;
+            }
+        }
+}

@@ -287,6 +287,129 @@ int oracle_haar_inv(const double *y, double *x, int64_t B, int64_t C, int64_t T,
 }
 
 /*
+ * Adjoints (transposes), for gradients.  Each level of the forward is a
+ * replication R (frame 0 copied in front) followed by pair butterflies P; the
+ * butterfly matrix [[s, s], [s, -s]] is symmetric, so P^T = P^-1 is the inverse
+ * butterfly, and R^T adds the copy's gradient into frame 0.  So the adjoint of a
+ * level is the inverse level with the first reconstructed frame ADDED to frame
+ * 0 instead of dropped, and the adjoint of the two-level patcher applies the
+ * level-2 adjoint first.  The unpatcher is (drop the first frame) after inverse
+ * butterflies, per level, level 2 first; its adjoint puts a zero frame in front
+ * (the dropped frame gets no gradient) and applies the forward butterflies,
+ * level 1 first.
+ */
+static void level3d_adj(const double *o, double *v, int64_t C, int64_t To, int64_t Ho, int64_t Wo)
+{
+    const int64_t T = 2 * To - 1, H = 2 * Ho, W = 2 * Wo;
+    for (int64_t c = 0; c < C; ++c)
+        for (int64_t j = 0; j < To; ++j)
+            for (int64_t i = 0; i < Ho; ++i)
+                for (int64_t k = 0; k < Wo; ++k) {
+                    double g[2][2][2];
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            for (int bx = 0; bx < 2; ++bx)
+                                g[bt][by][bx] = o[((((int64_t)(4 * bt + 2 * by + bx) * C + c) * To + j) * Ho + i) * Wo + k];
+                    for (int bt = 0; bt < 2; ++bt) /* P^T along x */
+                        for (int by = 0; by < 2; ++by)
+                            haar_unpair(g[bt][by][0], g[bt][by][1], &g[bt][by][0], &g[bt][by][1]);
+                    for (int bt = 0; bt < 2; ++bt) /* along y */
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_unpair(g[bt][0][dx], g[bt][1][dx], &g[bt][0][dx], &g[bt][1][dx]);
+                    for (int dy = 0; dy < 2; ++dy) /* along t */
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_unpair(g[0][dy][dx], g[1][dy][dx], &g[0][dy][dx], &g[1][dy][dx]);
+                    for (int dt = 0; dt < 2; ++dt) {
+                        const int64_t pt = 2 * j + dt;
+                        const int64_t vt = (pt == 0) ? 0 : pt - 1; /* R^T: the copy lands on frame 0 */
+                        for (int dy = 0; dy < 2; ++dy)
+                            for (int dx = 0; dx < 2; ++dx) {
+                                double *dst = &v[((c * T + vt) * H + (2 * i + dy)) * W + (2 * k + dx)];
+                                if (pt == 0)
+                                    *dst = g[dt][dy][dx];
+                                else if (pt == 1)
+                                    *dst += g[dt][dy][dx];
+                                else
+                                    *dst = g[dt][dy][dx];
+                            }
+                    }
+                }
+}
+
+/* Adjoint of level3d_inv: v[C][2To-1][2Ho][2Wo] -> o[8C][To][Ho][Wo]. */
+static void level3d_inv_adj(const double *v, double *o, int64_t C, int64_t To, int64_t Ho, int64_t Wo)
+{
+    const int64_t T = 2 * To - 1, H = 2 * Ho, W = 2 * Wo;
+    for (int64_t c = 0; c < C; ++c)
+        for (int64_t j = 0; j < To; ++j)
+            for (int64_t i = 0; i < Ho; ++i)
+                for (int64_t k = 0; k < Wo; ++k) {
+                    double g[2][2][2];
+                    for (int dt = 0; dt < 2; ++dt) {
+                        const int64_t pt = 2 * j + dt; /* the dropped frame p_0 has no gradient */
+                        for (int dy = 0; dy < 2; ++dy)
+                            for (int dx = 0; dx < 2; ++dx)
+                                g[dt][dy][dx] =
+                                    pt == 0 ? 0.0 : v[((c * T + (pt - 1)) * H + (2 * i + dy)) * W + (2 * k + dx)];
+                    }
+                    for (int dy = 0; dy < 2; ++dy) /* along t: the inverse butterfly's transpose */
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_pair(g[0][dy][dx], g[1][dy][dx], &g[0][dy][dx], &g[1][dy][dx]);
+                    for (int bt = 0; bt < 2; ++bt) /* along y */
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_pair(g[bt][0][dx], g[bt][1][dx], &g[bt][0][dx], &g[bt][1][dx]);
+                    for (int bt = 0; bt < 2; ++bt) /* along x */
+                        for (int by = 0; by < 2; ++by)
+                            haar_pair(g[bt][by][0], g[bt][by][1], &g[bt][by][0], &g[bt][by][1]);
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            for (int bx = 0; bx < 2; ++bx)
+                                o[((((int64_t)(4 * bt + 2 * by + bx) * C + c) * To + j) * Ho + i) * Wo + k] =
+                                    g[bt][by][bx];
+                }
+}
+
+/* Gradient of the two-level patcher: gy (coefficient shape) -> gx (pixel shape). Video only. */
+int oracle_haar_fwd_adjoint(const double *gy, double *gx, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W)
+{
+    if (!shape_ok(B, C, T, H, W) || T == 1)
+        return ORACLE_BAD_SHAPE;
+    const int64_t nx = C * T * H * W, Tq = oracle_haar_out_frames(T), T1 = 2 * Tq - 1;
+    const int64_t n1 = 8 * C * T1 * (H / 2) * (W / 2), ny = 64 * C * Tq * (H / 4) * (W / 4);
+    if (nx == 0 || B == 0)
+        return ORACLE_OK;
+    double *mid = (double *)malloc((size_t)n1 * sizeof(double));
+    if (!mid)
+        return ORACLE_NO_MEMORY;
+    for (int64_t b = 0; b < B; ++b) {
+        level3d_adj(gy + b * ny, mid, 8 * C, Tq, H / 4, W / 4);
+        level3d_adj(mid, gx + b * nx, C, T1, H / 2, W / 2);
+    }
+    free(mid);
+    return ORACLE_OK;
+}
+
+/* Gradient of the two-level unpatcher: gx (pixel shape) -> gy (coefficient shape). Video only. */
+int oracle_haar_inv_adjoint(const double *gx, double *gy, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W)
+{
+    if (!shape_ok(B, C, T, H, W) || T == 1)
+        return ORACLE_BAD_SHAPE;
+    const int64_t nx = C * T * H * W, Tq = oracle_haar_out_frames(T), T1 = 2 * Tq - 1;
+    const int64_t n1 = 8 * C * T1 * (H / 2) * (W / 2), ny = 64 * C * Tq * (H / 4) * (W / 4);
+    if (nx == 0 || B == 0)
+        return ORACLE_OK;
+    double *mid = (double *)malloc((size_t)n1 * sizeof(double));
+    if (!mid)
+        return ORACLE_NO_MEMORY;
+    for (int64_t b = 0; b < B; ++b) {
+        level3d_inv_adj(gx + b * nx, mid, C, T1, H / 2, W / 2);
+        level3d_inv_adj(mid, gy + b * ny, 8 * C, Tq, H / 4, W / 4);
+    }
+    free(mid);
+    return ORACLE_OK;
+}
+
+/*
  * Second, independent statement of the two-level forward transform, used only
  * to pin the level-by-level form above.  It is derived from the definition:
  *   - two full-packet levels on four samples x0..x3 give the 4-point
