@@ -24,7 +24,9 @@ FSQ_DIM = 6
 
 # Every symbol include/tok.h declares.
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
-               "tok_haar_inv", "tok_haar_fwd_windows", "tok_haar_inv_windows", "tok_fsq_encode", "tok_fsq_decode")
+               "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
+               "tok_haar_inv_windows", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
+               "tok_fsq_encode_backward", "tok_fsq_decode_backward")
 
 _lib = None
 
@@ -55,9 +57,14 @@ def lib():
         L.tok_last_cuda_error.argtypes = []
         L.tok_check_device.restype = i32
         L.tok_check_device.argtypes = [vp]
-        for f in (L.tok_haar_fwd, L.tok_haar_inv):
+        for f in (L.tok_haar_fwd, L.tok_haar_inv, L.tok_haar_fwd_adjoint, L.tok_haar_inv_adjoint):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
+        L.tok_fsq_backward_workspace_size.restype = i64
+        L.tok_fsq_backward_workspace_size.argtypes = [i64, i64, i64]
+        for f in (L.tok_fsq_encode_backward, L.tok_fsq_decode_backward):
+            f.restype = i32
+            f.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
         for f in (L.tok_haar_fwd_windows, L.tok_haar_inv_windows):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, vp]
@@ -183,6 +190,28 @@ def tok_haar_inv_windows(y: torch.Tensor, x: torch.Tensor, t_begin: int, t_end: 
     return x
 
 
+def tok_haar_fwd_adjoint(gy: torch.Tensor, gx: torch.Tensor, stream=None):
+    """Gradient of the patcher: gy (coefficient shape) -> gx [B,C,T,H,W]."""
+    _cuda(gx, "gx"), _cuda(gy, "gy")
+    B, C, T, H, W = gx.shape
+    if gy.dtype != gx.dtype or tuple(gy.shape) != haar_coeff_shape(B, C, T, H, W):
+        raise ValueError("gy must have the coefficient shape and dtype of gx")
+    _check(lib().tok_haar_fwd_adjoint(_ptr(gy), _ptr(gx), _dtype_code(gx), B, C, T, H, W, _stream(gx, stream)),
+           "tok_haar_fwd_adjoint")
+    return gx
+
+
+def tok_haar_inv_adjoint(gx: torch.Tensor, gy: torch.Tensor, stream=None):
+    """Gradient of the unpatcher: gx [B,C,T,H,W] -> gy (coefficient shape)."""
+    _cuda(gx, "gx"), _cuda(gy, "gy")
+    B, C, T, H, W = gx.shape
+    if gy.dtype != gx.dtype or tuple(gy.shape) != haar_coeff_shape(B, C, T, H, W):
+        raise ValueError("gy must have the coefficient shape and dtype of gx")
+    _check(lib().tok_haar_inv_adjoint(_ptr(gx), _ptr(gy), _dtype_code(gx), B, C, T, H, W, _stream(gx, stream)),
+           "tok_haar_inv_adjoint")
+    return gy
+
+
 def _latent_dims(u: torch.Tensor):
     if u.dim() < 2:
         raise ValueError("latent must be [B, C, ...]")
@@ -226,6 +255,41 @@ def tok_fsq_decode(idx: torch.Tensor, w: torch.Tensor, out: torch.Tensor, bad_co
     return out
 
 
+def fsq_backward_workspace_size(B: int, C: int, S: int) -> int:
+    n = int(lib().tok_fsq_backward_workspace_size(B, C, S))
+    if n < 0:
+        raise ValueError(f"no FSQ backward for B={B}, C={C}, S={S} (1 <= C <= 16)")
+    return n
+
+
+def tok_fsq_encode_backward(u, w, grad_codes, grad_u, grad_w, workspace, stream=None):
+    """Straight-through encode backward into grad_u [B,C,...] and grad_w [6,C]; workspace: uint8 CUDA tensor."""
+    for t, n in ((u, "u"), (w, "w"), (grad_codes, "grad_codes"), (grad_u, "grad_u"), (grad_w, "grad_w"),
+                 (workspace, "workspace")):
+        _cuda(t, n)
+    B, C, S = _latent_dims(u)
+    if grad_u.shape != u.shape or grad_codes.numel() != B * FSQ_DIM * S or tuple(grad_w.shape) != (FSQ_DIM, C):
+        raise ValueError("shapes: grad_u like u, grad_codes [B,6,...], grad_w [6,C]")
+    _check(lib().tok_fsq_encode_backward(_ptr(u), _ptr(w), _ptr(grad_codes), _ptr(grad_u), _ptr(grad_w),
+                                         _ptr(workspace), workspace.numel() * workspace.element_size(), B, C, S,
+                                         _stream(u, stream)), "tok_fsq_encode_backward")
+    return grad_u, grad_w
+
+
+def tok_fsq_decode_backward(idx, w, grad_out, grad_codes, grad_w, workspace, stream=None):
+    """Decode backward into grad_codes [B,6,...] and grad_w [6,C]; workspace: uint8 CUDA tensor."""
+    for t, n in ((idx, "idx"), (w, "w"), (grad_out, "grad_out"), (grad_codes, "grad_codes"), (grad_w, "grad_w"),
+                 (workspace, "workspace")):
+        _cuda(t, n)
+    B, C, S = _latent_dims(grad_out)
+    if idx.numel() != B * S or grad_codes.numel() != B * FSQ_DIM * S or tuple(grad_w.shape) != (FSQ_DIM, C):
+        raise ValueError("shapes: idx [B,...], grad_codes [B,6,...], grad_w [6,C]")
+    _check(lib().tok_fsq_decode_backward(_ptr(idx), _ptr(w), _ptr(grad_out), _ptr(grad_codes), _ptr(grad_w),
+                                         _ptr(workspace), workspace.numel() * workspace.element_size(), B, C, S,
+                                         _stream(idx, stream)), "tok_fsq_decode_backward")
+    return grad_codes, grad_w
+
+
 # ---------------------------------------------------------------------------
 # Allocating wrappers.
 # ---------------------------------------------------------------------------
@@ -252,3 +316,33 @@ def fsq_encode(u: torch.Tensor, w: torch.Tensor, with_codes: bool = False, strea
 def fsq_decode(idx: torch.Tensor, w: torch.Tensor, bad_count: torch.Tensor = None, stream=None) -> torch.Tensor:
     out = torch.empty((idx.shape[0], w.shape[1]) + tuple(idx.shape[1:]), dtype=torch.float32, device=idx.device)
     return tok_fsq_decode(idx, w, out, bad_count, stream)
+
+
+def haar_fwd_adjoint(gy: torch.Tensor, T: int, H: int, W: int, stream=None) -> torch.Tensor:
+    B = gy.shape[0]
+    C = gy.shape[1] // (16 if T == 1 else 64)
+    gx = torch.empty((B, C, T, H, W), dtype=gy.dtype, device=gy.device)
+    return tok_haar_fwd_adjoint(gy, gx, stream)
+
+
+def haar_inv_adjoint(gx: torch.Tensor, stream=None) -> torch.Tensor:
+    gy = torch.empty(haar_coeff_shape(*gx.shape), dtype=gx.dtype, device=gx.device)
+    return tok_haar_inv_adjoint(gx, gy, stream)
+
+
+def _workspace(B, C, S, device):
+    return torch.empty(max(fsq_backward_workspace_size(B, C, S), 1), dtype=torch.uint8, device=device)
+
+
+def fsq_encode_backward(u: torch.Tensor, w: torch.Tensor, grad_codes: torch.Tensor, stream=None):
+    B, C, S = _latent_dims(u)
+    grad_u = torch.empty_like(u)
+    grad_w = torch.empty_like(w)
+    return tok_fsq_encode_backward(u, w, grad_codes, grad_u, grad_w, _workspace(B, C, S, u.device), stream)
+
+
+def fsq_decode_backward(idx: torch.Tensor, w: torch.Tensor, grad_out: torch.Tensor, stream=None):
+    B, C, S = _latent_dims(grad_out)
+    grad_codes = torch.empty((B, FSQ_DIM) + tuple(grad_out.shape[2:]), dtype=torch.float32, device=idx.device)
+    grad_w = torch.empty_like(w)
+    return tok_fsq_decode_backward(idx, w, grad_out, grad_codes, grad_w, _workspace(B, C, S, idx.device), stream)

@@ -79,7 +79,8 @@ struct Geometry {
 // grid.x covers the (i, jn) items of one latent frame, grid.y the latent frame,
 // grid.z the (b, c) pair; y and z loop when the grid is capped.
 // ---------------------------------------------------------------------------
-template <typename T, int NB, bool VEC>
+// ADJ: the unpatcher's adjoint (window 0 takes (0, 0, 0, frame 0) in time).
+template <typename T, int NB, bool VEC, bool ADJ>
 __global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restrict__ x, T *__restrict__ y, Geometry g)
 {
     const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restric
         {
             float v[NB][4][4][4]; // [block][t][y][x]
             if (tq == 0) {
-                // Output frame 0 reads frame 0 four times.
+                // Output frame 0 reads frame 0 four times (the adjoint: once, as the last sample).
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
                     float row[4 * NB];
@@ -109,9 +110,9 @@ __global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restric
 #pragma unroll
                         for (int d = 0; d < 4; ++d) {
                             const float s = row[4 * nb + d];
-                            v[nb][0][r][d] = s;
-                            v[nb][1][r][d] = s;
-                            v[nb][2][r][d] = s;
+                            v[nb][0][r][d] = ADJ ? 0.0f : s;
+                            v[nb][1][r][d] = ADJ ? 0.0f : s;
+                            v[nb][2][r][d] = ADJ ? 0.0f : s;
                             v[nb][3][r][d] = s;
                         }
                 }
@@ -164,7 +165,8 @@ __global__ void __launch_bounds__(kThreads) haar3d_fwd_kernel(const T *__restric
 // ---------------------------------------------------------------------------
 // Inverse, video: y [B,64C,Tq,h,w] -> x [B,C,T,H,W].
 // ---------------------------------------------------------------------------
-template <typename T, int NB, bool VEC>
+// ADJ: the patcher's adjoint (frame 0 receives the sum of window 0's four rebuilt frames).
+template <typename T, int NB, bool VEC, bool ADJ>
 __global__ void __launch_bounds__(kThreads) haar3d_inv_kernel(const T *__restrict__ y, T *__restrict__ x, Geometry g)
 {
     const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -212,6 +214,15 @@ __global__ void __launch_bounds__(kThreads) haar3d_inv_kernel(const T *__restric
                         haar4(v[nb][0][r][d], v[nb][1][r][d], v[nb][2][r][d], v[nb][3][r][d]);
             }
             // Window 0 rebuilds frame 0 as its last sample; window t' >= 1 rebuilds frames 4t'-3 .. 4t'.
+            if (ADJ && tq == 0) {
+#pragma unroll
+                for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            v[nb][3][r][d] = ((v[nb][0][r][d] + v[nb][1][r][d]) + v[nb][2][r][d]) + v[nb][3][r][d];
+            }
             const int a_first = (tq == 0) ? 3 : 0;
 #pragma unroll
             for (int a = 0; a < 4; ++a) {
@@ -339,7 +350,7 @@ __global__ void __launch_bounds__(kThreads) haar2d_inv_kernel(const T *__restric
 // ---------------------------------------------------------------------------
 constexpr int64_t kMaxGridYZ = 65535;
 
-template <typename T, int NB, bool VEC>
+template <typename T, int NB, bool VEC, bool ADJ>
 tok_status launch3d(bool fwd, const void *in, void *out, Geometry g, cudaStream_t stream)
 {
     g.wn = g.w / NB;
@@ -353,9 +364,9 @@ tok_status launch3d(bool fwd, const void *in, void *out, Geometry g, cudaStream_
         return TOK_ERR_SHAPE;
     const dim3 grid((unsigned)gx, gy, (unsigned)gz);
     if (fwd)
-        haar3d_fwd_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+        haar3d_fwd_kernel<T, NB, VEC, ADJ><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
     else
-        haar3d_inv_kernel<T, NB, VEC><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+        haar3d_inv_kernel<T, NB, VEC, ADJ><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
     return launch_status();
 }
 
@@ -379,8 +390,16 @@ tok_status launch2d(bool fwd, const void *in, void *out, Geometry g, cudaStream_
 }
 
 // Latent frames [t_begin, t_end) of the full tensors; t_end < 0 means "through the last".
-tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
-                     int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream)
+template <typename T, int NB, bool VEC>
+tok_status launch3d_any(bool fwd, bool adj, const void *in, void *out, Geometry g, cudaStream_t stream)
+{
+    return adj ? launch3d<T, NB, VEC, true>(fwd, in, out, g, stream) : launch3d<T, NB, VEC, false>(fwd, in, out, g, stream);
+}
+
+// fwd: pixels -> coefficients.  adj: the adjoint variants (the gradient of the other
+// direction's operation); on images the transform is orthogonal and adj changes nothing.
+tok_status haar_call(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                     int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream)
 {
     if (dt != TOK_F32 && dt != TOK_BF16)
         return TOK_ERR_DTYPE;
@@ -417,7 +436,7 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
 
     const HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, g.tq0, g.nq};
     if (haar_tma_eligible(in, out, dt, dims))
-        return haar_tma_launch(fwd, in, out, dt, dims, stream);
+        return haar_tma_launch(fwd, adj, in, out, dt, dims, stream);
 
     // Register path: any 4-aligned W and element-aligned pointers.
     const bool a16 = aligned(in, 16) && aligned(out, 16);
@@ -425,10 +444,10 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
         // Two adjacent blocks per thread: 8 input elements per row, pairs per plane.
         const bool vec = a16 && W % 8 == 0;
         if (dt == TOK_BF16)
-            return vec ? launch3d<__nv_bfloat16, 2, true>(fwd, in, out, g, stream)
-                       : launch3d<__nv_bfloat16, 1, false>(fwd, in, out, g, stream);
-        return vec ? launch3d<float, 2, true>(fwd, in, out, g, stream)
-                   : launch3d<float, 1, false>(fwd, in, out, g, stream);
+            return vec ? launch3d_any<__nv_bfloat16, 2, true>(fwd, adj, in, out, g, stream)
+                       : launch3d_any<__nv_bfloat16, 1, false>(fwd, adj, in, out, g, stream);
+        return vec ? launch3d_any<float, 2, true>(fwd, adj, in, out, g, stream)
+                   : launch3d_any<float, 1, false>(fwd, adj, in, out, g, stream);
     }
     // Image path: four adjacent blocks per thread: 16 input elements per row, quads per plane.
     const bool vec = a16 && W % 16 == 0;
@@ -444,13 +463,25 @@ tok_status haar_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t 
 extern "C" tok_status tok_haar_fwd(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                                    int64_t W, cudaStream_t stream)
 {
-    return tok::haar_call(true, x, y, dt, B, C, T, H, W, 0, -1, stream);
+    return tok::haar_call(true, false, x, y, dt, B, C, T, H, W, 0, -1, stream);
 }
 
 extern "C" tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
                                    int64_t W, cudaStream_t stream)
 {
-    return tok::haar_call(false, y, x, dt, B, C, T, H, W, 0, -1, stream);
+    return tok::haar_call(false, false, y, x, dt, B, C, T, H, W, 0, -1, stream);
+}
+
+extern "C" tok_status tok_haar_fwd_adjoint(const void *gy, void *gx, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, cudaStream_t stream)
+{
+    return tok::haar_call(false, true, gy, gx, dt, B, C, T, H, W, 0, -1, stream);
+}
+
+extern "C" tok_status tok_haar_inv_adjoint(const void *gx, void *gy, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, cudaStream_t stream)
+{
+    return tok::haar_call(true, true, gx, gy, dt, B, C, T, H, W, 0, -1, stream);
 }
 
 extern "C" tok_status tok_haar_fwd_windows(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
@@ -458,7 +489,7 @@ extern "C" tok_status tok_haar_fwd_windows(const void *x, void *y, tok_dtype dt,
 {
     if (t_end < 0)
         return TOK_ERR_SHAPE;
-    return tok::haar_call(true, x, y, dt, B, C, T, H, W, t_begin, t_end, stream);
+    return tok::haar_call(true, false, x, y, dt, B, C, T, H, W, t_begin, t_end, stream);
 }
 
 extern "C" tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
@@ -466,5 +497,5 @@ extern "C" tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt,
 {
     if (t_end < 0)
         return TOK_ERR_SHAPE;
-    return tok::haar_call(false, y, x, dt, B, C, T, H, W, t_begin, t_end, stream);
+    return tok::haar_call(false, false, y, x, dt, B, C, T, H, W, t_begin, t_end, stream);
 }

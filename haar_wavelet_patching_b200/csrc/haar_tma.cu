@@ -146,7 +146,12 @@ template <bool VIDEO> struct TileRows {
     static constexpr int RW = VIDEO ? 1 : 4;
 };
 
-template <typename T, bool VIDEO, bool FWD>
+// FWD: pixels -> coefficients (the patcher, or with ADJ the unpatcher's adjoint);
+// !FWD: coefficients -> pixels (the unpatcher, or with ADJ the patcher's adjoint).
+// ADJ changes window 0 only: its time samples are (0, 0, 0, frame 0) instead of four
+// copies of frame 0, and frame 0 receives the sum of the four rebuilt samples
+// instead of the last one.
+template <typename T, bool VIDEO, bool FWD, bool ADJ>
 __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
                     const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
@@ -223,8 +228,15 @@ __global__ void __launch_bounds__(32)
                 for (int a = 0; a < NA; ++a) {
                     const int fa = (VIDEO && tq > 0) ? a : 0; // window 0 reads frame 0 four times
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr)
-                        SRow<T>::load(tin + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                    for (int rr = 0; rr < 4; ++rr) {
+                        if (ADJ && VIDEO && tq == 0 && a != 3) {
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                v[a][rr][d] = make_float2(0.0f, 0.0f);
+                        } else {
+                            SRow<T>::load(tin + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                        }
+                    }
                 }
             } else {
 #pragma unroll
@@ -272,8 +284,21 @@ __global__ void __launch_bounds__(32)
                     gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
                 }
             } else {
-                // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only.
+                // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only
+                // (the adjoint: the sum of its four frames).
                 T *xb = out + (bc * tg.T) * tg.H * tg.W + (4 * row) * tg.W + 4 * j0;
+                if (ADJ && VIDEO && tq == 0) {
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        float2 o[4];
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            o[d] = __fmul2_rn(add2(add2(add2(v[0][rr][d], v[1][rr][d]), v[2][rr][d]), v[3][rr][d]),
+                                              scale);
+                        gstore_row(xb + rr * tg.W, o);
+                    }
+                    continue;
+                }
 #pragma unroll
                 for (int a = 0; a < NA; ++a) {
                     if (VIDEO && tq == 0 && a != 3)
@@ -304,7 +329,8 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+template <typename T, bool VIDEO, bool FWD, bool ADJ>
+tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     using P = WarpTiles<T>;
     constexpr int G = VIDEO ? 64 : 16, RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
@@ -348,13 +374,13 @@ template <typename T, bool VIDEO, bool FWD> tok_status launch(const void *in, vo
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err =
-        cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+        cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_tma_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
+    haar_tma_kernel<T, VIDEO, FWD, ADJ><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
     return launch_status();
 }
 
@@ -376,19 +402,26 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
     return sm_count() > 0;
 }
 
-tok_status haar_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream)
+tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
+                           cudaStream_t stream)
 {
     const bool video = d.T > 1;
     if (dt == TOK_BF16) {
-        if (video)
-            return fwd ? launch<__nv_bfloat16, true, true>(in, out, d, stream)
-                       : launch<__nv_bfloat16, true, false>(in, out, d, stream);
-        return fwd ? launch<__nv_bfloat16, false, true>(in, out, d, stream)
-                   : launch<__nv_bfloat16, false, false>(in, out, d, stream);
+        using B16 = __nv_bfloat16;
+        if (!video)
+            return fwd ? launch<B16, false, true, false>(in, out, d, stream)
+                       : launch<B16, false, false, false>(in, out, d, stream);
+        if (adj)
+            return fwd ? launch<B16, true, true, true>(in, out, d, stream)
+                       : launch<B16, true, false, true>(in, out, d, stream);
+        return fwd ? launch<B16, true, true, false>(in, out, d, stream) : launch<B16, true, false, false>(in, out, d, stream);
     }
-    if (video)
-        return fwd ? launch<float, true, true>(in, out, d, stream) : launch<float, true, false>(in, out, d, stream);
-    return fwd ? launch<float, false, true>(in, out, d, stream) : launch<float, false, false>(in, out, d, stream);
+    if (!video)
+        return fwd ? launch<float, false, true, false>(in, out, d, stream)
+                   : launch<float, false, false, false>(in, out, d, stream);
+    if (adj)
+        return fwd ? launch<float, true, true, true>(in, out, d, stream) : launch<float, true, false, true>(in, out, d, stream);
+    return fwd ? launch<float, true, true, false>(in, out, d, stream) : launch<float, true, false, false>(in, out, d, stream);
 }
 
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)

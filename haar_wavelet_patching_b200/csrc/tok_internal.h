@@ -18,7 +18,9 @@ struct HaarDims {
 
 // The TMA path takes 16-byte-aligned tensors whose rows are multiples of 16 bytes.
 bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
-tok_status haar_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream);
+// fwd: pixels -> coefficients; adj: the adjoint variant (video only; images are orthogonal).
+tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
+                           cudaStream_t stream);
 
 // Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
 // Haar (resp. FSQ) kernels since the last call, and clear them.

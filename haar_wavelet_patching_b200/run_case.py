@@ -16,7 +16,9 @@ import haar_wavelet_patching_b200 as hwp
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", required=True, choices=("haar_fwd", "haar_inv", "fsq_encode", "fsq_decode"))
+    ap.add_argument("--op", required=True, choices=("haar_fwd", "haar_inv", "haar_fwd_adjoint", "haar_inv_adjoint",
+                                                     "fsq_encode", "fsq_decode", "fsq_encode_backward",
+                                                     "fsq_decode_backward"))
     ap.add_argument("--shape", required=True, help="B,C,T,H,W for haar ops; B,C,S for fsq ops")
     ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
     ap.add_argument("--iters", type=int, default=3)
@@ -27,15 +29,15 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op in ("haar_fwd", "haar_inv"):
+    if a.op.startswith("haar"):
         B, C, T, H, W = shape
         x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
         y = torch.empty(hwp.haar_coeff_shape(*shape), dtype=dt, device=dev)
-        if a.op == "haar_inv":
+        if a.op in ("haar_inv", "haar_fwd_adjoint"):
             y.copy_((torch.rand(y.shape, generator=g, device=dev) * 2 - 1).to(dt))
-            run = lambda: hwp.tok_haar_inv(y, x)  # noqa: E731
-        else:
-            run = lambda: hwp.tok_haar_fwd(x, y)  # noqa: E731
+        run = {"haar_fwd": lambda: hwp.tok_haar_fwd(x, y), "haar_inv": lambda: hwp.tok_haar_inv(y, x),
+               "haar_fwd_adjoint": lambda: hwp.tok_haar_fwd_adjoint(y, x),
+               "haar_inv_adjoint": lambda: hwp.tok_haar_inv_adjoint(x, y)}[a.op]
         nbytes = (x.numel() + y.numel()) * x.element_size()
     else:
         B, C, S = shape
@@ -46,9 +48,20 @@ def main():
         if a.op == "fsq_encode":
             run = lambda: hwp.tok_fsq_encode(u, w, idx, codes)  # noqa: E731
             nbytes = (u.numel() + idx.numel() + (codes.numel() if codes is not None else 0)) * 4
-        else:
+        elif a.op == "fsq_decode":
             run = lambda: hwp.tok_fsq_decode(idx, w, u)  # noqa: E731
             nbytes = (u.numel() + idx.numel()) * 4
+        else:
+            ws = torch.empty(max(hwp.fsq_backward_workspace_size(B, C, S), 1), dtype=torch.uint8, device=dev)
+            gw = torch.empty_like(w)
+            g6 = torch.randn(B, 6, S, generator=g, device=dev)
+            gout = torch.empty_like(u)
+            if a.op == "fsq_encode_backward":
+                run = lambda: hwp.tok_fsq_encode_backward(u, w, g6, gout, gw, ws)  # noqa: E731
+                nbytes = (2 * u.numel() + g6.numel()) * 4
+            else:
+                run = lambda: hwp.tok_fsq_decode_backward(idx, w, u, g6, gw, ws)  # noqa: E731
+                nbytes = (u.numel() + idx.numel() + g6.numel()) * 4
 
     run()
     torch.cuda.synchronize()

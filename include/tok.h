@@ -130,6 +130,27 @@ TOK_API tok_status tok_haar_inv(const void *y, void *x, tok_dtype dt, int64_t B,
                         int64_t W, cudaStream_t stream);
 
 /*
+ * tok_haar_fwd_adjoint / tok_haar_inv_adjoint -- the gradients (transposes) of
+ * the patcher and of the unpatcher, for training through them.  [guide] 7.1:
+ * the patcher replicates frame 0 and pairs samples with the symmetric
+ * orthonormal butterfly, so its transpose is the unpatcher's butterflies with
+ * the replica's gradient ADDED to frame 0: window 0 gives frame 0 the sum of
+ * its four rebuilt frames.  The unpatcher drops the replica, so its transpose
+ * feeds window 0 the time samples (0, 0, 0, g_0) and applies the patcher's
+ * butterflies.  On images (T == 1) both transforms are orthogonal and the
+ * adjoints equal tok_haar_inv and tok_haar_fwd.  The round (straight-through)
+ * has no part here: the patcher is linear.
+ *
+ *   tok_haar_fwd_adjoint: gy (coefficient layout, input) -> gx [B, C, T, H, W]
+ *   tok_haar_inv_adjoint: gx [B, C, T, H, W] (input)    -> gy (coefficient layout)
+ * Same shape rule, dtypes and errors as tok_haar_fwd.
+ */
+TOK_API tok_status tok_haar_fwd_adjoint(const void *gy, void *gx, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                        int64_t H, int64_t W, cudaStream_t stream);
+TOK_API tok_status tok_haar_inv_adjoint(const void *gx, void *gy, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                        int64_t H, int64_t W, cudaStream_t stream);
+
+/*
  * tok_haar_fwd_windows / tok_haar_inv_windows -- the same transforms restricted
  * to latent frames [t_begin, t_end), 0 <= t_begin <= t_end <= T' (T' = 1 on
  * images).  x and y are the full tensors with the extents above; only latent
@@ -184,6 +205,48 @@ TOK_API tok_status tok_fsq_encode(const float *u, const float *w, int32_t *idx, 
  */
 TOK_API tok_status tok_fsq_decode(const int32_t *idx, const float *w, float *out, int32_t *bad_count, int64_t B,
                           int64_t C, int64_t S, cudaStream_t stream);
+
+/*
+ * FSQ backward (training).  [guide] 7.2: the bound uses tanh and round_ste
+ * keeps a straight-through gradient -- the rounding passes the gradient
+ * unchanged -- so d zhat_i / d z_i = half_i * sech^2(z_i + shift_i) / floor(L_i/2)
+ * with the constants of tok_fsq_encode.  The weight gradient is a sum over all
+ * tokens; it is reduced deterministically (a fixed partition of the tokens and a
+ * fixed summation order, independent of the device) through a caller-provided
+ * workspace of tok_fsq_backward_workspace_size() bytes, device memory that the
+ * call overwrites.  grad_w is overwritten, not accumulated.  1 <= C <= 16.
+ */
+
+/* Workspace bytes for a backward call on [B, C, S]; -1 for an invalid shape. */
+TOK_API int64_t tok_fsq_backward_workspace_size(int64_t B, int64_t C, int64_t S);
+
+/*
+ * tok_fsq_encode_backward -- gradients of tok_fsq_encode's codes output.
+ *   u          : [B, C, S] fp32, the forward's latent (input)
+ *   w          : [6, C] fp32 (input)
+ *   grad_codes : [B, 6, S] fp32, gradient of the normalized codes (input)
+ *   grad_u     : [B, C, S] fp32, sum_i w[i][c] * t_i (output)
+ *   grad_w     : [6, C] fp32, sum over tokens of t_i * u[c] (output)
+ * with t_i = grad_codes_i * d zhat_i / d z_i and z the forward's fp32 chain.
+ * Errors: as tok_fsq_encode, plus TOK_ERR_SHAPE for C > 16 or a workspace that
+ * is too small, TOK_ERR_ALIAS if any buffer overlaps an output or the workspace.
+ */
+TOK_API tok_status tok_fsq_encode_backward(const float *u, const float *w, const float *grad_codes, float *grad_u,
+                                           float *grad_w, void *workspace, int64_t workspace_bytes, int64_t B,
+                                           int64_t C, int64_t S, cudaStream_t stream);
+
+/*
+ * tok_fsq_decode_backward -- gradients of tok_fsq_decode.
+ *   idx        : [B, S] int32 (input)
+ *   w          : [6, C] fp32 (input)
+ *   grad_out   : [B, C, S] fp32, gradient of the decoded latent (input)
+ *   grad_codes : [B, 6, S] fp32, sum_c w[i][c] * grad_out[c]; 0 for invalid indices (output)
+ *   grad_w     : [6, C] fp32, sum over tokens of zhat_i * grad_out[c] (output)
+ */
+TOK_API tok_status tok_fsq_decode_backward(const int32_t *idx, const float *w, const float *grad_out,
+                                           float *grad_codes, float *grad_w, void *workspace,
+                                           int64_t workspace_bytes, int64_t B, int64_t C, int64_t S,
+                                           cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -98,6 +98,23 @@ def test_haar_window_rules(lib):
     assert iw(A, A, 1, 1, 3, 9, 64, 64, 0, 1, NULL) == hwp.TOK_ERR_ALIAS
 
 
+def test_backward_argument_rules(lib):
+    ws = lib.tok_fsq_backward_workspace_size
+    assert ws(64, 16, 56320) == ((64 * 56320 + 2047) // 2048) * 96 * 4
+    assert ws(1, 17, 8) == -1 and ws(1, 0, 8) == -1 and ws(-1, 16, 8) == -1
+    assert ws(0, 16, 8) == 0
+    eb, db = lib.tok_fsq_encode_backward, lib.tok_fsq_decode_backward
+    U, Wt, G, GU, GW, WS = F(0x100000), F(0x200000), F(0x300000), F(0x400000), F(0x500000), F(0x600000)
+    need = ws(1, 16, 128)
+    assert eb(U, Wt, G, GU, GW, WS, need - 4, 1, 16, 128, NULL) == hwp.TOK_ERR_SHAPE    # workspace too small
+    assert eb(U, Wt, G, GU, GW, WS, need, 1, 17, 128, NULL) == hwp.TOK_ERR_SHAPE        # C > 16
+    assert eb(U, Wt, G, NULL, GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_NULL
+    assert eb(U, Wt, G, F(0x100000 + 64), GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS  # grad_u in u
+    assert eb(U, Wt, G, GU, GW, F(0x400000 + 8), need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS   # workspace in grad_u
+    assert db(U, Wt, G, GU, GW, WS, need - 4, 1, 16, 128, NULL) == hwp.TOK_ERR_SHAPE
+    assert db(U, Wt, G, F(0x300000 + 4), GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS
+
+
 def test_fsq_argument_rules(lib):
     enc, dec = lib.tok_fsq_encode, lib.tok_fsq_decode
     assert enc(A, Bp, F(0x20000000), NULL, 1, 0, 16, NULL) == hwp.TOK_ERR_SHAPE       # C >= 1
