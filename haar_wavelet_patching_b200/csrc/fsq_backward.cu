@@ -17,8 +17,9 @@
 // partition does not depend on the device), each thread accumulates its tokens
 // in registers in order, a shuffle tree and shared memory reduce a CTA's
 // threads in a fixed order into one row of the caller's workspace
-// [blocks][6C], and a second kernel sums the rows in order, in double.  The
-// result is therefore the same on every run and every B200.
+// [blocks][6C], and a second kernel sums the rows in double in a fixed order
+// (strided per thread, then a pairwise tree).  The result is therefore the same
+// on every run and every B200.
 //
 // Memory: encode backward reads u (4C B), g (24 B) and writes grad_u (4C B)
 // per token; decode backward reads the index (4 B) and g (4C B) and writes
@@ -195,19 +196,29 @@ __global__ void __launch_bounds__(kThreads)
     reduce_rows(acc, C, red, partial + (int64_t)blockIdx.x * 6 * C);
 }
 
-// grad_w[k] = sum over the rows of partial, in row order, in double.
-__global__ void fsq_bwd_sum_rows_kernel(const float *__restrict__ partial, int64_t rows, int K, float *__restrict__ out)
+// grad_w[k] = sum over the rows of partial, in double, in a fixed order: one CTA
+// per entry k; thread t sums rows t, t + 256, ... in order, then a pairwise tree
+// over the threads.
+constexpr int kSumThreads = 256;
+__global__ void __launch_bounds__(kSumThreads)
+    fsq_bwd_sum_rows_kernel(const float *__restrict__ partial, int64_t rows, int K, float *__restrict__ out)
 {
-    const int k = blockIdx.x * blockDim.x + threadIdx.x;
-    if (k >= K)
-        return;
+    __shared__ double part[kSumThreads];
+    const int k = blockIdx.x;
     double s = 0.0;
-    for (int64_t r = 0; r < rows; ++r)
+    for (int64_t r = threadIdx.x; r < rows; r += kSumThreads)
         s += (double)partial[r * K + k];
-    out[k] = (float)s;
+    part[threadIdx.x] = s;
+    __syncthreads();
+    for (int half = kSumThreads / 2; half > 0; half >>= 1) {
+        if (threadIdx.x < half)
+            part[threadIdx.x] += part[threadIdx.x + half];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0)
+        out[k] = (float)part[0];
 }
 
-// Tokens N = B*S; false on a bad extent or if a tensor's byte size overflows.
 bool shape_ok(int64_t B, int64_t C, int64_t S, int64_t *N)
 {
     int64_t bytes;
@@ -268,7 +279,8 @@ extern "C" tok_status tok_fsq_encode_backward(const float *u, const float *w, co
     if (rows > 0)
         fsq_encode_bwd_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(u, w, grad_codes, grad_u, (float *)workspace, B,
                                                                        (int)C, S, slope_consts());
-    fsq_bwd_sum_rows_kernel<<<1, 128, 0, stream>>>((const float *)workspace, rows, (int)(6 * C), grad_w);
+    fsq_bwd_sum_rows_kernel<<<(unsigned)(6 * C), kSumThreads, 0, stream>>>((const float *)workspace, rows,
+                                                                             (int)(6 * C), grad_w);
     return launch_status();
 }
 
@@ -308,6 +320,7 @@ extern "C" tok_status tok_fsq_decode_backward(const int32_t *idx, const float *w
     if (rows > 0)
         fsq_decode_bwd_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(idx, w, grad_out, grad_codes,
                                                                        (float *)workspace, B, (int)C, S);
-    fsq_bwd_sum_rows_kernel<<<1, 128, 0, stream>>>((const float *)workspace, rows, (int)(6 * C), grad_w);
+    fsq_bwd_sum_rows_kernel<<<(unsigned)(6 * C), kSumThreads, 0, stream>>>((const float *)workspace, rows,
+                                                                             (int)(6 * C), grad_w);
     return launch_status();
 }
