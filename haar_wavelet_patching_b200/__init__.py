@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtok.so")
 
 (TOK_OK, TOK_ERR_NULL, TOK_ERR_SHAPE, TOK_ERR_ALIGN, TOK_ERR_DTYPE, TOK_ERR_ALIAS, TOK_ERR_CUDA,
- TOK_ERR_TIMEOUT) = range(8)
+ TOK_ERR_TIMEOUT, TOK_ERR_TOO_LARGE) = range(9)
 TOK_F32, TOK_BF16 = 0, 1
 FSQ_CODEBOOK = 64000
 FSQ_DIM = 6
@@ -26,7 +26,7 @@ FSQ_DIM = 6
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
                "tok_haar_inv_windows", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
-               "tok_fsq_encode_backward", "tok_fsq_decode_backward")
+               "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
 _lib = None
 
@@ -65,6 +65,8 @@ def lib():
         for f in (L.tok_fsq_encode_backward, L.tok_fsq_decode_backward):
             f.restype = i32
             f.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, vp]
+        L.tok_fsq_encode_backward_noalloc.restype = i32
+        L.tok_fsq_encode_backward_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, vp]
         for f in (L.tok_haar_fwd_windows, L.tok_haar_inv_windows):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, vp]
@@ -273,6 +275,19 @@ def tok_fsq_encode_backward(u, w, grad_codes, grad_u, grad_w, workspace, stream=
     _check(lib().tok_fsq_encode_backward(_ptr(u), _ptr(w), _ptr(grad_codes), _ptr(grad_u), _ptr(grad_w),
                                          _ptr(workspace), workspace.numel() * workspace.element_size(), B, C, S,
                                          _stream(u, stream)), "tok_fsq_encode_backward")
+    return grad_u, grad_w
+
+
+def tok_fsq_encode_backward_noalloc(u, w, grad_codes, grad_u, grad_w, stream=None):
+    """tok_fsq_encode_backward using the library's fixed scratch instead of a workspace (allocates nothing;
+    at most 8,388,608 tokens; concurrent calls must be serialized by the caller)."""
+    for t, n in ((u, "u"), (w, "w"), (grad_codes, "grad_codes"), (grad_u, "grad_u"), (grad_w, "grad_w")):
+        _cuda(t, n)
+    B, C, S = _latent_dims(u)
+    if grad_u.shape != u.shape or grad_codes.numel() != B * FSQ_DIM * S or tuple(grad_w.shape) != (FSQ_DIM, C):
+        raise ValueError("shapes: grad_u like u, grad_codes [B,6,...], grad_w [6,C]")
+    _check(lib().tok_fsq_encode_backward_noalloc(_ptr(u), _ptr(w), _ptr(grad_codes), _ptr(grad_u), _ptr(grad_w),
+                                                 B, C, S, _stream(u, stream)), "tok_fsq_encode_backward_noalloc")
     return grad_u, grad_w
 
 

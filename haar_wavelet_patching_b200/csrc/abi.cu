@@ -112,6 +112,9 @@ extern "C" const char *tok_status_str(tok_status status)
         return "TOK_ERR_CUDA: a CUDA call or kernel launch failed";
     case TOK_ERR_TIMEOUT:
         return "TOK_ERR_TIMEOUT: a kernel stopped after a barrier wait ran out; its output is incomplete";
+    case TOK_ERR_TOO_LARGE:
+        return "TOK_ERR_TOO_LARGE: more tokens than the fixed scratch of the allocation-free call holds "
+               "(at most 8388608)";
     }
     return "unknown tok_status";
 }

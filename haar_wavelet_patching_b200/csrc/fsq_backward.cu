@@ -25,6 +25,7 @@
 // per token; decode backward reads the index (4 B) and g (4C B) and writes
 // grad_codes (24 B).  Both are HBM-bound.
 #include <cmath>
+#include <mutex>
 
 #include "tok_common.cuh"
 #include "tok_internal.h"
@@ -238,6 +239,92 @@ int64_t fsq_backward_workspace_bytes(int64_t B, int64_t C, int64_t S)
 }
 
 } // namespace tok
+
+// ---------------------------------------------------------------------------
+// Allocation-free form of the encode backward (tok_fsq_encode_backward_noalloc).
+//
+// Some callers cannot allocate device memory at the point where they need a
+// gradient: a host framework that owns every device allocation and hands its
+// plugins only their inputs and outputs, a service that fixes its memory at
+// start-up and must not allocate (cudaMalloc may synchronize the device) while
+// requests run, or an embedded pipeline with no allocator at all.  For them the
+// workspace lives in a fixed array compiled into this library: every GPU that
+// loads the library holds it, 1.5 MB, until the process exits.
+// ---------------------------------------------------------------------------
+namespace tok {
+namespace {
+
+constexpr int64_t kNoAllocMaxRows = 4096; // token blocks: at most 4096 * 2048 = 8,388,608 tokens
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxRows * 6 * kMaxC];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+float *g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+tok_status noalloc_scratch(float **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices)
+        return TOK_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            record_cuda_error(e);
+            return TOK_ERR_CUDA;
+        }
+        g_noalloc_addr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return TOK_OK;
+}
+
+} // namespace
+} // namespace tok
+
+extern "C" tok_status tok_fsq_encode_backward_noalloc(const float *u, const float *w, const float *grad_codes,
+                                                      float *grad_u, float *grad_w, int64_t B, int64_t C, int64_t S,
+                                                      cudaStream_t stream)
+{
+    using namespace tok;
+    int64_t N;
+    if (!shape_ok(B, C, S, &N))
+        return TOK_ERR_SHAPE;
+    const int64_t rows = blocks_for(N);
+    if (rows > kNoAllocMaxRows)
+        return TOK_ERR_TOO_LARGE;
+    if (!w || !grad_w || (N > 0 && (!u || !grad_codes || !grad_u)))
+        return TOK_ERR_NULL;
+    if (!aligned(u, 4) || !aligned(w, 4) || !aligned(grad_codes, 4) || !aligned(grad_u, 4) || !aligned(grad_w, 4))
+        return TOK_ERR_ALIGN;
+    const int64_t bu = N * C * 4, bg = N * 24, bw = 6 * C * 4;
+    const void *ins[3] = {u, w, grad_codes};
+    const int64_t inb[3] = {bu, bw, bg};
+    for (int a = 0; a < 3; ++a)
+        if ((inb[a] && bu && overlaps(ins[a], inb[a], grad_u, bu)) || overlaps(ins[a], inb[a], grad_w, bw))
+            return TOK_ERR_ALIAS;
+    if (bu && overlaps(grad_u, bu, grad_w, bw))
+        return TOK_ERR_ALIAS;
+    float *scratch = nullptr;
+    const tok_status st = noalloc_scratch(&scratch);
+    if (st != TOK_OK)
+        return st;
+    // Every row the sum reads is written first by the same call, so nothing is cleared.
+    if (rows > 0)
+        fsq_encode_bwd_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(u, w, grad_codes, grad_u, scratch, B, (int)C,
+                                                                       S, slope_consts());
+    fsq_bwd_sum_rows_kernel<<<(unsigned)(6 * C), kSumThreads, 0, stream>>>(scratch, rows, (int)(6 * C), grad_w);
+    return launch_status();
+}
 
 extern "C" int64_t tok_fsq_backward_workspace_size(int64_t B, int64_t C, int64_t S)
 {

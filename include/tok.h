@@ -66,7 +66,8 @@ typedef enum {
     TOK_ERR_DTYPE = 4, /* unknown tok_dtype */
     TOK_ERR_ALIAS = 5, /* an input buffer overlaps an output buffer */
     TOK_ERR_CUDA = 6,   /* a CUDA call or kernel launch failed; see tok_last_cuda_error() */
-    TOK_ERR_TIMEOUT = 7 /* reported by tok_check_device(): a kernel stopped after a bounded wait ran out */
+    TOK_ERR_TIMEOUT = 7, /* reported by tok_check_device(): a kernel stopped after a bounded wait ran out */
+    TOK_ERR_TOO_LARGE = 8 /* the problem exceeds the fixed scratch of tok_fsq_encode_backward_noalloc */
 } tok_status;
 
 typedef enum {
@@ -234,6 +235,32 @@ TOK_API int64_t tok_fsq_backward_workspace_size(int64_t B, int64_t C, int64_t S)
 TOK_API tok_status tok_fsq_encode_backward(const float *u, const float *w, const float *grad_codes, float *grad_u,
                                            float *grad_w, void *workspace, int64_t workspace_bytes, int64_t B,
                                            int64_t C, int64_t S, cudaStream_t stream);
+
+/*
+ * tok_fsq_encode_backward_noalloc -- tok_fsq_encode_backward without a
+ * workspace argument, for callers that cannot allocate device memory when they
+ * need the gradient: a host framework that owns every device allocation and
+ * hands its plugins only inputs and outputs, a service that fixes its memory
+ * at start-up and must not call cudaMalloc (which may synchronize the device)
+ * while it serves, an embedded pipeline without an allocator.  The pages have
+ * no counterpart: it is a deployment form of the same computation.
+ *
+ * The workspace is a fixed array compiled into the library (1.5 MB, held by
+ * every GPU that loads the library until the process exits), so:
+ *   - at most 4096 * 2048 = 8,388,608 tokens (B * S); larger calls return
+ *     TOK_ERR_TOO_LARGE before anything runs;
+ *   - every call uses the same array: calls that may overlap on the GPU
+ *     (concurrent streams, other host threads) race and must be serialized by
+ *     the caller; a call overwrites whatever an earlier call left there;
+ *   - the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and caches it; make that first call before any
+ *     stream capture.
+ * It allocates nothing.  Arguments, outputs and results are those of
+ * tok_fsq_encode_backward.
+ */
+TOK_API tok_status tok_fsq_encode_backward_noalloc(const float *u, const float *w, const float *grad_codes,
+                                                   float *grad_u, float *grad_w, int64_t B, int64_t C, int64_t S,
+                                                   cudaStream_t stream);
 
 /*
  * tok_fsq_decode_backward -- gradients of tok_fsq_decode.

@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(lib):
 
 def test_version_and_status_strings(lib):
     assert lib.tok_abi_version() == 1
-    for code in range(8):
+    for code in range(9):
         assert lib.tok_status_str(code).decode().startswith("TOK_")
     assert lib.tok_last_cuda_error() == 0
 
@@ -113,6 +113,12 @@ def test_backward_argument_rules(lib):
     assert eb(U, Wt, G, GU, GW, F(0x400000 + 8), need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS   # workspace in grad_u
     assert db(U, Wt, G, GU, GW, WS, need - 4, 1, 16, 128, NULL) == hwp.TOK_ERR_SHAPE
     assert db(U, Wt, G, F(0x300000 + 4), GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS
+    nb = lib.tok_fsq_encode_backward_noalloc
+    assert nb(U, Wt, G, GU, GW, 1, 16, 4096 * 2048 + 1, NULL) == hwp.TOK_ERR_TOO_LARGE     # beyond the fixed scratch
+    assert nb(U, Wt, G, GU, GW, 2, 16, 4096 * 1024 + 1, NULL) == hwp.TOK_ERR_TOO_LARGE
+    assert nb(U, Wt, G, GU, GW, 1, 17, 128, NULL) == hwp.TOK_ERR_SHAPE
+    assert nb(U, Wt, G, NULL, GW, 1, 16, 128, NULL) == hwp.TOK_ERR_NULL
+    assert nb(U, Wt, G, F(0x100000 + 64), GW, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS
 
 
 def test_fsq_argument_rules(lib):
