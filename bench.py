@@ -328,6 +328,43 @@ def make_e2e_step(torch, hwp, x_host, u_host, w_dev, x, y, xr, u, idx, ur, y_hos
 
     step.join = join
     return step
+GRAD_ITERS = 20
+
+
+def time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev, iters=GRAD_ITERS):
+    """The gradient calls on the headline workload, each timed alone (CUDA events on the
+    launching stream, mean over `iters` launches after one warm-up), outside the step's timed
+    region.  Buffers of the step are reused as inputs and outputs; returns per call the mean ms,
+    the algorithmic bytes per call (inputs read once, outputs written once; the FSQ workspace
+    rows are not counted) and the kernel launches per call."""
+    B, _, S = u.shape
+    g6 = torch.randn(B, 6, S, device=dev, generator=torch.Generator(device=dev).manual_seed(7))
+    gcodes = torch.empty_like(g6)
+    gw = torch.empty_like(w_dev)
+    ws = torch.empty(max(hwp.fsq_backward_workspace_size(B, u.shape[1], S), 1), dtype=torch.uint8, device=dev)
+    hb = x.numel() * x.element_size() + y.numel() * y.element_size()
+    calls = {
+        "haar_fwd_adjoint": (lambda: hwp.tok_haar_fwd_adjoint(y, xr), hb, 1),
+        "haar_inv_adjoint": (lambda: hwp.tok_haar_inv_adjoint(x, y), hb, 1),
+        "fsq_encode_backward": (lambda: hwp.tok_fsq_encode_backward(u, w_dev, g6, ur, gw, ws),
+                                (2 * u.numel() + g6.numel()) * 4, 2),
+        "fsq_decode_backward": (lambda: hwp.tok_fsq_decode_backward(idx, w_dev, u, gcodes, gw, ws),
+                                (u.numel() + idx.numel() + gcodes.numel()) * 4, 2),
+    }
+    out = {}
+    for name, (call, nbytes, launches) in calls.items():
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "bytes": nbytes, "launches": launches}
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -429,6 +466,9 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     barrier()
 
+    grads = time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev)
+    barrier()
+
     if rank != 0:
         return 0
     peak, peak_kind = measured_peak()
@@ -458,6 +498,9 @@ def run_ours(args, rank, world, local_rank):
                         "(H2D / kernels / D2H), tok_haar_*_windows per chunk"},
         "gpu_launches": 4 * K,
         "clocks": clocks,
+        "gradients": {n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
+                          "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
+                          "bytes": g["bytes"], "launches": g["launches"]} for n, g in grads.items()},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

@@ -280,7 +280,7 @@ def tok_fsq_encode_backward(u, w, grad_codes, grad_u, grad_w, workspace, stream=
 
 def tok_fsq_encode_backward_noalloc(u, w, grad_codes, grad_u, grad_w, stream=None):
     """tok_fsq_encode_backward using the library's fixed scratch instead of a workspace (allocates nothing;
-    at most 8,388,608 tokens; concurrent calls must be serialized by the caller)."""
+    its 3 MB scratch holds at most 8,388,608 tokens at C = 16; concurrent calls must be serialized by the caller)."""
     for t, n in ((u, "u"), (w, "w"), (grad_codes, "grad_codes"), (grad_u, "grad_u"), (grad_w, "grad_w")):
         _cuda(t, n)
     B, C, S = _latent_dims(u)

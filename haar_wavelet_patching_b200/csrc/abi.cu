@@ -84,13 +84,15 @@ extern "C" int tok_last_cuda_error(void) { return tok::g_last_cuda_error; }
 
 extern "C" tok_status tok_check_device(cudaStream_t stream)
 {
-    unsigned int nh = 0, nf = 0;
+    unsigned int nh = 0, nf = 0, nb = 0;
     tok_status st = tok::read_and_clear_haar_timeouts(stream, &nh);
     if (st == TOK_OK)
         st = tok::read_and_clear_fsq_timeouts(stream, &nf);
+    if (st == TOK_OK)
+        st = tok::read_and_clear_fsq_bwd_timeouts(stream, &nb);
     if (st != TOK_OK)
         return st;
-    return (nh || nf) ? TOK_ERR_TIMEOUT : TOK_OK;
+    return (nh || nf || nb) ? TOK_ERR_TIMEOUT : TOK_OK;
 }
 
 extern "C" const char *tok_status_str(tok_status status)
@@ -113,8 +115,8 @@ extern "C" const char *tok_status_str(tok_status status)
     case TOK_ERR_TIMEOUT:
         return "TOK_ERR_TIMEOUT: a kernel stopped after a barrier wait ran out; its output is incomplete";
     case TOK_ERR_TOO_LARGE:
-        return "TOK_ERR_TOO_LARGE: more tokens than the fixed scratch of the allocation-free call holds "
-               "(at most 8388608)";
+        return "TOK_ERR_TOO_LARGE: the call needs more than the 3 MB fixed scratch of the allocation-free call "
+               "(at most 8388608 tokens at C = 16)";
     }
     return "unknown tok_status";
 }

@@ -23,9 +23,10 @@ tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dt
                            cudaStream_t stream);
 
 // Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
-// Haar (resp. FSQ) kernels since the last call, and clear them.
+// Haar (resp. FSQ, FSQ backward) kernels since the last call, and clear them.
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count);
 tok_status read_and_clear_fsq_timeouts(cudaStream_t stream, unsigned int *count);
+tok_status read_and_clear_fsq_bwd_timeouts(cudaStream_t stream, unsigned int *count);
 
 // Remembers a CUDA error for tok_last_cuda_error().
 void record_cuda_error(cudaError_t e);

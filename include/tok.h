@@ -245,10 +245,12 @@ TOK_API tok_status tok_fsq_encode_backward(const float *u, const float *w, const
  * while it serves, an embedded pipeline without an allocator.  The pages have
  * no counterpart: it is a deployment form of the same computation.
  *
- * The workspace is a fixed array compiled into the library (1.5 MB, held by
+ * The workspace is a fixed array compiled into the library (3 MB, held by
  * every GPU that loads the library until the process exits), so:
- *   - at most 4096 * 2048 = 8,388,608 tokens (B * S); larger calls return
- *     TOK_ERR_TOO_LARGE before anything runs;
+ *   - the workspace tok_fsq_backward_workspace_size(B, C, S) reports must fit
+ *     in 3 MB: at most 8,388,608 tokens (B * S) at C = 16 when S is a multiple
+ *     of 128 (each batch row's last 128-token tile counts whole; smaller C
+ *     allows more); larger calls return TOK_ERR_TOO_LARGE before anything runs;
  *   - every call uses the same array: calls that may overlap on the GPU
  *     (concurrent streams, other host threads) race and must be serialized by
  *     the caller; a call overwrites whatever an earlier call left there;

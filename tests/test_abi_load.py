@@ -100,7 +100,11 @@ def test_haar_window_rules(lib):
 
 def test_backward_argument_rules(lib):
     ws = lib.tok_fsq_backward_workspace_size
-    assert ws(64, 16, 56320) == ((64 * 56320 + 2047) // 2048) * 96 * 4
+    def rows(B, S):  # register path: 2048 tokens per row; TMA path: 8 tiles of 128 tokens of a batch row
+        return max((B * S + 2047) // 2048, (B * ((S + 127) // 128) + 7) // 8)
+    assert ws(64, 16, 56320) == rows(64, 56320) * 96 * 4 == 3520 * 384
+    assert ws(3, 16, 1000) == rows(3, 1000) * 96 * 4 == 3 * 384
+    assert ws(1, 5, 4097) == rows(1, 4097) * 30 * 4
     assert ws(1, 17, 8) == -1 and ws(1, 0, 8) == -1 and ws(-1, 16, 8) == -1
     assert ws(0, 16, 8) == 0
     eb, db = lib.tok_fsq_encode_backward, lib.tok_fsq_decode_backward

@@ -92,7 +92,13 @@ def test_image_adjoints_are_the_other_direction():
     assert torch.equal(hwp.haar_fwd_adjoint(y, 1, 32, 64), hwp.haar_inv(y, 1, 32, 64))
 
 
-@pytest.mark.parametrize("B,C,S", [(2, 16, 4096), (3, 16, 1000), (1, 5, 777), (16, 16, 56320)])
+# C = 16 with S % 4 == 0 takes the TMA kernels (ragged last tile at S = 1000, a single
+# mostly empty tile at S = 4, workspace rows spanning batch rows at B = 3); S = 1001 and
+# C = 5 take the register kernels.
+CASES = [(2, 16, 4096), (3, 16, 1000), (1, 16, 4), (2, 16, 1001), (1, 5, 777), (16, 16, 56320)]
+
+
+@pytest.mark.parametrize("B,C,S", CASES)
 def test_fsq_encode_backward_matches_oracle(B, C, S):
     u = synth.normal((B, C, S), seed=41 + C, std=1.3)
     w = synth.fsq_weight(C)
@@ -108,7 +114,7 @@ def test_fsq_encode_backward_matches_oracle(B, C, S):
     assert (np.abs(got_w - ref_w) <= tol_w).all(), (np.abs(got_w - ref_w) / tol_w).max()
 
 
-@pytest.mark.parametrize("B,C,S", [(2, 16, 4096), (3, 16, 1000), (1, 5, 777), (16, 16, 56320)])
+@pytest.mark.parametrize("B,C,S", CASES)
 def test_fsq_decode_backward_matches_oracle(B, C, S):
     idx = synth.uniform((B, S), seed=47, lo=0, hi=64000, dtype=synth.F64).astype(np.int32)
     idx.reshape(-1)[::997] = -3                                          # some invalid indices
