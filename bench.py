@@ -66,10 +66,19 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_digest():
+# The sources each timed kernel is compiled from (its .cu file and the headers it includes).
+KERNEL_SOURCES = {
+    "haar_fwd": ("haar_tma.cu", "tma.cuh", "tok_common.cuh", "tok_internal.h"),
+    "haar_inv": ("haar_tma.cu", "tma.cuh", "tok_common.cuh", "tok_internal.h"),
+    "fsq_encode": ("fsq.cu", "tma.cuh", "tok_common.cuh", "tok_internal.h"),
+    "fsq_decode": ("fsq.cu", "tma.cuh", "tok_common.cuh", "tok_internal.h"),
+}
+
+
+def kernel_source_digest(kernel):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "haar_wavelet_patching_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -82,7 +91,7 @@ def recorded_traffic(kernel):
         lines = open(path).read().splitlines()
     except OSError:
         return None
-    digest = kernel_source_digest()
+    digest = kernel_source_digest(kernel)
     for ln in lines:
         parts = [p.strip() for p in ln.strip().strip("|").split("|")]
         if len(parts) >= 3 and parts[0] == kernel and parts[2] == digest:

@@ -10,8 +10,9 @@
 // Decode backward, per token (zhat from the index; invalid indices count as zero):
 //   grad_codes_i = sum_c w[i][c] g_c;  grad_w[i][c] = sum_tokens zhat_i g_c.
 //
-// sech^2(x) is evaluated as 4a / (1 + a)^2 with a = exp(-2|x|): accurate where
-// tanh saturates, unlike 1 - tanh^2.
+// sech^2(x) is evaluated as 4a / (1 + a)^2 with a = exp(-2|x|) = 2^(-2 log2(e) |x|):
+// accurate where tanh saturates, unlike 1 - tanh^2.  Both paths round the same
+// sequence of fp32 operations, so they give the same t bit for bit.
 //
 // Reduction of grad_w: tokens are cut into fixed blocks of kTokensPerCta (the
 // partition does not depend on the device), each thread accumulates its tokens
@@ -27,13 +28,22 @@
 //
 // Main path (C = 16, S % 4 == 0, 16-byte-aligned tensors): single-warp CTAs,
 // each owning a fixed run of kTilesPerRow = 8 tiles of 128 tokens (tile order:
-// batch row, then position).
-// A two-stage ring of TMA loads brings a tile's inputs into shared memory while
-// the previous tile is computed; each lane owns 4 consecutive tokens, reads
-// them with 16-byte shared loads and writes its outputs with 16-byte global
-// stores.  The grad_w accumulators stay in registers across the CTA's tiles and
-// are reduced by a shuffle butterfly into the CTA's workspace row.  Other
-// shapes take the register kernels (2048 tokens per CTA, 128 threads).
+// batch row, then position).  A two-stage ring of TMA loads brings a tile's
+// inputs into shared memory while the previous tile is computed; each lane owns
+// 4 consecutive tokens, reads them with 16-byte shared loads, computes with
+// packed f32x2 operations and writes with 16-byte global stores.  The grad_w
+// accumulators stay in registers across the CTA's tiles and are reduced by a
+// shuffle butterfly into the CTA's workspace row.  Other shapes take the
+// register kernels (2048 tokens per CTA, 128 threads).
+//
+// The workspace holds one row of 6C sums per CTA, partial[row * 6C + k] with
+// k = i*C + c (a CTA writes its row as a contiguous block, the cheapest pattern
+// for the row kernel).  The summing kernel (one CTA per entry) is launched as a
+// programmatic dependent of the row kernel, so its launch is prepared while the
+// row kernel runs; it waits for the row kernel's completion before reading.
+// (Measured: letting the row kernel release it early, a grouped summing kernel
+// with 16-byte loads, and entry-major or sector-grouped workspace layouts were
+// all slower.)
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -58,8 +68,8 @@ constexpr int kStages = 2;
 static __device__ unsigned int g_bwd_wait_timeouts;
 
 struct SlopeConsts {
-    float shift[6]; // atanh(off / half)
-    float scale[6]; // half / floor(L / 2)
+    float shift[6];  // atanh(off / half)
+    float scale4[6]; // 4 * half / floor(L / 2)
 };
 
 SlopeConsts slope_consts()
@@ -70,27 +80,56 @@ SlopeConsts slope_consts()
         const double half = (L[i] - 1) * (1.0 + 1e-3) / 2.0;
         const double off = (L[i] % 2 == 0) ? 0.5 : 0.0;
         k.shift[i] = (float)std::atanh(off / half);
-        k.scale[i] = (float)(half / (double)(L[i] / 2));
+        k.scale4[i] = (float)(4.0 * half / (double)(L[i] / 2));
     }
     return k;
 }
 
-// sech^2(x) = 4a / (1 + a)^2 with a = e^{-2|x|} in (0, 1]: the quotient's
-// denominator lies in [1, 4], where the fast division is accurate to a few ulp;
-// the fast exponential's relative error grows like |x| * 2^-24, so sech^2 keeps
-// about 1e-6 relative accuracy for |x| <= 20 (beyond, a < 5e-18 is negligible
-// next to the slopes that matter).
-__device__ __forceinline__ float sech2(float x)
+// 2^x and 1/x from the hardware approximations (relative error about 2^-22).
+__device__ __forceinline__ float ex2_approx(float x)
 {
-    const float a = __expf(-2.0f * fabsf(x));
-    const float d = 1.0f + a;
-    return __fdividef(4.0f * a, d * d);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+constexpr float kMinus2Log2e = -2.88539008f; // -2 log2(e): e^{-2|x|} = 2^(kMinus2Log2e |x|)
+
+// t = g * slope(z) with slope = scale4 * a / (1 + a)^2, a = e^{-2|z + shift|} in (0, 1]:
+// the denominator lies in [1, 4], so the approximate reciprocal is accurate there; the
+// rounding of the exponent's argument costs about |x| * 2^-24 relative, which matters
+// only where the slope itself is negligible.  Relative accuracy about 1e-6.
+__device__ __forceinline__ float ste_grad(float z, float g, float shift, float scale4)
+{
+    const float x = z + shift;
+    const float a = ex2_approx(kMinus2Log2e * fabsf(x));
+    const float d = a + 1.0f;
+    const float r = rcp_approx(d * d);
+    return g * ((a * r) * scale4);
+}
+
+// The same for two tokens, in packed f32x2 operations with the same roundings.
+__device__ __forceinline__ float2 ste_grad2(float2 z, float2 g, float2 shift, float2 scale4)
+{
+    const float2 x = __fadd2_rn(z, shift);
+    const float2 a = make_float2(ex2_approx(kMinus2Log2e * fabsf(x.x)), ex2_approx(kMinus2Log2e * fabsf(x.y)));
+    const float2 d = __fadd2_rn(a, make_float2(1.0f, 1.0f));
+    const float2 dd = __fmul2_rn(d, d);
+    const float2 r = make_float2(rcp_approx(dd.x), rcp_approx(dd.y));
+    return __fmul2_rn(g, __fmul2_rn(__fmul2_rn(a, r), scale4));
 }
 
 // Reduces the per-thread accumulators acc[i * kMaxC + c] over the CTA in a fixed
-// order and writes the CTA's row of 6*C sums, row[i * C + c].  All indices into
+// order and writes the CTA's row of 6*C sums, partial[row * 6C + i * C + c].  All indices into
 // acc are compile-time constants, so it stays in registers.
-__device__ __forceinline__ void reduce_rows(const float (&acc)[6 * kMaxC], int C, float *red, float *row)
+__device__ __forceinline__ void reduce_rows(const float (&acc)[6 * kMaxC], int C, float *red, float *partial)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 #pragma unroll
@@ -110,7 +149,7 @@ __device__ __forceinline__ void reduce_rows(const float (&acc)[6 * kMaxC], int C
         float s = 0.0f;
         for (int w = 0; w < kThreads / 32; ++w)
             s += red[w * 6 * kMaxC + k];
-        row[k] = s;
+        partial[(int64_t)blockIdx.x * 6 * C + k] = s;
     }
 }
 
@@ -148,7 +187,7 @@ __global__ void __launch_bounds__(kThreads)
             for (int c = 0; c < kMaxC; ++c)
                 if (c < C)
                     z = fmaf(ws[i * C + c], uc[c], z);
-            t[i] = g[(b * 6 + i) * S + s] * (k.scale[i] * sech2(z + k.shift[i]));
+            t[i] = ste_grad(z, g[(b * 6 + i) * S + s], k.shift[i], k.scale4[i]);
         }
 #pragma unroll
         for (int c = 0; c < kMaxC; ++c) {
@@ -163,7 +202,7 @@ __global__ void __launch_bounds__(kThreads)
             gu[(b * C + c) * S + s] = acc_u;
         }
     }
-    reduce_rows(acc, C, red, partial + (int64_t)blockIdx.x * 6 * C);
+    reduce_rows(acc, C, red, partial);
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -219,31 +258,61 @@ __global__ void __launch_bounds__(kThreads)
             gcodes[(b * 6 + i) * S + s] = valid ? a : 0.0f;
         }
     }
-    reduce_rows(acc, C, red, partial + (int64_t)blockIdx.x * 6 * C);
+    reduce_rows(acc, C, red, partial);
 }
 
 // grad_w[k] = sum over the rows of partial, in double, in a fixed order: one CTA
-// per entry k; thread t sums rows t, t + 256, ... in order, then a pairwise tree
-// over the threads.
-constexpr int kSumThreads = 256;
+// per entry k; thread t sums rows t, t + 512, ... in order, each warp then sums its
+// 32 threads by a shuffle butterfly, and one warp sums the 16 warp totals the same
+// way.  Launched as a programmatic dependent of the row kernel: it waits for that
+// grid's completion (and the visibility of its writes) before it reads.
+constexpr int kSumThreads = 512;
+
+__device__ __forceinline__ double warp_sum(double v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+        v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    return v;
+}
+
 __global__ void __launch_bounds__(kSumThreads)
     fsq_bwd_sum_rows_kernel(const float *__restrict__ partial, int64_t rows, int K, float *__restrict__ out)
 {
-    __shared__ double part[kSumThreads];
-    const int k = blockIdx.x;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    __shared__ double warps[kSumThreads / 32];
+    const int t = threadIdx.x, k = blockIdx.x;
     double s = 0.0;
 #pragma unroll 8
-    for (int64_t r = threadIdx.x; r < rows; r += kSumThreads)
+    for (int64_t r = t; r < rows; r += kSumThreads)
         s += (double)partial[r * K + k];
-    part[threadIdx.x] = s;
+    s = warp_sum(s);
+    if ((t & 31) == 0)
+        warps[t >> 5] = s;
     __syncthreads();
-    for (int half = kSumThreads / 2; half > 0; half >>= 1) {
-        if (threadIdx.x < half)
-            part[threadIdx.x] += part[threadIdx.x + half];
-        __syncthreads();
+    if (t < 32) {
+        double v = t < kSumThreads / 32 ? warps[t] : 0.0;
+        v = warp_sum(v);
+        if (t == 0)
+            out[k] = (float)v;
     }
-    if (threadIdx.x == 0)
-        out[k] = (float)part[0];
+}
+
+// Launches the sum of `rows` rows of K entries into out[K] on `stream` as a
+// programmatic dependent of the preceding kernel.
+cudaError_t launch_sum_rows(const float *partial, int64_t rows, int K, float *out, cudaStream_t stream)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)K);
+    cfg.blockDim = dim3(kSumThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fsq_bwd_sum_rows_kernel, partial, rows, K, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -252,45 +321,61 @@ __global__ void __launch_bounds__(kSumThreads)
 
 // grad_w on the main path.  A pair of lanes (2p, 2p + 1) covers the pair's 8 tokens
 // 8p .. 8p + 7 of the tile; lane 2p + h accumulates the channels c = 8h .. 8h + 7, so
-// a lane holds 48 sums acc[i * 8 + cc] (c = 8h + cc) instead of 96.
+// a lane holds 48 sums, as f32x2 pairs acc2[ip][cc] = (acc[2ip][8h + cc], acc[2ip + 1][8h + cc]).
 constexpr int kHalfC = 8;
 
-// Sums acc over the 16 lanes of the same half (xor butterfly over lane bits 1..4:
-// every lane ends with the same sums in the same order) and writes them to
-// row[i * 16 + 8h + cc], three entries per lane.
-__device__ __forceinline__ void warp_row_half(float (&acc)[6 * kHalfC], float *row)
+// Sums acc2 over the 16 lanes of the same half (xor butterfly over lane bits 1..4:
+// every lane ends with the same sums in the same order) and writes entry
+// k = i * 16 + 8h + cc of this CTA's row to partial[row * 96 + k], three per lane.
+__device__ __forceinline__ void warp_row_half(const float2 (&acc2)[3][kHalfC], float *partial)
 {
     const int lane = threadIdx.x & 31, h = lane & 1;
 #pragma unroll
     for (int q = 0; q < 6 * kHalfC; ++q) {
-        float v = acc[q];
+        const int i = q / kHalfC, cc = q % kHalfC;
+        float v = (i & 1) ? acc2[i >> 1][cc].y : acc2[i >> 1][cc].x;
 #pragma unroll
         for (int off = 16; off > 1; off >>= 1)
             v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
         if ((q & 15) == (lane >> 1))
-            row[(q / kHalfC) * 16 + kHalfC * h + (q % kHalfC)] = v;
+            partial[(int64_t)blockIdx.x * 6 * kMaxC + i * 16 + kHalfC * h + cc] = v;
     }
 }
 
-// Weights in shared memory as ws[c * 8 + i] = w[i][c] (i < 6; 6 and 7 are zero),
-// so one 16-byte and one 8-byte load give a channel's six weights.
-__device__ __forceinline__ void stage_ws16(const float *__restrict__ w, float *ws)
+// Shared tables after the stages: the weights with each entry twice,
+// wd[c * 12 + 2i + e] = w[i][c] (e = 0, 1), so three 16-byte loads give a channel's six
+// weights as (w, w) pairs for the packed FMAs; then kd[i] = (shift, shift, scale4, scale4).
+constexpr int kTableBytes = 16 * 12 * 4 + 6 * 16;
+
+__device__ __forceinline__ void stage_weights(const float *__restrict__ w, float *wd)
 {
-    for (int q = threadIdx.x; q < 16 * 8; q += 32) {
-        const int c = q >> 3, i = q & 7;
-        ws[q] = i < 6 ? w[i * 16 + c] : 0.0f;
+    for (int q = threadIdx.x; q < 16 * 12; q += 32) {
+        const int c = q / 12, i = (q % 12) >> 1;
+        wd[q] = w[i * 16 + c];
     }
 }
 
-__device__ __forceinline__ void weights_of(const float *ws, int c, float (&wc)[6])
+__device__ __forceinline__ void stage_slopes(const SlopeConsts &k, float *wd)
 {
-    const float4 wa = *reinterpret_cast<const float4 *>(ws + c * 8);
-    const float2 wb = *reinterpret_cast<const float2 *>(ws + c * 8 + 4);
-    wc[0] = wa.x, wc[1] = wa.y, wc[2] = wa.z, wc[3] = wa.w, wc[4] = wb.x, wc[5] = wb.y;
+    float4 *kd = reinterpret_cast<float4 *>(wd + 16 * 12);
+#pragma unroll
+    for (int i = 0; i < 6; ++i) // constant indices keep the parameter in the constant bank
+        if (threadIdx.x == i)
+            kd[i] = make_float4(k.shift[i], k.shift[i], k.scale4[i], k.scale4[i]);
 }
 
-// Digits of a valid index, as normalized codes; an invalid index gives zeros.
-__device__ __forceinline__ void zhat_of(int32_t id, float (&zh)[6])
+__device__ __forceinline__ void wpairs_of(const float *wd, int c, float2 (&wp)[6])
+{
+    const float4 a = *reinterpret_cast<const float4 *>(wd + c * 12);
+    const float4 b = *reinterpret_cast<const float4 *>(wd + c * 12 + 4);
+    const float4 e = *reinterpret_cast<const float4 *>(wd + c * 12 + 8);
+    wp[0] = make_float2(a.x, a.y), wp[1] = make_float2(a.z, a.w), wp[2] = make_float2(b.x, b.y);
+    wp[3] = make_float2(b.z, b.w), wp[4] = make_float2(e.x, e.y), wp[5] = make_float2(e.z, e.w);
+}
+
+// Normalized codes of an index as channel pairs (zh0, zh1), (zh2, zh3), (zh4, zh5);
+// an invalid index gives zeros.
+__device__ __forceinline__ void zhat_pairs(int32_t id, float2 (&zp)[3])
 {
     const bool valid = (uint32_t)id < (uint32_t)TOK_FSQ_CODEBOOK;
     uint32_t r = valid ? (uint32_t)id : 0u;
@@ -301,12 +386,9 @@ __device__ __forceinline__ void zhat_of(int32_t id, float (&zh)[6])
     const int d4 = r % 5u; r /= 5u;
     const int d5 = (int)r;
     const float v = valid ? 1.0f : 0.0f;
-    zh[0] = v * ((float)(d0 - 4) * 0.25f);
-    zh[1] = v * ((float)(d1 - 4) * 0.25f);
-    zh[2] = v * ((float)(d2 - 4) * 0.25f);
-    zh[3] = v * ((float)(d3 - 2) * 0.5f);
-    zh[4] = v * ((float)(d4 - 2) * 0.5f);
-    zh[5] = v * ((float)(d5 - 2) * 0.5f);
+    zp[0] = make_float2(v * ((float)(d0 - 4) * 0.25f), v * ((float)(d1 - 4) * 0.25f));
+    zp[1] = make_float2(v * ((float)(d2 - 4) * 0.25f), v * ((float)(d3 - 2) * 0.5f));
+    zp[2] = make_float2(v * ((float)(d4 - 2) * 0.5f), v * ((float)(d5 - 2) * 0.5f));
 }
 
 // Ring bookkeeping shared by both kernels: tile j of the CTA sits in stage j % STAGES
@@ -326,9 +408,10 @@ __device__ __forceinline__ void ring_drain(const uint64_t *bars, int j, int coun
     __syncwarp();
 }
 
-// Encode backward, C = 16.  Stage layout: u tile [16][128] then g tile [6][128] (fp32);
-// each lane overwrites its own tokens' g with t = g * slope(z), which the lane pair
-// then reads back for grad_w.
+// Encode backward, C = 16.  Stage layout: u tile [16][128] then g tile [6][128] (fp32).
+// Once every lane has read its g, each lane writes t = g * slope(z) of its four tokens
+// over the g tile as channel pairs, tp[ip][m] = (t[2ip][m], t[2ip + 1][m]), which the
+// lane pair then reads back for grad_w.
 template <int TPR, int STAGES>
 __global__ void __launch_bounds__(32)
     fsq_encode_bwd_tma_kernel(const __grid_constant__ CUtensorMap umap, const __grid_constant__ CUtensorMap gmap,
@@ -338,7 +421,8 @@ __global__ void __launch_bounds__(32)
     constexpr int U_BYTES = 16 * kTileTokens * 4, STAGE = U_BYTES + 6 * kTileTokens * 4;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + STAGES * STAGE);
-    float *ws = reinterpret_cast<float *>(smem_raw + STAGES * STAGE + 16 * STAGES); // 16-byte aligned
+    float *wd = reinterpret_cast<float *>(smem_raw + STAGES * STAGE + 16 * STAGES); // 16-byte aligned
+    const float4 *kd = reinterpret_cast<const float4 *>(wd + 16 * 12);
     const int lane = threadIdx.x, h = lane & 1;
     const uint32_t first = blockIdx.x * (uint32_t)TPR;
     const int count = (int)min((uint32_t)TPR, ntiles - first);
@@ -357,13 +441,16 @@ __global__ void __launch_bounds__(32)
         for (int j = 0; j < count && j < STAGES; ++j)
             issue(j);
     }
-    stage_ws16(w, ws);
+    stage_weights(w, wd);
+    stage_slopes(k, wd);
     __syncwarp();
 
-    float acc[6 * kHalfC];
+    float2 acc2[3][kHalfC];
 #pragma unroll
-    for (int q = 0; q < 6 * kHalfC; ++q)
-        acc[q] = 0.0f;
+    for (int ip = 0; ip < 3; ++ip)
+#pragma unroll
+        for (int cc = 0; cc < kHalfC; ++cc)
+            acc2[ip][cc] = make_float2(0.0f, 0.0f);
 
     int j = 0;
     for (; j < count; ++j) {
@@ -383,26 +470,30 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const float4 q = *reinterpret_cast<const float4 *>(tu + c * kTileTokens + 4 * lane);
-                float wc[6];
-                weights_of(ws, c, wc);
+                float2 wp[6];
+                wpairs_of(wd, c, wp);
 #pragma unroll
                 for (int i = 0; i < 6; ++i) {
-                    const float2 wi = make_float2(wc[i], wc[i]);
-                    z[i][0] = __ffma2_rn(wi, make_float2(q.x, q.y), z[i][0]);
-                    z[i][1] = __ffma2_rn(wi, make_float2(q.z, q.w), z[i][1]);
+                    z[i][0] = __ffma2_rn(wp[i], make_float2(q.x, q.y), z[i][0]);
+                    z[i][1] = __ffma2_rn(wp[i], make_float2(q.z, q.w), z[i][1]);
                 }
             }
-            // t_i = g_i * slope_i(z_i), kept in registers and written over g.
-            float t[6][4];
+            // t_i = g_i * slope_i(z_i).
+            float2 t2[6][2];
 #pragma unroll
             for (int i = 0; i < 6; ++i) {
-                float4 *gp = reinterpret_cast<float4 *>(tg + i * kTileTokens + 4 * lane);
-                const float4 gq = *gp;
-                const float zz[4] = {z[i][0].x, z[i][0].y, z[i][1].x, z[i][1].y}, gg[4] = {gq.x, gq.y, gq.z, gq.w};
+                const float4 gq = *reinterpret_cast<const float4 *>(tg + i * kTileTokens + 4 * lane);
+                const float4 kq = kd[i];
+                const float2 shift = make_float2(kq.x, kq.y), scale4 = make_float2(kq.z, kq.w);
+                t2[i][0] = ste_grad2(z[i][0], make_float2(gq.x, gq.y), shift, scale4);
+                t2[i][1] = ste_grad2(z[i][1], make_float2(gq.z, gq.w), shift, scale4);
+            }
+            __syncwarp(); // every lane has read its g: the tile may now hold t
 #pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    t[i][m] = gg[m] * (k.scale[i] * sech2(zz[m] + k.shift[i]));
-                *gp = make_float4(t[i][0], t[i][1], t[i][2], t[i][3]);
+            for (int ip = 0; ip < 3; ++ip) {
+                float4 *dst = reinterpret_cast<float4 *>(tg + (ip * kTileTokens + 4 * lane) * 2);
+                dst[0] = make_float4(t2[2 * ip][0].x, t2[2 * ip + 1][0].x, t2[2 * ip][0].y, t2[2 * ip + 1][0].y);
+                dst[1] = make_float4(t2[2 * ip][1].x, t2[2 * ip + 1][1].x, t2[2 * ip][1].y, t2[2 * ip + 1][1].y);
             }
             // grad_u = sum_i w[i][c] t_i, the chain over i from 0, for the lane's tokens.
             const int64_t t0 = (int64_t)tx * kTileTokens + 4 * lane;
@@ -410,42 +501,43 @@ __global__ void __launch_bounds__(32)
                 float *gub = gu + (int64_t)b * 16 * S + t0;
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    float wc[6];
-                    weights_of(ws, c, wc);
-                    float o[4];
+                    float2 wp[6];
+                    wpairs_of(wd, c, wp);
+                    float2 o0 = make_float2(0.0f, 0.0f), o1 = o0;
 #pragma unroll
-                    for (int m = 0; m < 4; ++m) {
-                        float a = 0.0f;
-#pragma unroll
-                        for (int i = 0; i < 6; ++i)
-                            a = fmaf(wc[i], t[i][m], a);
-                        o[m] = a;
+                    for (int i = 0; i < 6; ++i) {
+                        o0 = __ffma2_rn(wp[i], t2[i][0], o0);
+                        o1 = __ffma2_rn(wp[i], t2[i][1], o1);
                     }
-                    *reinterpret_cast<float4 *>(gub) = make_float4(o[0], o[1], o[2], o[3]);
+                    *reinterpret_cast<float4 *>(gub) = make_float4(o0.x, o0.y, o1.x, o1.y);
                     gub += S;
                 }
             }
         }
         __syncwarp(); // t of the partner lane is in shared memory
-        // grad_w: the pair's 8 tokens, channels 8h .. 8h + 7, tokens in increasing order.
+        // grad_w: the pair's 8 tokens in increasing order, channels 8h .. 8h + 7.
 #pragma unroll
         for (int g2 = 0; g2 < 2; ++g2) {
             const int col = 4 * ((lane & ~1) + g2);
-            float t[6][4];
+            float2 tp[3][4];
 #pragma unroll
-            for (int i = 0; i < 6; ++i) {
-                const float4 tq = *reinterpret_cast<const float4 *>(tg + i * kTileTokens + col);
-                t[i][0] = tq.x, t[i][1] = tq.y, t[i][2] = tq.z, t[i][3] = tq.w;
+            for (int ip = 0; ip < 3; ++ip) {
+                const float4 *src = reinterpret_cast<const float4 *>(tg + (ip * kTileTokens + col) * 2);
+                const float4 a = src[0], e = src[1];
+                tp[ip][0] = make_float2(a.x, a.y), tp[ip][1] = make_float2(a.z, a.w);
+                tp[ip][2] = make_float2(e.x, e.y), tp[ip][3] = make_float2(e.z, e.w);
             }
 #pragma unroll
             for (int cc = 0; cc < kHalfC; ++cc) {
                 const float4 q = *reinterpret_cast<const float4 *>(tu + (kHalfC * h + cc) * kTileTokens + col);
                 const float uq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                for (int i = 0; i < 6; ++i)
+                for (int m = 0; m < 4; ++m) {
+                    const float2 ub = make_float2(uq[m], uq[m]);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        acc[i * kHalfC + cc] = fmaf(t[i][m], uq[m], acc[i * kHalfC + cc]);
+                    for (int ip = 0; ip < 3; ++ip)
+                        acc2[ip][cc] = __ffma2_rn(tp[ip][m], ub, acc2[ip][cc]);
+                }
             }
         }
         __syncwarp(); // every lane has read this stage
@@ -456,7 +548,7 @@ __global__ void __launch_bounds__(32)
     }
     if (j < count)
         ring_drain<STAGES>(bars, j, count);
-    warp_row_half(acc, partial + (int64_t)blockIdx.x * 6 * kMaxC);
+    warp_row_half(acc2, partial);
 }
 
 // Decode backward, C = 16.  Stage layout: g tile [16][128] (fp32) then the 128 indices.
@@ -469,7 +561,7 @@ __global__ void __launch_bounds__(32)
     constexpr int G_BYTES = 16 * kTileTokens * 4, STAGE = G_BYTES + kTileTokens * 4;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + STAGES * STAGE);
-    float *ws = reinterpret_cast<float *>(smem_raw + STAGES * STAGE + 16 * STAGES); // 16-byte aligned
+    float *wd = reinterpret_cast<float *>(smem_raw + STAGES * STAGE + 16 * STAGES); // 16-byte aligned
     const int lane = threadIdx.x, h = lane & 1;
     const uint32_t first = blockIdx.x * (uint32_t)TPR;
     const int count = (int)min((uint32_t)TPR, ntiles - first);
@@ -488,13 +580,15 @@ __global__ void __launch_bounds__(32)
         for (int j = 0; j < count && j < STAGES; ++j)
             issue(j);
     }
-    stage_ws16(w, ws);
+    stage_weights(w, wd);
     __syncwarp();
 
-    float acc[6 * kHalfC];
+    float2 acc2[3][kHalfC];
 #pragma unroll
-    for (int q = 0; q < 6 * kHalfC; ++q)
-        acc[q] = 0.0f;
+    for (int ip = 0; ip < 3; ++ip)
+#pragma unroll
+        for (int cc = 0; cc < kHalfC; ++cc)
+            acc2[ip][cc] = make_float2(0.0f, 0.0f);
 
     int j = 0;
     for (; j < count; ++j) {
@@ -509,54 +603,51 @@ __global__ void __launch_bounds__(32)
         const int64_t t0 = (int64_t)tx * kTileTokens + 4 * lane;
         if (t0 < S) {
             const int4 iq = *reinterpret_cast<const int4 *>(tid + 4 * lane);
-            const bool valid[4] = {(uint32_t)iq.x < (uint32_t)TOK_FSQ_CODEBOOK,
-                                   (uint32_t)iq.y < (uint32_t)TOK_FSQ_CODEBOOK,
-                                   (uint32_t)iq.z < (uint32_t)TOK_FSQ_CODEBOOK,
-                                   (uint32_t)iq.w < (uint32_t)TOK_FSQ_CODEBOOK};
-            float gc[6][4];
+            const bool v0 = (uint32_t)iq.x < (uint32_t)TOK_FSQ_CODEBOOK, v1 = (uint32_t)iq.y < (uint32_t)TOK_FSQ_CODEBOOK;
+            const bool v2 = (uint32_t)iq.z < (uint32_t)TOK_FSQ_CODEBOOK, v3 = (uint32_t)iq.w < (uint32_t)TOK_FSQ_CODEBOOK;
+            float2 gc2[6][2];
 #pragma unroll
             for (int i = 0; i < 6; ++i)
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    gc[i][m] = 0.0f;
+                gc2[i][0] = gc2[i][1] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const float4 q = *reinterpret_cast<const float4 *>(tgl + c * kTileTokens + 4 * lane);
-                const float gq[4] = {q.x, q.y, q.z, q.w};
-                float wc[6];
-                weights_of(ws, c, wc);
+                float2 wp[6];
+                wpairs_of(wd, c, wp);
 #pragma unroll
-                for (int i = 0; i < 6; ++i)
-#pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        gc[i][m] = fmaf(wc[i], gq[m], gc[i][m]);
+                for (int i = 0; i < 6; ++i) {
+                    gc2[i][0] = __ffma2_rn(wp[i], make_float2(q.x, q.y), gc2[i][0]);
+                    gc2[i][1] = __ffma2_rn(wp[i], make_float2(q.z, q.w), gc2[i][1]);
+                }
             }
             float *gcb = gcodes + (int64_t)b * 6 * S + t0;
 #pragma unroll
             for (int i = 0; i < 6; ++i)
                 *reinterpret_cast<float4 *>(gcb + (int64_t)i * S) =
-                    make_float4(valid[0] ? gc[i][0] : 0.0f, valid[1] ? gc[i][1] : 0.0f, valid[2] ? gc[i][2] : 0.0f,
-                                valid[3] ? gc[i][3] : 0.0f);
+                    make_float4(v0 ? gc2[i][0].x : 0.0f, v1 ? gc2[i][0].y : 0.0f, v2 ? gc2[i][1].x : 0.0f,
+                                v3 ? gc2[i][1].y : 0.0f);
         }
-        // grad_w: the pair's 8 tokens, channels 8h .. 8h + 7, tokens in increasing order.
+        // grad_w: the pair's 8 tokens in increasing order, channels 8h .. 8h + 7.
 #pragma unroll
         for (int g2 = 0; g2 < 2; ++g2) {
             const int col = 4 * ((lane & ~1) + g2);
             const int4 iq = *reinterpret_cast<const int4 *>(tid + col);
-            const int32_t ids[4] = {iq.x, iq.y, iq.z, iq.w};
-            float zh[4][6];
-#pragma unroll
-            for (int m = 0; m < 4; ++m)
-                zhat_of(ids[m], zh[m]);
+            float2 zp[4][3];
+            zhat_pairs(iq.x, zp[0]);
+            zhat_pairs(iq.y, zp[1]);
+            zhat_pairs(iq.z, zp[2]);
+            zhat_pairs(iq.w, zp[3]);
 #pragma unroll
             for (int cc = 0; cc < kHalfC; ++cc) {
                 const float4 q = *reinterpret_cast<const float4 *>(tgl + (kHalfC * h + cc) * kTileTokens + col);
                 const float gq[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-                for (int i = 0; i < 6; ++i)
+                for (int m = 0; m < 4; ++m) {
+                    const float2 gb = make_float2(gq[m], gq[m]);
 #pragma unroll
-                    for (int m = 0; m < 4; ++m)
-                        acc[i * kHalfC + cc] = fmaf(zh[m][i], gq[m], acc[i * kHalfC + cc]);
+                    for (int ip = 0; ip < 3; ++ip)
+                        acc2[ip][cc] = __ffma2_rn(zp[m][ip], gb, acc2[ip][cc]);
+                }
             }
         }
         __syncwarp(); // every lane has read this stage
@@ -567,19 +658,19 @@ __global__ void __launch_bounds__(32)
     }
     if (j < count)
         ring_drain<STAGES>(bars, j, count);
-    warp_row_half(acc, partial + (int64_t)blockIdx.x * 6 * kMaxC);
+    warp_row_half(acc2, partial);
 }
 
 // Shared memory: the stages (multiples of 128 bytes), one 16-byte slot per stage for
-// its barrier, then the weights.
-template <int STAGES> constexpr int enc_smem() { return STAGES * (22 * kTileTokens * 4 + 16) + 16 * 8 * 4; }
-template <int STAGES> constexpr int dec_smem() { return STAGES * (17 * kTileTokens * 4 + 16) + 16 * 8 * 4; }
+// its barrier, then the tables.
+template <int STAGES> constexpr int enc_smem() { return STAGES * (22 * kTileTokens * 4 + 16) + kTableBytes; }
+template <int STAGES> constexpr int dec_smem() { return STAGES * (17 * kTileTokens * 4 + 16) + kTableBytes; }
 
 // Tiles of the main path: B * ceil(S / 128).
 int64_t tma_tiles(int64_t B, int64_t S) { return B * ((S + kTileTokens - 1) / kTileTokens); }
 
-// The main path takes C = 16 with S % 4 == 0 (16-byte rows for TMA and for the
-// lanes' 16-byte stores) and 16-byte-aligned tensors.
+// The main path takes C = 16 with S % 4 == 0 (TMA needs rows of a multiple of 16
+// bytes) and 16-byte-aligned tensors.
 bool bwd_tma_eligible(int64_t B, int64_t C, int64_t S, const void *a, const void *b, const void *c)
 {
     return C == 16 && S % 4 == 0 && S < ((int64_t)1 << 31) && B < ((int64_t)1 << 31) &&
@@ -709,7 +800,11 @@ tok_status encode_bwd_run(const float *u, const float *w, const float *g, float 
     if (!done && rows > 0)
         fsq_encode_bwd_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(u, w, g, gu, partial, B, (int)C, S,
                                                                        slope_consts());
-    fsq_bwd_sum_rows_kernel<<<(unsigned)(6 * C), kSumThreads, 0, stream>>>(partial, rows, (int)(6 * C), gw);
+    const cudaError_t e = launch_sum_rows(partial, rows, (int)(6 * C), gw, stream);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -728,7 +823,11 @@ tok_status decode_bwd_run(const int32_t *idx, const float *w, const float *g, fl
     }
     if (!done && rows > 0)
         fsq_decode_bwd_kernel<<<(unsigned)rows, kThreads, 0, stream>>>(idx, w, g, gc, partial, B, (int)C, S);
-    fsq_bwd_sum_rows_kernel<<<(unsigned)(6 * C), kSumThreads, 0, stream>>>(partial, rows, (int)(6 * C), gw);
+    const cudaError_t e = launch_sum_rows(partial, rows, (int)(6 * C), gw, stream);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
     return launch_status();
 }
 

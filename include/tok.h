@@ -214,8 +214,9 @@ TOK_API tok_status tok_fsq_decode(const int32_t *idx, const float *w, float *out
  * with the constants of tok_fsq_encode.  The weight gradient is a sum over all
  * tokens; it is reduced deterministically (a fixed partition of the tokens and a
  * fixed summation order, independent of the device) through a caller-provided
- * workspace of tok_fsq_backward_workspace_size() bytes, device memory that the
- * call overwrites.  grad_w is overwritten, not accumulated.  1 <= C <= 16.
+ * workspace of tok_fsq_backward_workspace_size() bytes, 4-byte-aligned device
+ * memory that the call overwrites (nothing in it needs to be initialized).
+ * grad_w is overwritten, not accumulated.  1 <= C <= 16.
  */
 
 /* Workspace bytes for a backward call on [B, C, S]; -1 for an invalid shape. */
@@ -271,6 +272,7 @@ TOK_API tok_status tok_fsq_encode_backward_noalloc(const float *u, const float *
  *   grad_out   : [B, C, S] fp32, gradient of the decoded latent (input)
  *   grad_codes : [B, 6, S] fp32, sum_c w[i][c] * grad_out[c]; 0 for invalid indices (output)
  *   grad_w     : [6, C] fp32, sum over tokens of zhat_i * grad_out[c] (output)
+ * Errors: as tok_fsq_encode_backward.
  */
 TOK_API tok_status tok_fsq_decode_backward(const int32_t *idx, const float *w, const float *grad_out,
                                            float *grad_codes, float *grad_w, void *workspace,

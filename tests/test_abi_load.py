@@ -104,7 +104,7 @@ def test_backward_argument_rules(lib):
         return max((B * S + 2047) // 2048, (B * ((S + 127) // 128) + 7) // 8)
     assert ws(64, 16, 56320) == rows(64, 56320) * 96 * 4 == 3520 * 384
     assert ws(3, 16, 1000) == rows(3, 1000) * 96 * 4 == 3 * 384
-    assert ws(1, 5, 4097) == rows(1, 4097) * 30 * 4
+    assert ws(1, 5, 4097) == rows(1, 4097) * 30 * 4 == 5 * 120
     assert ws(1, 17, 8) == -1 and ws(1, 0, 8) == -1 and ws(-1, 16, 8) == -1
     assert ws(0, 16, 8) == 0
     eb, db = lib.tok_fsq_encode_backward, lib.tok_fsq_decode_backward
@@ -115,6 +115,8 @@ def test_backward_argument_rules(lib):
     assert eb(U, Wt, G, NULL, GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_NULL
     assert eb(U, Wt, G, F(0x100000 + 64), GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS  # grad_u in u
     assert eb(U, Wt, G, GU, GW, F(0x400000 + 8), need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS   # workspace in grad_u
+    assert eb(U, Wt, G, GU, GW, F(0x600000 + 2), need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIGN
+    assert db(U, Wt, G, GU, GW, F(0x600000 + 2), need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIGN
     assert db(U, Wt, G, GU, GW, WS, need - 4, 1, 16, 128, NULL) == hwp.TOK_ERR_SHAPE
     assert db(U, Wt, G, F(0x300000 + 4), GW, WS, need, 1, 16, 128, NULL) == hwp.TOK_ERR_ALIAS
     nb = lib.tok_fsq_encode_backward_noalloc

@@ -94,8 +94,9 @@ def test_image_adjoints_are_the_other_direction():
 
 # C = 16 with S % 4 == 0 takes the TMA kernels (ragged last tile at S = 1000, a single
 # mostly empty tile at S = 4, workspace rows spanning batch rows at B = 3); S = 1001 and
-# C = 5 take the register kernels.
-CASES = [(2, 16, 4096), (3, 16, 1000), (1, 16, 4), (2, 16, 1001), (1, 5, 777), (16, 16, 56320)]
+# C = 4, 5 take the register kernels.  6C % 8 == 0 (C = 4, 16) sums the rows in groups of
+# 8 entries, C = 5 entry by entry.
+CASES = [(2, 16, 4096), (3, 16, 1000), (1, 16, 4), (2, 16, 1001), (2, 4, 1000), (1, 5, 777), (16, 16, 56320)]
 
 
 @pytest.mark.parametrize("B,C,S", CASES)
@@ -129,6 +130,40 @@ def test_fsq_decode_backward_matches_oracle(B, C, S):
     assert (np.abs(got_c - ref_c) <= tol_c).all()
     tol_w = 1e-5 * g64.sum(axis=(0, 2))[None, :] + 1e-30
     assert (np.abs(got_w - ref_w) <= tol_w).all()
+
+
+def misaligned(a):
+    """A contiguous device copy of `a` whose address is 4 bytes past a 16-byte boundary, so the
+    library takes its register kernels instead of the TMA kernels."""
+    t = torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    buf = torch.empty(t.numel() + 4, dtype=t.dtype, device="cuda")
+    out = buf[1:1 + t.numel()].view(t.shape)
+    out.copy_(t)
+    assert out.data_ptr() % 16 != 0
+    return out
+
+
+def test_fsq_backward_paths_agree_bit_for_bit():
+    """The TMA kernels and the register kernels round the same fp32 operations in the same
+    order per token, so grad_u and grad_codes agree bit for bit; grad_w differs only in the
+    partition of its sums."""
+    B, C, S = 2, 16, 4096
+    u = synth.normal((B, C, S), seed=71, std=1.4)
+    w = synth.fsq_weight(C)
+    g = synth.normal((B, 6, S), seed=73)
+    gu_a, gw_a = hwp.fsq_encode_backward(dev(u), dev(w), dev(g))
+    gu_b, gw_b = hwp.fsq_encode_backward(misaligned(u), dev(w), misaligned(g))
+    assert torch.equal(gu_a, gu_b)
+    gs = np.abs(g.astype(np.float64)) * SCALE[None, :, None]
+    tol_w = 2e-5 * np.einsum("bis,bcs->ic", gs, np.abs(u.astype(np.float64)))  # each side within 1e-5
+    assert (np.abs(gw_a.double().cpu().numpy() - gw_b.double().cpu().numpy()) <= tol_w).all()
+    idx = synth.uniform((B, S), seed=79, lo=0, hi=64000, dtype=synth.F64).astype(np.int32)
+    go = synth.normal((B, C, S), seed=83)
+    gc_a, gw_a = hwp.fsq_decode_backward(dev(idx), dev(w), dev(go))
+    gc_b, gw_b = hwp.fsq_decode_backward(misaligned(idx), dev(w), misaligned(go))
+    assert torch.equal(gc_a, gc_b)
+    tol_w = 2e-5 * np.abs(go.astype(np.float64)).sum(axis=(0, 2))[None, :]
+    assert (np.abs(gw_a.double().cpu().numpy() - gw_b.double().cpu().numpy()) <= tol_w).all()
 
 
 def test_fsq_backward_is_deterministic():
