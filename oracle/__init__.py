@@ -37,6 +37,19 @@ def _load():
             f = getattr(lib, name)
             f.restype = ctypes.c_int
             f.argtypes = [dp, dp, i64, i64, i64, i64, i64]
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        lib.oracle_haar_padded_extents.restype = ctypes.c_int
+        lib.oracle_haar_padded_extents.argtypes = [i64, i64, i64, i64, i64, i64p, i64p, i64p]
+        lib.oracle_haar_pad.restype = ctypes.c_int
+        lib.oracle_haar_pad.argtypes = [dp, dp, i64, i64, i64, i64, i64, i64, i64, i64]
+        for name in ("oracle_haar_fwd_padded", "oracle_haar_inv_cropped"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [dp, dp, i64, i64, i64, i64, i64, i64, i64]
+        for name in ("oracle_haar_fwd_chunk", "oracle_haar_inv_chunk"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [dp, dp, i64, i64, i64, i64, i64, ctypes.c_int]
         lib.oracle_haar_level_fwd.restype = ctypes.c_int
         lib.oracle_haar_level_fwd.argtypes = [dp, dp, i64, i64, i64, i64]
         lib.oracle_haar_out_frames.restype = i64
@@ -247,3 +260,75 @@ def fsq_decode_backward(idx: np.ndarray, w: np.ndarray, g: np.ndarray):
     _load().oracle_fsq_decode_backward(_ptr(idx, ctypes.c_int32), _ptr(w, ctypes.c_float), _ptr(g, ctypes.c_float),
                                        B, C, S, _ptr(gc, ctypes.c_double), _ptr(gw, ctypes.c_double))
     return gc, gw
+
+
+def padded_extents(T: int, H: int, W: int, ms: int = 4, mt: int = 4):
+    """(Tp, Hp, Wp): zeros to multiples of ms in space, reflection to Tp = 1 (mod mt) in time."""
+    Tp, Hp, Wp = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    if not _load().oracle_haar_padded_extents(T, H, W, ms, mt, ctypes.byref(Tp), ctypes.byref(Hp), ctypes.byref(Wp)):
+        raise ValueError("padded_extents: invalid multiples or shape")
+    return Tp.value, Hp.value, Wp.value
+
+
+def haar_pad(x: np.ndarray, ms: int = 4, mt: int = 4) -> np.ndarray:
+    """The padded clip [B, C, Tp, Hp, Wp] the padded patcher transforms."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, C, T, H, W = x.shape
+    Tp, Hp, Wp = padded_extents(T, H, W, ms, mt)
+    xp = np.zeros((B, C, Tp, Hp, Wp))
+    _check(_load().oracle_haar_pad(_ptr(x, ctypes.c_double), _ptr(xp, ctypes.c_double), B, C, T, H, W, Tp, Hp, Wp),
+           "haar_pad")
+    return xp
+
+
+def haar_fwd_padded(x: np.ndarray, ms: int = 4, mt: int = 4) -> np.ndarray:
+    """Patcher on a clip of any extents: pad (zeros in space, reflection in time), then transform."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, C, T, H, W = x.shape
+    Tp, Hp, Wp = padded_extents(T, H, W, ms, mt)
+    y = np.zeros(haar_out_shape(B, C, Tp, Hp, Wp))
+    _check(_load().oracle_haar_fwd_padded(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double), B, C, T, H, W, ms, mt),
+           "haar_fwd_padded")
+    return y
+
+
+def haar_inv_cropped(y: np.ndarray, T: int, H: int, W: int, ms: int = 4, mt: int = 4) -> np.ndarray:
+    """Unpatcher on the padded extents, cropped to [B, C, T, H, W]."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    Tp, Hp, Wp = padded_extents(T, H, W, ms, mt)
+    B = y.shape[0]
+    C = y.shape[1] // (16 if Tp == 1 else 64)
+    if y.shape != haar_out_shape(B, C, Tp, Hp, Wp):
+        raise ValueError("haar_inv_cropped: coefficient shape does not match the padded extents")
+    x = np.zeros((B, C, T, H, W))
+    _check(_load().oracle_haar_inv_cropped(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), B, C, T, H, W, ms, mt),
+           "haar_inv_cropped")
+    return x
+
+
+def chunk_out_shape(B, C, T, H, W, first):
+    """Streaming chunks are always video: 64C channels, (T + 3) // 4 latent frames (first) or T // 4."""
+    return (B, 64 * C, (T + 3) // 4 if first else T // 4, H // 4, W // 4)
+
+
+def haar_fwd_chunk(x: np.ndarray, first: bool) -> np.ndarray:
+    """Streaming chunk of a video: first -> T = 1 + 4k frames with the frame-0 replicas (3D even
+    for one frame); else 4k frames, no replica."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    B, C, T, H, W = x.shape
+    y = np.zeros(chunk_out_shape(B, C, T, H, W, first))
+    _check(_load().oracle_haar_fwd_chunk(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double), B, C, T, H, W,
+                                         int(bool(first))), "haar_fwd_chunk")
+    return y
+
+
+def haar_inv_chunk(y: np.ndarray, T: int, H: int, W: int, first: bool) -> np.ndarray:
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    B = y.shape[0]
+    C = y.shape[1] // 64
+    if y.shape != chunk_out_shape(B, C, T, H, W, first):
+        raise ValueError("haar_inv_chunk: shape mismatch")
+    x = np.zeros((B, C, T, H, W))
+    _check(_load().oracle_haar_inv_chunk(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), B, C, T, H, W,
+                                         int(bool(first))), "haar_inv_chunk")
+    return x

@@ -474,3 +474,241 @@ int oracle_haar_fwd_blockform(const double *x, double *y, int64_t B, int64_t C, 
                                 }
     return ORACLE_OK;
 }
+
+/*
+ * Arbitrary extents and streaming time ("NVIDIA Cosmos Tokenizer 完全指南",
+ * section 6.3: videos of any size are padded -- zeros in space, reflection at the
+ * temporal edge -- to aligned extents before the network, and the result is
+ * cropped back afterwards; long videos run window by window).
+ *
+ * Readings where the pages are silent (parity unpinned by the pages for the
+ * choice of multiples and of the reflection form; these are conventions shared
+ * with the CUDA path):
+ *   - spatial padding appends zero rows at the bottom and zero columns at the
+ *     right up to multiples of `ms` (a multiple of 4);
+ *   - temporal padding appends frames at the end, up to the smallest Tp >= T
+ *     with (Tp - 1) % mt == 0 (mt a multiple of 4), each a mirror image about
+ *     the last frame without repeating it (frame T-1+k is frame T-1-k), the
+ *     mirroring repeated with period 2(T-1) when more frames are needed than
+ *     the clip has; images (T == 1) get no temporal padding;
+ *   - the padded clip goes through the two-level patcher unchanged; the
+ *     unpatcher's output is cropped to the first T frames, H rows, W columns;
+ *   - a continuation chunk (streaming) is a run of 4k frames that follows
+ *     earlier frames: it is transformed level by level with no frame-0
+ *     replica (frames paired as they come), giving k latent frames; the first
+ *     chunk (1 + 4k frames, k >= 0) is the start of a video and always takes
+ *     the 3D levels, so a one-frame first chunk gives latent frame 0.
+ */
+
+/* Padded extents; returns 0 if the multiples or the shape are invalid. */
+int oracle_haar_padded_extents(int64_t T, int64_t H, int64_t W, int64_t ms, int64_t mt, int64_t *Tp, int64_t *Hp,
+                               int64_t *Wp)
+{
+    if (T < 1 || H < 0 || W < 0 || ms < 4 || ms % 4 != 0 || mt < 4 || mt % 4 != 0)
+        return 0;
+    *Hp = (H + ms - 1) / ms * ms;
+    *Wp = (W + ms - 1) / ms * ms;
+    *Tp = (T == 1) ? 1 : 1 + (T - 1 + mt - 1) / mt * mt;
+    return 1;
+}
+
+/* Source frame of padded frame t (mirror about the last frame, period 2(T-1)). */
+static int64_t reflect_frame(int64_t t, int64_t T)
+{
+    if (t < T)
+        return t;
+    if (T == 1)
+        return 0;
+    const int64_t period = 2 * (T - 1);
+    const int64_t r = t % period;
+    return r < T ? r : period - r;
+}
+
+/* x [B][C][T][H][W] -> xp [B][C][Tp][Hp][Wp]. */
+int oracle_haar_pad(const double *x, double *xp, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W, int64_t Tp,
+                    int64_t Hp, int64_t Wp)
+{
+    if (Tp < T || Hp < H || Wp < W)
+        return ORACLE_BAD_SHAPE;
+    for (int64_t bc = 0; bc < B * C; ++bc)
+        for (int64_t t = 0; t < Tp; ++t) {
+            const int64_t ts = reflect_frame(t, T);
+            for (int64_t y = 0; y < Hp; ++y)
+                for (int64_t xx = 0; xx < Wp; ++xx)
+                    xp[((bc * Tp + t) * Hp + y) * Wp + xx] =
+                        (y < H && xx < W) ? x[((bc * T + ts) * H + y) * W + xx] : 0.0;
+        }
+    return ORACLE_OK;
+}
+
+/* Padded patcher: pad, then the two-level patcher on [B][C][Tp][Hp][Wp]. */
+int oracle_haar_fwd_padded(const double *x, double *y, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W,
+                           int64_t ms, int64_t mt)
+{
+    int64_t Tp, Hp, Wp;
+    if (B < 0 || C < 0 || !oracle_haar_padded_extents(T, H, W, ms, mt, &Tp, &Hp, &Wp))
+        return ORACLE_BAD_SHAPE;
+    if (B * C * Tp * Hp * Wp == 0)
+        return ORACLE_OK;
+    double *xp = (double *)malloc((size_t)(B * C * Tp * Hp * Wp) * sizeof(double));
+    if (!xp)
+        return ORACLE_NO_MEMORY;
+    int rc = oracle_haar_pad(x, xp, B, C, T, H, W, Tp, Hp, Wp);
+    if (rc == ORACLE_OK)
+        rc = oracle_haar_fwd(xp, y, B, C, Tp, Hp, Wp);
+    free(xp);
+    return rc;
+}
+
+/* Cropped unpatcher: the two-level unpatcher on the padded extents, then the first
+ * T frames, H rows and W columns. */
+int oracle_haar_inv_cropped(const double *y, double *x, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W,
+                            int64_t ms, int64_t mt)
+{
+    int64_t Tp, Hp, Wp;
+    if (B < 0 || C < 0 || !oracle_haar_padded_extents(T, H, W, ms, mt, &Tp, &Hp, &Wp))
+        return ORACLE_BAD_SHAPE;
+    if (B * C * Tp * Hp * Wp == 0)
+        return ORACLE_OK;
+    double *xp = (double *)malloc((size_t)(B * C * Tp * Hp * Wp) * sizeof(double));
+    if (!xp)
+        return ORACLE_NO_MEMORY;
+    const int rc = oracle_haar_inv(y, xp, B, C, Tp, Hp, Wp);
+    if (rc == ORACLE_OK)
+        for (int64_t bc = 0; bc < B * C; ++bc)
+            for (int64_t t = 0; t < T; ++t)
+                for (int64_t yy = 0; yy < H; ++yy)
+                    for (int64_t xx = 0; xx < W; ++xx)
+                        x[((bc * T + t) * H + yy) * W + xx] = xp[((bc * Tp + t) * Hp + yy) * Wp + xx];
+    free(xp);
+    return rc;
+}
+
+/*
+ * One level of the 3D DWT without the frame-0 replica (continuation chunks):
+ * v[C][T][H][W] -> o[8C][T/2][H/2][W/2], T even; frames 2j and 2j+1 form pair j.
+ * Same butterflies and subband order as level3d_fwd.
+ */
+static void level3d_fwd_norep(const double *v, double *o, int64_t C, int64_t T, int64_t H, int64_t W)
+{
+    const int64_t To = T / 2, Ho = H / 2, Wo = W / 2;
+    for (int64_t c = 0; c < C; ++c)
+        for (int64_t j = 0; j < To; ++j)
+            for (int64_t i = 0; i < Ho; ++i)
+                for (int64_t k = 0; k < Wo; ++k) {
+                    double g[2][2][2];
+                    for (int dt = 0; dt < 2; ++dt)
+                        for (int dy = 0; dy < 2; ++dy)
+                            for (int dx = 0; dx < 2; ++dx)
+                                g[dt][dy][dx] = v[((c * T + 2 * j + dt) * H + (2 * i + dy)) * W + (2 * k + dx)];
+                    for (int dy = 0; dy < 2; ++dy)
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_pair(g[0][dy][dx], g[1][dy][dx], &g[0][dy][dx], &g[1][dy][dx]);
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_pair(g[bt][0][dx], g[bt][1][dx], &g[bt][0][dx], &g[bt][1][dx]);
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            haar_pair(g[bt][by][0], g[bt][by][1], &g[bt][by][0], &g[bt][by][1]);
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            for (int bx = 0; bx < 2; ++bx)
+                                o[((((4 * bt + 2 * by + bx) * C + c) * To + j) * Ho + i) * Wo + k] = g[bt][by][bx];
+                }
+}
+
+/* Inverse of level3d_fwd_norep: o[8C][To][Ho][Wo] -> v[C][2To][2Ho][2Wo], no frame dropped. */
+static void level3d_inv_norep(const double *o, double *v, int64_t C, int64_t To, int64_t Ho, int64_t Wo)
+{
+    const int64_t T = 2 * To, H = 2 * Ho, W = 2 * Wo;
+    for (int64_t c = 0; c < C; ++c)
+        for (int64_t j = 0; j < To; ++j)
+            for (int64_t i = 0; i < Ho; ++i)
+                for (int64_t k = 0; k < Wo; ++k) {
+                    double g[2][2][2];
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            for (int bx = 0; bx < 2; ++bx)
+                                g[bt][by][bx] = o[((((4 * bt + 2 * by + bx) * C + c) * To + j) * Ho + i) * Wo + k];
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int by = 0; by < 2; ++by)
+                            haar_unpair(g[bt][by][0], g[bt][by][1], &g[bt][by][0], &g[bt][by][1]);
+                    for (int bt = 0; bt < 2; ++bt)
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_unpair(g[bt][0][dx], g[bt][1][dx], &g[bt][0][dx], &g[bt][1][dx]);
+                    for (int dy = 0; dy < 2; ++dy)
+                        for (int dx = 0; dx < 2; ++dx)
+                            haar_unpair(g[0][dy][dx], g[1][dy][dx], &g[0][dy][dx], &g[1][dy][dx]);
+                    for (int dt = 0; dt < 2; ++dt)
+                        for (int dy = 0; dy < 2; ++dy)
+                            for (int dx = 0; dx < 2; ++dx)
+                                v[((c * T + 2 * j + dt) * H + (2 * i + dy)) * W + (2 * k + dx)] = g[dt][dy][dx];
+                }
+}
+
+/*
+ * Streaming chunk of a video: first != 0 is the start of the video, T = 1 + 4k
+ * frames (k >= 0), transformed by the two 3D levels with their frame-0 replicas
+ * (a one-frame first chunk gives the video's latent frame 0, not the image
+ * transform); first == 0 is a continuation chunk of T = 4k frames (k >= 1),
+ * transformed by two levels without replicas.  Output [B][64C][(T+3)/4 or T/4][H/4][W/4].
+ */
+static int chunk_shape_ok(int64_t B, int64_t C, int64_t T, int64_t H, int64_t W, int first)
+{
+    if (B < 0 || C < 0 || H < 0 || W < 0 || H % 4 != 0 || W % 4 != 0)
+        return 0;
+    return first ? (T >= 1 && T % 4 == 1) : (T >= 4 && T % 4 == 0);
+}
+
+int oracle_haar_fwd_chunk(const double *x, double *y, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W,
+                          int first)
+{
+    if (!chunk_shape_ok(B, C, T, H, W, first))
+        return ORACLE_BAD_SHAPE;
+    const int64_t T1 = first ? (T + 1) / 2 : T / 2, Tq = first ? (T1 + 1) / 2 : T1 / 2;
+    const int64_t nx = C * T * H * W, n1 = 8 * C * T1 * (H / 2) * (W / 2);
+    const int64_t ny = 64 * C * Tq * (H / 4) * (W / 4);
+    if (nx == 0 || B == 0)
+        return ORACLE_OK;
+    double *mid = (double *)malloc((size_t)n1 * sizeof(double));
+    if (!mid)
+        return ORACLE_NO_MEMORY;
+    for (int64_t b = 0; b < B; ++b) {
+        if (first) {
+            level3d_fwd(x + b * nx, mid, C, T, H, W);
+            level3d_fwd(mid, y + b * ny, 8 * C, T1, H / 2, W / 2);
+        } else {
+            level3d_fwd_norep(x + b * nx, mid, C, T, H, W);
+            level3d_fwd_norep(mid, y + b * ny, 8 * C, T1, H / 2, W / 2);
+        }
+    }
+    free(mid);
+    return ORACLE_OK;
+}
+
+/* Inverse of oracle_haar_fwd_chunk (T, H, W: the chunk's pixel extents). */
+int oracle_haar_inv_chunk(const double *y, double *x, int64_t B, int64_t C, int64_t T, int64_t H, int64_t W,
+                          int first)
+{
+    if (!chunk_shape_ok(B, C, T, H, W, first))
+        return ORACLE_BAD_SHAPE;
+    const int64_t T1 = first ? (T + 1) / 2 : T / 2, Tq = first ? (T1 + 1) / 2 : T1 / 2;
+    const int64_t nx = C * T * H * W, n1 = 8 * C * T1 * (H / 2) * (W / 2);
+    const int64_t ny = 64 * C * Tq * (H / 4) * (W / 4);
+    if (nx == 0 || B == 0)
+        return ORACLE_OK;
+    double *mid = (double *)malloc((size_t)n1 * sizeof(double));
+    if (!mid)
+        return ORACLE_NO_MEMORY;
+    for (int64_t b = 0; b < B; ++b) {
+        if (first) {
+            level3d_inv(y + b * ny, mid, 8 * C, Tq, H / 4, W / 4);
+            level3d_inv(mid, x + b * nx, C, T1, H / 2, W / 2);
+        } else {
+            level3d_inv_norep(y + b * ny, mid, 8 * C, Tq, H / 4, W / 4);
+            level3d_inv_norep(mid, x + b * nx, C, T1, H / 2, W / 2);
+        }
+    }
+    free(mid);
+    return ORACLE_OK;
+}

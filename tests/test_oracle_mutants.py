@@ -39,6 +39,10 @@ MUTANTS = [
      "acc += (double)w[(c * FSQ_DIM + i) % (FSQ_DIM * C)] * gc;"),
     ("decode forgets the offset", "fsq.c", "zhat[i] = (double)(digits[i] - half_width) / (double)half_width;",
      "zhat[i] = (double)(digits[i]) / (double)half_width;"),
+    ("temporal padding repeats the edge frame", "haar.c", "return r < T ? r : period - r;",
+     "return r < T ? r : period - r + 1;"),
+    ("continuation chunk pairs frames in reverse", "haar.c", "(c * T + 2 * j + dt) * H",
+     "(c * T + 2 * j + 1 - dt) * H"),
 ]
 
 
@@ -58,6 +62,7 @@ def test_pins_catch_planted_mistake(tmp_path, name, fname, orig, mutated):
                     str(tmp_path / "haar.c"), str(tmp_path / "fsq.c"), "-lm"], check=True)
     env = dict(os.environ, ORACLE_SO=str(so))
     r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                        "tests/test_oracle_haar.py", "tests/test_oracle_fsq.py", "tests/test_oracle_backward.py"],
+                        "tests/test_oracle_haar.py", "tests/test_oracle_fsq.py", "tests/test_oracle_backward.py",
+                        "tests/test_oracle_padding.py"],
                        cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, f"pins did not catch the planted mistake '{name}'"
