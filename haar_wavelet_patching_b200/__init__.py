@@ -25,7 +25,8 @@ FSQ_DIM = 6
 # Every symbol include/tok.h declares.
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
-               "tok_haar_inv_windows", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
+               "tok_haar_inv_windows", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
+               "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
                "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
 _lib = None
@@ -70,6 +71,15 @@ def lib():
         for f in (L.tok_haar_fwd_windows, L.tok_haar_inv_windows):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, vp]
+        i64p = ctypes.POINTER(ctypes.c_int64)
+        L.tok_haar_padded_extents.restype = i32
+        L.tok_haar_padded_extents.argtypes = [i64, i64, i64, i64, i64, i64p, i64p, i64p]
+        for f in (L.tok_haar_fwd_padded, L.tok_haar_inv_cropped):
+            f.restype = i32
+            f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i64, i64, vp]
+        for f in (L.tok_haar_fwd_chunk, L.tok_haar_inv_chunk):
+            f.restype = i32
+            f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i32, vp]
         L.tok_fsq_encode.restype = i32
         L.tok_fsq_encode.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
         L.tok_fsq_decode.restype = i32
@@ -189,6 +199,77 @@ def tok_haar_fwd_windows(x: torch.Tensor, y: torch.Tensor, t_begin: int, t_end: 
 def tok_haar_inv_windows(y: torch.Tensor, x: torch.Tensor, t_begin: int, t_end: int, stream=None):
     """Inverse restricted to latent frames [t_begin, t_end): writes only those windows' pixel frames."""
     _haar_windows(False, x, y, t_begin, t_end, stream)
+    return x
+
+
+def padded_extents(T: int, H: int, W: int, spatial_multiple: int = 4, temporal_multiple: int = 4):
+    """(Tp, Hp, Wp) of tok_haar_fwd_padded: zeros in space, a mirrored tail in time."""
+    Tp, Hp, Wp = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    _check(lib().tok_haar_padded_extents(T, H, W, spatial_multiple, temporal_multiple, ctypes.byref(Tp),
+                                         ctypes.byref(Hp), ctypes.byref(Wp)), "tok_haar_padded_extents")
+    return Tp.value, Hp.value, Wp.value
+
+
+def padded_coeff_shape(B, C, T, H, W, spatial_multiple=4, temporal_multiple=4):
+    Tp, Hp, Wp = padded_extents(T, H, W, spatial_multiple, temporal_multiple)
+    return haar_coeff_shape(B, C, Tp, Hp, Wp)
+
+
+def tok_haar_fwd_padded(x: torch.Tensor, y: torch.Tensor, spatial_multiple: int = 4, temporal_multiple: int = 4,
+                        stream=None):
+    """x [B,C,T,H,W] of any extents -> y, the patcher of the padded clip (see padded_coeff_shape)."""
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != padded_coeff_shape(B, C, T, H, W, spatial_multiple, temporal_multiple):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected "
+                         f"{padded_coeff_shape(B, C, T, H, W, spatial_multiple, temporal_multiple)}")
+    _check(lib().tok_haar_fwd_padded(_ptr(x), _ptr(y), _dtype_code(x), B, C, T, H, W, spatial_multiple,
+                                     temporal_multiple, _stream(x, stream)), "tok_haar_fwd_padded")
+    return y
+
+
+def tok_haar_inv_cropped(y: torch.Tensor, x: torch.Tensor, spatial_multiple: int = 4, temporal_multiple: int = 4,
+                         stream=None):
+    """Coefficients of a padded clip -> x [B,C,T,H,W], the unpatcher cropped to x's extents."""
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != padded_coeff_shape(B, C, T, H, W, spatial_multiple, temporal_multiple):
+        raise ValueError("y does not have the padded coefficient shape of x")
+    _check(lib().tok_haar_inv_cropped(_ptr(y), _ptr(x), _dtype_code(x), B, C, T, H, W, spatial_multiple,
+                                      temporal_multiple, _stream(x, stream)), "tok_haar_inv_cropped")
+    return x
+
+
+def chunk_coeff_shape(B, C, T, H, W, first):
+    """Streaming chunks are video: 64C channels, (T + 3) // 4 latent frames (first) or T // 4."""
+    return (B, 64 * C, (T + 3) // 4 if first else T // 4, H // 4, W // 4)
+
+
+def _haar_chunk(fwd, x, y, first, stream):
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != chunk_coeff_shape(B, C, T, H, W, first):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {chunk_coeff_shape(B, C, T, H, W, first)}")
+    f = lib().tok_haar_fwd_chunk if fwd else lib().tok_haar_inv_chunk
+    src, dst = (x, y) if fwd else (y, x)
+    _check(f(_ptr(src), _ptr(dst), _dtype_code(x), B, C, T, H, W, int(bool(first)), _stream(x, stream)),
+           "tok_haar_fwd_chunk" if fwd else "tok_haar_inv_chunk")
+
+
+def tok_haar_fwd_chunk(x: torch.Tensor, y: torch.Tensor, first: bool, stream=None):
+    """A chunk of a video: first -> T = 1 + 4k frames with the frame-0 replicas; else 4k frames, none."""
+    _haar_chunk(True, x, y, first, stream)
+    return y
+
+
+def tok_haar_inv_chunk(y: torch.Tensor, x: torch.Tensor, first: bool, stream=None):
+    _haar_chunk(False, x, y, first, stream)
     return x
 
 
@@ -331,6 +412,30 @@ def fsq_encode(u: torch.Tensor, w: torch.Tensor, with_codes: bool = False, strea
 def fsq_decode(idx: torch.Tensor, w: torch.Tensor, bad_count: torch.Tensor = None, stream=None) -> torch.Tensor:
     out = torch.empty((idx.shape[0], w.shape[1]) + tuple(idx.shape[1:]), dtype=torch.float32, device=idx.device)
     return tok_fsq_decode(idx, w, out, bad_count, stream)
+
+
+def haar_fwd_padded(x: torch.Tensor, spatial_multiple: int = 4, temporal_multiple: int = 4,
+                    stream=None) -> torch.Tensor:
+    y = torch.empty(padded_coeff_shape(*x.shape, spatial_multiple, temporal_multiple), dtype=x.dtype, device=x.device)
+    return tok_haar_fwd_padded(x, y, spatial_multiple, temporal_multiple, stream)
+
+
+def haar_inv_cropped(y: torch.Tensor, T: int, H: int, W: int, spatial_multiple: int = 4, temporal_multiple: int = 4,
+                     stream=None) -> torch.Tensor:
+    B = y.shape[0]
+    C = y.shape[1] // (16 if T == 1 else 64)
+    x = torch.empty((B, C, T, H, W), dtype=y.dtype, device=y.device)
+    return tok_haar_inv_cropped(y, x, spatial_multiple, temporal_multiple, stream)
+
+
+def haar_fwd_chunk(x: torch.Tensor, first: bool, stream=None) -> torch.Tensor:
+    y = torch.empty(chunk_coeff_shape(*x.shape, first), dtype=x.dtype, device=x.device)
+    return tok_haar_fwd_chunk(x, y, first, stream)
+
+
+def haar_inv_chunk(y: torch.Tensor, T: int, H: int, W: int, first: bool, stream=None) -> torch.Tensor:
+    x = torch.empty((y.shape[0], y.shape[1] // 64, T, H, W), dtype=y.dtype, device=y.device)
+    return tok_haar_inv_chunk(y, x, first, stream)
 
 
 def haar_fwd_adjoint(gy: torch.Tensor, T: int, H: int, W: int, stream=None) -> torch.Tensor:

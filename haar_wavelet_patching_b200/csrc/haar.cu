@@ -434,7 +434,8 @@ tok_status haar_call(bool fwd, bool adj, const void *in, void *out, tok_dtype dt
     if (overlaps(in, bytes_in, out, bytes_out))
         return TOK_ERR_ALIAS;
 
-    const HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, g.tq0, g.nq};
+    HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, g.tq0, g.nq};
+    dims.video = T > 1;
     if (haar_tma_eligible(in, out, dt, dims))
         return haar_tma_launch(fwd, adj, in, out, dt, dims, stream);
 
@@ -455,6 +456,217 @@ tok_status haar_call(bool fwd, bool adj, const void *in, void *out, tok_dtype dt
         return vec ? launch2d<__nv_bfloat16, 4, true>(fwd, in, out, g, stream)
                    : launch2d<__nv_bfloat16, 1, false>(fwd, in, out, g, stream);
     return vec ? launch2d<float, 4, true>(fwd, in, out, g, stream) : launch2d<float, 1, false>(fwd, in, out, g, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Extended form, register path: padding / cropping and streaming chunks for the
+// shapes the TMA path cannot take (rows not a multiple of 16 bytes, unaligned
+// pointers).  One thread per block; element loads with bounds (zeros past the
+// pixel tensor's rows and columns, frames mirrored past its last frame) and
+// element stores with bounds (the inverse crops).  Same butterflies and order.
+// ---------------------------------------------------------------------------
+struct ExtGeometry {
+    int64_t BC, C;
+    int64_t T, H, W;  // pixel tensor
+    int64_t Tq, h, w; // latent tensor
+    int64_t fbase;    // first frame of window tq (not the replica window): 4*tq + fbase
+    int rep;          // window 0 is the frame-0 replica window
+};
+
+__device__ __forceinline__ int64_t mirror_frame_ext(int64_t f, int64_t T)
+{
+    if (f < T)
+        return f;
+    if (T == 1)
+        return 0;
+    const int64_t period = 2 * (T - 1), r = f % period;
+    return r < T ? r : period - r;
+}
+
+template <typename T> __device__ __forceinline__ float elem_to_f(T v);
+template <> __device__ __forceinline__ float elem_to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float elem_to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T f_to_elem(float v);
+template <> __device__ __forceinline__ float f_to_elem<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 f_to_elem<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+template <typename T, bool VIDEO, bool FWD>
+__global__ void __launch_bounds__(kThreads) haar_ext_kernel(const T *__restrict__ in, T *__restrict__ out, ExtGeometry g)
+{
+    constexpr int NA = VIDEO ? 4 : 1, G = VIDEO ? 64 : 16;
+    constexpr float SCALE = VIDEO ? 0.125f : 0.25f;
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.w)
+        return;
+    const int64_t i = item / g.w, j = item - i * g.w;
+    const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y; // (b, c, t')
+    if (pair >= g.BC * g.Tq)
+        return;
+    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t b = bc / g.C, c = bc - b * g.C;
+    const bool replica = VIDEO && g.rep && tq == 0;
+    const int64_t plane_lat = g.Tq * g.h * g.w, cstride = g.C * plane_lat;
+    const int64_t lat0 = (b * G * g.C + c) * plane_lat + (tq * g.h + i) * g.w + j;
+
+    float v[NA][4][4];
+    if constexpr (FWD) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            const int64_t f = !VIDEO ? 0 : replica ? 0 : mirror_frame_ext(4 * tq + g.fbase + a, g.T);
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int d = 0; d < 4; ++d) {
+                    const int64_t yy = 4 * i + r, xx = 4 * j + d;
+                    v[a][r][d] = (yy < g.H && xx < g.W) ? elem_to_f(in[((bc * g.T + f) * g.H + yy) * g.W + xx]) : 0.0f;
+                }
+        }
+    } else {
+#pragma unroll
+        for (int grp = 0; grp < G; ++grp) {
+            const float p = elem_to_f(in[lat0 + grp * cstride]);
+            if constexpr (VIDEO)
+                v[kt_of(grp)][ky_of(grp)][kx_of(grp)] = p;
+            else
+                v[0][ky2_of(grp)][kx2_of(grp)] = p;
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            haar4(v[a][r][0], v[a][r][1], v[a][r][2], v[a][r][3]);
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+            haar4(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
+    if constexpr (VIDEO) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                haar4(v[0][r][d], v[1][r][d], v[2][r][d], v[3][r][d]);
+    }
+    if constexpr (FWD) {
+#pragma unroll
+        for (int grp = 0; grp < G; ++grp) {
+            const float p = VIDEO ? v[kt_of(grp)][ky_of(grp)][kx_of(grp)] : v[0][ky2_of(grp)][kx2_of(grp)];
+            out[lat0 + grp * cstride] = f_to_elem<T>(p * SCALE);
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            if (replica && a != 3)
+                continue;
+            const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + g.fbase + a;
+            if (f >= g.T)
+                continue;
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+#pragma unroll
+                for (int d = 0; d < 4; ++d) {
+                    const int64_t yy = 4 * i + r, xx = 4 * j + d;
+                    if (yy < g.H && xx < g.W)
+                        out[((bc * g.T + f) * g.H + yy) * g.W + xx] = f_to_elem<T>(v[a][r][d] * SCALE);
+                }
+        }
+    }
+}
+
+template <typename T, bool VIDEO, bool FWD>
+tok_status launch_ext(const void *in, void *out, const ExtGeometry &g, cudaStream_t stream)
+{
+    const int64_t items = g.h * g.w, pairs = g.BC * g.Tq;
+    const int64_t gy = pairs < 65535 ? pairs : 65535, gz = (pairs + gy - 1) / gy;
+    if ((items + kThreads - 1) / kThreads > 0x7FFFFFFF || gz > 65535)
+        return TOK_ERR_SHAPE;
+    const dim3 grid((unsigned)((items + kThreads - 1) / kThreads), (unsigned)gy, (unsigned)gz);
+    haar_ext_kernel<T, VIDEO, FWD><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    return launch_status();
+}
+
+// Extended call: pixels [B, C, T, H, W] <-> coefficients [B, G*C, Tq, Hp/4, Wp/4] with
+// (Tp, Hp, Wp) the padded extents, windows as described for ExtGeometry.
+tok_status haar_ext_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                         int64_t H, int64_t W, int64_t Tp, int64_t Hp, int64_t Wp, int64_t fbase, int rep, bool video,
+                         cudaStream_t stream)
+{
+    if (dt != TOK_F32 && dt != TOK_BF16)
+        return TOK_ERR_DTYPE;
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    ExtGeometry g{};
+    g.C = C;
+    g.T = T;
+    g.H = H;
+    g.W = W;
+    g.Tq = !video ? 1 : rep ? 1 + (Tp - 1) / 4 : Tp / 4;
+    g.h = Hp / 4;
+    g.w = Wp / 4;
+    g.fbase = fbase;
+    g.rep = rep;
+    int64_t nx, ny, bytes_x, bytes_y;
+    if (!prod_ok({B, C}, &g.BC) || !prod_ok({g.BC, T, H, W}, &nx) || !prod_ok({nx, es}, &bytes_x) ||
+        !prod_ok({g.BC, video ? 64 : 16, g.Tq, g.h, g.w}, &ny) || !prod_ok({ny, es}, &bytes_y))
+        return TOK_ERR_SHAPE;
+    if (nx == 0 || ny == 0)
+        return TOK_OK;
+    if (!in || !out)
+        return TOK_ERR_NULL;
+    if (!aligned(in, es) || !aligned(out, es))
+        return TOK_ERR_ALIGN;
+    const int64_t bytes_in = fwd ? bytes_x : bytes_y, bytes_out = fwd ? bytes_y : bytes_x;
+    if (overlaps(in, bytes_in, out, bytes_out))
+        return TOK_ERR_ALIAS;
+
+    HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, 0, g.Tq};
+    dims.fbase = fbase;
+    dims.rep = rep;
+    dims.video = video;
+    dims.ext = true;
+    if (haar_tma_eligible(in, out, dt, dims))
+        return haar_tma_launch(fwd, false, in, out, dt, dims, stream);
+    if (dt == TOK_BF16) {
+        using B16 = __nv_bfloat16;
+        if (video)
+            return fwd ? launch_ext<B16, true, true>(in, out, g, stream) : launch_ext<B16, true, false>(in, out, g, stream);
+        return fwd ? launch_ext<B16, false, true>(in, out, g, stream) : launch_ext<B16, false, false>(in, out, g, stream);
+    }
+    if (video)
+        return fwd ? launch_ext<float, true, true>(in, out, g, stream) : launch_ext<float, true, false>(in, out, g, stream);
+    return fwd ? launch_ext<float, false, true>(in, out, g, stream) : launch_ext<float, false, false>(in, out, g, stream);
+}
+
+bool padded_extents(int64_t T, int64_t H, int64_t W, int64_t ms, int64_t mt, int64_t *Tp, int64_t *Hp, int64_t *Wp)
+{
+    if (T < 1 || H < 0 || W < 0 || ms < 4 || ms % 4 != 0 || mt < 4 || mt % 4 != 0)
+        return false;
+    if (H > ((int64_t)1 << 40) || W > ((int64_t)1 << 40) || T > ((int64_t)1 << 40) || ms > ((int64_t)1 << 20) ||
+        mt > ((int64_t)1 << 20))
+        return false;
+    *Hp = (H + ms - 1) / ms * ms;
+    *Wp = (W + ms - 1) / ms * ms;
+    *Tp = T == 1 ? 1 : 1 + (T - 1 + mt - 1) / mt * mt;
+    return true;
+}
+
+tok_status padded_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                       int64_t W, int64_t ms, int64_t mt, cudaStream_t stream)
+{
+    int64_t Tp, Hp, Wp;
+    if (B < 0 || C < 0 || !padded_extents(T, H, W, ms, mt, &Tp, &Hp, &Wp))
+        return TOK_ERR_SHAPE;
+    return haar_ext_call(fwd, in, out, dt, B, C, T, H, W, Tp, Hp, Wp, -3, 1, T > 1, stream);
+}
+
+tok_status chunk_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                      int64_t W, int first, cudaStream_t stream)
+{
+    if (B < 0 || C < 0 || H < 0 || W < 0 || H % 4 || W % 4)
+        return TOK_ERR_SHAPE;
+    if (first ? (T < 1 || T % 4 != 1) : (T < 4 || T % 4 != 0))
+        return TOK_ERR_SHAPE;
+    return haar_ext_call(fwd, in, out, dt, B, C, T, H, W, T, H, W, first ? -3 : 0, first ? 1 : 0, true, stream);
 }
 
 } // namespace
@@ -498,4 +710,38 @@ extern "C" tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt,
     if (t_end < 0)
         return TOK_ERR_SHAPE;
     return tok::haar_call(false, false, y, x, dt, B, C, T, H, W, t_begin, t_end, stream);
+}
+
+extern "C" tok_status tok_haar_padded_extents(int64_t T, int64_t H, int64_t W, int64_t spatial_multiple,
+                                              int64_t temporal_multiple, int64_t *Tp, int64_t *Hp, int64_t *Wp)
+{
+    if (!Tp || !Hp || !Wp)
+        return TOK_ERR_NULL;
+    return tok::padded_extents(T, H, W, spatial_multiple, temporal_multiple, Tp, Hp, Wp) ? TOK_OK : TOK_ERR_SHAPE;
+}
+
+extern "C" tok_status tok_haar_fwd_padded(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                          int64_t H, int64_t W, int64_t spatial_multiple, int64_t temporal_multiple,
+                                          cudaStream_t stream)
+{
+    return tok::padded_call(true, x, y, dt, B, C, T, H, W, spatial_multiple, temporal_multiple, stream);
+}
+
+extern "C" tok_status tok_haar_inv_cropped(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, int64_t spatial_multiple, int64_t temporal_multiple,
+                                           cudaStream_t stream)
+{
+    return tok::padded_call(false, y, x, dt, B, C, T, H, W, spatial_multiple, temporal_multiple, stream);
+}
+
+extern "C" tok_status tok_haar_fwd_chunk(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                         int64_t H, int64_t W, int first, cudaStream_t stream)
+{
+    return tok::chunk_call(true, x, y, dt, B, C, T, H, W, first, stream);
+}
+
+extern "C" tok_status tok_haar_inv_chunk(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                         int64_t H, int64_t W, int first, cudaStream_t stream)
+{
+    return tok::chunk_call(false, y, x, dt, B, C, T, H, W, first, stream);
 }

@@ -57,7 +57,24 @@ struct TileGrid {
     int T, Tq, tq0;          // frames, latent frames of the tensor, first latent frame processed
     int64_t H, W, h, w;
     uint32_t ntiles;
+    // Extended form (padding, cropping, streaming chunks): a window tq that is not the
+    // frame-0 replica window reads frames 4*tq + fbase .. + 3 of the T-frame pixel tensor,
+    // mirrored about frame T - 1 past its end; window 0 is the replica window iff rep.
+    // The pixel tensor [T][H][W] may be smaller than the 4h x 4w blocks: the forward
+    // reads zeros there (TMA fill), the inverse does not write there.
+    int fbase, rep;
 };
+
+// Source frame of frame f of a T-frame clip mirrored about its last frame (period 2(T-1)).
+__device__ __forceinline__ int mirror_frame(int f, int T)
+{
+    if (f < T)
+        return f;
+    if (T == 1)
+        return 0;
+    const int period = 2 * (T - 1), r = f % period;
+    return r < T ? r : period - r;
+}
 
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 // a - b, exactly as a subtraction rounds (the product b * -1 is exact).
@@ -123,6 +140,10 @@ template <> struct SRow<float> {
     static __device__ __forceinline__ void store_pair(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
 };
 
+template <typename T> __device__ __forceinline__ T to_elem(float v);
+template <> __device__ __forceinline__ float to_elem<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 to_elem<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
 // Global stores of results: two coefficients (blocks j, j+1) of one plane, or one
 // pixel row of 8 elements (4 of block j, 4 of block j+1).
 __device__ __forceinline__ void gstore_pair(__nv_bfloat16 *p, float2 v)
@@ -150,12 +171,14 @@ template <bool VIDEO> struct TileRows {
 // !FWD: coefficients -> pixels (the unpatcher, or with ADJ the patcher's adjoint).
 // ADJ changes window 0 only: its time samples are (0, 0, 0, frame 0) instead of four
 // copies of frame 0, and frame 0 receives the sum of the four rebuilt samples
-// instead of the last one.
-template <typename T, bool VIDEO, bool FWD, bool ADJ>
+// instead of the last one.  EXT: the extended form of TileGrid (padding, cropping,
+// streaming chunks).
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
 __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
                     const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
 {
+    static_assert(!(EXT && ADJ), "the adjoints take the plain form");
     using P = WarpTiles<T>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
@@ -191,7 +214,21 @@ __global__ void __launch_bounds__(32)
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
             const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
-            if constexpr (FWD) {
+            if constexpr (FWD && EXT && VIDEO) {
+                if (tg.rep && tq == 0) {
+                    mbar_expect_tx(bar, FRAME_BYTES);
+                    tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
+                } else if (4 * tq + tg.fbase + 3 < tg.T) {
+                    mbar_expect_tx(bar, NA * FRAME_BYTES);
+                    tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq + tg.fbase), bar);
+                } else {
+                    // The window runs past the clip: frame by frame, mirrored about the last frame.
+                    mbar_expect_tx(bar, NA * FRAME_BYTES);
+                    for (int a = 0; a < NA; ++a)
+                        tma_load_3d(dst + a * FRAME_BYTES, &xmap1, 4 * WT * tx, 4 * RW * ty,
+                                    (int)(bc * tg.T + mirror_frame(4 * tq + tg.fbase + a, tg.T)), bar);
+                }
+            } else if constexpr (FWD) {
                 if (VIDEO && tq > 0) {
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
                     tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
@@ -219,6 +256,7 @@ __global__ void __launch_bounds__(32)
         const T *tin = in_buf + s * kTileElems;
         const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
         const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
+        const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0); // window 0 of a video
 
 #pragma unroll
         for (int rw = 0; rw < RW; ++rw) {
@@ -226,7 +264,7 @@ __global__ void __launch_bounds__(32)
             if constexpr (FWD) {
 #pragma unroll
                 for (int a = 0; a < NA; ++a) {
-                    const int fa = (VIDEO && tq > 0) ? a : 0; // window 0 reads frame 0 four times
+                    const int fa = replica ? 0 : a; // window 0 reads frame 0 four times
 #pragma unroll
                     for (int rr = 0; rr < 4; ++rr) {
                         if (ADJ && VIDEO && tq == 0 && a != 3) {
@@ -287,7 +325,7 @@ __global__ void __launch_bounds__(32)
                 // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only
                 // (the adjoint: the sum of its four frames).
                 T *xb = out + (bc * tg.T) * tg.H * tg.W + (4 * row) * tg.W + 4 * j0;
-                if (ADJ && VIDEO && tq == 0) {
+                if (ADJ && replica) {
 #pragma unroll
                     for (int rr = 0; rr < 4; ++rr) {
                         float2 o[4];
@@ -301,16 +339,31 @@ __global__ void __launch_bounds__(32)
                 }
 #pragma unroll
                 for (int a = 0; a < NA; ++a) {
-                    if (VIDEO && tq == 0 && a != 3)
+                    if (replica && a != 3)
                         continue;
-                    const int64_t f = VIDEO ? (tq == 0 ? 0 : 4 * tq - 3 + a) : 0;
+                    const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
+                    if (EXT && f >= tg.T) // cropped frames
+                        continue;
 #pragma unroll
                     for (int rr = 0; rr < 4; ++rr) {
                         float2 o[4];
 #pragma unroll
                         for (int d = 0; d < 4; ++d)
                             o[d] = __fmul2_rn(v[a][rr][d], scale);
-                        gstore_row(xb + f * tg.H * tg.W + rr * tg.W, o);
+                        T *dst = xb + f * tg.H * tg.W + rr * tg.W;
+                        if (!EXT) {
+                            gstore_row(dst, o);
+                        } else if (4 * row + rr < tg.H) { // cropped rows and columns
+                            const int64_t col = 4 * j0;
+                            if (col + 8 <= tg.W) {
+                                gstore_row(dst, o);
+                            } else {
+#pragma unroll
+                                for (int d = 0; d < 8; ++d)
+                                    if (col + d < tg.W)
+                                        dst[d] = to_elem<T>(d < 4 ? o[d].x : o[d - 4].y);
+                            }
+                        }
                     }
                 }
             }
@@ -329,7 +382,7 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-template <typename T, bool VIDEO, bool FWD, bool ADJ>
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
 tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     using P = WarpTiles<T>;
@@ -345,8 +398,10 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
         const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
         const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
         const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
+        // The 4-frame box serves windows with four frames of the clip, so a frame axis
+        // shorter than 4 never uses it and it is not encoded.
         if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
-            (VIDEO && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
+            (VIDEO && xdims[2] >= 4 && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
             return TOK_ERR_SHAPE;
     } else {
         const uint64_t ydims[5] = {(uint64_t)d.w, (uint64_t)d.h, (uint64_t)d.Tq, (uint64_t)d.C, (uint64_t)(G * d.B)};
@@ -371,16 +426,18 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.h = d.h;
     tg.w = d.w;
     tg.ntiles = (uint32_t)(ntx * nty * d.nq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
+    tg.fbase = (int)d.fbase;
+    tg.rep = d.rep;
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err =
-        cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+        cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_tma_kernel<T, VIDEO, FWD, ADJ><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
+    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
     return launch_status();
 }
 
@@ -391,7 +448,7 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
     const int64_t es = dt == TOK_F32 ? 4 : 2;
     if (!aligned(in, 16) || !aligned(out, 16))
         return false;
-    if ((d.w * es) % 16 != 0) // row strides of both tensors must be multiples of 16 bytes
+    if ((d.w * es) % 16 != 0 || (d.W * es) % 16 != 0) // row strides of both tensors: multiples of 16 bytes
         return false;
     // Coordinates are 32-bit: frames of the flattened [B*C*T] axis and the group axis must fit,
     // tiles are numbered in 32 bits, and the 64 planes of one channel lie within a 32-bit offset.
@@ -405,23 +462,41 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
 tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
                            cudaStream_t stream)
 {
-    const bool video = d.T > 1;
+    const bool video = d.video;
+    if (d.ext) {
+        if (dt == TOK_BF16) {
+            using B16 = __nv_bfloat16;
+            if (video)
+                return fwd ? launch<B16, true, true, false, true>(in, out, d, stream)
+                           : launch<B16, true, false, false, true>(in, out, d, stream);
+            return fwd ? launch<B16, false, true, false, true>(in, out, d, stream)
+                       : launch<B16, false, false, false, true>(in, out, d, stream);
+        }
+        if (video)
+            return fwd ? launch<float, true, true, false, true>(in, out, d, stream)
+                       : launch<float, true, false, false, true>(in, out, d, stream);
+        return fwd ? launch<float, false, true, false, true>(in, out, d, stream)
+                   : launch<float, false, false, false, true>(in, out, d, stream);
+    }
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (!video)
-            return fwd ? launch<B16, false, true, false>(in, out, d, stream)
-                       : launch<B16, false, false, false>(in, out, d, stream);
+            return fwd ? launch<B16, false, true, false, false>(in, out, d, stream)
+                       : launch<B16, false, false, false, false>(in, out, d, stream);
         if (adj)
-            return fwd ? launch<B16, true, true, true>(in, out, d, stream)
-                       : launch<B16, true, false, true>(in, out, d, stream);
-        return fwd ? launch<B16, true, true, false>(in, out, d, stream) : launch<B16, true, false, false>(in, out, d, stream);
+            return fwd ? launch<B16, true, true, true, false>(in, out, d, stream)
+                       : launch<B16, true, false, true, false>(in, out, d, stream);
+        return fwd ? launch<B16, true, true, false, false>(in, out, d, stream)
+                   : launch<B16, true, false, false, false>(in, out, d, stream);
     }
     if (!video)
-        return fwd ? launch<float, false, true, false>(in, out, d, stream)
-                   : launch<float, false, false, false>(in, out, d, stream);
+        return fwd ? launch<float, false, true, false, false>(in, out, d, stream)
+                   : launch<float, false, false, false, false>(in, out, d, stream);
     if (adj)
-        return fwd ? launch<float, true, true, true>(in, out, d, stream) : launch<float, true, false, true>(in, out, d, stream);
-    return fwd ? launch<float, true, true, false>(in, out, d, stream) : launch<float, true, false, false>(in, out, d, stream);
+        return fwd ? launch<float, true, true, true, false>(in, out, d, stream)
+                   : launch<float, true, false, true, false>(in, out, d, stream);
+    return fwd ? launch<float, true, true, false, false>(in, out, d, stream)
+               : launch<float, true, false, false, false>(in, out, d, stream);
 }
 
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)

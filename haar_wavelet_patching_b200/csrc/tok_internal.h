@@ -10,10 +10,18 @@ namespace tok {
 
 // Extents of one Haar call: pixels [B, C, T, H, W], coefficients [B, G*C, Tq, h, w];
 // the call processes latent frames [tq0, tq0 + nq).
+// Extended form (ext): the pixel tensor may be smaller than the 4h x 4w blocks (the
+// forward pads with zeros, the inverse crops), a window tq that is not the frame-0
+// replica window reads frames 4*tq + fbase .. + 3 (mirrored past frame T - 1), and
+// window 0 is the replica window iff rep.  video: 3D transform (else the 2D path).
 struct HaarDims {
     int64_t B, C, T, H, W;
     int64_t Tq, h, w;
     int64_t tq0, nq;
+    int64_t fbase = -3;
+    int rep = 1;
+    bool video = true;
+    bool ext = false;
 };
 
 // The TMA path takes 16-byte-aligned tensors whose rows are multiples of 16 bytes.

@@ -171,6 +171,68 @@ TOK_API tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, in
                                         int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream);
 
 /*
+ * Clips of any extents ([guide] 6.3: before the network a clip is padded --
+ * zeros in space, reflection at the temporal edge -- to aligned extents, and the
+ * result is cropped back to the original size afterwards).
+ *
+ * tok_haar_padded_extents -- the padded extents: Hp, Wp = H, W rounded up to
+ * multiples of spatial_multiple; Tp = the smallest T' >= T with
+ * (T' - 1) % temporal_multiple == 0 (images, T == 1, stay at 1).  Both
+ * multiples must be positive multiples of 4 (4 for the patcher alone; 8 or 16
+ * to match a network's total downsampling).  TOK_ERR_SHAPE for invalid
+ * arguments, TOK_ERR_NULL for a NULL output pointer.
+ */
+TOK_API tok_status tok_haar_padded_extents(int64_t T, int64_t H, int64_t W, int64_t spatial_multiple,
+                                           int64_t temporal_multiple, int64_t *Tp, int64_t *Hp, int64_t *Wp);
+
+/*
+ * tok_haar_fwd_padded -- the patcher on a clip of any extents.
+ *   x : [B, C, T, H, W] (input, any T >= 1, H, W >= 0)
+ *   y : [B, 64C, 1 + (Tp-1)/4, Hp/4, Wp/4] (T > 1) or [B, 16C, 1, Hp/4, Wp/4]
+ *       (T == 1), extents from tok_haar_padded_extents (output)
+ * equal to tok_haar_fwd on the padded clip: rows H .. Hp-1 and columns
+ * W .. Wp-1 are zero; frames T .. Tp-1 mirror the clip about its last frame
+ * (frame T-1+k is frame T-1-k, repeated with period 2(T-1) if the padding is
+ * longer than the clip).  The padded clip is never stored: the kernels read
+ * zeros and mirrored frames in place.  Errors as tok_haar_fwd (no divisibility
+ * rule on T, H, W).
+ *
+ * tok_haar_inv_cropped -- the unpatcher on the padded extents, keeping the
+ * first T frames, H rows and W columns: y as above (input), x [B, C, T, H, W]
+ * (output).  The inverse of tok_haar_fwd_padded on its output.
+ */
+TOK_API tok_status tok_haar_fwd_padded(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                       int64_t H, int64_t W, int64_t spatial_multiple, int64_t temporal_multiple,
+                                       cudaStream_t stream);
+TOK_API tok_status tok_haar_inv_cropped(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                        int64_t H, int64_t W, int64_t spatial_multiple, int64_t temporal_multiple,
+                                        cudaStream_t stream);
+
+/*
+ * Streaming chunks of a video ([guide] 6.3: long videos run window by window).
+ * Unlike the windowed calls, a chunk call sees only the chunk's own frames, so
+ * a long video never has to be resident in device memory at once.
+ *
+ * tok_haar_fwd_chunk --
+ *   first != 0: the start of a video, T = 1 + 4k frames (k >= 0): the patcher
+ *     with its frame-0 replicas, always the 3D transform (a one-frame first
+ *     chunk gives the video's latent frame 0, not the image transform);
+ *     y [B, 64C, 1 + k, H/4, W/4].
+ *   first == 0: a continuation, T = 4k frames (k >= 1) that follow earlier
+ *     frames; latent frame j reads frames 4j .. 4j+3 of the chunk, no replica;
+ *     y [B, 64C, k, H/4, W/4].
+ * Chunks of 1 + 4k0, 4k1, 4k2, ... frames give exactly the latent frames of the
+ * whole video, in order.  H % 4 == 0, W % 4 == 0; other errors as tok_haar_fwd.
+ *
+ * tok_haar_inv_chunk -- the inverse of tok_haar_fwd_chunk (T, H, W: the chunk's
+ * pixel extents): y as above (input) -> x [B, C, T, H, W] (output).
+ */
+TOK_API tok_status tok_haar_fwd_chunk(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                      int64_t H, int64_t W, int first, cudaStream_t stream);
+TOK_API tok_status tok_haar_inv_chunk(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                      int64_t H, int64_t W, int first, cudaStream_t stream);
+
+/*
  * tok_fsq_encode -- fused 1x1 projection + FSQ quantization + index pack.
  * [guide] 7.2 (bound with tanh, rounding, levels [8,8,8,5,5,5], implicit
  * codebook of 64000, mixed-radix codes_to_indices), [guide] 6.2 (indices

@@ -155,3 +155,32 @@ def test_host_shape_logic():
     assert hwp.haar_coeff_shape(16, 3, 1, 1024, 1024) == (16, 48, 1, 256, 256)
     with pytest.raises(ValueError):
         hwp.latent_frames(7)
+
+
+def test_padded_and_chunk_rules(lib):
+    T, H, W = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
+    ext = lib.tok_haar_padded_extents
+    assert ext(10, 5, 6, 4, 4, ctypes.byref(T), ctypes.byref(H), ctypes.byref(W)) == hwp.TOK_OK
+    assert (T.value, H.value, W.value) == (13, 8, 8)
+    assert ext(10, 5, 6, 16, 8, ctypes.byref(T), ctypes.byref(H), ctypes.byref(W)) == hwp.TOK_OK
+    assert (T.value, H.value, W.value) == (17, 16, 16)
+    assert ext(1, 1080, 1920, 16, 8, ctypes.byref(T), ctypes.byref(H), ctypes.byref(W)) == hwp.TOK_OK
+    assert (T.value, H.value, W.value) == (1, 1088, 1920)
+    for bad in [(10, 5, 6, 6, 4), (10, 5, 6, 4, 0), (10, 5, 6, 0, 4), (0, 5, 6, 4, 4), (10, -1, 6, 4, 4)]:
+        assert ext(*bad, ctypes.byref(T), ctypes.byref(H), ctypes.byref(W)) == hwp.TOK_ERR_SHAPE
+    assert ext(10, 5, 6, 4, 4, None, ctypes.byref(H), ctypes.byref(W)) == hwp.TOK_ERR_NULL
+    fp, ic = lib.tok_haar_fwd_padded, lib.tok_haar_inv_cropped
+    assert fp(A, Bp, 1, 1, 3, 10, 5, 6, 6, 4, NULL) == hwp.TOK_ERR_SHAPE      # spatial multiple 6
+    assert fp(A, Bp, 7, 1, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_ERR_DTYPE
+    assert fp(NULL, Bp, 1, 1, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_ERR_NULL
+    assert fp(F(0x10001), Bp, 1, 1, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_ERR_ALIGN
+    assert fp(A, A, 1, 1, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_ERR_ALIAS
+    assert ic(A, A, 1, 1, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_ERR_ALIAS
+    assert fp(NULL, NULL, 1, 0, 3, 10, 5, 6, 4, 4, NULL) == hwp.TOK_OK        # empty: nothing to do
+    fc, iv = lib.tok_haar_fwd_chunk, lib.tok_haar_inv_chunk
+    assert fc(A, Bp, 1, 1, 3, 8, 64, 64, 1, NULL) == hwp.TOK_ERR_SHAPE        # first chunk: 1 + 4k frames
+    assert fc(A, Bp, 1, 1, 3, 6, 64, 64, 0, NULL) == hwp.TOK_ERR_SHAPE        # continuation: 4k frames
+    assert fc(A, Bp, 1, 1, 3, 0, 64, 64, 0, NULL) == hwp.TOK_ERR_SHAPE
+    assert fc(A, Bp, 1, 1, 3, 8, 62, 64, 0, NULL) == hwp.TOK_ERR_SHAPE       # H % 4
+    assert fc(NULL, Bp, 1, 1, 3, 8, 64, 64, 0, NULL) == hwp.TOK_ERR_NULL
+    assert iv(A, A, 1, 1, 3, 8, 64, 64, 0, NULL) == hwp.TOK_ERR_ALIAS
