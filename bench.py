@@ -374,6 +374,42 @@ def time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev, iters=G
     return out
 
 
+STREAM_CLIP = (1, 3, 120, 720, 1280)  # 120 frames: one mirrored frame makes 121; also 30 continuation windows
+
+
+def time_streaming(torch, hwp, stream, dev, iters=GRAD_ITERS):
+    """The arbitrary-extent and streaming calls on a 120-frame 720p clip (bf16), each timed alone
+    like the gradients: the padded patcher / cropped unpatcher (spatial multiple 16, temporal 8:
+    one frame mirrored in, 121 frames' worth of windows) and the same 120 frames as one
+    continuation chunk (30 windows, no replica).  Algorithmic bytes: the clip read or written once
+    plus the coefficients written or read once."""
+    B, C, T, H, W = STREAM_CLIP
+    g = torch.Generator(device=dev).manual_seed(11)
+    x = (torch.rand(STREAM_CLIP, generator=g, device=dev) * 2 - 1).to(torch.bfloat16)
+    xr = torch.empty_like(x)
+    yp = torch.empty(hwp.padded_coeff_shape(B, C, T, H, W, 16, 8), dtype=torch.bfloat16, device=dev)
+    yc = torch.empty(hwp.chunk_coeff_shape(B, C, T, H, W, False), dtype=torch.bfloat16, device=dev)
+    xb = x.numel() * 2
+    calls = {
+        "haar_fwd_padded": (lambda: hwp.tok_haar_fwd_padded(x, yp, 16, 8), xb + yp.numel() * 2),
+        "haar_inv_cropped": (lambda: hwp.tok_haar_inv_cropped(yp, xr, 16, 8), xb + yp.numel() * 2),
+        "haar_fwd_chunk": (lambda: hwp.tok_haar_fwd_chunk(x, yc, False), xb + yc.numel() * 2),
+        "haar_inv_chunk": (lambda: hwp.tok_haar_inv_chunk(yc, xr, False), xb + yc.numel() * 2),
+    }
+    out = {}
+    for name, (call, nbytes) in calls.items():
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "bytes": nbytes, "launches": 1}
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -476,6 +512,7 @@ def run_ours(args, rank, world, local_rank):
     barrier()
 
     grads = time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev)
+    streaming = time_streaming(torch, hwp, stream, dev)
     barrier()
 
     if rank != 0:
@@ -510,6 +547,10 @@ def run_ours(args, rank, world, local_rank):
         "gradients": {n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
                           "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
                           "bytes": g["bytes"], "launches": g["launches"]} for n, g in grads.items()},
+        "streaming": {"clip": list(STREAM_CLIP), "dtype": "bf16",
+                      **{n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
+                             "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
+                             "bytes": g["bytes"]} for n, g in streaming.items()}},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

@@ -2,6 +2,7 @@
 
     python -m haar_wavelet_patching_b200.run_case --op haar_inv --shape 1,3,33,704,1280 --dtype bf16 --iters 3
     python -m haar_wavelet_patching_b200.run_case --op fsq_encode --shape 48,16,56320 --iters 3
+    python -m haar_wavelet_patching_b200.run_case --op haar_fwd_padded --shape 1,3,120,720,1280 --ms 16 --mt 8
 
 Inputs are random tensors made on the device by torch (their values do not
 change the kernels' work).  Prints the mean CUDA-event time per launch and the
@@ -17,19 +18,36 @@ import haar_wavelet_patching_b200 as hwp
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=("haar_fwd", "haar_inv", "haar_fwd_adjoint", "haar_inv_adjoint",
-                                                     "fsq_encode", "fsq_decode", "fsq_encode_backward",
-                                                     "fsq_decode_backward"))
+                                                     "haar_fwd_padded", "haar_inv_cropped", "haar_fwd_chunk",
+                                                     "haar_inv_chunk", "fsq_encode", "fsq_decode",
+                                                     "fsq_encode_backward", "fsq_decode_backward"))
     ap.add_argument("--shape", required=True, help="B,C,T,H,W for haar ops; B,C,S for fsq ops")
     ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--codes", action="store_true", help="fsq_encode: also write the codes")
+    ap.add_argument("--ms", type=int, default=4, help="padded ops: spatial multiple")
+    ap.add_argument("--mt", type=int, default=4, help="padded ops: temporal multiple")
+    ap.add_argument("--first", action="store_true", help="chunk ops: the first chunk (1 + 4k frames)")
     a = ap.parse_args()
     shape = tuple(int(v) for v in a.shape.split(","))
     dev = torch.device("cuda", 0)
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op.startswith("haar"):
+    if a.op in ("haar_fwd_padded", "haar_inv_cropped", "haar_fwd_chunk", "haar_inv_chunk"):
+        B, C, T, H, W = shape
+        x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
+        if a.op.endswith(("padded", "cropped")):
+            yshape = hwp.padded_coeff_shape(B, C, T, H, W, a.ms, a.mt)
+        else:
+            yshape = hwp.chunk_coeff_shape(B, C, T, H, W, a.first)
+        y = (torch.rand(yshape, generator=g, device=dev) * 2 - 1).to(dt)
+        run = {"haar_fwd_padded": lambda: hwp.tok_haar_fwd_padded(x, y, a.ms, a.mt),
+               "haar_inv_cropped": lambda: hwp.tok_haar_inv_cropped(y, x, a.ms, a.mt),
+               "haar_fwd_chunk": lambda: hwp.tok_haar_fwd_chunk(x, y, a.first),
+               "haar_inv_chunk": lambda: hwp.tok_haar_inv_chunk(y, x, a.first)}[a.op]
+        nbytes = (x.numel() + y.numel()) * x.element_size()
+    elif a.op.startswith("haar"):
         B, C, T, H, W = shape
         x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
         y = torch.empty(hwp.haar_coeff_shape(*shape), dtype=dt, device=dev)
