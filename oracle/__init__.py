@@ -50,8 +50,10 @@ def _load():
             f = getattr(lib, name)
             f.restype = ctypes.c_int
             f.argtypes = [dp, dp, i64, i64, i64, i64, i64, ctypes.c_int]
-        lib.oracle_haar_level_fwd.restype = ctypes.c_int
-        lib.oracle_haar_level_fwd.argtypes = [dp, dp, i64, i64, i64, i64]
+        for name in ("oracle_haar_level_fwd", "oracle_haar_level_inv"):
+            f = getattr(lib, name)
+            f.restype = ctypes.c_int
+            f.argtypes = [dp, dp, i64, i64, i64, i64]
         lib.oracle_haar_out_frames.restype = i64
         lib.oracle_haar_out_frames.argtypes = [i64]
         lib.oracle_fsq_levels.restype = ctypes.c_int
@@ -172,6 +174,30 @@ def haar_level_fwd(x: np.ndarray) -> np.ndarray:
     _check(_load().oracle_haar_level_fwd(_ptr(x, ctypes.c_double), _ptr(y, ctypes.c_double), C, T, H, W),
            "haar_level_fwd")
     return y
+
+
+def haar_level_inv(y: np.ndarray, T: int, H: int, W: int) -> np.ndarray:
+    """Inverse of one level, T, H, W the pixel extents: -> [C, T, H, W]."""
+    y = np.ascontiguousarray(y, dtype=np.float64)
+    C = y.shape[0] // (4 if T == 1 else 8)
+    x = np.zeros((C, T, H, W), dtype=np.float64)
+    _check(_load().oracle_haar_level_inv(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), C, T, H, W),
+           "haar_level_inv")
+    return x
+
+
+def single_out_shape(B, C, T, H, W):
+    """The single-level patcher (patch_size=2): [B, 8C, (T+1)/2, H/2, W/2], images [B, 4C, 1, H/2, W/2]."""
+    return (B, 4 * C, 1, H // 2, W // 2) if T == 1 else (B, 8 * C, (T + 1) // 2, H // 2, W // 2)
+
+
+def haar_single_fwd(x: np.ndarray) -> np.ndarray:
+    """The single-level patcher on a batch [B, C, T, H, W]: one level per item."""
+    return np.stack([haar_level_fwd(xb) for xb in np.asarray(x, dtype=np.float64)])
+
+
+def haar_single_inv(y: np.ndarray, T: int, H: int, W: int) -> np.ndarray:
+    return np.stack([haar_level_inv(yb, T, H, W) for yb in np.asarray(y, dtype=np.float64)])
 
 
 def fsq_basis():

@@ -224,6 +224,21 @@ int oracle_haar_level_fwd(const double *x, double *y, int64_t C, int64_t T, int6
 }
 
 /*
+ * Single level inverse (the unpatcher with patch_size=2), T, H, W the pixel
+ * extents: y [4C][1][H/2][W/2] (T == 1) or [8C][(T+1)/2][H/2][W/2] -> x [C][T][H][W].
+ */
+int oracle_haar_level_inv(const double *y, double *x, int64_t C, int64_t T, int64_t H, int64_t W)
+{
+    if (C < 0 || T < 1 || H % 2 || W % 2 || (T > 1 && T % 2 == 0))
+        return ORACLE_BAD_SHAPE;
+    if (T == 1)
+        level2d_inv(y, x, C, H / 2, W / 2);
+    else
+        level3d_inv(y, x, C, (T + 1) / 2, H / 2, W / 2);
+    return ORACLE_OK;
+}
+
+/*
  * Two-level patcher (patch_size=4): the single level applied twice, the second
  * time to all 8C (or 4C) first-level channels.
  */
