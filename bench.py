@@ -377,6 +377,29 @@ def time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev, iters=G
 STREAM_CLIP = (1, 3, 120, 720, 1280)  # 120 frames: one mirrored frame makes 121; also 30 continuation windows
 
 
+def time_single(torch, hwp, stream, x, dev, iters=GRAD_ITERS):
+    """The single-level patcher / unpatcher (patch_size=2) on the headline clip, timed alone:
+    [1,3,121,704,1280] <-> [1,24,61,352,640] bf16; algorithmic bytes: the clip plus the
+    coefficients, each once."""
+    y1 = torch.empty(hwp.single_coeff_shape(*x.shape), dtype=x.dtype, device=dev)
+    xr = torch.empty_like(x)
+    nbytes = (x.numel() + y1.numel()) * x.element_size()
+    out = {}
+    for name, call in (("haar_fwd_single", lambda: hwp.tok_haar_fwd_single(x, y1)),
+                       ("haar_inv_single", lambda: hwp.tok_haar_inv_single(y1, xr))):
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "bytes": nbytes}
+    del y1, xr
+    return out
+
+
 def time_streaming(torch, hwp, stream, dev, iters=GRAD_ITERS):
     """The arbitrary-extent and streaming calls on a 120-frame 720p clip (bf16), each timed alone
     like the gradients: the padded patcher / cropped unpatcher (spatial multiple 16, temporal 8:
@@ -513,6 +536,7 @@ def run_ours(args, rank, world, local_rank):
 
     grads = time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev)
     streaming = time_streaming(torch, hwp, stream, dev)
+    single = time_single(torch, hwp, stream, x, dev)
     barrier()
 
     if rank != 0:
@@ -551,6 +575,9 @@ def run_ours(args, rank, world, local_rank):
                       **{n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
                              "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
                              "bytes": g["bytes"]} for n, g in streaming.items()}},
+        "single_level": {n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
+                             "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
+                             "bytes": g["bytes"]} for n, g in single.items()},
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()

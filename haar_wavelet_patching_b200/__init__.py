@@ -25,7 +25,7 @@ FSQ_DIM = 6
 # Every symbol include/tok.h declares.
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
-               "tok_haar_inv_windows", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
+               "tok_haar_inv_windows", "tok_haar_fwd_single", "tok_haar_inv_single", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
                "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
                "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
@@ -58,7 +58,8 @@ def lib():
         L.tok_last_cuda_error.argtypes = []
         L.tok_check_device.restype = i32
         L.tok_check_device.argtypes = [vp]
-        for f in (L.tok_haar_fwd, L.tok_haar_inv, L.tok_haar_fwd_adjoint, L.tok_haar_inv_adjoint):
+        for f in (L.tok_haar_fwd, L.tok_haar_inv, L.tok_haar_fwd_adjoint, L.tok_haar_inv_adjoint,
+                  L.tok_haar_fwd_single, L.tok_haar_inv_single):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
         L.tok_fsq_backward_workspace_size.restype = i64
@@ -199,6 +200,35 @@ def tok_haar_fwd_windows(x: torch.Tensor, y: torch.Tensor, t_begin: int, t_end: 
 def tok_haar_inv_windows(y: torch.Tensor, x: torch.Tensor, t_begin: int, t_end: int, stream=None):
     """Inverse restricted to latent frames [t_begin, t_end): writes only those windows' pixel frames."""
     _haar_windows(False, x, y, t_begin, t_end, stream)
+    return x
+
+
+def single_coeff_shape(B, C, T, H, W):
+    """The single-level patcher's output: [B, 8C, (T+1)/2, H/2, W/2], images [B, 4C, 1, H/2, W/2]."""
+    return (B, 4 * C, 1, H // 2, W // 2) if T == 1 else (B, 8 * C, (T + 1) // 2, H // 2, W // 2)
+
+
+def _haar_single(fwd, x, y, stream):
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != single_coeff_shape(B, C, T, H, W):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {single_coeff_shape(B, C, T, H, W)}")
+    f = lib().tok_haar_fwd_single if fwd else lib().tok_haar_inv_single
+    src, dst = (x, y) if fwd else (y, x)
+    _check(f(_ptr(src), _ptr(dst), _dtype_code(x), B, C, T, H, W, _stream(x, stream)),
+           "tok_haar_fwd_single" if fwd else "tok_haar_inv_single")
+
+
+def tok_haar_fwd_single(x: torch.Tensor, y: torch.Tensor, stream=None):
+    """The single-level patcher (patch_size=2): x [B,C,T,H,W] -> y (single_coeff_shape)."""
+    _haar_single(True, x, y, stream)
+    return y
+
+
+def tok_haar_inv_single(y: torch.Tensor, x: torch.Tensor, stream=None):
+    _haar_single(False, x, y, stream)
     return x
 
 
@@ -412,6 +442,16 @@ def fsq_encode(u: torch.Tensor, w: torch.Tensor, with_codes: bool = False, strea
 def fsq_decode(idx: torch.Tensor, w: torch.Tensor, bad_count: torch.Tensor = None, stream=None) -> torch.Tensor:
     out = torch.empty((idx.shape[0], w.shape[1]) + tuple(idx.shape[1:]), dtype=torch.float32, device=idx.device)
     return tok_fsq_decode(idx, w, out, bad_count, stream)
+
+
+def haar_fwd_single(x: torch.Tensor, stream=None) -> torch.Tensor:
+    y = torch.empty(single_coeff_shape(*x.shape), dtype=x.dtype, device=x.device)
+    return tok_haar_fwd_single(x, y, stream)
+
+
+def haar_inv_single(y: torch.Tensor, T: int, H: int, W: int, stream=None) -> torch.Tensor:
+    x = torch.empty((y.shape[0], y.shape[1] // (4 if T == 1 else 8), T, H, W), dtype=y.dtype, device=y.device)
+    return tok_haar_inv_single(y, x, stream)
 
 
 def haar_fwd_padded(x: torch.Tensor, spatial_multiple: int = 4, temporal_multiple: int = 4,

@@ -637,6 +637,157 @@ tok_status haar_ext_call(bool fwd, const void *in, void *out, tok_dtype dt, int6
     return fwd ? launch_ext<float, false, true>(in, out, g, stream) : launch_ext<float, false, false>(in, out, g, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Single level (patch_size=2), register path for shapes the TMA kernel cannot take:
+// one thread per 2x2x2 block (2x2 on images), element loads and stores.
+// ---------------------------------------------------------------------------
+struct SingleGeometry {
+    int64_t BC, C, T, H, W, Tq, h, w;
+};
+
+template <typename T, bool VIDEO, bool FWD>
+__global__ void __launch_bounds__(kThreads)
+    haar_single_reg_kernel(const T *__restrict__ in, T *__restrict__ out, SingleGeometry g)
+{
+    constexpr int NA = VIDEO ? 2 : 1, G = VIDEO ? 8 : 4;
+    constexpr float SCALE = VIDEO ? 0.353553390593273762f : 0.5f;
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.w)
+        return;
+    const int64_t i = item / g.w, j = item - i * g.w;
+    const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if (pair >= g.BC * g.Tq)
+        return;
+    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t b = bc / g.C, c = bc - b * g.C;
+    const bool replica = VIDEO && tq == 0;
+    const int64_t plane = g.Tq * g.h * g.w, cstride = g.C * plane;
+    const int64_t lat0 = (b * G * g.C + c) * plane + (tq * g.h + i) * g.w + j;
+    float v[NA][2][2];
+    if constexpr (FWD) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            const int64_t f = !VIDEO ? 0 : replica ? 0 : 2 * tq - 1 + a;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+                    v[a][r][d] = elem_to_f(in[((bc * g.T + f) * g.H + 2 * i + r) * g.W + 2 * j + d]);
+        }
+    } else {
+#pragma unroll
+        for (int grp = 0; grp < G; ++grp) {
+            const float p = elem_to_f(in[lat0 + grp * cstride]);
+            if constexpr (VIDEO)
+                v[grp >> 2][(grp >> 1) & 1][grp & 1] = p;
+            else
+                v[0][grp >> 1][grp & 1] = p;
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float l = v[a][r][0] + v[a][r][1], hgh = v[a][r][0] - v[a][r][1];
+            v[a][r][0] = l, v[a][r][1] = hgh;
+        }
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int d = 0; d < 2; ++d) {
+            const float l = v[a][0][d] + v[a][1][d], hgh = v[a][0][d] - v[a][1][d];
+            v[a][0][d] = l, v[a][1][d] = hgh;
+        }
+    if constexpr (VIDEO) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int d = 0; d < 2; ++d) {
+                const float l = v[0][r][d] + v[1][r][d], hgh = v[0][r][d] - v[1][r][d];
+                v[0][r][d] = l, v[1][r][d] = hgh;
+            }
+    }
+    if constexpr (FWD) {
+#pragma unroll
+        for (int grp = 0; grp < G; ++grp) {
+            const float p = VIDEO ? v[grp >> 2][(grp >> 1) & 1][grp & 1] : v[0][grp >> 1][grp & 1];
+            out[lat0 + grp * cstride] = f_to_elem<T>(p * SCALE);
+        }
+    } else {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+            if (replica && a != 1)
+                continue;
+            const int64_t f = !VIDEO ? 0 : replica ? 0 : 2 * tq - 1 + a;
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+                    out[((bc * g.T + f) * g.H + 2 * i + r) * g.W + 2 * j + d] = f_to_elem<T>(v[a][r][d] * SCALE);
+        }
+    }
+}
+
+template <typename T, bool VIDEO, bool FWD>
+tok_status launch_single_reg(const void *in, void *out, const SingleGeometry &g, cudaStream_t stream)
+{
+    const int64_t items = g.h * g.w, pairs = g.BC * g.Tq;
+    const int64_t gy = pairs < 65535 ? pairs : 65535, gz = (pairs + gy - 1) / gy;
+    if ((items + kThreads - 1) / kThreads > 0x7FFFFFFF || gz > 65535)
+        return TOK_ERR_SHAPE;
+    const dim3 grid((unsigned)((items + kThreads - 1) / kThreads), (unsigned)gy, (unsigned)gz);
+    haar_single_reg_kernel<T, VIDEO, FWD><<<grid, kThreads, 0, stream>>>((const T *)in, (T *)out, g);
+    return launch_status();
+}
+
+tok_status single_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                       int64_t H, int64_t W, cudaStream_t stream)
+{
+    if (dt != TOK_F32 && dt != TOK_BF16)
+        return TOK_ERR_DTYPE;
+    if (B < 0 || C < 0 || T < 1 || H < 0 || W < 0 || H % 2 || W % 2 || (T != 1 && T % 2 == 0))
+        return TOK_ERR_SHAPE;
+    const bool video = T > 1;
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    SingleGeometry g{};
+    g.C = C;
+    g.T = T;
+    g.H = H;
+    g.W = W;
+    g.Tq = video ? (T + 1) / 2 : 1;
+    g.h = H / 2;
+    g.w = W / 2;
+    int64_t nx, ny, bytes_x, bytes_y;
+    if (!prod_ok({B, C}, &g.BC) || !prod_ok({g.BC, T, H, W}, &nx) || !prod_ok({nx, es}, &bytes_x) ||
+        !prod_ok({g.BC, video ? 8 : 4, g.Tq, g.h, g.w}, &ny) || !prod_ok({ny, es}, &bytes_y))
+        return TOK_ERR_SHAPE;
+    if (nx == 0)
+        return TOK_OK;
+    if (!in || !out)
+        return TOK_ERR_NULL;
+    if (!aligned(in, es) || !aligned(out, es))
+        return TOK_ERR_ALIGN;
+    if (overlaps(in, fwd ? bytes_x : bytes_y, out, fwd ? bytes_y : bytes_x))
+        return TOK_ERR_ALIAS;
+    HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, 0, g.Tq};
+    dims.video = video;
+    if (haar_single_tma_eligible(in, out, dt, dims))
+        return haar_single_tma_launch(fwd, in, out, dt, dims, stream);
+    if (dt == TOK_BF16) {
+        using B16 = __nv_bfloat16;
+        if (video)
+            return fwd ? launch_single_reg<B16, true, true>(in, out, g, stream)
+                       : launch_single_reg<B16, true, false>(in, out, g, stream);
+        return fwd ? launch_single_reg<B16, false, true>(in, out, g, stream)
+                   : launch_single_reg<B16, false, false>(in, out, g, stream);
+    }
+    if (video)
+        return fwd ? launch_single_reg<float, true, true>(in, out, g, stream)
+                   : launch_single_reg<float, true, false>(in, out, g, stream);
+    return fwd ? launch_single_reg<float, false, true>(in, out, g, stream)
+               : launch_single_reg<float, false, false>(in, out, g, stream);
+}
+
 bool padded_extents(int64_t T, int64_t H, int64_t W, int64_t ms, int64_t mt, int64_t *Tp, int64_t *Hp, int64_t *Wp)
 {
     if (T < 1 || H < 0 || W < 0 || ms < 4 || ms % 4 != 0 || mt < 4 || mt % 4 != 0)
@@ -744,4 +895,16 @@ extern "C" tok_status tok_haar_inv_chunk(const void *y, void *x, tok_dtype dt, i
                                          int64_t H, int64_t W, int first, cudaStream_t stream)
 {
     return tok::chunk_call(false, y, x, dt, B, C, T, H, W, first, stream);
+}
+
+extern "C" tok_status tok_haar_fwd_single(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                          int64_t H, int64_t W, cudaStream_t stream)
+{
+    return tok::single_call(true, x, y, dt, B, C, T, H, W, stream);
+}
+
+extern "C" tok_status tok_haar_inv_single(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                          int64_t H, int64_t W, cudaStream_t stream)
+{
+    return tok::single_call(false, y, x, dt, B, C, T, H, W, stream);
 }

@@ -380,6 +380,179 @@ __global__ void __launch_bounds__(32)
 }
 
 // ---------------------------------------------------------------------------
+// Single-level patcher / unpatcher (patch_size=2: one DWT; guide 7.1).  Same design
+// as the two-level kernel with 2x2x2 blocks (2x2 on images): a warp tile is 64
+// horizontally adjacent blocks across (128 pixels) and 8 block rows of one (b, c, t')
+// window (16 on images), 4096 elements on either side; each lane owns blocks 2*lane
+// and 2*lane + 1 as f32x2 pairs.  Window 0 of a video reads frame 0 twice (the
+// replica) and its inverse keeps the second sample.  The three +-1 butterflies are
+// followed by one fp32 multiply by 1/(2 sqrt 2) on video (the three 1/sqrt 2 taps),
+// by the exact 1/2 on images.
+// ---------------------------------------------------------------------------
+template <bool VIDEO> struct SingleRows {
+    static constexpr int RB = VIDEO ? 8 : 16; // block rows of a tile
+};
+
+template <typename T, bool VIDEO, bool FWD>
+__global__ void __launch_bounds__(32)
+    haar_single_kernel(const __grid_constant__ CUtensorMap xmap2, const __grid_constant__ CUtensorMap xmap1,
+                       const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
+{
+    using P = WarpTiles<T>;
+    constexpr int KT = P::KT, WT = kTileBlocks;
+    constexpr int RB = SingleRows<VIDEO>::RB;
+    constexpr int G = VIDEO ? 8 : 4;
+    constexpr int NA = VIDEO ? 2 : 1;
+    constexpr int FRAME = 2 * RB * 2 * WT; // elements of one frame slice of the tile
+    static_assert(G * RB * WT == kTileElems && NA * FRAME == kTileElems, "tile sizes");
+    constexpr uint32_t TILE_BYTES = kTileElems * sizeof(T), FRAME_BYTES = FRAME * sizeof(T);
+    constexpr float SCALE = VIDEO ? 0.353553390593273762f : 0.5f;
+
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const int lane = threadIdx.x;
+    T *in_buf = reinterpret_cast<T *>(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * TILE_BYTES);
+
+    auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
+        const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
+        tx = (int)(n - q1 * tg.ntx.d);
+        ty = (int)(q1 - q2 * tg.nty.d);
+        tq = (int)(q2 - q3 * tg.nq.d);
+        bc = q3;
+    };
+
+    const uint32_t first = blockIdx.x * (uint32_t)KT;
+    const int count = (int)min((uint32_t)KT, tg.ntiles - first);
+
+    if (lane == 0) {
+        for (int s = 0; s < KT; ++s)
+            mbar_init(smem_addr(bars + s), 1);
+        fence_barrier_init();
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t bc;
+            decode(first + s, tx, ty, tq, bc);
+            const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
+            if constexpr (FWD) {
+                if (VIDEO && tq > 0) {
+                    mbar_expect_tx(bar, NA * FRAME_BYTES);
+                    tma_load_3d(dst, &xmap2, 2 * WT * tx, 2 * RB * ty, (int)(bc * tg.T + 2 * tq - 1), bar);
+                } else {
+                    mbar_expect_tx(bar, FRAME_BYTES);
+                    tma_load_3d(dst, &xmap1, 2 * WT * tx, 2 * RB * ty, (int)(bc * tg.T), bar);
+                }
+            } else {
+                const int b = (int)tg.C.div((uint32_t)bc), c = (int)(bc - (int64_t)b * tg.C.d);
+                mbar_expect_tx(bar, TILE_BYTES);
+                tma_load_5d(dst, &ymap, WT * tx, RB * ty, tq, c, G * b, bar);
+            }
+        }
+    }
+    __syncwarp();
+
+    int s = 0;
+    for (; s < count; ++s) {
+        const bool ok = mbar_wait(smem_addr(bars + s), 0u);
+        if (__any_sync(0xFFFFFFFFu, !ok))
+            break;
+        int tx, ty, tq;
+        int64_t bc;
+        decode(first + s, tx, ty, tq, bc);
+        const T *tin = in_buf + s * kTileElems;
+        const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
+        const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
+        const bool replica = VIDEO && tq == 0;
+
+#pragma unroll 2
+        for (int rb = 0; rb < RB; ++rb) {
+            float2 v[NA][2][2]; // FWD: [t][y][x] pixels -> [bt][by][bx]; INV: the reverse
+            if constexpr (FWD) {
+#pragma unroll
+                for (int a = 0; a < NA; ++a) {
+                    const int fa = replica ? 0 : a;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const T *src = tin + (fa * 2 * RB + 2 * rb + r) * 2 * WT + 4 * lane;
+                        const float2 p01 = SRow<T>::load_pair(src), p23 = SRow<T>::load_pair(src + 2);
+                        v[a][r][0] = make_float2(p01.x, p23.x); // pixel 0 of blocks j0, j0 + 1
+                        v[a][r][1] = make_float2(p01.y, p23.y); // pixel 1
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 p = SRow<T>::load_pair(tin + (g * RB + rb) * WT + 2 * lane);
+                    if constexpr (VIDEO)
+                        v[g >> 2][(g >> 1) & 1][g & 1] = p;
+                    else
+                        v[0][g >> 1][g & 1] = p;
+                }
+            }
+            // one butterfly per axis: (a + b, a - b)
+#pragma unroll
+            for (int a = 0; a < NA; ++a)
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const float2 l = add2(v[a][r][0], v[a][r][1]), hgh = sub2(v[a][r][0], v[a][r][1]);
+                    v[a][r][0] = l, v[a][r][1] = hgh;
+                }
+#pragma unroll
+            for (int a = 0; a < NA; ++a)
+#pragma unroll
+                for (int d = 0; d < 2; ++d) {
+                    const float2 l = add2(v[a][0][d], v[a][1][d]), hgh = sub2(v[a][0][d], v[a][1][d]);
+                    v[a][0][d] = l, v[a][1][d] = hgh;
+                }
+            if constexpr (VIDEO) {
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int d = 0; d < 2; ++d) {
+                        const float2 l = add2(v[0][r][d], v[1][r][d]), hgh = sub2(v[0][r][d], v[1][r][d]);
+                        v[0][r][d] = l, v[1][r][d] = hgh;
+                    }
+            }
+            const float2 scale = make_float2(SCALE, SCALE);
+            const int64_t row = (int64_t)ty * RB + rb; // block row
+            if (!col_ok || row >= tg.h)
+                continue;
+            if constexpr (FWD) {
+                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 p = VIDEO ? v[g >> 2][(g >> 1) & 1][g & 1] : v[0][g >> 1][g & 1];
+                    gstore_pair(yp + (int64_t)g * tg.C.d * plane, __fmul2_rn(p, scale));
+                }
+            } else {
+                T *xb = out + (bc * tg.T) * tg.H * tg.W + (2 * row) * tg.W + 2 * j0;
+#pragma unroll
+                for (int a = 0; a < NA; ++a) {
+                    if (replica && a != 1) // window 0 keeps its second sample (frame 0)
+                        continue;
+                    const int64_t f = !VIDEO ? 0 : replica ? 0 : 2 * tq - 1 + a;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const float2 q0 = __fmul2_rn(v[a][r][0], scale), q1 = __fmul2_rn(v[a][r][1], scale);
+                        T *dst = xb + f * tg.H * tg.W + r * tg.W;
+                        SRow<T>::store_pair(dst, make_float2(q0.x, q1.x));     // block j0: pixels 0, 1
+                        SRow<T>::store_pair(dst + 2, make_float2(q0.y, q1.y)); // block j0 + 1
+                    }
+                }
+            }
+        }
+    }
+
+    if (s < count && lane == 0) {
+        for (int r = s; r < count; ++r)
+            mbar_wait(smem_addr(bars + r), 0u);
+        atomicAdd(&g_wait_timeouts, 1u);
+    }
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
 template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
@@ -515,6 +688,94 @@ tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count
         return TOK_ERR_CUDA;
     }
     return TOK_OK;
+}
+
+} // namespace tok
+
+namespace tok {
+namespace {
+
+template <typename T, bool VIDEO, bool FWD>
+tok_status launch_single(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    using P = WarpTiles<T>;
+    constexpr int G = VIDEO ? 8 : 4, RB = SingleRows<VIDEO>::RB, WT = kTileBlocks;
+    const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const uint64_t es = sizeof(T);
+    CUtensorMap xm2, xm1, ym;
+    memset(&xm2, 0, sizeof xm2);
+    memset(&xm1, 0, sizeof xm1);
+    memset(&ym, 0, sizeof ym);
+    if (FWD) {
+        const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
+        const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
+        const uint32_t box2[3] = {2u * WT, 2u * RB, 2u}, box1[3] = {2u * WT, 2u * RB, 1u};
+        if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
+            (VIDEO && !encode_tensor_map(&xm2, dt, 3, in, xdims, xstr, box2)))
+            return TOK_ERR_SHAPE;
+    } else {
+        const uint64_t ydims[5] = {(uint64_t)d.w, (uint64_t)d.h, (uint64_t)d.Tq, (uint64_t)d.C, (uint64_t)(G * d.B)};
+        const uint64_t plane = d.Tq * d.h * d.w * es;
+        const uint64_t ystr[4] = {d.w * es, d.h * d.w * es, plane, d.C * plane};
+        const uint32_t ybox[5] = {(uint32_t)WT, (uint32_t)RB, 1u, 1u, (uint32_t)G};
+        if (!encode_tensor_map(&ym, dt, 5, in, ydims, ystr, ybox))
+            return TOK_ERR_SHAPE;
+    }
+    const int64_t ntx = (d.w + WT - 1) / WT, nty = (d.h + RB - 1) / RB;
+    TileGrid tg{};
+    tg.ntx = FastDiv((uint32_t)ntx);
+    tg.nty = FastDiv((uint32_t)nty);
+    tg.nq = FastDiv((uint32_t)d.Tq);
+    tg.C = FastDiv((uint32_t)d.C);
+    tg.T = (int)d.T;
+    tg.Tq = (int)d.Tq;
+    tg.tq0 = 0;
+    tg.H = d.H;
+    tg.W = d.W;
+    tg.h = d.h;
+    tg.w = d.w;
+    tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B * d.C);
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_single_kernel<T, VIDEO, FWD>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+    if (attr_err != cudaSuccess) {
+        record_cuda_error(attr_err);
+        return TOK_ERR_CUDA;
+    }
+    const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
+    haar_single_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm2, xm1, ym, (T *)out, tg);
+    return launch_status();
+}
+
+} // namespace
+
+bool haar_single_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
+{
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    if (!aligned(in, 16) || !aligned(out, 16) || (d.w * es) % 16 != 0 || (d.W * es) % 16 != 0)
+        return false;
+    const int64_t ntiles = ((d.w + 63) / 64) * (d.h / 8 + 1) * d.Tq * d.B * d.C;
+    if (d.B * d.C * d.T >= (int64_t)1 << 31 || 8 * d.B >= (int64_t)1 << 31 || d.W >= (int64_t)1 << 31 ||
+        d.H >= (int64_t)1 << 31 || ntiles >= (int64_t)1 << 32)
+        return false;
+    return sm_count() > 0;
+}
+
+tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d,
+                                  cudaStream_t stream)
+{
+    if (dt == TOK_BF16) {
+        using B16 = __nv_bfloat16;
+        if (d.video)
+            return fwd ? launch_single<B16, true, true>(in, out, d, stream)
+                       : launch_single<B16, true, false>(in, out, d, stream);
+        return fwd ? launch_single<B16, false, true>(in, out, d, stream)
+                   : launch_single<B16, false, false>(in, out, d, stream);
+    }
+    if (d.video)
+        return fwd ? launch_single<float, true, true>(in, out, d, stream)
+                   : launch_single<float, true, false>(in, out, d, stream);
+    return fwd ? launch_single<float, false, true>(in, out, d, stream)
+               : launch_single<float, false, false>(in, out, d, stream);
 }
 
 } // namespace tok

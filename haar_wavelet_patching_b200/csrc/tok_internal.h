@@ -30,6 +30,12 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
 tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
                            cudaStream_t stream);
 
+// Single-level patcher / unpatcher (patch_size=2): pixels [B, C, T, H, W] <->
+// coefficients [B, G*C, Tq, h, w] with G = 8 (video), 4 (images), Tq = (T + 1) / 2, h = H/2.
+bool haar_single_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
+tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d,
+                                  cudaStream_t stream);
+
 // Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
 // Haar (resp. FSQ, FSQ backward) kernels since the last call, and clear them.
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count);

@@ -171,6 +171,24 @@ TOK_API tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, in
                                         int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream);
 
 /*
+ * tok_haar_fwd_single / tok_haar_inv_single -- the single-level patcher and
+ * unpatcher (patch_size=2: one DWT; [guide] 7.1: one 2D DWT turns c channels into
+ * 4c at half size, one 3D DWT into 8c with the first frame repeated for causal
+ * alignment).  Same conventions as tok_haar_fwd for one level:
+ *   x : [B, C, T, H, W], T == 1 (image) or T odd, H and W even
+ *   y : [B, 8C, (T+1)/2, H/2, W/2] (video) or [B, 4C, 1, H/2, W/2] (image)
+ * channel s*C + c with subband s = 4*bt + 2*by + bx (2*by + bx on images), bit 1
+ * the high band (a - b)/sqrt 2 of an axis; latent frame 0 reads frame 0 twice,
+ * frame t' >= 1 reads frames 2t'-1 and 2t'; the inverse keeps the later copy of
+ * frame 0.  Two single levels (the second on all 8C channels) equal tok_haar_fwd.
+ * Errors as tok_haar_fwd (H, W even instead of multiples of 4; T odd).
+ */
+TOK_API tok_status tok_haar_fwd_single(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                       int64_t H, int64_t W, cudaStream_t stream);
+TOK_API tok_status tok_haar_inv_single(const void *y, void *x, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                       int64_t H, int64_t W, cudaStream_t stream);
+
+/*
  * Clips of any extents ([guide] 6.3: before the network a clip is padded --
  * zeros in space, reflection at the temporal edge -- to aligned extents, and the
  * result is cropped back to the original size afterwards).

@@ -184,3 +184,14 @@ def test_padded_and_chunk_rules(lib):
     assert fc(A, Bp, 1, 1, 3, 8, 62, 64, 0, NULL) == hwp.TOK_ERR_SHAPE       # H % 4
     assert fc(NULL, Bp, 1, 1, 3, 8, 64, 64, 0, NULL) == hwp.TOK_ERR_NULL
     assert iv(A, A, 1, 1, 3, 8, 64, 64, 0, NULL) == hwp.TOK_ERR_ALIAS
+
+
+def test_single_level_rules(lib):
+    fs, iv = lib.tok_haar_fwd_single, lib.tok_haar_inv_single
+    assert fs(A, Bp, 1, 1, 3, 4, 64, 64, NULL) == hwp.TOK_ERR_SHAPE    # T even
+    assert fs(A, Bp, 1, 1, 3, 5, 63, 64, NULL) == hwp.TOK_ERR_SHAPE    # H odd
+    assert fs(A, Bp, 7, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_DTYPE
+    assert fs(NULL, Bp, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_NULL
+    assert fs(A, A, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
+    assert iv(A, A, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
+    assert fs(NULL, NULL, 1, 0, 3, 5, 64, 64, NULL) == hwp.TOK_OK      # empty
