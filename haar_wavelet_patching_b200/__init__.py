@@ -25,7 +25,7 @@ FSQ_DIM = 6
 # Every symbol include/tok.h declares.
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
-               "tok_haar_inv_windows", "tok_haar_fwd_single", "tok_haar_inv_single", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
+               "tok_haar_inv_windows", "tok_haar_fwd_single", "tok_haar_inv_single", "tok_haar_fwd_channels_last", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
                "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
                "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
@@ -59,7 +59,7 @@ def lib():
         L.tok_check_device.restype = i32
         L.tok_check_device.argtypes = [vp]
         for f in (L.tok_haar_fwd, L.tok_haar_inv, L.tok_haar_fwd_adjoint, L.tok_haar_inv_adjoint,
-                  L.tok_haar_fwd_single, L.tok_haar_inv_single):
+                  L.tok_haar_fwd_single, L.tok_haar_inv_single, L.tok_haar_fwd_channels_last):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, vp]
         L.tok_fsq_backward_workspace_size.restype = i64
@@ -201,6 +201,30 @@ def tok_haar_inv_windows(y: torch.Tensor, x: torch.Tensor, t_begin: int, t_end: 
     """Inverse restricted to latent frames [t_begin, t_end): writes only those windows' pixel frames."""
     _haar_windows(False, x, y, t_begin, t_end, stream)
     return x
+
+
+def channels_last_shape(B, C, T, H, W):
+    """tok_haar_fwd_channels_last's output: [B, T', H/4, W/4, 64C] (images [B, 1, H/4, W/4, 16C])."""
+    b, k, t, h, w = haar_coeff_shape(B, C, T, H, W)
+    return (b, t, h, w, k)
+
+
+def tok_haar_fwd_channels_last(x: torch.Tensor, y: torch.Tensor, stream=None):
+    """x [B,C,T,H,W] -> y [B,T',H/4,W/4,64C]: the patcher's coefficients, channels last."""
+    _cuda(x, "x"), _cuda(y, "y")
+    if x.dim() != 5 or y.dtype != x.dtype:
+        raise ValueError("x must be [B, C, T, H, W] and y of the same dtype")
+    B, C, T, H, W = x.shape
+    if tuple(y.shape) != channels_last_shape(B, C, T, H, W):
+        raise ValueError(f"y has shape {tuple(y.shape)}, expected {channels_last_shape(B, C, T, H, W)}")
+    _check(lib().tok_haar_fwd_channels_last(_ptr(x), _ptr(y), _dtype_code(x), B, C, T, H, W, _stream(x, stream)),
+           "tok_haar_fwd_channels_last")
+    return y
+
+
+def haar_fwd_channels_last(x: torch.Tensor, stream=None) -> torch.Tensor:
+    y = torch.empty(channels_last_shape(*x.shape), dtype=x.dtype, device=x.device)
+    return tok_haar_fwd_channels_last(x, y, stream)
 
 
 def single_coeff_shape(B, C, T, H, W):

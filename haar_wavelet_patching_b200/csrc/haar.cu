@@ -788,6 +788,114 @@ tok_status single_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_
                : launch_single_reg<float, false, false>(in, out, g, stream);
 }
 
+// ---------------------------------------------------------------------------
+// Channels-last two-level patcher, register path (any C, shapes the TMA kernel
+// cannot take): one thread per block of one (b, c, t'); element loads, the 64 (16)
+// results stored at y[b][t'][i][j][g*C + c].
+// ---------------------------------------------------------------------------
+template <typename T, bool VIDEO>
+__global__ void __launch_bounds__(kThreads) haar_cl_reg_kernel(const T *__restrict__ x, T *__restrict__ y, Geometry g)
+{
+    constexpr int NA = VIDEO ? 4 : 1, G = VIDEO ? 64 : 16;
+    constexpr float SCALE = VIDEO ? 0.125f : 0.25f;
+    const int64_t item = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (item >= g.h * g.w)
+        return;
+    const int64_t i = item / g.w, j = item - i * g.w;
+    const int64_t pair = (int64_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if (pair >= g.BC * g.Tq)
+        return;
+    const int64_t bc = pair / g.Tq, tq = pair - bc * g.Tq;
+    const int64_t b = bc / g.C, c = bc - b * g.C;
+    float v[NA][4][4];
+#pragma unroll
+    for (int a = 0; a < NA; ++a) {
+        const int64_t f = (!VIDEO || tq == 0) ? 0 : 4 * tq - 3 + a;
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                v[a][r][d] = elem_to_f(x[((bc * g.T + f) * g.H + 4 * i + r) * g.W + 4 * j + d]);
+    }
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            haar4(v[a][r][0], v[a][r][1], v[a][r][2], v[a][r][3]);
+#pragma unroll
+    for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+            haar4(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
+    if constexpr (VIDEO) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int d = 0; d < 4; ++d)
+                haar4(v[0][r][d], v[1][r][d], v[2][r][d], v[3][r][d]);
+    }
+    T *yb = y + (((b * g.Tq + tq) * g.h + i) * g.w + j) * G * g.C + c;
+#pragma unroll
+    for (int grp = 0; grp < G; ++grp) {
+        const float p = VIDEO ? v[kt_of(grp)][ky_of(grp)][kx_of(grp)] : v[0][ky2_of(grp)][kx2_of(grp)];
+        yb[grp * g.C] = f_to_elem<T>(p * SCALE);
+    }
+}
+
+tok_status channels_last_call(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T, int64_t H,
+                              int64_t W, cudaStream_t stream)
+{
+    if (dt != TOK_F32 && dt != TOK_BF16)
+        return TOK_ERR_DTYPE;
+    if (B < 0 || C < 0 || T < 1 || H < 0 || W < 0 || H % 4 || W % 4 || (T != 1 && T % 4 != 1))
+        return TOK_ERR_SHAPE;
+    const bool video = T > 1;
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    Geometry g{};
+    g.C = C;
+    g.T = T;
+    g.H = H;
+    g.W = W;
+    g.Tq = video ? 1 + (T - 1) / 4 : 1;
+    g.h = H / 4;
+    g.w = W / 4;
+    g.tq0 = 0;
+    g.nq = g.Tq;
+    int64_t nx, ny, bytes_x, bytes_y;
+    if (!prod_ok({B, C}, &g.BC) || !prod_ok({g.BC, T, H, W}, &nx) || !prod_ok({nx, es}, &bytes_x) ||
+        !prod_ok({g.BC, video ? 64 : 16, g.Tq, g.h, g.w}, &ny) || !prod_ok({ny, es}, &bytes_y))
+        return TOK_ERR_SHAPE;
+    if (nx == 0)
+        return TOK_OK;
+    if (!x || !y)
+        return TOK_ERR_NULL;
+    if (!aligned(x, es) || !aligned(y, es))
+        return TOK_ERR_ALIGN;
+    if (overlaps(x, bytes_x, y, bytes_y))
+        return TOK_ERR_ALIAS;
+    HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, 0, g.Tq};
+    dims.video = video;
+    if (haar_cl_tma_eligible(x, y, dt, dims))
+        return haar_cl_tma_launch(x, y, dt, dims, stream);
+    const int64_t items = g.h * g.w, pairs = g.BC * g.Tq;
+    const int64_t gy = pairs < 65535 ? pairs : 65535, gz = (pairs + gy - 1) / gy;
+    if ((items + kThreads - 1) / kThreads > 0x7FFFFFFF || gz > 65535)
+        return TOK_ERR_SHAPE;
+    const dim3 grid((unsigned)((items + kThreads - 1) / kThreads), (unsigned)gy, (unsigned)gz);
+    if (dt == TOK_BF16) {
+        using B16 = __nv_bfloat16;
+        if (video)
+            haar_cl_reg_kernel<B16, true><<<grid, kThreads, 0, stream>>>((const B16 *)x, (B16 *)y, g);
+        else
+            haar_cl_reg_kernel<B16, false><<<grid, kThreads, 0, stream>>>((const B16 *)x, (B16 *)y, g);
+    } else if (video) {
+        haar_cl_reg_kernel<float, true><<<grid, kThreads, 0, stream>>>((const float *)x, (float *)y, g);
+    } else {
+        haar_cl_reg_kernel<float, false><<<grid, kThreads, 0, stream>>>((const float *)x, (float *)y, g);
+    }
+    return launch_status();
+}
+
 bool padded_extents(int64_t T, int64_t H, int64_t W, int64_t ms, int64_t mt, int64_t *Tp, int64_t *Hp, int64_t *Wp)
 {
     if (T < 1 || H < 0 || W < 0 || ms < 4 || ms % 4 != 0 || mt < 4 || mt % 4 != 0)
@@ -907,4 +1015,10 @@ extern "C" tok_status tok_haar_inv_single(const void *y, void *x, tok_dtype dt, 
                                           int64_t H, int64_t W, cudaStream_t stream)
 {
     return tok::single_call(false, y, x, dt, B, C, T, H, W, stream);
+}
+
+extern "C" tok_status tok_haar_fwd_channels_last(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C,
+                                                 int64_t T, int64_t H, int64_t W, cudaStream_t stream)
+{
+    return tok::channels_last_call(x, y, dt, B, C, T, H, W, stream);
 }

@@ -380,6 +380,160 @@ __global__ void __launch_bounds__(32)
 }
 
 // ---------------------------------------------------------------------------
+// Channels-last patcher: y [B, Tq, h, w, G*C] (G = 64 on video, 16 on images),
+// channel g*C + c as in the planar layout, so a block's G*C coefficients are
+// contiguous.  A tile is one block row (four on images) of 64 blocks across with
+// all NC input channels: NC TMA loads on one barrier.  Per channel, each lane
+// transforms its two blocks as in the planar kernel and, once the warp has read
+// that channel's pixels, writes the results back over them as [row][g][block]
+// pairs (4-byte shared stores, consecutive across lanes); the warp then gathers
+// each block's G*C run from the NC staged channels and writes it with 16-byte
+// global stores.
+// ---------------------------------------------------------------------------
+template <typename T, int NC> struct ClTiles {
+    static constexpr int REGION_BYTES = kTileElems * sizeof(T);
+    static constexpr int KT = (32768 / (NC * REGION_BYTES)) > 0 ? 32768 / (NC * REGION_BYTES) : 1;
+    static constexpr int SMEM = KT * NC * REGION_BYTES + 8 * KT;
+};
+
+template <typename T, bool VIDEO, int NC>
+__global__ void __launch_bounds__(32)
+    haar_cl_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
+                   T *__restrict__ out, const TileGrid tg)
+{
+    using P = ClTiles<T, NC>;
+    constexpr int KT = P::KT, WT = kTileBlocks;
+    constexpr int RW = TileRows<VIDEO>::RW;
+    constexpr int G = VIDEO ? 64 : 16;
+    constexpr int NA = VIDEO ? 4 : 1;
+    constexpr int FRAME = 16 * RW * WT;
+    constexpr uint32_t FRAME_BYTES = FRAME * sizeof(T);
+    constexpr float SCALE = VIDEO ? 0.125f : 0.25f;
+    constexpr int VEC = 16 / (int)sizeof(T); // elements per 16-byte store
+    static_assert((G * NC) % VEC == 0, "a block's run is whole 16-byte pieces");
+
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const int lane = threadIdx.x;
+    T *buf = reinterpret_cast<T *>(smem_raw);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * NC * P::REGION_BYTES);
+
+    auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &b) {
+        const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
+        tx = (int)(n - q1 * tg.ntx.d);
+        ty = (int)(q1 - q2 * tg.nty.d);
+        tq = (int)(q2 - q3 * tg.nq.d);
+        b = q3;
+    };
+
+    const uint32_t first = blockIdx.x * (uint32_t)KT;
+    const int count = (int)min((uint32_t)KT, tg.ntiles - first);
+
+    if (lane == 0) {
+        for (int s = 0; s < KT; ++s)
+            mbar_init(smem_addr(bars + s), 1);
+        fence_barrier_init();
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t b;
+            decode(first + s, tx, ty, tq, b);
+            const uint32_t bar = smem_addr(bars + s);
+            const bool full = VIDEO && tq > 0;
+            mbar_expect_tx(bar, NC * (full ? NA * FRAME_BYTES : FRAME_BYTES));
+            for (int c = 0; c < NC; ++c) {
+                const uint32_t dst = smem_addr(buf + (s * NC + c) * kTileElems);
+                const int frame0 = (int)((b * NC + c) * tg.T);
+                if (full)
+                    tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, frame0 + 4 * tq - 3, bar);
+                else
+                    tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, frame0, bar);
+            }
+        }
+    }
+    __syncwarp();
+
+    int s = 0;
+    for (; s < count; ++s) {
+        const bool ok = mbar_wait(smem_addr(bars + s), 0u);
+        if (__any_sync(0xFFFFFFFFu, !ok))
+            break;
+        int tx, ty, tq;
+        int64_t b;
+        decode(first + s, tx, ty, tq, b);
+        const int64_t j0 = (int64_t)tx * WT + 2 * lane;
+        const bool col_ok = j0 < tg.w;
+        const bool replica = VIDEO && tq == 0;
+
+#pragma unroll 1
+        for (int c = 0; c < NC; ++c) {
+            T *region = buf + (s * NC + c) * kTileElems;
+#pragma unroll
+            for (int rw = 0; rw < RW; ++rw) {
+                float2 v[NA][4][4];
+#pragma unroll
+                for (int a = 0; a < NA; ++a) {
+                    const int fa = replica ? 0 : a;
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+                        SRow<T>::load(region + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                }
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+                        haar4x2(v[a][rr][0], v[a][rr][1], v[a][rr][2], v[a][rr][3]);
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+#pragma unroll
+                    for (int d = 0; d < 4; ++d)
+                        haar4x2(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
+                if constexpr (VIDEO) {
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            haar4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
+                }
+                __syncwarp(); // this row's pixels are read: the row may now hold results
+                const float2 scale = make_float2(SCALE, SCALE);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
+                    SRow<T>::store_pair(region + (rw * G + g) * WT + 2 * lane, __fmul2_rn(p, scale));
+                }
+            }
+        }
+        __syncwarp(); // every channel is staged
+#pragma unroll
+        for (int rw = 0; rw < RW; ++rw) {
+            const int64_t row = (int64_t)ty * RW + rw;
+            if (!col_ok || row >= tg.h)
+                continue;
+            T *yb = out + (((b * tg.Tq + tq) * tg.h + row) * tg.w + j0) * (G * NC);
+#pragma unroll 4
+            for (int q = 0; q < G * NC / VEC; ++q) {
+                T e0[VEC], e1[VEC];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    const int k = q * VEC + e, g = k / NC, c = k - g * NC;
+                    const T *st = buf + (s * NC + c) * kTileElems + (rw * G + g) * WT + 2 * lane;
+                    e0[e] = st[0];
+                    e1[e] = st[1];
+                }
+                *reinterpret_cast<uint4 *>(yb + q * VEC) = *reinterpret_cast<const uint4 *>(e0);
+                *reinterpret_cast<uint4 *>(yb + G * NC + q * VEC) = *reinterpret_cast<const uint4 *>(e1);
+            }
+        }
+    }
+
+    if (s < count && lane == 0) {
+        for (int r = s; r < count; ++r)
+            mbar_wait(smem_addr(bars + r), 0u);
+        atomicAdd(&g_wait_timeouts, 1u);
+    }
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // Single-level patcher / unpatcher (patch_size=2: one DWT; guide 7.1).  Same design
 // as the two-level kernel with 2x2x2 blocks (2x2 on images): a warp tile is 64
 // horizontally adjacent blocks across (128 pixels) and 8 block rows of one (b, c, t')
@@ -776,6 +930,81 @@ tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype
                    : launch_single<float, true, false>(in, out, d, stream);
     return fwd ? launch_single<float, false, true>(in, out, d, stream)
                : launch_single<float, false, false>(in, out, d, stream);
+}
+
+} // namespace tok
+
+namespace tok {
+namespace {
+
+template <typename T, bool VIDEO, int NC>
+tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    using P = ClTiles<T, NC>;
+    constexpr int RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
+    const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const uint64_t es = sizeof(T);
+    CUtensorMap xm4, xm1;
+    memset(&xm4, 0, sizeof xm4);
+    memset(&xm1, 0, sizeof xm1);
+    const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
+    const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
+    const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
+    if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
+        (VIDEO && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
+        return TOK_ERR_SHAPE;
+    const int64_t ntx = (d.w + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
+    TileGrid tg{};
+    tg.ntx = FastDiv((uint32_t)ntx);
+    tg.nty = FastDiv((uint32_t)nty);
+    tg.nq = FastDiv((uint32_t)d.Tq);
+    tg.C = FastDiv((uint32_t)d.C);
+    tg.T = (int)d.T;
+    tg.Tq = (int)d.Tq;
+    tg.H = d.H;
+    tg.W = d.W;
+    tg.h = d.h;
+    tg.w = d.w;
+    tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B);
+    const cudaError_t attr_err =
+        cudaFuncSetAttribute(haar_cl_kernel<T, VIDEO, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+    if (attr_err != cudaSuccess) {
+        record_cuda_error(attr_err);
+        return TOK_ERR_CUDA;
+    }
+    const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
+    haar_cl_kernel<T, VIDEO, NC><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, (T *)out, tg);
+    return launch_status();
+}
+
+template <typename T, bool VIDEO>
+tok_status launch_cl_c(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    switch (d.C) {
+    case 1:
+        return launch_cl<T, VIDEO, 1>(in, out, d, stream);
+    case 2:
+        return launch_cl<T, VIDEO, 2>(in, out, d, stream);
+    case 3:
+        return launch_cl<T, VIDEO, 3>(in, out, d, stream);
+    default:
+        return launch_cl<T, VIDEO, 4>(in, out, d, stream);
+    }
+}
+
+} // namespace
+
+bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
+{
+    return d.C >= 1 && d.C <= 4 && haar_tma_eligible(in, out, dt, d);
+}
+
+tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream)
+{
+    if (dt == TOK_BF16)
+        return d.video ? launch_cl_c<__nv_bfloat16, true>(in, out, d, stream)
+                       : launch_cl_c<__nv_bfloat16, false>(in, out, d, stream);
+    return d.video ? launch_cl_c<float, true>(in, out, d, stream) : launch_cl_c<float, false>(in, out, d, stream);
 }
 
 } // namespace tok

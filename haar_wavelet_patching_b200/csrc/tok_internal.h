@@ -36,6 +36,10 @@ bool haar_single_tma_eligible(const void *in, const void *out, tok_dtype dt, con
 tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d,
                                   cudaStream_t stream);
 
+// Channels-last two-level patcher: pixels [B, C, T, H, W] -> [B, Tq, h, w, G*C] (1 <= C <= 4).
+bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
+tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream);
+
 // Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
 // Haar (resp. FSQ, FSQ backward) kernels since the last call, and clear them.
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count);

@@ -18,7 +18,7 @@ import haar_wavelet_patching_b200 as hwp
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", required=True, choices=("haar_fwd", "haar_inv", "haar_fwd_adjoint", "haar_inv_adjoint",
-                                                     "haar_fwd_single", "haar_inv_single",
+                                                     "haar_fwd_single", "haar_inv_single", "haar_fwd_channels_last",
                                                      "haar_fwd_padded", "haar_inv_cropped", "haar_fwd_chunk",
                                                      "haar_inv_chunk", "fsq_encode", "fsq_decode",
                                                      "fsq_encode_backward", "fsq_decode_backward"))
@@ -35,7 +35,12 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op in ("haar_fwd_single", "haar_inv_single"):
+    if a.op == "haar_fwd_channels_last":
+        x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
+        y = torch.empty(hwp.channels_last_shape(*shape), dtype=dt, device=dev)
+        run = lambda: hwp.tok_haar_fwd_channels_last(x, y)  # noqa: E731
+        nbytes = (x.numel() + y.numel()) * x.element_size()
+    elif a.op in ("haar_fwd_single", "haar_inv_single"):
         x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
         y = (torch.rand(hwp.single_coeff_shape(*shape), generator=g, device=dev) * 2 - 1).to(dt)
         run = (lambda: hwp.tok_haar_fwd_single(x, y)) if a.op == "haar_fwd_single" else \

@@ -171,6 +171,17 @@ TOK_API tok_status tok_haar_inv_windows(const void *y, void *x, tok_dtype dt, in
                                         int64_t H, int64_t W, int64_t t_begin, int64_t t_end, cudaStream_t stream);
 
 /*
+ * tok_haar_fwd_channels_last -- tok_haar_fwd with a channels-last output, the
+ * layout a following convolution reads its input channels from:
+ *   x : [B, C, T, H, W] as tok_haar_fwd (input)
+ *   y : [B, T', H/4, W/4, 64C] (video) or [B, 1, H/4, W/4, 16C] (image), element
+ *       [b][t'][i][j][k] = tok_haar_fwd's y[b][k][t'][i][j] (output)
+ * Not on the pages' API: a layout of the same result.  Errors as tok_haar_fwd.
+ */
+TOK_API tok_status tok_haar_fwd_channels_last(const void *x, void *y, tok_dtype dt, int64_t B, int64_t C, int64_t T,
+                                              int64_t H, int64_t W, cudaStream_t stream);
+
+/*
  * tok_haar_fwd_single / tok_haar_inv_single -- the single-level patcher and
  * unpatcher (patch_size=2: one DWT; [guide] 7.1: one 2D DWT turns c channels into
  * 4c at half size, one 3D DWT into 8c with the first frame repeated for causal

@@ -358,3 +358,9 @@ def haar_inv_chunk(y: np.ndarray, T: int, H: int, W: int, first: bool) -> np.nda
     _check(_load().oracle_haar_inv_chunk(_ptr(y, ctypes.c_double), _ptr(x, ctypes.c_double), B, C, T, H, W,
                                          int(bool(first))), "haar_inv_chunk")
     return x
+
+
+def haar_fwd_channels_last(x: np.ndarray) -> np.ndarray:
+    """The patcher's coefficients in channels-last order [B, T', h, w, 64C]: haar_fwd with the
+    channel axis moved last (a layout of the same values; numpy does the permutation)."""
+    return np.ascontiguousarray(np.moveaxis(haar_fwd(x), 1, -1))

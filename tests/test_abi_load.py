@@ -195,3 +195,13 @@ def test_single_level_rules(lib):
     assert fs(A, A, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
     assert iv(A, A, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
     assert fs(NULL, NULL, 1, 0, 3, 5, 64, 64, NULL) == hwp.TOK_OK      # empty
+
+
+def test_channels_last_rules(lib):
+    f = lib.tok_haar_fwd_channels_last
+    assert f(A, Bp, 1, 1, 3, 8, 64, 64, NULL) == hwp.TOK_ERR_SHAPE     # T % 4 != 1
+    assert f(A, Bp, 1, 1, 3, 5, 62, 64, NULL) == hwp.TOK_ERR_SHAPE     # H % 4
+    assert f(A, Bp, 9, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_DTYPE
+    assert f(NULL, Bp, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_NULL
+    assert f(A, A, 1, 1, 3, 5, 64, 64, NULL) == hwp.TOK_ERR_ALIAS
+    assert f(NULL, NULL, 1, 1, 0, 5, 64, 64, NULL) == hwp.TOK_OK         # empty

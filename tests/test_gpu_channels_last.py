@@ -1,0 +1,52 @@
+"""GPU parity of the channels-last patcher: the same coefficients as tok_haar_fwd, laid out
+[B, T', h, w, 64C].  The kernels run the same butterflies as the planar ones, so the result
+equals the planar call's output permuted, bit for bit; one case is also checked against
+the oracle with the planar tolerances."""
+import numpy as np
+import pytest
+import torch
+
+import haar_wavelet_patching_b200 as hwp
+import oracle
+import synth
+from tests.helpers import block_abs_sums, expand_to_channels, haar_bf16_tolerance, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    ((1, 3, 9, 32, 64), torch.bfloat16, "TMA, C = 3"),
+    ((2, 1, 5, 16, 96), torch.bfloat16, "TMA, C = 1, partial tile"),
+    ((1, 2, 13, 20, 64), torch.float32, "TMA fp32, C = 2"),
+    ((1, 4, 5, 8, 32), torch.bfloat16, "TMA, C = 4"),
+    ((2, 3, 1, 36, 64), torch.bfloat16, "TMA image, partial block rows"),
+    ((1, 5, 9, 16, 64), torch.bfloat16, "register, C = 5"),
+    ((1, 3, 9, 12, 44), torch.float32, "register, ragged row"),
+    ((1, 2, 1, 8, 20), torch.bfloat16, "register image"),
+]
+
+
+@pytest.mark.parametrize("shape,dtype,note", CASES, ids=[c[2] for c in CASES])
+def test_channels_last_is_the_planar_result_permuted(shape, dtype, note):
+    x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
+    y_cl = hwp.haar_fwd_channels_last(x)
+    hwp.tok_check_device()
+    assert torch.equal(y_cl, hwp.haar_fwd(x).permute(0, 2, 3, 4, 1))
+
+
+def test_channels_last_matches_oracle():
+    shape = (1, 3, 9, 32, 64)
+    x_np = synth.uniform(shape, seed=17, dtype=synth.BF16)
+    x64 = synth.to_f64(x_np, synth.BF16)
+    got = to_f64(hwp.haar_fwd_channels_last(to_device(x_np, synth.BF16)))
+    ref = oracle.haar_fwd_channels_last(x64)
+    tol = np.moveaxis(haar_bf16_tolerance(oracle.haar_fwd(x64), expand_to_channels(block_abs_sums(x64), 64), True),
+                      1, -1)
+    assert got.shape == ref.shape and (np.abs(got - ref) <= tol).all()
+
+
+def test_channels_last_bad_arguments_raise():
+    with pytest.raises(ValueError):
+        hwp.tok_haar_fwd_channels_last(torch.zeros(1, 3, 9, 32, 64, device="cuda"),
+                                       torch.zeros(1, 192, 3, 8, 16, device="cuda"))
+    with pytest.raises((ValueError, hwp.TokError)):  # T % 4 != 1: the shape helper or the library refuses
+        hwp.haar_fwd_channels_last(torch.zeros(1, 3, 8, 32, 64, device="cuda"))
