@@ -26,7 +26,8 @@ FSQ_DIM = 6
 ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
                "tok_haar_inv_windows", "tok_haar_fwd_single", "tok_haar_inv_single", "tok_haar_fwd_channels_last", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
-               "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
+               "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_conv_spatial", "tok_conv_temporal_causal",
+               "tok_conv_factorized", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
                "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
 _lib = None
@@ -81,6 +82,11 @@ def lib():
         for f in (L.tok_haar_fwd_chunk, L.tok_haar_inv_chunk):
             f.restype = i32
             f.argtypes = [vp, vp, i32, i64, i64, i64, i64, i64, i32, vp]
+        for f in (L.tok_conv_spatial, L.tok_conv_temporal_causal):
+            f.restype = i32
+            f.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp]
+        L.tok_conv_factorized.restype = i32
+        L.tok_conv_factorized.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp]
         L.tok_fsq_encode.restype = i32
         L.tok_fsq_encode.argtypes = [vp, vp, vp, vp, i64, i64, i64, vp]
         L.tok_fsq_decode.restype = i32
@@ -325,6 +331,57 @@ def tok_haar_fwd_chunk(x: torch.Tensor, y: torch.Tensor, first: bool, stream=Non
 def tok_haar_inv_chunk(y: torch.Tensor, x: torch.Tensor, first: bool, stream=None):
     _haar_chunk(False, x, y, first, stream)
     return x
+
+
+def _conv_dims(x, name):
+    _cuda(x, name)
+    if x.dim() != 5 or x.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be a channels-last bf16 tensor [B, T, h, w, C]")
+    return x.shape
+
+
+def tok_conv_spatial(x: torch.Tensor, ws: torch.Tensor, y: torch.Tensor, stream=None):
+    """1 x k x k convolution, 'same' zero padding: x [B,T,h,w,Cin], ws [Cout,k,k,Cin] -> y [B,T,h,w,Cout]."""
+    B, T, h, w, Cin = _conv_dims(x, "x")
+    _conv_dims(y, "y"), _cuda(ws, "ws")
+    Cout, k = ws.shape[0], ws.shape[1]
+    if tuple(ws.shape) != (Cout, k, k, Cin) or tuple(y.shape) != (B, T, h, w, Cout) or ws.dtype != torch.bfloat16:
+        raise ValueError("ws must be bf16 [Cout, k, k, Cin] and y [B, T, h, w, Cout]")
+    _check(lib().tok_conv_spatial(_ptr(x), _ptr(ws), _ptr(y), B, T, h, w, Cin, Cout, k, _stream(x, stream)),
+           "tok_conv_spatial")
+    return y
+
+
+def tok_conv_temporal_causal(x: torch.Tensor, wt: torch.Tensor, y: torch.Tensor, stream=None):
+    """k x 1 x 1 convolution over time, frame t reading t-k+1 .. t: wt [Cout, k, Cin]."""
+    B, T, h, w, Cin = _conv_dims(x, "x")
+    _conv_dims(y, "y"), _cuda(wt, "wt")
+    Cout, k = wt.shape[0], wt.shape[1]
+    if tuple(wt.shape) != (Cout, k, Cin) or tuple(y.shape) != (B, T, h, w, Cout) or wt.dtype != torch.bfloat16:
+        raise ValueError("wt must be bf16 [Cout, k, Cin] and y [B, T, h, w, Cout]")
+    _check(lib().tok_conv_temporal_causal(_ptr(x), _ptr(wt), _ptr(y), B, T, h, w, Cin, Cout, k,
+                                          _stream(x, stream)), "tok_conv_temporal_causal")
+    return y
+
+
+def tok_conv_factorized(x, ws, wt, mid, y, stream=None):
+    """The spatial convolution into mid, then the causal temporal convolution into y."""
+    B, T, h, w, Cin = _conv_dims(x, "x")
+    _conv_dims(mid, "mid"), _conv_dims(y, "y"), _cuda(ws, "ws"), _cuda(wt, "wt")
+    Cmid, k, Cout = ws.shape[0], ws.shape[1], wt.shape[0]
+    if (tuple(ws.shape) != (Cmid, k, k, Cin) or tuple(wt.shape) != (Cout, k, Cmid)
+            or tuple(mid.shape) != (B, T, h, w, Cmid) or tuple(y.shape) != (B, T, h, w, Cout)):
+        raise ValueError("shapes: ws [Cmid,k,k,Cin], wt [Cout,k,Cmid], mid [B,T,h,w,Cmid], y [B,T,h,w,Cout]")
+    _check(lib().tok_conv_factorized(_ptr(x), _ptr(ws), _ptr(wt), _ptr(mid), _ptr(y), B, T, h, w, Cin, Cmid, Cout,
+                                     k, _stream(x, stream)), "tok_conv_factorized")
+    return y
+
+
+def conv_factorized(x, ws, wt, stream=None):
+    B, T, h, w, _ = x.shape
+    mid = torch.empty((B, T, h, w, ws.shape[0]), dtype=torch.bfloat16, device=x.device)
+    y = torch.empty((B, T, h, w, wt.shape[0]), dtype=torch.bfloat16, device=x.device)
+    return tok_conv_factorized(x, ws, wt, mid, y, stream)
 
 
 def tok_haar_fwd_adjoint(gy: torch.Tensor, gx: torch.Tensor, stream=None):

@@ -29,21 +29,48 @@ def _nvcc():
     return "nvcc"
 
 
+# Files whose kernels come from CUTLASS's sm100 templates (header-only, vendored in the image).
+CUTLASS_SOURCES = ("conv.cu",)
+
+
+def cutlass_includes():
+    """Include directories of the CUTLASS tree vendored with flashinfer in this image."""
+    import importlib.util
+    spec = importlib.util.find_spec("flashinfer")
+    roots = [os.path.join(os.path.dirname(spec.origin), "data", "cutlass")] if spec and spec.origin else []
+    for root in roots:
+        inc, util = os.path.join(root, "include"), os.path.join(root, "tools", "util", "include")
+        if os.path.exists(os.path.join(inc, "cutlass", "conv", "collective", "builders", "sm100_umma_builder.inl")):
+            return [inc, util]
+    raise RuntimeError("CUTLASS headers with the sm100 convolution builders were not found")
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    deps = sources + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
-    if not force and os.path.exists(TARGET) and os.path.getmtime(TARGET) >= max(os.path.getmtime(d) for d in deps):
-        return TARGET
+    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
+        glob.glob(os.path.join(INCLUDE, "*.h"))
+    newest_header = max(os.path.getmtime(d) for d in headers)
     os.makedirs(BUILD, exist_ok=True)
     nvcc = _nvcc()
-    objs = []
+    objs, rebuilt = [], False
     for src in sources:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        objs.append(obj)
+        if not force and os.path.exists(obj) and \
+                os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header):
+            continue
         cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+        if os.path.basename(src) in CUTLASS_SOURCES:
+            for inc in cutlass_includes():
+                cmd += ["-I", inc]
+            cmd += ["-diag-suppress", "20012"]  # CUTLASS's defaulted host-device constructors
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)
-        objs.append(obj)
+        rebuilt = True
+    if not rebuilt and os.path.exists(TARGET) and \
+            os.path.getmtime(TARGET) >= max(os.path.getmtime(o) for o in objs):
+        return TARGET
     subprocess.run([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static",
                     "-o", TARGET + ".tmp", *objs], check=True)
     os.replace(TARGET + ".tmp", TARGET)

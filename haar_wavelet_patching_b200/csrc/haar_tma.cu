@@ -511,16 +511,34 @@ __global__ void __launch_bounds__(32)
             T *yb = out + (((b * tg.Tq + tq) * tg.h + row) * tg.w + j0) * (G * NC);
 #pragma unroll 4
             for (int q = 0; q < G * NC / VEC; ++q) {
-                T e0[VEC], e1[VEC];
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
+                // Each staged pair holds (block j0, block j0 + 1) of one channel k = g*NC + c.
+                auto staged = [&](int e) {
                     const int k = q * VEC + e, g = k / NC, c = k - g * NC;
-                    const T *st = buf + (s * NC + c) * kTileElems + (rw * G + g) * WT + 2 * lane;
-                    e0[e] = st[0];
-                    e1[e] = st[1];
+                    return buf + (s * NC + c) * kTileElems + (rw * G + g) * WT + 2 * lane;
+                };
+                uint4 r0, r1;
+                if constexpr (sizeof(T) == 2) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        w[e] = *reinterpret_cast<const uint32_t *>(staged(e));
+                    // low halves: block j0; high halves: block j0 + 1
+                    r0 = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
+                                    __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
+                    r1 = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
+                                    __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                } else {
+                    float2 p[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        p[e] = *reinterpret_cast<const float2 *>(staged(e));
+                    r0 = make_uint4(__float_as_uint(p[0].x), __float_as_uint(p[1].x), __float_as_uint(p[2].x),
+                                    __float_as_uint(p[3].x));
+                    r1 = make_uint4(__float_as_uint(p[0].y), __float_as_uint(p[1].y), __float_as_uint(p[2].y),
+                                    __float_as_uint(p[3].y));
                 }
-                *reinterpret_cast<uint4 *>(yb + q * VEC) = *reinterpret_cast<const uint4 *>(e0);
-                *reinterpret_cast<uint4 *>(yb + G * NC + q * VEC) = *reinterpret_cast<const uint4 *>(e1);
+                *reinterpret_cast<uint4 *>(yb + q * VEC) = r0;
+                *reinterpret_cast<uint4 *>(yb + G * NC + q * VEC) = r1;
             }
         }
     }

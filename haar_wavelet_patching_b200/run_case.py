@@ -21,8 +21,10 @@ def main():
                                                      "haar_fwd_single", "haar_inv_single", "haar_fwd_channels_last",
                                                      "haar_fwd_padded", "haar_inv_cropped", "haar_fwd_chunk",
                                                      "haar_inv_chunk", "fsq_encode", "fsq_decode",
-                                                     "fsq_encode_backward", "fsq_decode_backward"))
-    ap.add_argument("--shape", required=True, help="B,C,T,H,W for haar ops; B,C,S for fsq ops")
+                                                     "fsq_encode_backward", "fsq_decode_backward",
+                                                     "conv_spatial", "conv_temporal", "conv_factorized"))
+    ap.add_argument("--shape", required=True,
+                    help="B,C,T,H,W for haar ops; B,C,S for fsq ops; B,T,h,w,Cin,Cmid,Cout for conv ops")
     ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--codes", action="store_true", help="fsq_encode: also write the codes")
@@ -35,7 +37,26 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op == "haar_fwd_channels_last":
+    if a.op.startswith("conv"):
+        B, T, h, w, Cin, Cmid, Cout = shape
+        bf = torch.bfloat16
+        x = (torch.randn((B, T, h, w, Cin), generator=g, device=dev) * 0.5).to(bf)
+        ws = (torch.randn((Cmid, 3, 3, Cin), generator=g, device=dev) * (9 * Cin) ** -0.5).to(bf)
+        wt = (torch.randn((Cout, 3, Cmid), generator=g, device=dev) * (3 * Cmid) ** -0.5).to(bf)
+        mid = torch.empty((B, T, h, w, Cmid), dtype=bf, device=dev)
+        y = torch.empty((B, T, h, w, Cout), dtype=bf, device=dev)
+        pos = B * T * h * w
+        if a.op == "conv_spatial":
+            run = lambda: hwp.tok_conv_spatial(x, ws, mid)  # noqa: E731
+            flops, nbytes = 2 * pos * Cmid * 9 * Cin, (x.numel() + mid.numel() + ws.numel()) * 2
+        elif a.op == "conv_temporal":
+            run = lambda: hwp.tok_conv_temporal_causal(mid, wt, y)  # noqa: E731
+            flops, nbytes = 2 * pos * Cout * 3 * Cmid, (mid.numel() + y.numel() + wt.numel()) * 2
+        else:
+            run = lambda: hwp.tok_conv_factorized(x, ws, wt, mid, y)  # noqa: E731
+            flops = 2 * pos * (Cmid * 9 * Cin + Cout * 3 * Cmid)
+            nbytes = (x.numel() + 2 * mid.numel() + y.numel() + ws.numel() + wt.numel()) * 2
+    elif a.op == "haar_fwd_channels_last":
         x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
         y = torch.empty(hwp.channels_last_shape(*shape), dtype=dt, device=dev)
         run = lambda: hwp.tok_haar_fwd_channels_last(x, y)  # noqa: E731
@@ -102,7 +123,8 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.iters
-    print(f"{a.op} {shape} {a.dtype}: {ms * 1e3:.1f} us per launch, {nbytes / ms / 1e6:.1f} GB/s")
+    extra = f", {flops / ms / 1e9:.1f} TFLOP/s" if a.op.startswith("conv") else ""
+    print(f"{a.op} {shape} {a.dtype}: {ms * 1e3:.1f} us per launch, {nbytes / ms / 1e6:.1f} GB/s{extra}")
 
 
 if __name__ == "__main__":

@@ -262,6 +262,34 @@ TOK_API tok_status tok_haar_inv_chunk(const void *y, void *x, tok_dtype dt, int6
                                       int64_t H, int64_t W, int first, cudaStream_t stream);
 
 /*
+ * The first causal factorized convolution after the patcher ([notes] model
+ * architecture item 1: a 1 x k x k spatial convolution, then a k x 1 x 1 temporal
+ * convolution padded by k - 1 on the past side only), on the tensor cores:
+ * channels-last bf16 activations, bf16 weights, fp32 accumulation, bf16 results.
+ * Cross-correlation (no kernel flip), no bias.  Channel counts are multiples of 8
+ * (at least 8); all pointers are 16-byte aligned device memory.  Errors:
+ * TOK_ERR_SHAPE (channels, k, or 32-bit extents), TOK_ERR_NULL, TOK_ERR_ALIGN,
+ * TOK_ERR_ALIAS (an input overlaps the output), TOK_ERR_CUDA.  Not on the pages'
+ * API: the layer the pages name, with weights the caller provides.
+ *
+ * tok_conv_spatial -- y[b,t,i,j,n] = sum_{dy,dx,c} ws[n][dy][dx][c] *
+ *   x[b, t, i+dy-(k-1)/2, j+dx-(k-1)/2, c], zero outside the frame; k odd.
+ *   x [B, T, h, w, Cin], ws [Cout, k, k, Cin], y [B, T, h, w, Cout].
+ * tok_conv_temporal_causal -- y[b,t,i,j,n] = sum_{dt,c} wt[n][dt][c] *
+ *   x[b, t-(k-1)+dt, i, j, c], zero before frame 0 (output frame t reads frames
+ *   t-k+1 .. t).  x [B, T, h, w, Cin], wt [Cout, k, Cin], y [B, T, h, w, Cout].
+ * tok_conv_factorized -- tok_conv_spatial into the caller's mid [B, T, h, w, Cmid]
+ *   (overwritten), then tok_conv_temporal_causal into y.
+ */
+TOK_API tok_status tok_conv_spatial(const void *x, const void *ws, void *y, int64_t B, int64_t T, int64_t h,
+                                    int64_t w, int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream);
+TOK_API tok_status tok_conv_temporal_causal(const void *x, const void *wt, void *y, int64_t B, int64_t T, int64_t h,
+                                            int64_t w, int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream);
+TOK_API tok_status tok_conv_factorized(const void *x, const void *ws, const void *wt, void *mid, void *y, int64_t B,
+                                       int64_t T, int64_t h, int64_t w, int64_t Cin, int64_t Cmid, int64_t Cout,
+                                       int64_t k, cudaStream_t stream);
+
+/*
  * tok_fsq_encode -- fused 1x1 projection + FSQ quantization + index pack.
  * [guide] 7.2 (bound with tanh, rounding, levels [8,8,8,5,5,5], implicit
  * codebook of 64000, mixed-radix codes_to_indices), [guide] 6.2 (indices
