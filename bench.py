@@ -400,6 +400,46 @@ def time_single(torch, hwp, stream, x, dev, iters=GRAD_ITERS):
     return out
 
 
+CONV_CH = (256, 256)  # C_mid, C_out of the factorized convolution after the patcher (k = 3)
+
+
+def time_patch_embed(torch, hwp, stream, x, dev, iters=10):
+    """The patcher's channels-last output feeding the first causal factorized convolution
+    (1x3x3 then 3x1x1 causal) on the headline clip, each call timed alone: flops of the two
+    implicit GEMMs, 2 * positions * (C_mid * 9 * C_in + C_out * 3 * C_mid)."""
+    B, C, T, H, W = x.shape
+    Cmid, Cout = CONV_CH
+    y_cl = torch.empty(hwp.channels_last_shape(B, C, T, H, W), dtype=torch.bfloat16, device=dev)
+    Bq, Tq, h, w, Cin = y_cl.shape
+    g = torch.Generator(device=dev).manual_seed(13)
+    ws = (torch.randn((Cmid, 3, 3, Cin), generator=g, device=dev) * (9 * Cin) ** -0.5).to(torch.bfloat16)
+    wt = (torch.randn((Cout, 3, Cmid), generator=g, device=dev) * (3 * Cmid) ** -0.5).to(torch.bfloat16)
+    mid = torch.empty((Bq, Tq, h, w, Cmid), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((Bq, Tq, h, w, Cout), dtype=torch.bfloat16, device=dev)
+    pos = Bq * Tq * h * w
+    calls = {
+        "haar_fwd_channels_last": (lambda: hwp.tok_haar_fwd_channels_last(x, y_cl), 0,
+                                   (x.numel() + y_cl.numel()) * 2, 1),
+        "conv_spatial": (lambda: hwp.tok_conv_spatial(y_cl, ws, mid), 2 * pos * Cmid * 9 * Cin,
+                         (y_cl.numel() + mid.numel()) * 2, 1),
+        "conv_temporal_causal": (lambda: hwp.tok_conv_temporal_causal(mid, wt, out), 2 * pos * Cout * 3 * Cmid,
+                                 (mid.numel() + out.numel()) * 2, 1),
+    }
+    res = {}
+    for name, (call, flops, nbytes, launches) in calls.items():
+        call()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(iters):
+            call()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        res[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "flops": flops, "bytes": nbytes}
+    del y_cl, mid, out
+    return res
+
+
 def time_streaming(torch, hwp, stream, dev, iters=GRAD_ITERS):
     """The arbitrary-extent and streaming calls on a 120-frame 720p clip (bf16), each timed alone
     like the gradients: the padded patcher / cropped unpatcher (spatial multiple 16, temporal 8:
@@ -430,6 +470,32 @@ def time_streaming(torch, hwp, stream, dev, iters=GRAD_ITERS):
         e1.record(stream)
         torch.cuda.synchronize()
         out[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "bytes": nbytes, "launches": 1}
+    return out
+
+
+def tensor_peak():
+    """(burst, sustained) bf16 TFLOP/s from MEASURED_PEAKS.json, else the recipe's fallback."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, 1400.0, "fallback"
+
+
+def patch_embed_report(embed, hbm_peak):
+    burst, sustained, kind = tensor_peak()
+    out = {"channels": {"C_in": 192, "C_mid": CONV_CH[0], "C_out": CONV_CH[1], "k": 3},
+           "tensor_peak_tflops": burst, "tensor_peak_sustained_tflops": sustained, "peak_source": kind}
+    for n, g in embed.items():
+        e = {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1)}
+        if g["flops"]:
+            tf = g["flops"] / (g["ms"] / 1e3) / 1e12
+            e.update({"TFLOP/s": round(tf, 1), "frac_of_tensor_peak": round(tf / burst, 4),
+                      "frac_of_sustained": round(tf / sustained, 4), "flops": g["flops"]})
+        else:
+            e["frac_of_hbm_peak"] = round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / hbm_peak, 4)
+        out[n] = e
     return out
 
 
@@ -537,6 +603,7 @@ def run_ours(args, rank, world, local_rank):
     grads = time_gradients(torch, hwp, stream, x, y, xr, u, idx, ur, w_dev, dev)
     streaming = time_streaming(torch, hwp, stream, dev)
     single = time_single(torch, hwp, stream, x, dev)
+    embed = time_patch_embed(torch, hwp, stream, x, dev)
     barrier()
 
     if rank != 0:
@@ -578,6 +645,7 @@ def run_ours(args, rank, world, local_rank):
         "single_level": {n: {"ms": round(g["ms"], 4), "GB/s": round(g["bytes"] / (g["ms"] / 1e3) / 1e9, 1),
                              "frac_of_peak": round(g["bytes"] / (g["ms"] / 1e3) / 1e9 / peak, 4),
                              "bytes": g["bytes"]} for n, g in single.items()},
+        "patch_embed": patch_embed_report(embed, peak),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
