@@ -386,12 +386,17 @@ __global__ void __launch_bounds__(32)
 // all NC input channels: NC TMA loads on one barrier.  Per channel, each lane
 // transforms its two blocks as in the planar kernel and, once the warp has read
 // that channel's pixels, writes the results back over them as [row][g][block]
-// pairs (4-byte shared stores, consecutive across lanes); the warp then gathers
-// each block's G*C run from the NC staged channels and writes it with 16-byte
-// global stores.
+// pairs, rows padded to 66 elements (4-byte shared stores, consecutive across
+// lanes).  The copy-out gives each lane a (block pair, 16-byte piece of the run):
+// consecutive lanes take consecutive pieces, so a warp's store covers about two
+// contiguous runs instead of 32 scattered sectors, and the padding puts the pieces'
+// different (g, c) sources in different banks.
 // ---------------------------------------------------------------------------
+constexpr int kClPitch = 66; // staged row length in elements (64 blocks + 2 of padding)
+
 template <typename T, int NC> struct ClTiles {
-    static constexpr int REGION_BYTES = kTileElems * sizeof(T);
+    static constexpr int REGION_ELEMS = 64 * kClPitch; // >= kTileElems; a multiple of 128 bytes
+    static constexpr int REGION_BYTES = REGION_ELEMS * sizeof(T);
     static constexpr int KT = (32768 / (NC * REGION_BYTES)) > 0 ? 32768 / (NC * REGION_BYTES) : 1;
     static constexpr int SMEM = KT * NC * REGION_BYTES + 8 * KT;
 };
@@ -440,7 +445,7 @@ __global__ void __launch_bounds__(32)
             const bool full = VIDEO && tq > 0;
             mbar_expect_tx(bar, NC * (full ? NA * FRAME_BYTES : FRAME_BYTES));
             for (int c = 0; c < NC; ++c) {
-                const uint32_t dst = smem_addr(buf + (s * NC + c) * kTileElems);
+                const uint32_t dst = smem_addr(buf + (s * NC + c) * P::REGION_ELEMS);
                 const int frame0 = (int)((b * NC + c) * tg.T);
                 if (full)
                     tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, frame0 + 4 * tq - 3, bar);
@@ -459,15 +464,16 @@ __global__ void __launch_bounds__(32)
         int tx, ty, tq;
         int64_t b;
         decode(first + s, tx, ty, tq, b);
-        const int64_t j0 = (int64_t)tx * WT + 2 * lane;
-        const bool col_ok = j0 < tg.w;
         const bool replica = VIDEO && tq == 0;
 
 #pragma unroll 1
         for (int c = 0; c < NC; ++c) {
-            T *region = buf + (s * NC + c) * kTileElems;
+            T *region = buf + (s * NC + c) * P::REGION_ELEMS;
+            // Block rows in descending order: with the padded rows, the results of block row rw
+            // reach past its own pixels into those of rows above it, which are then already read.
 #pragma unroll
-            for (int rw = 0; rw < RW; ++rw) {
+            for (int rr_ = 0; rr_ < RW; ++rr_) {
+                const int rw = RW - 1 - rr_;
                 float2 v[NA][4][4];
 #pragma unroll
                 for (int a = 0; a < NA; ++a) {
@@ -498,47 +504,51 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
-                    SRow<T>::store_pair(region + (rw * G + g) * WT + 2 * lane, __fmul2_rn(p, scale));
+                    SRow<T>::store_pair(region + (rw * G + g) * kClPitch + 2 * lane, __fmul2_rn(p, scale));
                 }
             }
         }
         __syncwarp(); // every channel is staged
-#pragma unroll
+        constexpr int PIECES = G * NC / VEC; // 16-byte pieces of one block's run
+        const int64_t nblk = min((int64_t)WT, tg.w - (int64_t)tx * WT); // even: w is
+#pragma unroll 1
         for (int rw = 0; rw < RW; ++rw) {
             const int64_t row = (int64_t)ty * RW + rw;
-            if (!col_ok || row >= tg.h)
+            if (row >= tg.h)
                 continue;
-            T *yb = out + (((b * tg.Tq + tq) * tg.h + row) * tg.w + j0) * (G * NC);
-#pragma unroll 4
-            for (int q = 0; q < G * NC / VEC; ++q) {
-                // Each staged pair holds (block j0, block j0 + 1) of one channel k = g*NC + c.
+            T *yrow = out + (((b * tg.Tq + tq) * tg.h + row) * tg.w + (int64_t)tx * WT) * (G * NC);
+            const int total = (int)(nblk / 2) * PIECES; // (block pair, piece) items
+#pragma unroll 2
+            for (int it = lane; it < total; it += 32) {
+                const int pr = it / PIECES, q = it - pr * PIECES; // block pair, piece
                 auto staged = [&](int e) {
                     const int k = q * VEC + e, g = k / NC, c = k - g * NC;
-                    return buf + (s * NC + c) * kTileElems + (rw * G + g) * WT + 2 * lane;
+                    return buf + (s * NC + c) * P::REGION_ELEMS + (rw * G + g) * kClPitch + 2 * pr;
                 };
                 uint4 r0, r1;
                 if constexpr (sizeof(T) == 2) {
-                    uint32_t w[8];
+                    uint32_t wv[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        w[e] = *reinterpret_cast<const uint32_t *>(staged(e));
-                    // low halves: block j0; high halves: block j0 + 1
-                    r0 = make_uint4(__byte_perm(w[0], w[1], 0x5410), __byte_perm(w[2], w[3], 0x5410),
-                                    __byte_perm(w[4], w[5], 0x5410), __byte_perm(w[6], w[7], 0x5410));
-                    r1 = make_uint4(__byte_perm(w[0], w[1], 0x7632), __byte_perm(w[2], w[3], 0x7632),
-                                    __byte_perm(w[4], w[5], 0x7632), __byte_perm(w[6], w[7], 0x7632));
+                        wv[e] = *reinterpret_cast<const uint32_t *>(staged(e));
+                    // low halves: block 2*pr; high halves: block 2*pr + 1
+                    r0 = make_uint4(__byte_perm(wv[0], wv[1], 0x5410), __byte_perm(wv[2], wv[3], 0x5410),
+                                    __byte_perm(wv[4], wv[5], 0x5410), __byte_perm(wv[6], wv[7], 0x5410));
+                    r1 = make_uint4(__byte_perm(wv[0], wv[1], 0x7632), __byte_perm(wv[2], wv[3], 0x7632),
+                                    __byte_perm(wv[4], wv[5], 0x7632), __byte_perm(wv[6], wv[7], 0x7632));
                 } else {
-                    float2 p[4];
+                    float2 pv[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        p[e] = *reinterpret_cast<const float2 *>(staged(e));
-                    r0 = make_uint4(__float_as_uint(p[0].x), __float_as_uint(p[1].x), __float_as_uint(p[2].x),
-                                    __float_as_uint(p[3].x));
-                    r1 = make_uint4(__float_as_uint(p[0].y), __float_as_uint(p[1].y), __float_as_uint(p[2].y),
-                                    __float_as_uint(p[3].y));
+                        pv[e] = *reinterpret_cast<const float2 *>(staged(e));
+                    r0 = make_uint4(__float_as_uint(pv[0].x), __float_as_uint(pv[1].x), __float_as_uint(pv[2].x),
+                                    __float_as_uint(pv[3].x));
+                    r1 = make_uint4(__float_as_uint(pv[0].y), __float_as_uint(pv[1].y), __float_as_uint(pv[2].y),
+                                    __float_as_uint(pv[3].y));
                 }
-                *reinterpret_cast<uint4 *>(yb + q * VEC) = r0;
-                *reinterpret_cast<uint4 *>(yb + G * NC + q * VEC) = r1;
+                T *dst = yrow + (int64_t)(2 * pr) * (G * NC) + q * VEC;
+                *reinterpret_cast<uint4 *>(dst) = r0;
+                *reinterpret_cast<uint4 *>(dst + G * NC) = r1;
             }
         }
     }
