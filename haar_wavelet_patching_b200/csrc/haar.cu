@@ -436,8 +436,9 @@ tok_status haar_call(bool fwd, bool adj, const void *in, void *out, tok_dtype dt
 
     HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, g.tq0, g.nq};
     dims.video = T > 1;
-    if (haar_tma_eligible(in, out, dt, dims))
-        return haar_tma_launch(fwd, adj, in, out, dt, dims, stream);
+    const HaarTmaForm form = haar_tma_form(fwd, in, out, dt, dims);
+    if (form != HaarTmaForm::none)
+        return haar_tma_launch(fwd, adj, form, in, out, dt, dims, stream);
 
     // Register path: any 4-aligned W and element-aligned pointers.
     const bool a16 = aligned(in, 16) && aligned(out, 16);
@@ -624,8 +625,9 @@ tok_status haar_ext_call(bool fwd, const void *in, void *out, tok_dtype dt, int6
     dims.rep = rep;
     dims.video = video;
     dims.ext = true;
-    if (haar_tma_eligible(in, out, dt, dims))
-        return haar_tma_launch(fwd, false, in, out, dt, dims, stream);
+    const HaarTmaForm form = haar_tma_form(fwd, in, out, dt, dims);
+    if (form != HaarTmaForm::none)
+        return haar_tma_launch(fwd, false, form, in, out, dt, dims, stream);
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (video)

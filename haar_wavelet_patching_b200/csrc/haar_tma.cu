@@ -63,6 +63,7 @@ struct TileGrid {
     // The pixel tensor [T][H][W] may be smaller than the 4h x 4w blocks: the forward
     // reads zeros there (TMA fill), the inverse does not write there.
     int fbase, rep;
+    int64_t n_src; // elements of the source tensor (the row form stops its copies at its end)
 };
 
 // Source frame of frame f of a T-frame clip mirrored about its last frame (period 2(T-1)).
@@ -162,6 +163,166 @@ __device__ __forceinline__ void gstore_row(float *p, const float2 *v)
     *reinterpret_cast<float4 *>(p + 4) = make_float4(v[0].y, v[1].y, v[2].y, v[3].y);
 }
 
+// ---------------------------------------------------------------------------
+// Row form.  When the source's rows are not whole 16-byte units, a tile cannot be one
+// TMA box (a tensor map needs 16-byte strides): its rows start at arbitrary 2- or
+// 4-byte offsets.  The row form stages each source row of the tile with one bulk copy
+// (cp.async.bulk: 16-byte-aligned addresses and size, no tensor map) from the 16-byte
+// boundary at or below the row, with 16 bytes of slack, records the row's offset in
+// its staged copy, and reads it back realigned.  The copy stops at the tensor's end
+// (the issuing lane copies a last partial 16 bytes element by element).  Stores pick
+// their width from the destination address at run time.
+// ---------------------------------------------------------------------------
+template <typename T, bool FWD, bool ROWS> struct TileSmem {
+    static constexpr int KT = WarpTiles<T>::KT;
+    static constexpr int NR = FWD ? 16 : 64;                              // staged rows of a tile
+    static constexpr int ROW = (FWD ? 256 : 64) * (int)sizeof(T) + 16;     // a source row and its slack
+    static constexpr int TILE = ROWS ? NR * ROW : kTileElems * (int)sizeof(T);
+    static constexpr int SMEM = KT * TILE + 8 * KT + (ROWS ? 64 * KT : 0); // tiles, barriers, row offsets
+    static_assert(ROW % 16 == 0 && TILE % 16 == 0, "16-byte bulk-copy destinations");
+};
+constexpr unsigned char kRowSkipped = 0xFF; // a staged row that was not loaded (past the tensor edge)
+
+// 16 bytes at byte offset o (even) of a 16-byte-aligned staged row.  The branch on o's
+// alignment is uniform across a warp (lanes differ by multiples of 16 bytes).
+__device__ __forceinline__ uint4 lds16_at(const unsigned char *row, uint32_t o)
+{
+    if ((o & 15) == 0)
+        return *reinterpret_cast<const uint4 *>(row + o);
+    if ((o & 7) == 0) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(row + o), b = *reinterpret_cast<const uint2 *>(row + o + 8);
+        return make_uint4(a.x, a.y, b.x, b.y);
+    }
+    if ((o & 3) == 0) {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o);
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o - 2);
+    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
+    return make_uint4(__funnelshift_r(w0, w1, 16), __funnelshift_r(w1, w2, 16), __funnelshift_r(w2, w3, 16),
+                      __funnelshift_r(w3, w4, 16));
+}
+
+// Eight elements (blocks j, j+1 of one pixel row) from a staged row -> four pairs, as SRow::load.
+__device__ __forceinline__ void staged_row8(const unsigned char *row, uint32_t o, __nv_bfloat16 *, float2 *v)
+{
+    const uint4 r = lds16_at(row, o);
+    v[0] = make_float2(bf16_lo(r.x), bf16_lo(r.z));
+    v[1] = make_float2(bf16_hi(r.x), bf16_hi(r.z));
+    v[2] = make_float2(bf16_lo(r.y), bf16_lo(r.w));
+    v[3] = make_float2(bf16_hi(r.y), bf16_hi(r.w));
+}
+__device__ __forceinline__ void staged_row8(const unsigned char *row, uint32_t o, float *, float2 *v)
+{
+    const uint4 a = lds16_at(row, o), b = lds16_at(row, o + 16);
+    v[0] = make_float2(__uint_as_float(a.x), __uint_as_float(b.x));
+    v[1] = make_float2(__uint_as_float(a.y), __uint_as_float(b.y));
+    v[2] = make_float2(__uint_as_float(a.z), __uint_as_float(b.z));
+    v[3] = make_float2(__uint_as_float(a.w), __uint_as_float(b.w));
+}
+
+// Two adjacent elements (one coefficient of blocks j, j+1) from a staged row.
+__device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t o, __nv_bfloat16 *)
+{
+    uint32_t r;
+    if ((o & 3) == 0) {
+        r = *reinterpret_cast<const uint32_t *>(row + o);
+    } else {
+        const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o - 2);
+        r = __funnelshift_r(w[0], w[1], 16);
+    }
+    return make_float2(bf16_lo(r), bf16_hi(r));
+}
+__device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t o, float *)
+{
+    if ((o & 7) == 0)
+        return *reinterpret_cast<const float2 *>(row + o);
+    const float *w = reinterpret_cast<const float *>(row + o);
+    return make_float2(w[0], w[1]);
+}
+
+// Global stores whose alignment is known only at run time (the destination's rows are
+// not multiples of the vector width): the widest stores the address allows.
+__device__ __forceinline__ void gstore_pair_any(__nv_bfloat16 *p, float2 v)
+{
+    const uint32_t u = pack_bf16x2(v.x, v.y);
+    if (((uintptr_t)p & 3) == 0) {
+        *reinterpret_cast<uint32_t *>(p) = u;
+    } else {
+        reinterpret_cast<unsigned short *>(p)[0] = (unsigned short)(u & 0xFFFFu);
+        reinterpret_cast<unsigned short *>(p)[1] = (unsigned short)(u >> 16);
+    }
+}
+__device__ __forceinline__ void gstore_pair_any(float *p, float2 v)
+{
+    if (((uintptr_t)p & 7) == 0) {
+        *reinterpret_cast<float2 *>(p) = v;
+    } else {
+        p[0] = v.x;
+        p[1] = v.y;
+    }
+}
+__device__ __forceinline__ void gstore_row_any(__nv_bfloat16 *p, const float2 *v)
+{
+    const uint32_t w0 = pack_bf16x2(v[0].x, v[1].x), w1 = pack_bf16x2(v[2].x, v[3].x);
+    const uint32_t w2 = pack_bf16x2(v[0].y, v[1].y), w3 = pack_bf16x2(v[2].y, v[3].y);
+    const uintptr_t a = (uintptr_t)p;
+    if ((a & 15) == 0) {
+        *reinterpret_cast<uint4 *>(p) = make_uint4(w0, w1, w2, w3);
+    } else if ((a & 7) == 0) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(w0, w1);
+        *reinterpret_cast<uint2 *>(p + 4) = make_uint2(w2, w3);
+    } else if ((a & 3) == 0) {
+        uint32_t *q = reinterpret_cast<uint32_t *>(p);
+        q[0] = w0;
+        q[1] = w1;
+        q[2] = w2;
+        q[3] = w3;
+    } else {
+        unsigned short *q = reinterpret_cast<unsigned short *>(p);
+        const uint32_t w[4] = {w0, w1, w2, w3};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            q[2 * k] = (unsigned short)(w[k] & 0xFFFFu);
+            q[2 * k + 1] = (unsigned short)(w[k] >> 16);
+        }
+    }
+}
+__device__ __forceinline__ void gstore_row_any(float *p, const float2 *v)
+{
+    const uintptr_t a = (uintptr_t)p;
+    if ((a & 15) == 0) {
+        gstore_row(p, v);
+    } else if ((a & 7) == 0) {
+#pragma unroll
+        for (int k = 0; k < 4; k += 2) {
+            *reinterpret_cast<float2 *>(p + k) = make_float2(v[k].x, v[k + 1].x);
+            *reinterpret_cast<float2 *>(p + 4 + k) = make_float2(v[k].y, v[k + 1].y);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            p[k] = v[k].x;
+            p[4 + k] = v[k].y;
+        }
+    }
+}
+
+// One pixel row of blocks j, j+1 (only block j when `both` is false, at the right edge of
+// an odd w); the row form does not know the destination's alignment at compile time.
+template <bool ROWS, typename T> __device__ __forceinline__ void store_pixel_row(T *p, const float2 *o, bool both)
+{
+    if constexpr (!ROWS) {
+        gstore_row(p, o);
+    } else if (both) {
+        gstore_row_any(p, o);
+    } else {
+#pragma unroll
+        for (int d = 0; d < 4; ++d)
+            p[d] = to_elem<T>(o[d].x);
+    }
+}
+
 // Video: one block row (tile rows = 1); images: four block rows, done one after another.
 template <bool VIDEO> struct TileRows {
     static constexpr int RW = VIDEO ? 1 : 4;
@@ -172,14 +333,17 @@ template <bool VIDEO> struct TileRows {
 // ADJ changes window 0 only: its time samples are (0, 0, 0, frame 0) instead of four
 // copies of frame 0, and frame 0 receives the sum of the four rebuilt samples
 // instead of the last one.  EXT: the extended form of TileGrid (padding, cropping,
-// streaming chunks).
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
+// streaming chunks).  ROWS: the row form (source rows at any element offset, destination
+// stores of any alignment, w may be odd); it reads the source through `src` (tg.n_src
+// elements) instead of the tensor maps.
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS>
 __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
-                    const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
+                    const __grid_constant__ CUtensorMap ymap, const T *__restrict__ src, T *__restrict__ out,
+                    const TileGrid tg)
 {
     static_assert(!(EXT && ADJ), "the adjoints take the plain form");
-    using P = WarpTiles<T>;
+    using P = TileSmem<T, FWD, ROWS>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
     constexpr int G = VIDEO ? 64 : 16;  // channel groups
@@ -191,8 +355,8 @@ __global__ void __launch_bounds__(32)
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int lane = threadIdx.x;
-    T *in_buf = reinterpret_cast<T *>(smem_raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * TILE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * P::TILE);
+    unsigned char *row_off = reinterpret_cast<unsigned char *>(bars + KT); // ROWS: [tile][staged row]
 
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
         const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
@@ -205,7 +369,81 @@ __global__ void __launch_bounds__(32)
     const uint32_t first = blockIdx.x * (uint32_t)KT;
     const int count = (int)min((uint32_t)KT, tg.ntiles - first); // tiles of this CTA
 
-    if (lane == 0) {
+    if constexpr (ROWS) {
+        if (lane == 0) {
+            for (int s = 0; s < KT; ++s)
+                mbar_init(smem_addr(bars + s), 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        constexpr int VE = 16 / (int)sizeof(T); // elements per 16 bytes
+        constexpr int PER = FWD ? 1 : 2;        // staged rows issued per lane (16 or 64 per tile)
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t bc;
+            decode(first + s, tx, ty, tq, bc);
+            const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0);
+            int64_t start[PER]; // byte offset of each staged row in the source (16-byte aligned)
+            uint32_t nbulk[PER];
+            bool ok[PER];
+            uint32_t tx_bytes = 0;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int r = lane + 32 * k;
+                int64_t off = 0;
+                if constexpr (FWD) {
+                    // Staged row r: frame slot r / (4 RW), pixel row 4 RW ty + r % (4 RW).
+                    const int a = r / (4 * RW);
+                    const int64_t y = (int64_t)4 * RW * ty + r % (4 * RW);
+                    int64_t f = 0;
+                    bool loaded = r < P::NR && y < tg.H;
+                    if (VIDEO && replica)
+                        loaded = loaded && a == 0; // window 0 reads frame 0 only
+                    else if (VIDEO)
+                        f = EXT ? mirror_frame(4 * tq + tg.fbase + a, tg.T) : 4 * tq - 3 + a;
+                    ok[k] = loaded;
+                    off = ((bc * tg.T + f) * tg.H + y) * tg.W + (int64_t)4 * WT * tx;
+                } else {
+                    // Staged row r: group r / RW, block row RW ty + r % RW.
+                    const int g = r / RW;
+                    const int64_t row = (int64_t)RW * ty + r % RW;
+                    const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                    const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                    ok[k] = row < tg.h;
+                    off = ((b * G + g) * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + (int64_t)WT * tx;
+                }
+                const int mis = (int)(off % VE);
+                start[k] = (off - mis) * (int64_t)sizeof(T);
+                // Bytes the bulk copy takes: the staged row, or up to the last 16-byte boundary
+                // before the tensor's end (a valid row starts before the end).
+                const int64_t avail = tg.n_src * (int64_t)sizeof(T) - start[k];
+                nbulk[k] = !ok[k] ? 0u : avail >= P::ROW ? (uint32_t)P::ROW : (uint32_t)(avail & ~(int64_t)15);
+                if (r < P::NR)
+                    row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T)) : kRowSkipped;
+                tx_bytes += __reduce_add_sync(0xFFFFFFFFu, nbulk[k]);
+            }
+            const uint32_t bar = smem_addr(bars + s);
+            if (lane == 0)
+                mbar_expect_tx(bar, tx_bytes);
+            __syncwarp();
+            unsigned char *tile = smem_raw + s * P::TILE;
+            const unsigned char *src_b = reinterpret_cast<const unsigned char *>(src);
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                if (!ok[k])
+                    continue;
+                unsigned char *dst = tile + (lane + 32 * k) * P::ROW;
+                if (nbulk[k] > 0)
+                    bulk_load(smem_addr(dst), src_b + start[k], nbulk[k], bar);
+                if (nbulk[k] < (uint32_t)P::ROW) {
+                    // The row reaches the tensor's last, partial 16 bytes: copy those elements.
+                    const int64_t end = min(tg.n_src * (int64_t)sizeof(T) - start[k], (int64_t)P::ROW);
+                    for (int64_t b = nbulk[k]; b < end; b += (int64_t)sizeof(T))
+                        *reinterpret_cast<T *>(dst + b) = *reinterpret_cast<const T *>(src_b + start[k] + b);
+                }
+            }
+        }
+    } else if (lane == 0) {
         for (int s = 0; s < KT; ++s)
             mbar_init(smem_addr(bars + s), 1);
         fence_barrier_init();
@@ -213,7 +451,7 @@ __global__ void __launch_bounds__(32)
             int tx, ty, tq;
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
-            const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
+            const uint32_t dst = smem_addr(smem_raw + s * P::TILE), bar = smem_addr(bars + s);
             if constexpr (FWD && EXT && VIDEO) {
                 if (tg.rep && tq == 0) {
                     mbar_expect_tx(bar, FRAME_BYTES);
@@ -253,9 +491,11 @@ __global__ void __launch_bounds__(32)
         int tx, ty, tq;
         int64_t bc;
         decode(first + s, tx, ty, tq, bc);
-        const T *tin = in_buf + s * kTileElems;
+        const unsigned char *tile = smem_raw + s * P::TILE;
+        const T *tin = reinterpret_cast<const T *>(tile);
         const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
-        const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
+        const bool col_ok = j0 < tg.w;
+        const bool pair_ok = !ROWS || j0 + 1 < tg.w;    // block j0 + 1 exists (w is even outside the row form)
         const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0); // window 0 of a video
 
 #pragma unroll
@@ -271,6 +511,31 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
                             for (int d = 0; d < 4; ++d)
                                 v[a][rr][d] = make_float2(0.0f, 0.0f);
+                        } else if constexpr (ROWS) {
+                            const int r = fa * 4 * RW + 4 * rw + rr;
+                            const unsigned mb = row_off[s * 64 + r];
+                            if (mb == kRowSkipped) { // a row past the clip's last row: zeros
+#pragma unroll
+                                for (int d = 0; d < 4; ++d)
+                                    v[a][rr][d] = make_float2(0.0f, 0.0f);
+                            } else {
+                                staged_row8(tile + r * P::ROW, mb + lane * 8 * (uint32_t)sizeof(T), (T *)nullptr,
+                                            v[a][rr]);
+                                if (EXT) {
+                                    // Columns past the clip's last column read as zeros (the staged
+                                    // row runs on into the next one).
+                                    const int64_t c0 = (int64_t)4 * WT * tx + 8 * lane;
+                                    if (c0 + 8 > tg.W) {
+#pragma unroll
+                                        for (int d = 0; d < 4; ++d) {
+                                            if (c0 + d >= tg.W)
+                                                v[a][rr][d].x = 0.0f;
+                                            if (c0 + 4 + d >= tg.W)
+                                                v[a][rr][d].y = 0.0f;
+                                        }
+                                    }
+                                }
+                            }
                         } else {
                             SRow<T>::load(tin + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
                         }
@@ -279,7 +544,16 @@ __global__ void __launch_bounds__(32)
             } else {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float2 p = SRow<T>::load_pair(tin + (g * RW + rw) * WT + 2 * lane);
+                    float2 p;
+                    if constexpr (ROWS) {
+                        // A skipped row lies past the last block row: its results are not stored.
+                        const unsigned mb = row_off[s * 64 + g * RW + rw];
+                        p = mb == kRowSkipped ? make_float2(0.0f, 0.0f)
+                                              : staged_pair(tile + (g * RW + rw) * P::ROW,
+                                                            mb + lane * 2 * (uint32_t)sizeof(T), (T *)nullptr);
+                    } else {
+                        p = SRow<T>::load_pair(tin + (g * RW + rw) * WT + 2 * lane);
+                    }
                     if constexpr (VIDEO)
                         v[kt_of(g)][ky_of(g)][kx_of(g)] = p;
                     else
@@ -319,7 +593,16 @@ __global__ void __launch_bounds__(32)
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
-                    gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
+                    T *dst = yp + (uint64_t)((uint32_t)g * cstride);
+                    if constexpr (ROWS) {
+                        const float2 q = __fmul2_rn(p, scale);
+                        if (pair_ok)
+                            gstore_pair_any(dst, q);
+                        else
+                            dst[0] = to_elem<T>(q.x);
+                    } else {
+                        gstore_pair(dst, __fmul2_rn(p, scale));
+                    }
                 }
             } else {
                 // x[bc][frame][4*row + rr][4*j0 .. 4*j0 + 7]; window 0 keeps its last frame only
@@ -333,7 +616,7 @@ __global__ void __launch_bounds__(32)
                         for (int d = 0; d < 4; ++d)
                             o[d] = __fmul2_rn(add2(add2(add2(v[0][rr][d], v[1][rr][d]), v[2][rr][d]), v[3][rr][d]),
                                               scale);
-                        gstore_row(xb + rr * tg.W, o);
+                        store_pixel_row<ROWS>(xb + rr * tg.W, o, pair_ok);
                     }
                     continue;
                 }
@@ -352,11 +635,11 @@ __global__ void __launch_bounds__(32)
                             o[d] = __fmul2_rn(v[a][rr][d], scale);
                         T *dst = xb + f * tg.H * tg.W + rr * tg.W;
                         if (!EXT) {
-                            gstore_row(dst, o);
+                            store_pixel_row<ROWS>(dst, o, pair_ok);
                         } else if (4 * row + rr < tg.H) { // cropped rows and columns
                             const int64_t col = 4 * j0;
                             if (col + 8 <= tg.W) {
-                                gstore_row(dst, o);
+                                store_pixel_row<ROWS>(dst, o, true);
                             } else {
 #pragma unroll
                                 for (int d = 0; d < 8; ++d)
@@ -737,10 +1020,10 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS>
 tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    using P = WarpTiles<T>;
+    using P = TileSmem<T, FWD, ROWS>;
     constexpr int G = VIDEO ? 64 : 16, RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
@@ -749,7 +1032,9 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     memset(&xm4, 0, sizeof xm4);
     memset(&xm1, 0, sizeof xm1);
     memset(&ym, 0, sizeof ym);
-    if (FWD) {
+    if (ROWS) {
+        // The row form reads the source through its pointer (bulk copies); no tensor map.
+    } else if (FWD) {
         const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
         const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
         const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
@@ -783,17 +1068,35 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.ntiles = (uint32_t)(ntx * nty * d.nq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
     tg.fbase = (int)d.fbase;
     tg.rep = d.rep;
+    tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
 
     // Per call: the attribute belongs to the current device.
-    const cudaError_t attr_err =
-        cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (T *)out, tg);
+    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS>
+        <<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (const T *)in, (T *)out, tg);
     return launch_status();
+}
+
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
+tok_status launch_form(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    return rows ? launch<T, VIDEO, FWD, ADJ, EXT, true>(in, out, d, stream)
+                : launch<T, VIDEO, FWD, ADJ, EXT, false>(in, out, d, stream);
+}
+
+// Limits shared by both forms: 32-bit frame, group and tile numbers, and the 64 planes of
+// one channel within a 32-bit element offset.
+bool tma_limits_ok(const HaarDims &d)
+{
+    const int64_t ntiles = ((d.w + 63) / 64) * ((d.h + 3) / 4 + d.h) * d.Tq * d.B * d.C; // generous bound
+    return d.B * d.C * d.T < (int64_t)1 << 31 && 64 * d.B < (int64_t)1 << 31 && d.W < (int64_t)1 << 31 &&
+           d.H < (int64_t)1 << 31 && ntiles < (int64_t)1 << 32 && 64 * d.C * d.Tq * d.h * d.w < (int64_t)1 << 32;
 }
 
 } // namespace
@@ -805,53 +1108,62 @@ bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const Haar
         return false;
     if ((d.w * es) % 16 != 0 || (d.W * es) % 16 != 0) // row strides of both tensors: multiples of 16 bytes
         return false;
-    // Coordinates are 32-bit: frames of the flattened [B*C*T] axis and the group axis must fit,
-    // tiles are numbered in 32 bits, and the 64 planes of one channel lie within a 32-bit offset.
-    const int64_t ntiles = ((d.w + 63) / 64) * ((d.h + 3) / 4 + d.h) * d.Tq * d.B * d.C; // generous bound
-    if (d.B * d.C * d.T >= (int64_t)1 << 31 || 64 * d.B >= (int64_t)1 << 31 || d.W >= (int64_t)1 << 31 ||
-        d.H >= (int64_t)1 << 31 || ntiles >= (int64_t)1 << 32 || 64 * d.C * d.Tq * d.h * d.w >= (int64_t)1 << 32)
-        return false;
-    return sm_count() > 0;
+    return tma_limits_ok(d) && sm_count() > 0;
 }
 
-tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
-                           cudaStream_t stream)
+HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
-    const bool video = d.video;
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    if (!tma_limits_ok(d) || sm_count() <= 0)
+        return HaarTmaForm::none;
+    // Box form: the source's rows are whole 16-byte units (one TMA box per tile); the forward
+    // stores coefficient pairs (w even), the inverse 16-byte pixel rows.
+    const bool boxes = fwd ? aligned(in, 16) && (d.W * es) % 16 == 0 && aligned(out, 2 * es) && d.w % 2 == 0
+                           : aligned(in, 16) && (d.w * es) % 16 == 0 && aligned(out, 16) && (d.W * es) % 16 == 0;
+    if (boxes)
+        return HaarTmaForm::boxes;
+    // Row form: any 16-byte-aligned source.
+    return aligned(in, 16) ? HaarTmaForm::rows : HaarTmaForm::none;
+}
+
+tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
+                           const HaarDims &d, cudaStream_t stream)
+{
+    const bool video = d.video, rows = form == HaarTmaForm::rows;
     if (d.ext) {
         if (dt == TOK_BF16) {
             using B16 = __nv_bfloat16;
             if (video)
-                return fwd ? launch<B16, true, true, false, true>(in, out, d, stream)
-                           : launch<B16, true, false, false, true>(in, out, d, stream);
-            return fwd ? launch<B16, false, true, false, true>(in, out, d, stream)
-                       : launch<B16, false, false, false, true>(in, out, d, stream);
+                return fwd ? launch_form<B16, true, true, false, true>(rows, in, out, d, stream)
+                           : launch_form<B16, true, false, false, true>(rows, in, out, d, stream);
+            return fwd ? launch_form<B16, false, true, false, true>(rows, in, out, d, stream)
+                       : launch_form<B16, false, false, false, true>(rows, in, out, d, stream);
         }
         if (video)
-            return fwd ? launch<float, true, true, false, true>(in, out, d, stream)
-                       : launch<float, true, false, false, true>(in, out, d, stream);
-        return fwd ? launch<float, false, true, false, true>(in, out, d, stream)
-                   : launch<float, false, false, false, true>(in, out, d, stream);
+            return fwd ? launch_form<float, true, true, false, true>(rows, in, out, d, stream)
+                       : launch_form<float, true, false, false, true>(rows, in, out, d, stream);
+        return fwd ? launch_form<float, false, true, false, true>(rows, in, out, d, stream)
+                   : launch_form<float, false, false, false, true>(rows, in, out, d, stream);
     }
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (!video)
-            return fwd ? launch<B16, false, true, false, false>(in, out, d, stream)
-                       : launch<B16, false, false, false, false>(in, out, d, stream);
+            return fwd ? launch_form<B16, false, true, false, false>(rows, in, out, d, stream)
+                       : launch_form<B16, false, false, false, false>(rows, in, out, d, stream);
         if (adj)
-            return fwd ? launch<B16, true, true, true, false>(in, out, d, stream)
-                       : launch<B16, true, false, true, false>(in, out, d, stream);
-        return fwd ? launch<B16, true, true, false, false>(in, out, d, stream)
-                   : launch<B16, true, false, false, false>(in, out, d, stream);
+            return fwd ? launch_form<B16, true, true, true, false>(rows, in, out, d, stream)
+                       : launch_form<B16, true, false, true, false>(rows, in, out, d, stream);
+        return fwd ? launch_form<B16, true, true, false, false>(rows, in, out, d, stream)
+                   : launch_form<B16, true, false, false, false>(rows, in, out, d, stream);
     }
     if (!video)
-        return fwd ? launch<float, false, true, false, false>(in, out, d, stream)
-                   : launch<float, false, false, false, false>(in, out, d, stream);
+        return fwd ? launch_form<float, false, true, false, false>(rows, in, out, d, stream)
+                   : launch_form<float, false, false, false, false>(rows, in, out, d, stream);
     if (adj)
-        return fwd ? launch<float, true, true, true, false>(in, out, d, stream)
-                   : launch<float, true, false, true, false>(in, out, d, stream);
-    return fwd ? launch<float, true, true, false, false>(in, out, d, stream)
-               : launch<float, true, false, false, false>(in, out, d, stream);
+        return fwd ? launch_form<float, true, true, true, false>(rows, in, out, d, stream)
+                   : launch_form<float, true, false, true, false>(rows, in, out, d, stream);
+    return fwd ? launch_form<float, true, true, false, false>(rows, in, out, d, stream)
+               : launch_form<float, true, false, false, false>(rows, in, out, d, stream);
 }
 
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)

@@ -24,11 +24,18 @@ struct HaarDims {
     bool ext = false;
 };
 
-// The TMA path takes 16-byte-aligned tensors whose rows are multiples of 16 bytes.
+// Strict test (the channels-last kernel): 16-byte-aligned tensors whose rows are multiples
+// of 16 bytes on both sides.
 bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
+
+// Which form of the TMA kernel takes a planar call in direction fwd: boxes (the source's
+// rows are whole 16-byte units), rows (a 16-byte-aligned source of fewer than 2^31
+// elements, any row length, any element-aligned destination) or none (register kernels).
+enum class HaarTmaForm { none, boxes, rows };
+HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d);
 // fwd: pixels -> coefficients; adj: the adjoint variant (video only; images are orthogonal).
-tok_status haar_tma_launch(bool fwd, bool adj, const void *in, void *out, tok_dtype dt, const HaarDims &d,
-                           cudaStream_t stream);
+tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
+                           const HaarDims &d, cudaStream_t stream);
 
 // Single-level patcher / unpatcher (patch_size=2): pixels [B, C, T, H, W] <->
 // coefficients [B, G*C, Tq, h, w] with G = 8 (video), 4 (images), Tq = (T + 1) / 2, h = H/2.

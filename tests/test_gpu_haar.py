@@ -74,8 +74,9 @@ def check_inv(y: torch.Tensor, T, H, W, label):
 
 
 SMALL = [
-    # (shape, dtype, note).  TMA path: 16-byte-aligned tensors with W*elem/4 a multiple of 16 bytes
-    # (bf16: W % 32 == 0, fp32: W % 16 == 0); the others take the register kernels.
+    # (shape, dtype, note).  TMA box form: the source's rows are whole 16-byte units (forward:
+    # W * elem, with w even; inverse: w * elem and W * elem); other 16-byte-aligned sources take
+    # the TMA row form.  The register kernels take misaligned views (tests below).
     ((1, 3, 9, 64, 64), synth.F32, "config 1"),
     ((2, 3, 13, 40, 96), synth.BF16, "TMA bf16, partial tiles in x and y"),
     ((1, 2, 9, 36, 80), synth.F32, "TMA fp32, partial tiles"),
@@ -83,14 +84,14 @@ SMALL = [
     ((1, 1, 5, 4, 32), synth.BF16, "TMA bf16, one block row"),
     ((3, 2, 1, 24, 160), synth.BF16, "TMA image path, partial tiles"),
     ((2, 1, 1, 20, 48), synth.F32, "TMA image path fp32"),
-    ((2, 3, 13, 64, 264), synth.F32, "vector path, 5 CTAs per frame, ragged tail"),
-    ((2, 3, 13, 64, 264), synth.BF16, "vector path bf16"),
-    ((1, 2, 9, 16, 44), synth.BF16, "W % 8 == 4: element-wise path"),
-    ((1, 2, 9, 16, 44), synth.F32, "element-wise path fp32"),
+    ((2, 3, 13, 64, 264), synth.F32, "box forward, row-form inverse, ragged tail"),
+    ((2, 3, 13, 64, 264), synth.BF16, "box forward, row-form inverse, bf16"),
+    ((1, 2, 9, 16, 44), synth.BF16, "W % 8 == 4: row form, odd w"),
+    ((1, 2, 9, 16, 44), synth.F32, "row form fp32, odd w"),
     ((1, 1, 5, 4, 4), synth.F32, "smallest video"),
-    ((3, 2, 1, 64, 192), synth.BF16, "image path, vector"),
+    ((3, 2, 1, 64, 192), synth.BF16, "image path, boxes both ways"),
     ((3, 2, 1, 64, 192), synth.F32, "image path fp32"),
-    ((2, 3, 1, 36, 40), synth.BF16, "image path, W % 16 == 8: element-wise"),
+    ((2, 3, 1, 36, 40), synth.BF16, "image path, W % 16 == 8: row-form inverse"),
     ((1, 1, 1, 4, 4), synth.F32, "smallest image"),
     ((1, 5, 21, 24, 1032), synth.BF16, "odd channel count, long row"),
 ]
@@ -157,7 +158,7 @@ def test_tma_and_register_paths_agree_bitwise(shape, dtype):
 
 @pytest.mark.parametrize("shape,dtype,chunks", [
     ((1, 3, 41, 64, 128), torch.bfloat16, [(0, 1), (1, 4), (4, 7), (7, 11)]),    # TMA path
-    ((2, 2, 29, 40, 72), torch.bfloat16, [(0, 3), (3, 8)]),                      # register path (W % 32 != 0)
+    ((2, 2, 29, 40, 72), torch.bfloat16, [(0, 3), (3, 8)]),                      # row-form inverse (W % 32 != 0)
     ((1, 2, 21, 32, 64), torch.float32, [(0, 2), (2, 2), (2, 6)]),               # fp32, an empty chunk
     ((2, 3, 1, 32, 64), torch.bfloat16, [(0, 1)]),                               # image: one window
 ])

@@ -36,9 +36,9 @@ PADDED = [
     ((2, 1, 6, 30, 256), synth.BF16, 16, 8, "TMA bf16, zero rows, mirrored frames"),
     ((1, 2, 7, 20, 32), synth.F32, 8, 4, "TMA fp32, zero rows"),
     ((1, 1, 2, 8, 64), synth.BF16, 4, 8, "TMA bf16, mirror longer than the clip"),
-    ((1, 2, 7, 21, 45), synth.BF16, 4, 4, "register bf16, ragged rows and columns"),
-    ((1, 2, 11, 13, 30), synth.F32, 8, 8, "register fp32"),
-    ((2, 3, 1, 30, 50), synth.BF16, 4, 4, "image, register"),
+    ((1, 2, 7, 21, 45), synth.BF16, 4, 4, "row form bf16, ragged rows and columns"),
+    ((1, 2, 11, 13, 30), synth.F32, 8, 8, "row form fp32"),
+    ((2, 3, 1, 30, 50), synth.BF16, 4, 4, "image, row form"),
     ((1, 2, 1, 24, 64), synth.F32, 16, 4, "image, TMA, zero rows"),
 ]
 
@@ -79,7 +79,7 @@ def test_no_padding_needed_is_the_plain_call_bit_for_bit(shape, dtype):
 CHUNKS = [
     # (shape of the whole video, dtype, frames per chunk: 1 + 4k first, then multiples of 4)
     ((2, 2, 21, 16, 64), synth.BF16, [1, 8, 4, 8]),      # TMA path; a one-frame first chunk
-    ((1, 2, 13, 8, 20), synth.F32, [5, 4, 4]),           # register path (w * 4 bytes not a multiple of 16)
+    ((1, 2, 13, 8, 20), synth.F32, [5, 4, 4]),           # row form (w * 4 bytes not a multiple of 16)
     ((1, 3, 25, 12, 96), synth.BF16, [9, 16]),
 ]
 
