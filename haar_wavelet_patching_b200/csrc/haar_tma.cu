@@ -174,7 +174,9 @@ __device__ __forceinline__ void gstore_row(float *p, const float2 *v)
 // their width from the destination address at run time.
 // ---------------------------------------------------------------------------
 template <typename T, bool FWD, bool ROWS> struct TileSmem {
-    static constexpr int KT = WarpTiles<T>::KT;
+    // The row form spends more instructions per tile (row offsets, realigned reads, stores of
+    // run-time width), so it trades tiles per CTA for resident warps: ~17 KB per CTA.
+    static constexpr int KT = !ROWS ? WarpTiles<T>::KT : sizeof(T) == 2 ? 2 : 1;
     static constexpr int NR = FWD ? 16 : 64;                              // staged rows of a tile
     static constexpr int ROW = (FWD ? 256 : 64) * (int)sizeof(T) + 16;     // a source row and its slack
     static constexpr int TILE = ROWS ? NR * ROW : kTileElems * (int)sizeof(T);
@@ -241,27 +243,8 @@ __device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t
     return make_float2(w[0], w[1]);
 }
 
-// Global stores whose alignment is known only at run time (the destination's rows are
-// not multiples of the vector width): the widest stores the address allows.
-__device__ __forceinline__ void gstore_pair_any(__nv_bfloat16 *p, float2 v)
-{
-    const uint32_t u = pack_bf16x2(v.x, v.y);
-    if (((uintptr_t)p & 3) == 0) {
-        *reinterpret_cast<uint32_t *>(p) = u;
-    } else {
-        reinterpret_cast<unsigned short *>(p)[0] = (unsigned short)(u & 0xFFFFu);
-        reinterpret_cast<unsigned short *>(p)[1] = (unsigned short)(u >> 16);
-    }
-}
-__device__ __forceinline__ void gstore_pair_any(float *p, float2 v)
-{
-    if (((uintptr_t)p & 7) == 0) {
-        *reinterpret_cast<float2 *>(p) = v;
-    } else {
-        p[0] = v.x;
-        p[1] = v.y;
-    }
-}
+// A pixel-row store whose alignment is known only at run time (the destination's rows are
+// not multiples of 16 bytes): the widest stores the address allows.
 __device__ __forceinline__ void gstore_row_any(__nv_bfloat16 *p, const float2 *v)
 {
     const uint32_t w0 = pack_bf16x2(v[0].x, v[1].x), w1 = pack_bf16x2(v[2].x, v[3].x);
@@ -418,8 +401,12 @@ __global__ void __launch_bounds__(32)
                 // before the tensor's end (a valid row starts before the end).
                 const int64_t avail = tg.n_src * (int64_t)sizeof(T) - start[k];
                 nbulk[k] = !ok[k] ? 0u : avail >= P::ROW ? (uint32_t)P::ROW : (uint32_t)(avail & ~(int64_t)15);
+                // A row that is not loaded reads as zeros where its values are used (rows past the
+                // clip's last row on the padded forward); elsewhere its results are never stored
+                // and it is read at offset 0 of its (stale) staging row.
                 if (r < P::NR)
-                    row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T)) : kRowSkipped;
+                    row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T))
+                                                : FWD && EXT ? kRowSkipped : (unsigned char)0;
                 tx_bytes += __reduce_add_sync(0xFFFFFFFFu, nbulk[k]);
             }
             const uint32_t bar = smem_addr(bars + s);
@@ -514,7 +501,7 @@ __global__ void __launch_bounds__(32)
                         } else if constexpr (ROWS) {
                             const int r = fa * 4 * RW + 4 * rw + rr;
                             const unsigned mb = row_off[s * 64 + r];
-                            if (mb == kRowSkipped) { // a row past the clip's last row: zeros
+                            if (EXT && mb == kRowSkipped) { // a row past the clip's last row: zeros
 #pragma unroll
                                 for (int d = 0; d < 4; ++d)
                                     v[a][rr][d] = make_float2(0.0f, 0.0f);
@@ -546,11 +533,9 @@ __global__ void __launch_bounds__(32)
                 for (int g = 0; g < G; ++g) {
                     float2 p;
                     if constexpr (ROWS) {
-                        // A skipped row lies past the last block row: its results are not stored.
                         const unsigned mb = row_off[s * 64 + g * RW + rw];
-                        p = mb == kRowSkipped ? make_float2(0.0f, 0.0f)
-                                              : staged_pair(tile + (g * RW + rw) * P::ROW,
-                                                            mb + lane * 2 * (uint32_t)sizeof(T), (T *)nullptr);
+                        p = staged_pair(tile + (g * RW + rw) * P::ROW, mb + lane * 2 * (uint32_t)sizeof(T),
+                                        (T *)nullptr);
                     } else {
                         p = SRow<T>::load_pair(tin + (g * RW + rw) * WT + 2 * lane);
                     }
@@ -581,27 +566,52 @@ __global__ void __launch_bounds__(32)
             const float2 scale = make_float2(SCALE, SCALE);
 
             const int64_t row = (int64_t)ty * RW + rw; // block row
+            // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart, a 32-bit
+            // stride (checked on the host), so each address is one wide multiply-add.  (Addresses
+            // only; nothing is stored for lanes past the last block column or rows past h.)
+            const uint32_t cstride = (uint32_t)(tg.C.d * (int64_t)tg.Tq * tg.h * tg.w);
+            T *yp = nullptr;
+            bool pairs = true;
+            if constexpr (FWD) {
+                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                if constexpr (ROWS) {
+                    // A pair store is aligned iff its element offset is even, which alternates with g
+                    // only when the plane stride is odd.  One warp-wide choice per tile row (taken
+                    // before any lane leaves): pair stores when every storing lane's 64 pairs are
+                    // aligned and whole, element stores otherwise.
+                    const uintptr_t amask = 2 * sizeof(T) - 1;
+                    pairs = __all_sync(0xFFFFFFFFu, !col_ok || (pair_ok && ((uintptr_t)yp & amask) == 0 &&
+                                                                ((uintptr_t)(yp + cstride) & amask) == 0));
+                }
+            }
             if (!col_ok || row >= tg.h)
                 continue;
             if constexpr (FWD) {
-                // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart,
-                // a 32-bit stride (checked on the host), so each address is one wide multiply-add.
-                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
-                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
-                const uint32_t cstride = (uint32_t)(tg.C.d * plane);
-                T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                if constexpr (ROWS) {
+                    if (pairs) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
-                    T *dst = yp + (uint64_t)((uint32_t)g * cstride);
-                    if constexpr (ROWS) {
-                        const float2 q = __fmul2_rn(p, scale);
-                        if (pair_ok)
-                            gstore_pair_any(dst, q);
-                        else
-                            dst[0] = to_elem<T>(q.x);
+                        for (int g = 0; g < G; ++g) {
+                            const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
+                            gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
+                        }
                     } else {
-                        gstore_pair(dst, __fmul2_rn(p, scale));
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const float2 q = __fmul2_rn(
+                                VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)], scale);
+                            T *dst = yp + (uint64_t)((uint32_t)g * cstride);
+                            dst[0] = to_elem<T>(q.x);
+                            if (pair_ok)
+                                dst[1] = to_elem<T>(q.y);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
+                        gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
                     }
                 }
             } else {
