@@ -31,6 +31,7 @@
 // makes the warp stop, drain what it issued and count a timeout that
 // tok_check_device() reports.  No cluster multicast is used.
 #include <cstring>
+#include <numeric>
 
 #include "tma.cuh"
 #include "tok_common.cuh"
@@ -64,6 +65,10 @@ struct TileGrid {
     // reads zeros there (TMA fill), the inverse does not write there.
     int fbase, rep;
     int64_t n_src; // elements of the source tensor (the row form stops its copies at its end)
+    // Video forward, box form: when a coefficient row is not a whole number of 32-byte sectors
+    // (but a plane is), tiles of block row k = t' h + row start at column 64 tx - (k w mod salign)
+    // (salign = 32 bytes / element), so every warp's plane store starts on a sector; else 0.
+    int salign;
 };
 
 // Source frame of frame f of a T-frame clip mirrored about its last frame (period 2(T-1)).
@@ -185,61 +190,55 @@ template <typename T, bool FWD, bool ROWS> struct TileSmem {
 };
 constexpr unsigned char kRowSkipped = 0xFF; // a staged row that was not loaded (past the tensor edge)
 
-// 16 bytes at byte offset o (even) of a 16-byte-aligned staged row.  The branch on o's
-// alignment is uniform across a warp (lanes differ by multiples of 16 bytes).
-__device__ __forceinline__ uint4 lds16_at(const unsigned char *row, uint32_t o)
-{
-    if ((o & 15) == 0)
-        return *reinterpret_cast<const uint4 *>(row + o);
-    if ((o & 7) == 0) {
-        const uint2 a = *reinterpret_cast<const uint2 *>(row + o), b = *reinterpret_cast<const uint2 *>(row + o + 8);
-        return make_uint4(a.x, a.y, b.x, b.y);
-    }
-    if ((o & 3) == 0) {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o);
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o - 2);
-    const uint32_t w0 = w[0], w1 = w[1], w2 = w[2], w3 = w[3], w4 = w[4];
-    return make_uint4(__funnelshift_r(w0, w1, 16), __funnelshift_r(w1, w2, 16), __funnelshift_r(w2, w3, 16),
-                      __funnelshift_r(w3, w4, 16));
-}
+// Realigned reads from a 16-byte-aligned staged row, without branches, so the rows of a
+// tile are scheduled together: aligned 8- or 4-byte loads from at or below the offset,
+// then a select of the word offset and a funnel shift of the byte offset.
 
-// Eight elements (blocks j, j+1 of one pixel row) from a staged row -> four pairs, as SRow::load.
+// Eight elements (blocks j, j+1 of one pixel row) at byte offset o (even) -> four pairs, as
+// SRow::load.  Reads 24 bytes from the 8-byte boundary at or below o.
 __device__ __forceinline__ void staged_row8(const unsigned char *row, uint32_t o, __nv_bfloat16 *, float2 *v)
 {
-    const uint4 r = lds16_at(row, o);
-    v[0] = make_float2(bf16_lo(r.x), bf16_lo(r.z));
-    v[1] = make_float2(bf16_hi(r.x), bf16_hi(r.z));
-    v[2] = make_float2(bf16_lo(r.y), bf16_lo(r.w));
-    v[3] = make_float2(bf16_hi(r.y), bf16_hi(r.w));
+    const uint32_t base = o & ~7u, sh = (o & 3u) * 8u;
+    const bool odd = (o & 4u) != 0;
+    const uint2 a = *reinterpret_cast<const uint2 *>(row + base);
+    const uint2 b = *reinterpret_cast<const uint2 *>(row + base + 8);
+    const uint2 c = *reinterpret_cast<const uint2 *>(row + base + 16);
+    const uint32_t x0 = odd ? a.y : a.x, x1 = odd ? b.x : a.y, x2 = odd ? b.y : b.x, x3 = odd ? c.x : b.y,
+                   x4 = odd ? c.y : c.x;
+    const uint32_t r0 = __funnelshift_r(x0, x1, sh), r1 = __funnelshift_r(x1, x2, sh);
+    const uint32_t r2 = __funnelshift_r(x2, x3, sh), r3 = __funnelshift_r(x3, x4, sh);
+    v[0] = make_float2(bf16_lo(r0), bf16_lo(r2));
+    v[1] = make_float2(bf16_hi(r0), bf16_hi(r2));
+    v[2] = make_float2(bf16_lo(r1), bf16_lo(r3));
+    v[3] = make_float2(bf16_hi(r1), bf16_hi(r3));
 }
+// fp32: o is a multiple of 4; reads 40 bytes from the 8-byte boundary at or below o.
 __device__ __forceinline__ void staged_row8(const unsigned char *row, uint32_t o, float *, float2 *v)
 {
-    const uint4 a = lds16_at(row, o), b = lds16_at(row, o + 16);
-    v[0] = make_float2(__uint_as_float(a.x), __uint_as_float(b.x));
-    v[1] = make_float2(__uint_as_float(a.y), __uint_as_float(b.y));
-    v[2] = make_float2(__uint_as_float(a.z), __uint_as_float(b.z));
-    v[3] = make_float2(__uint_as_float(a.w), __uint_as_float(b.w));
+    const uint32_t base = o & ~7u;
+    const bool odd = (o & 4u) != 0;
+    float w[10];
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+        const float2 q = *reinterpret_cast<const float2 *>(row + base + 8 * k);
+        w[2 * k] = q.x;
+        w[2 * k + 1] = q.y;
+    }
+#pragma unroll
+    for (int d = 0; d < 4; ++d)
+        v[d] = make_float2(odd ? w[d + 1] : w[d], odd ? w[d + 5] : w[d + 4]);
 }
 
-// Two adjacent elements (one coefficient of blocks j, j+1) from a staged row.
+// Two adjacent elements (one coefficient of blocks j, j+1) at byte offset o.
 __device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t o, __nv_bfloat16 *)
 {
-    uint32_t r;
-    if ((o & 3) == 0) {
-        r = *reinterpret_cast<const uint32_t *>(row + o);
-    } else {
-        const uint32_t *w = reinterpret_cast<const uint32_t *>(row + o - 2);
-        r = __funnelshift_r(w[0], w[1], 16);
-    }
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (o & ~3u));
+    const uint32_t r = __funnelshift_r(w[0], w[1], (o & 3u) * 8u);
     return make_float2(bf16_lo(r), bf16_hi(r));
 }
 __device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t o, float *)
 {
-    if ((o & 7) == 0)
-        return *reinterpret_cast<const float2 *>(row + o);
-    const float *w = reinterpret_cast<const float *>(row + o);
+    const float *w = reinterpret_cast<const float *>(row + o); // o is a multiple of 4
     return make_float2(w[0], w[1]);
 }
 
@@ -341,6 +340,15 @@ __global__ void __launch_bounds__(32)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * P::TILE);
     unsigned char *row_off = reinterpret_cast<unsigned char *>(bars + KT); // ROWS: [tile][staged row]
 
+    // First block column of a tile (see TileGrid::salign).
+    auto col0 = [&](int tx, int ty, int tq) -> int {
+        if constexpr (FWD && VIDEO && !ROWS) {
+            if (tg.salign)
+                return WT * tx - (int)((((int64_t)tq * tg.h + ty) * tg.w) % tg.salign);
+        }
+        return WT * tx;
+    };
+
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
         const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
         tx = (int)(n - q1 * tg.ntx.d);
@@ -438,28 +446,29 @@ __global__ void __launch_bounds__(32)
             int tx, ty, tq;
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
+            const int x0 = 4 * col0(tx, ty, tq); // first pixel column (may be negative: TMA fills zeros)
             const uint32_t dst = smem_addr(smem_raw + s * P::TILE), bar = smem_addr(bars + s);
             if constexpr (FWD && EXT && VIDEO) {
                 if (tg.rep && tq == 0) {
                     mbar_expect_tx(bar, FRAME_BYTES);
-                    tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
+                    tma_load_3d(dst, &xmap1, x0, 4 * RW * ty, (int)(bc * tg.T), bar);
                 } else if (4 * tq + tg.fbase + 3 < tg.T) {
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
-                    tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq + tg.fbase), bar);
+                    tma_load_3d(dst, &xmap4, x0, 4 * RW * ty, (int)(bc * tg.T + 4 * tq + tg.fbase), bar);
                 } else {
                     // The window runs past the clip: frame by frame, mirrored about the last frame.
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
                     for (int a = 0; a < NA; ++a)
-                        tma_load_3d(dst + a * FRAME_BYTES, &xmap1, 4 * WT * tx, 4 * RW * ty,
+                        tma_load_3d(dst + a * FRAME_BYTES, &xmap1, x0, 4 * RW * ty,
                                     (int)(bc * tg.T + mirror_frame(4 * tq + tg.fbase + a, tg.T)), bar);
                 }
             } else if constexpr (FWD) {
                 if (VIDEO && tq > 0) {
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
-                    tma_load_3d(dst, &xmap4, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
+                    tma_load_3d(dst, &xmap4, x0, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
                 } else {
                     mbar_expect_tx(bar, FRAME_BYTES);
-                    tma_load_3d(dst, &xmap1, 4 * WT * tx, 4 * RW * ty, (int)(bc * tg.T), bar);
+                    tma_load_3d(dst, &xmap1, x0, 4 * RW * ty, (int)(bc * tg.T), bar);
                 }
             } else {
                 const int b = (int)tg.C.div((uint32_t)bc), c = (int)(bc - (int64_t)b * tg.C.d);
@@ -480,8 +489,8 @@ __global__ void __launch_bounds__(32)
         decode(first + s, tx, ty, tq, bc);
         const unsigned char *tile = smem_raw + s * P::TILE;
         const T *tin = reinterpret_cast<const T *>(tile);
-        const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
-        const bool col_ok = j0 < tg.w;
+        const int64_t j0 = (int64_t)col0(tx, ty, tq) + 2 * lane; // this lane's first block column
+        const bool col_ok = j0 >= 0 && j0 < tg.w;
         const bool pair_ok = !ROWS || j0 + 1 < tg.w;    // block j0 + 1 exists (w is even outside the row form)
         const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0); // window 0 of a video
 
@@ -1062,7 +1071,16 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
             return TOK_ERR_SHAPE;
     }
 
-    const int64_t ntx = (d.w + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
+    // Sector-aligned plane stores (TileGrid::salign): the shifts k w mod salign are multiples of
+    // gcd(w, salign), so a row needs at most ceil((w + salign - gcd) / 64) tiles.
+    int salign = 0;
+    if (FWD && VIDEO && !ROWS) {
+        const int64_t sa = 32 / (int64_t)es, plane = d.Tq * d.h * d.w;
+        if ((d.w * (int64_t)es) % 32 != 0 && (plane * (int64_t)es) % 32 == 0 && aligned(out, 32))
+            salign = (int)sa;
+    }
+    const int64_t smax = salign ? salign - std::gcd(d.w, (int64_t)salign) : 0;
+    const int64_t ntx = (d.w + smax + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
     TileGrid tg;
     tg.ntx = FastDiv((uint32_t)ntx);
     tg.nty = FastDiv((uint32_t)nty);
@@ -1079,6 +1097,7 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.fbase = (int)d.fbase;
     tg.rep = d.rep;
     tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
+    tg.salign = salign;
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS>,
@@ -1104,7 +1123,7 @@ tok_status launch_form(bool rows, const void *in, void *out, const HaarDims &d, 
 // one channel within a 32-bit element offset.
 bool tma_limits_ok(const HaarDims &d)
 {
-    const int64_t ntiles = ((d.w + 63) / 64) * ((d.h + 3) / 4 + d.h) * d.Tq * d.B * d.C; // generous bound
+    const int64_t ntiles = ((d.w + 16 + 63) / 64) * ((d.h + 3) / 4 + d.h) * d.Tq * d.B * d.C; // generous bound
     return d.B * d.C * d.T < (int64_t)1 << 31 && 64 * d.B < (int64_t)1 << 31 && d.W < (int64_t)1 << 31 &&
            d.H < (int64_t)1 << 31 && ntiles < (int64_t)1 << 32 && 64 * d.C * d.Tq * d.h * d.w < (int64_t)1 << 32;
 }

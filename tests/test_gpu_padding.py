@@ -40,6 +40,7 @@ PADDED = [
     ((1, 2, 11, 13, 30), synth.F32, 8, 8, "row form fp32"),
     ((2, 3, 1, 30, 50), synth.BF16, 4, 4, "image, row form"),
     ((1, 2, 1, 24, 64), synth.F32, 16, 4, "image, TMA, zero rows"),
+    ((1, 2, 5, 15, 88), synth.BF16, 4, 4, "TMA bf16, sector-shifted tiles (w = 22), zero rows"),
 ]
 
 
