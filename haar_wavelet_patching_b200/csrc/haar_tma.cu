@@ -67,7 +67,8 @@ struct TileGrid {
     int64_t n_src; // elements of the source tensor (the row form stops its copies at its end)
     // Video forward, box form: when a coefficient row is not a whole number of 32-byte sectors
     // (but a plane is), tiles of block row k = t' h + row start at column 64 tx - (k w mod salign)
-    // (salign = 32 bytes / element), so every warp's plane store starts on a sector; else 0.
+    // (salign = 32 bytes / element, a power of two), so every warp's plane store starts on a
+    // sector; else 0.
     int salign;
 };
 
@@ -343,8 +344,10 @@ __global__ void __launch_bounds__(32)
     // First block column of a tile (see TileGrid::salign).
     auto col0 = [&](int tx, int ty, int tq) -> int {
         if constexpr (FWD && VIDEO && !ROWS) {
+            // salign is a power of two, so (k w) mod salign needs only the low bits of k w.
             if (tg.salign)
-                return WT * tx - (int)((((int64_t)tq * tg.h + ty) * tg.w) % tg.salign);
+                return WT * tx - (int)((((uint32_t)tq * (uint32_t)tg.h + (uint32_t)ty) * (uint32_t)tg.w) &
+                                       (uint32_t)(tg.salign - 1));
         }
         return WT * tx;
     };
@@ -575,29 +578,28 @@ __global__ void __launch_bounds__(32)
             const float2 scale = make_float2(SCALE, SCALE);
 
             const int64_t row = (int64_t)ty * RW + rw; // block row
-            // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart, a 32-bit
-            // stride (checked on the host), so each address is one wide multiply-add.  (Addresses
-            // only; nothing is stored for lanes past the last block column or rows past h.)
-            const uint32_t cstride = (uint32_t)(tg.C.d * (int64_t)tg.Tq * tg.h * tg.w);
-            T *yp = nullptr;
             bool pairs = true;
-            if constexpr (FWD) {
+            if constexpr (FWD && ROWS) {
+                // A pair store is aligned iff its element offset is even, which alternates with g
+                // only when the plane stride is odd.  One warp-wide choice per tile row (taken before
+                // any lane leaves; addresses only): pair stores when every storing lane's 64 pairs
+                // are aligned and whole, element stores otherwise.
                 const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
                 const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
-                yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
-                if constexpr (ROWS) {
-                    // A pair store is aligned iff its element offset is even, which alternates with g
-                    // only when the plane stride is odd.  One warp-wide choice per tile row (taken
-                    // before any lane leaves): pair stores when every storing lane's 64 pairs are
-                    // aligned and whole, element stores otherwise.
-                    const uintptr_t amask = 2 * sizeof(T) - 1;
-                    pairs = __all_sync(0xFFFFFFFFu, !col_ok || (pair_ok && ((uintptr_t)yp & amask) == 0 &&
-                                                                ((uintptr_t)(yp + cstride) & amask) == 0));
-                }
+                const T *yq = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                const uintptr_t amask = 2 * sizeof(T) - 1;
+                pairs = __all_sync(0xFFFFFFFFu, !col_ok || (pair_ok && ((uintptr_t)yq & amask) == 0 &&
+                                                            ((uintptr_t)(yq + tg.C.d * plane) & amask) == 0));
             }
             if (!col_ok || row >= tg.h)
                 continue;
             if constexpr (FWD) {
+                // y[b][g*C + c][tq][row][j0 .. j0+1]; the 64 planes are C*plane elements apart, a
+                // 32-bit stride (checked on the host), so each address is one wide multiply-add.
+                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                const uint32_t cstride = (uint32_t)(tg.C.d * plane);
+                T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
                 if constexpr (ROWS) {
                     if (pairs) {
 #pragma unroll
