@@ -318,14 +318,17 @@ template <bool VIDEO> struct TileRows {
 // instead of the last one.  EXT: the extended form of TileGrid (padding, cropping,
 // streaming chunks).  ROWS: the row form (source rows at any element offset, destination
 // stores of any alignment, w may be odd); it reads the source through `src` (tg.n_src
-// elements) instead of the tensor maps.
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS>
+// elements) instead of the tensor maps.  ANYST (inverse, box form): the source takes the box
+// form but the pixel rows are not whole 16-byte units, so their stores take the row form's
+// run-time widths.
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false>
 __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
                     const __grid_constant__ CUtensorMap ymap, const T *__restrict__ src, T *__restrict__ out,
                     const TileGrid tg)
 {
     static_assert(!(EXT && ADJ), "the adjoints take the plain form");
+    static_assert(!(ANYST && (FWD || ROWS)), "ANYST: the inverse's box form only");
     using P = TileSmem<T, FWD, ROWS>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
@@ -637,7 +640,7 @@ __global__ void __launch_bounds__(32)
                         for (int d = 0; d < 4; ++d)
                             o[d] = __fmul2_rn(add2(add2(add2(v[0][rr][d], v[1][rr][d]), v[2][rr][d]), v[3][rr][d]),
                                               scale);
-                        store_pixel_row<ROWS>(xb + rr * tg.W, o, pair_ok);
+                        store_pixel_row<ROWS || ANYST>(xb + rr * tg.W, o, pair_ok);
                     }
                     continue;
                 }
@@ -656,11 +659,11 @@ __global__ void __launch_bounds__(32)
                             o[d] = __fmul2_rn(v[a][rr][d], scale);
                         T *dst = xb + f * tg.H * tg.W + rr * tg.W;
                         if (!EXT) {
-                            store_pixel_row<ROWS>(dst, o, pair_ok);
+                            store_pixel_row<ROWS || ANYST>(dst, o, pair_ok);
                         } else if (4 * row + rr < tg.H) { // cropped rows and columns
                             const int64_t col = 4 * j0;
                             if (col + 8 <= tg.W) {
-                                store_pixel_row<ROWS>(dst, o, true);
+                                store_pixel_row<ROWS || ANYST>(dst, o, true);
                             } else {
 #pragma unroll
                                 for (int d = 0; d < 8; ++d)
@@ -1041,7 +1044,7 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS>
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false>
 tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     using P = TileSmem<T, FWD, ROWS>;
@@ -1102,23 +1105,28 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.salign = salign;
 
     // Per call: the attribute belongs to the current device.
-    const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS>,
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS>
+    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST>
         <<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (const T *)in, (T *)out, tg);
     return launch_status();
 }
 
 template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT>
-tok_status launch_form(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+tok_status launch_form(HaarTmaForm form, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    return rows ? launch<T, VIDEO, FWD, ADJ, EXT, true>(in, out, d, stream)
-                : launch<T, VIDEO, FWD, ADJ, EXT, false>(in, out, d, stream);
+    if (form == HaarTmaForm::rows)
+        return launch<T, VIDEO, FWD, ADJ, EXT, true>(in, out, d, stream);
+    if constexpr (!FWD) {
+        if (form == HaarTmaForm::boxes_any_store)
+            return launch<T, VIDEO, FWD, ADJ, EXT, false, true>(in, out, d, stream);
+    }
+    return launch<T, VIDEO, FWD, ADJ, EXT, false>(in, out, d, stream);
 }
 
 // Limits shared by both forms: 32-bit frame, group and tile numbers, and the 64 planes of
@@ -1153,6 +1161,10 @@ HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype d
                            : aligned(in, 16) && (d.w * es) % 16 == 0 && aligned(out, 16) && (d.W * es) % 16 == 0;
     if (boxes)
         return HaarTmaForm::boxes;
+    // Inverse whose source takes the box form but whose pixel rows do not (cropped or chunked
+    // odd widths, a destination off a 16-byte boundary): box loads, stores of run-time width.
+    if (!fwd && aligned(in, 16) && (d.w * es) % 16 == 0)
+        return HaarTmaForm::boxes_any_store;
     // Row form: any 16-byte-aligned source.
     return aligned(in, 16) ? HaarTmaForm::rows : HaarTmaForm::none;
 }
@@ -1160,41 +1172,41 @@ HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype d
 tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
                            const HaarDims &d, cudaStream_t stream)
 {
-    const bool video = d.video, rows = form == HaarTmaForm::rows;
+    const bool video = d.video;
     if (d.ext) {
         if (dt == TOK_BF16) {
             using B16 = __nv_bfloat16;
             if (video)
-                return fwd ? launch_form<B16, true, true, false, true>(rows, in, out, d, stream)
-                           : launch_form<B16, true, false, false, true>(rows, in, out, d, stream);
-            return fwd ? launch_form<B16, false, true, false, true>(rows, in, out, d, stream)
-                       : launch_form<B16, false, false, false, true>(rows, in, out, d, stream);
+                return fwd ? launch_form<B16, true, true, false, true>(form, in, out, d, stream)
+                           : launch_form<B16, true, false, false, true>(form, in, out, d, stream);
+            return fwd ? launch_form<B16, false, true, false, true>(form, in, out, d, stream)
+                       : launch_form<B16, false, false, false, true>(form, in, out, d, stream);
         }
         if (video)
-            return fwd ? launch_form<float, true, true, false, true>(rows, in, out, d, stream)
-                       : launch_form<float, true, false, false, true>(rows, in, out, d, stream);
-        return fwd ? launch_form<float, false, true, false, true>(rows, in, out, d, stream)
-                   : launch_form<float, false, false, false, true>(rows, in, out, d, stream);
+            return fwd ? launch_form<float, true, true, false, true>(form, in, out, d, stream)
+                       : launch_form<float, true, false, false, true>(form, in, out, d, stream);
+        return fwd ? launch_form<float, false, true, false, true>(form, in, out, d, stream)
+                   : launch_form<float, false, false, false, true>(form, in, out, d, stream);
     }
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (!video)
-            return fwd ? launch_form<B16, false, true, false, false>(rows, in, out, d, stream)
-                       : launch_form<B16, false, false, false, false>(rows, in, out, d, stream);
+            return fwd ? launch_form<B16, false, true, false, false>(form, in, out, d, stream)
+                       : launch_form<B16, false, false, false, false>(form, in, out, d, stream);
         if (adj)
-            return fwd ? launch_form<B16, true, true, true, false>(rows, in, out, d, stream)
-                       : launch_form<B16, true, false, true, false>(rows, in, out, d, stream);
-        return fwd ? launch_form<B16, true, true, false, false>(rows, in, out, d, stream)
-                   : launch_form<B16, true, false, false, false>(rows, in, out, d, stream);
+            return fwd ? launch_form<B16, true, true, true, false>(form, in, out, d, stream)
+                       : launch_form<B16, true, false, true, false>(form, in, out, d, stream);
+        return fwd ? launch_form<B16, true, true, false, false>(form, in, out, d, stream)
+                   : launch_form<B16, true, false, false, false>(form, in, out, d, stream);
     }
     if (!video)
-        return fwd ? launch_form<float, false, true, false, false>(rows, in, out, d, stream)
-                   : launch_form<float, false, false, false, false>(rows, in, out, d, stream);
+        return fwd ? launch_form<float, false, true, false, false>(form, in, out, d, stream)
+                   : launch_form<float, false, false, false, false>(form, in, out, d, stream);
     if (adj)
-        return fwd ? launch_form<float, true, true, true, false>(rows, in, out, d, stream)
-                   : launch_form<float, true, false, true, false>(rows, in, out, d, stream);
-    return fwd ? launch_form<float, true, true, false, false>(rows, in, out, d, stream)
-               : launch_form<float, true, false, false, false>(rows, in, out, d, stream);
+        return fwd ? launch_form<float, true, true, true, false>(form, in, out, d, stream)
+                   : launch_form<float, true, false, true, false>(form, in, out, d, stream);
+    return fwd ? launch_form<float, true, true, false, false>(form, in, out, d, stream)
+               : launch_form<float, true, false, false, false>(form, in, out, d, stream);
 }
 
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)

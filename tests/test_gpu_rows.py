@@ -2,8 +2,10 @@
 
 The row form takes the planar calls whose rows are not whole 16-byte units (bf16 W % 8 != 0
 or w % 8 != 0, fp32 W % 4 != 0 or w % 4 != 0, odd w) on 16-byte-aligned sources: each source
-row of a tile is staged by 1D TMA boxes from the 16-byte boundary at or below it and read
-back realigned; stores take the widest width the destination address allows.
+row of a tile is staged by a bulk copy from the 16-byte boundary at or below it and read
+back realigned; stores take the widest width the destination address allows.  An inverse
+whose source rows are whole 16-byte units but whose pixel rows are not keeps the box loads
+and takes only the run-time store widths.
 
 Checked here: the oracle, element by element (same tolerances as the other Haar parity
 tests), and bit-for-bit agreement with the register kernels, which a view one element past
@@ -116,9 +118,12 @@ def test_rows_form_adjoints(shape, dtype):
 @pytest.mark.parametrize("shape,dtype,ms,mt", [((1, 2, 7, 21, 45), torch.bfloat16, 4, 4),
                                                ((1, 2, 11, 13, 30), torch.float32, 8, 8),
                                                ((2, 3, 1, 30, 50), torch.bfloat16, 4, 4),
-                                               ((1, 1, 6, 9, 1277), torch.bfloat16, 16, 8)])
+                                               ((1, 1, 6, 9, 1277), torch.bfloat16, 16, 8),
+                                               ((1, 2, 9, 12, 54), torch.bfloat16, 32, 4)])
 def test_rows_form_padded_and_cropped_equal_register_kernels(shape, dtype, ms, mt):
-    """Padding (zeros past the clip's rows and columns, mirrored frames) and cropping in the row form."""
+    """Padding (zeros past the clip's rows and columns, mirrored frames) and cropping in the row form;
+    where the padded coefficient rows are whole 16-byte units (w = 8, 16, 320 here) the cropped
+    inverse loads boxes and stores its odd-width pixel rows at run-time widths."""
     B, C, T, H, W = shape
     x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
     y = hwp.haar_fwd_padded(x, ms, mt)
