@@ -20,9 +20,12 @@
  *     TOK_ERR_CUDA; tok_last_cuda_error() gives the CUDA error code.
  *   - Inputs and outputs must not overlap (TOK_ERR_ALIAS).
  *   - Pointers need natural alignment of their element type (TOK_ERR_ALIGN
- *     otherwise).  16-byte-aligned buffers with suitable extents take the
- *     vectorized kernels; other layouts take element-wise GPU kernels with
- *     identical results.  There is no CPU path.
+ *     otherwise).  Every layout gives identical results; the kernel taken
+ *     depends on the layout: a 16-byte-aligned source whose rows are whole
+ *     16-byte units is loaded tile by tile with tensor copies; other
+ *     16-byte-aligned sources row by row with bulk copies; a source that is
+ *     not 16-byte aligned takes element-wise GPU kernels.  There is no CPU
+ *     path.
  *
  * Sources for the operations (page title, section):
  *   [guide] "NVIDIA Cosmos Tokenizer 完全指南" (a guide to the Cosmos Tokenizer
