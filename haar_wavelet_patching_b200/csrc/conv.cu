@@ -13,9 +13,12 @@
 // before the first frame and by nothing after the last, so output frame t reads
 // frames t - k + 1 .. t (M = B*T*h*w, N = C_out, K = k*C_mid).  They run CUTLASS's
 // sm100 implicit-GEMM kernels, instantiated here: TMA im2col loads of the activation
-// tile and tiled loads of the filter into shared memory, tcgen05.mma issued by one
-// thread with the accumulator in tensor memory, and a TMA store epilogue that rounds
-// to bf16.  One-CTA MMA and a 1 x 1 x 1 cluster: no cluster multicast anywhere.
+// tile and tiled loads of the filter into shared memory, tcgen05.mma with the
+// accumulator in tensor memory, and a TMA store epilogue that rounds to bf16.  The MMA
+// is the 2-SM form (cta_group::2): a pair of CTAs on a 2 x 1 x 1 cluster computes a
+// 256 x 256 tile, each CTA loading half of the activations and half of the filter, so
+// the filter crosses L2 half as often per flop as with 128 x 256 one-CTA tiles.  The
+// loads of a 2 x 1 x 1 cluster carry no multicast (plain cta_group::2 TMA loads).
 #include "cutlass/cutlass.h"
 #include "cutlass/kernel_hardware_info.hpp"
 #include "cute/tensor.hpp"
@@ -35,19 +38,19 @@ namespace {
 
 using namespace cute;
 using Elem = cutlass::bfloat16_t;
-using MmaTile = Shape<_128, _256, Shape<_64>>; // 128 output positions x 256 channels per CTA, K step 64
-using Cluster = Shape<_1, _1, _1>;
+using MmaTile = Shape<_256, _256, Shape<_64>>; // 256 output positions x 256 channels per CTA pair, K step 64
+using Cluster = Shape<_2, _1, _1>;             // the pair of a 2-SM MMA (no multicast loads)
 
 template <class Layout> struct Fprop {
     using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<
         cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, MmaTile, Cluster,
         cutlass::epilogue::collective::EpilogueTileAuto, float, float, Elem, Layout, 8, Elem, Layout, 8,
-        cutlass::epilogue::collective::EpilogueScheduleAuto>::CollectiveOp;
+        cutlass::epilogue::TmaWarpSpecialized2Sm>::CollectiveOp;
     using Mainloop = typename cutlass::conv::collective::CollectiveBuilder<
         cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, cutlass::conv::Operator::kFprop, Elem, Layout, 8,
         Elem, Layout, 8, float, MmaTile, Cluster,
         cutlass::conv::collective::StageCountAutoCarveout<sizeof(typename Epilogue::SharedStorage)>,
-        cutlass::conv::collective::KernelScheduleAuto>::CollectiveOp;
+        cutlass::conv::KernelImplicitTmaWarpSpecialized2SmSm100>::CollectiveOp;
     using Problem = cutlass::conv::ConvProblemShape<cutlass::conv::Operator::kFprop, Mainloop::NumSpatialDimensions>;
     using Kernel = cutlass::conv::kernel::ConvUniversal<Problem, Mainloop, Epilogue>;
     using Op = cutlass::conv::device::ConvUniversalAdapter<Kernel>;
