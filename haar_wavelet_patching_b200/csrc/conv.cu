@@ -18,7 +18,7 @@
 // is the 2-SM form (cta_group::2): a pair of CTAs on a 2 x 1 x 1 cluster computes a
 // 256 x 256 tile, each CTA loading half of the activations and half of the filter, so
 // the filter crosses L2 half as often per flop as with 128 x 256 one-CTA tiles.  The
-// loads of a 2 x 1 x 1 cluster carry no multicast (plain cta_group::2 TMA loads).
+// loads of a 2 x 1 x 1 cluster are plain cta_group::2 TMA loads, none broadcast to the pair.
 #include "cutlass/cutlass.h"
 #include "cutlass/kernel_hardware_info.hpp"
 #include "cute/tensor.hpp"
@@ -39,7 +39,7 @@ namespace {
 using namespace cute;
 using Elem = cutlass::bfloat16_t;
 using MmaTile = Shape<_256, _256, Shape<_64>>; // 256 output positions x 256 channels per CTA pair, K step 64
-using Cluster = Shape<_2, _1, _1>;             // the pair of a 2-SM MMA (no multicast loads)
+using Cluster = Shape<_2, _1, _1>;             // the pair of a 2-SM MMA (no broadcast loads)
 
 template <class Layout> struct Fprop {
     using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<

@@ -29,7 +29,7 @@
 //
 // Waits are bounded: a barrier that does not complete within kWaitPolls polls
 // makes the warp stop, drain what it issued and count a timeout that
-// tok_check_device() reports.  No cluster multicast is used.
+// tok_check_device() reports.  Every load fills only this CTA's own shared memory.
 #include <cstring>
 #include <numeric>
 

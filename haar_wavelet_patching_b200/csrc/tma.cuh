@@ -1,6 +1,6 @@
 // TMA (cp.async.bulk.tensor) and mbarrier primitives for sm_100a, as inline PTX,
 // plus the host-side tensor-map encoder (taken from the driver at run time, so
-// the library does not link libcuda).  No cluster multicast anywhere: every
+// the library does not link libcuda).  No load is broadcast to a cluster: every
 // load targets this CTA's own shared memory from this GPU's own memory.
 #pragma once
 
