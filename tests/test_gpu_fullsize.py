@@ -199,3 +199,34 @@ def test_fsq_backward_full_latent():
     assert (np.abs(gu.double().cpu().numpy() - ref_u) <= tol_u).all()
     tol_w = 1e-5 * np.einsum("bis,bcs->ic", gs, np.abs(u.astype(np.float64))) + 1e-30
     assert (np.abs(gw.double().cpu().numpy() - ref_w) <= tol_w).all()
+
+
+def test_image_beyond_the_tile_kernels_limits():
+    """A [1,1,1,32768,32768] bf16 image (2 GB): its 2^26 latent pixels put the 64 planes of a
+    channel past the 32-bit element offsets the TMA kernels use, so the vectorized register
+    kernels take it.  Checked bit for bit against the TMA kernels on 4096-row strips (tensors of
+    their own), and on sampled blocks against the oracle."""
+    H = W = 32768
+    g = torch.Generator(device="cuda").manual_seed(7)
+    x = (torch.rand((1, 1, 1, H, W), generator=g, device="cuda") * 2 - 1).to(torch.bfloat16)
+    y = hwp.haar_fwd(x)
+    xr = hwp.haar_inv(y, 1, H, W)
+    hwp.tok_check_device()
+    assert y.shape == (1, 16, 1, H // 4, W // 4)
+    for r0 in (0, H - 4096):
+        strip = x[:, :, :, r0:r0 + 4096].contiguous()
+        ys = hwp.haar_fwd(strip)
+        assert torch.equal(ys, y[:, :, :, r0 // 4:r0 // 4 + 1024])
+        xs = hwp.haar_inv(ys, 1, 4096, W)
+        assert torch.equal(xs, xr[:, :, :, r0:r0 + 4096])
+        del strip, ys, xs
+    rng = np.random.default_rng(7)
+    pos = [(int(rng.integers(H // 4)), int(rng.integers(W // 4))) for _ in range(400)]
+    pos += [(0, 0), (0, W // 4 - 1), (H // 4 - 1, 0), (H // 4 - 1, W // 4 - 1)]
+    blocks = np.stack([x[0, 0, 0, 4 * i:4 * i + 4, 4 * j:4 * j + 4].double().cpu().numpy() for i, j in pos])
+    ref = oracle.haar_fwd(blocks[:, None, None])  # [n, 16, 1, 1, 1]
+    got = np.stack([y[0, :, 0, i, j].double().cpu().numpy() for i, j in pos])
+    tol = haar_bf16_tolerance(ref[:, :, 0, 0, 0], np.abs(blocks).sum(axis=(1, 2))[:, None], False)
+    assert (np.abs(got - ref[:, :, 0, 0, 0]) <= tol).all()
+    del x, y, xr
+    torch.cuda.empty_cache()
