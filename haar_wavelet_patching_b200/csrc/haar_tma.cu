@@ -1098,7 +1098,7 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.W = d.W;
     tg.h = d.h;
     tg.w = d.w;
-    tg.ntiles = (uint32_t)(ntx * nty * d.nq * d.B * d.C); // < 2^32: checked by haar_tma_eligible
+    tg.ntiles = (uint32_t)(ntx * nty * d.nq * d.B * d.C); // < 2^32: checked by tma_limits_ok
     tg.fbase = (int)d.fbase;
     tg.rep = d.rep;
     tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
@@ -1139,16 +1139,6 @@ bool tma_limits_ok(const HaarDims &d)
 }
 
 } // namespace
-
-bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
-{
-    const int64_t es = dt == TOK_F32 ? 4 : 2;
-    if (!aligned(in, 16) || !aligned(out, 16))
-        return false;
-    if ((d.w * es) % 16 != 0 || (d.W * es) % 16 != 0) // row strides of both tensors: multiples of 16 bytes
-        return false;
-    return tma_limits_ok(d) && sm_count() > 0;
-}
 
 HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
@@ -1379,7 +1369,11 @@ tok_status launch_cl_c(const void *in, void *out, const HaarDims &d, cudaStream_
 
 bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
-    return d.C >= 1 && d.C <= 4 && haar_tma_eligible(in, out, dt, d);
+    // The pixel side takes the box form; a block's G*C outputs are whole 16-byte pieces at any w,
+    // and the copy-out works on block pairs (w even).
+    const int64_t es = dt == TOK_F32 ? 4 : 2;
+    return d.C >= 1 && d.C <= 4 && aligned(in, 16) && aligned(out, 16) && (d.W * es) % 16 == 0 && d.w % 2 == 0 &&
+           tma_limits_ok(d) && sm_count() > 0;
 }
 
 tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream)

@@ -24,10 +24,6 @@ struct HaarDims {
     bool ext = false;
 };
 
-// Strict test (the channels-last kernel): 16-byte-aligned tensors whose rows are multiples
-// of 16 bytes on both sides.
-bool haar_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
-
 // Which form of the TMA kernel takes a planar call in direction fwd: boxes (the source's
 // rows are whole 16-byte units, and so are the destination's where it stores 16-byte rows),
 // boxes_any_store (inverse: box loads, pixel-row stores of run-time width), rows (any

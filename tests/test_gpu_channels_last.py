@@ -19,6 +19,8 @@ CASES = [
     ((1, 2, 13, 20, 64), torch.float32, "TMA fp32, C = 2"),
     ((1, 4, 5, 8, 32), torch.bfloat16, "TMA, C = 4"),
     ((2, 3, 1, 36, 64), torch.bfloat16, "TMA image, partial block rows"),
+    ((1, 3, 9, 16, 72), torch.bfloat16, "TMA, w = 18 (coefficient rows not whole 16-byte units)"),
+    ((1, 2, 5, 8, 40), torch.float32, "TMA fp32, w = 10"),
     ((1, 5, 9, 16, 64), torch.bfloat16, "register, C = 5"),
     ((1, 3, 9, 12, 44), torch.float32, "register, ragged row"),
     ((1, 2, 1, 8, 20), torch.bfloat16, "register image"),
