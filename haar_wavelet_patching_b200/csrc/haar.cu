@@ -773,7 +773,7 @@ tok_status single_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_
         return TOK_ERR_ALIAS;
     HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, 0, g.Tq};
     dims.video = video;
-    if (haar_single_tma_eligible(in, out, dt, dims))
+    if (haar_single_tma_eligible(fwd, in, out, dt, dims))
         return haar_single_tma_launch(fwd, in, out, dt, dims, stream);
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;

@@ -1275,10 +1275,13 @@ tok_status launch_single(const void *in, void *out, const HaarDims &d, cudaStrea
 
 } // namespace
 
-bool haar_single_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
+bool haar_single_tma_eligible(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
+    // Only the source goes through TMA (pixels on the forward, coefficients on the inverse);
+    // both directions store element pairs (the forward's at even block columns, w even; the
+    // inverse's at even pixel columns, W even).
     const int64_t es = dt == TOK_F32 ? 4 : 2;
-    if (!aligned(in, 16) || !aligned(out, 16) || (d.w * es) % 16 != 0 || (d.W * es) % 16 != 0)
+    if (!aligned(in, 16) || !aligned(out, 2 * es) || ((fwd ? d.W : d.w) * es) % 16 != 0 || d.w % 2 != 0)
         return false;
     const int64_t ntiles = ((d.w + 63) / 64) * (d.h / 8 + 1) * d.Tq * d.B * d.C;
     if (d.B * d.C * d.T >= (int64_t)1 << 31 || 8 * d.B >= (int64_t)1 << 31 || d.W >= (int64_t)1 << 31 ||

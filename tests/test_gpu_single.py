@@ -40,6 +40,7 @@ CASES = [
     ((1, 2, 5, 36, 160), synth.BF16, "TMA bf16, ragged block rows"),
     ((2, 3, 1, 40, 96), synth.BF16, "TMA image"),
     ((1, 2, 1, 18, 24), synth.F32, "TMA image fp32"),
+    ((1, 2, 5, 12, 24), synth.BF16, "TMA forward (w = 12: coefficient rows not 16-byte units), register inverse"),
     ((1, 2, 9, 10, 22), synth.BF16, "register bf16"),
     ((1, 1, 3, 6, 14), synth.F32, "register fp32"),
     ((2, 2, 1, 6, 10), synth.BF16, "register image"),
