@@ -70,6 +70,9 @@ struct TileGrid {
     // (salign = 32 bytes / element, a power of two), so every warp's plane store starts on a
     // sector; else 0.
     int salign;
+    // Inverse, row form: the plane stride is a multiple of 16 bytes, so the staged rows of one
+    // block row (one per group) all sit at the same offset in their staged copies.
+    int planes_share_offset;
 };
 
 // Source frame of frame f of a T-frame clip mirrored about its last frame (period 2(T-1)).
@@ -544,20 +547,37 @@ __global__ void __launch_bounds__(32)
                     }
                 }
             } else {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float2 p;
-                    if constexpr (ROWS) {
-                        const unsigned mb = row_off[s * 64 + g * RW + rw];
-                        p = staged_pair(tile + (g * RW + rw) * P::ROW, mb + lane * 2 * (uint32_t)sizeof(T),
-                                        (T *)nullptr);
-                    } else {
-                        p = SRow<T>::load_pair(tin + (g * RW + rw) * WT + 2 * lane);
-                    }
+                auto put = [&](int g, float2 p) {
                     if constexpr (VIDEO)
                         v[kt_of(g)][ky_of(g)][kx_of(g)] = p;
                     else
                         v[0][ky2_of(g)][kx2_of(g)] = p;
+                };
+                if constexpr (ROWS) {
+                    // When the plane stride is a multiple of 16 bytes, the G staged rows of this block
+                    // row share one offset: hoisted, and one aligned load per pair when it allows.
+                    const uint32_t o0 = row_off[s * 64 + rw] + lane * 2 * (uint32_t)sizeof(T);
+                    const unsigned char *rows0 = tile + rw * P::ROW;
+                    if (tg.planes_share_offset && (o0 & (2 * sizeof(T) - 1)) == 0) {
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            put(g, SRow<T>::load_pair(reinterpret_cast<const T *>(rows0 + g * RW * P::ROW + o0)));
+                    } else if (tg.planes_share_offset) {
+#pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            put(g, staged_pair(rows0 + g * RW * P::ROW, o0, (T *)nullptr));
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const unsigned mb = row_off[s * 64 + g * RW + rw];
+                            put(g, staged_pair(tile + (g * RW + rw) * P::ROW, mb + lane * 2 * (uint32_t)sizeof(T),
+                                               (T *)nullptr));
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < G; ++g)
+                        put(g, SRow<T>::load_pair(tin + (g * RW + rw) * WT + 2 * lane));
                 }
             }
 
@@ -1103,6 +1123,7 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.rep = d.rep;
     tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
     tg.salign = salign;
+    tg.planes_share_offset = ((int64_t)d.C * d.Tq * d.h * d.w * (int64_t)es) % 16 == 0;
 
     // Per call: the attribute belongs to the current device.
     const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST>,
