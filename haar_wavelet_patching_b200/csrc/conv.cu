@@ -40,11 +40,14 @@ using namespace cute;
 using Elem = cutlass::bfloat16_t;
 using MmaTile = Shape<_256, _256, Shape<_64>>; // 256 output positions x 256 channels per CTA pair, K step 64
 using Cluster = Shape<_2, _1, _1>;             // the pair of a 2-SM MMA (no broadcast loads)
+// The epilogue stores 128 x 32 subtiles: its smaller shared-memory staging leaves room for a
+// sixth mainloop stage (measured 1-5% faster than the automatic 128 x 64 with five stages).
+using EpiTile = Shape<_128, _32>;
 
 template <class Layout> struct Fprop {
     using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<
-        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, MmaTile, Cluster,
-        cutlass::epilogue::collective::EpilogueTileAuto, float, float, Elem, Layout, 8, Elem, Layout, 8,
+        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, MmaTile, Cluster, EpiTile, float, float, Elem,
+        Layout, 8, Elem, Layout, 8,
         cutlass::epilogue::TmaWarpSpecialized2Sm>::CollectiveOp;
     using Mainloop = typename cutlass::conv::collective::CollectiveBuilder<
         cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, cutlass::conv::Operator::kFprop, Elem, Layout, 8,
