@@ -211,6 +211,52 @@ def cpu_baseline(reps=3):
             "sample": f"{sample_text(CPU_SAMPLE_FRAMES, CPU_SAMPLE_GRIDS)}; {reps} reps of {dt:.2f} s"}
 
 
+def oracle_step_parts(x64, lat, w, windows_per_part=1):
+    """The oracle step split into independent parts for a thread pool: per clip channel, the
+    windows in groups (the first chunk with the frame-0 replica, then chunks of 4k frames, the
+    oracle's streaming calls: together exactly the whole clip's transform), and the FSQ calls
+    per latent grid.  Each part returns its outputs (for the equivalence test)."""
+    import oracle
+    B, C, T, H, W = x64.shape
+    parts = []
+    for c in range(C):
+        f0 = 0
+        while f0 < T:
+            first = f0 == 0
+            f1 = min(T, (1 if first else f0) + 4 * windows_per_part)
+
+            def haar_part(c=c, f0=f0, f1=f1, first=first):
+                xs = x64[:, c:c + 1, f0:f1]
+                y = oracle.haar_fwd_chunk(xs, first)
+                return ("haar", c, f0, y, oracle.haar_inv_chunk(y, f1 - f0, H, W, first))
+            parts.append(haar_part)
+            f0 = f1
+    for g in range(lat.shape[0]):
+        def fsq_part(g=g):
+            idx, _, _ = oracle.fsq_encode(lat[g:g + 1], w)
+            return ("fsq", g, idx, oracle.fsq_decode(idx, w)[0])
+        parts.append(fsq_part)
+    return parts
+
+
+def cpu_baseline_threads(reps=3):
+    """The same sample as cpu_baseline, its independent parts on a pool of the host's cores
+    (ctypes releases the interpreter lock during each oracle call)."""
+    from concurrent.futures import ThreadPoolExecutor
+    x64, lat, w = oracle_sample_inputs()
+    parts = oracle_step_parts(x64, lat, w)
+    cores = len(os.sched_getaffinity(0))
+    with ThreadPoolExecutor(max_workers=cores) as pool:
+        list(pool.map(lambda f: f(), parts))  # warm
+        t = time.perf_counter()
+        for _ in range(reps):
+            list(pool.map(lambda f: f(), parts))
+        dt = (time.perf_counter() - t) / reps
+    return {"value": round(oracle_sample_bytes() / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{sample_text(CPU_SAMPLE_FRAMES, CPU_SAMPLE_GRIDS).replace('single-threaded', 'the same')}, "
+                      f"split into {len(parts)} independent parts on {cores} threads; {reps} reps of {dt:.2f} s"}
+
+
 def reference_sample(steps, warmup, budget_s=150.0):
     """Per-step sample (frames = 1 + 4m, grids) sized so steps + warmup oracle passes take about budget_s."""
     x64, lat, w = oracle_sample_inputs(5, 1)
@@ -649,6 +695,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+        line["cpu_baseline_threads"] = cpu_baseline_threads()
     print(json.dumps(line), flush=True)
     return 0
 

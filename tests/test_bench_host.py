@@ -62,3 +62,32 @@ def test_max_over_ranks_gloo_two_ranks():
 
 def test_single_process_max_is_identity():
     assert bench.max_over_ranks(3.5, "cpu") == 3.5
+
+
+def test_threaded_baseline_parts_are_the_whole_oracle_step():
+    """The parts the threaded CPU baseline times (per channel window chunks, per latent grid)
+    compute exactly the unsplit oracle step."""
+    import numpy as np
+
+    import oracle
+    import synth
+    x64 = synth.bf16_bits_to_f64(synth.smooth_field((1, 2, 13, 8, 16), seed=11))
+    lat = synth.fsq_input(4)[:3, :, :96]
+    w = synth.fsq_weight()
+    parts = bench.oracle_step_parts(x64, lat, w, windows_per_part=1)
+    assert len(parts) == 2 * 3 + 3  # per channel: windows 0-1 in the first chunk, then 2 and 3; 3 grids
+    out = [f() for f in parts]
+    y = oracle.haar_fwd(x64)
+    xr = oracle.haar_inv(y, 13, 8, 16)
+    C = 2
+    for kind, *rest in out:
+        if kind == "haar":
+            c, f0, yc, xc = rest
+            t0 = 0 if f0 == 0 else (f0 + 3) // 4
+            np.testing.assert_allclose(yc[0], y[0, c::C, t0:t0 + yc.shape[2]], rtol=0, atol=1e-12)
+            np.testing.assert_allclose(xc[0, 0], xr[0, c, f0:f0 + xc.shape[2]], rtol=0, atol=1e-12)
+        else:
+            g, idx, dec = rest
+            ref_idx, _, _ = oracle.fsq_encode(lat[g:g + 1], w)
+            assert np.array_equal(idx, ref_idx)
+            np.testing.assert_array_equal(dec, oracle.fsq_decode(ref_idx, w)[0])
