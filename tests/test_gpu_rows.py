@@ -92,6 +92,15 @@ def test_misaligned_destination_only(shape, dtype):
     hwp.tok_haar_inv(y, xo)
     hwp.tok_check_device()
     assert torch.equal(xo, hwp.haar_inv(y, *shape[2:]))
+    if shape[2] > 1:
+        # The adjoints the same way (the patcher's adjoint writes pixels like the inverse).
+        ao = empty_off(shape, dtype)
+        hwp.tok_haar_fwd_adjoint(y, ao)
+        bo = empty_off(y.shape, dtype)
+        hwp.tok_haar_inv_adjoint(x, bo)
+        hwp.tok_check_device()
+        assert torch.equal(ao, hwp.haar_fwd_adjoint(y, *shape[2:]))
+        assert torch.equal(bo, hwp.haar_inv_adjoint(x))
 
 
 @pytest.mark.parametrize("shape,dtype", [((1, 2, 9, 16, 44), torch.bfloat16), ((2, 1, 13, 8, 52), torch.float32)])
