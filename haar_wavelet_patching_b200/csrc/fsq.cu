@@ -25,8 +25,8 @@
 // ~96 FMAs and 33 compares per token, under the HBM roofline.
 //
 // Encode at C = 16 with 16-byte-aligned tensors (the main path): one-shot
-// single-warp CTAs, each owning two tiles of 128 consecutive tokens x 16
-// channel planes (8 KB); lane 0 issues both TMA loads at once, the lanes take
+// single-warp CTAs, each owning one tile of 128 consecutive tokens x 16
+// channel planes (8 KB); lane 0 issues its TMA load, the lanes take
 // 4 tokens each and run the projection as packed f32x2 fused multiply-adds
 // (two tokens per instruction, each lane of the pair the same fp32 chain).  A
 // grid of small CTAs in token order keeps the working set a compact, moving
@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(kThreads)
 // Encode, TMA path (C = 16).
 // ---------------------------------------------------------------------------
 constexpr int kEncTokens = 128; // tokens per tile: 16 planes x 512 bytes = 8 KB
-constexpr int kEncKT = 2;       // tiles per CTA, loaded at once
-constexpr int kEncSmem = kEncKT * 16 * kEncTokens * 4 + 8 * kEncKT + 16 * 8 * 4;
+constexpr int kEncKT = 1;       // tiles per CTA (one: more resident warps measured faster than two or four)
+constexpr int kEncSmem = kEncKT * 16 * kEncTokens * 4 + 16 * kEncKT + 16 * 8 * 4; // tiles, barriers, weights
 
 template <bool CODES>
 __global__ void __launch_bounds__(32)
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(32)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     float *tiles = reinterpret_cast<float *>(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + kEncKT * TILE * 4);
-    float *ws = reinterpret_cast<float *>(smem_raw + kEncKT * TILE * 4 + 8 * kEncKT); // [16][8]
+    float *ws = reinterpret_cast<float *>(smem_raw + kEncKT * TILE * 4 + 16 * kEncKT); // [16][8], 16-byte aligned
     const int lane = threadIdx.x;
     const uint32_t first = blockIdx.x * (uint32_t)kEncKT;
     const int count = (int)min((uint32_t)kEncKT, ntiles - first);
