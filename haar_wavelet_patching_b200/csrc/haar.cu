@@ -773,8 +773,9 @@ tok_status single_call(bool fwd, const void *in, void *out, tok_dtype dt, int64_
         return TOK_ERR_ALIAS;
     HaarDims dims{B, C, T, H, W, g.Tq, g.h, g.w, 0, g.Tq};
     dims.video = video;
-    if (haar_single_tma_eligible(fwd, in, out, dt, dims))
-        return haar_single_tma_launch(fwd, in, out, dt, dims, stream);
+    const HaarTmaForm form = haar_single_tma_form(fwd, in, out, dt, dims);
+    if (form != HaarTmaForm::none)
+        return haar_single_tma_launch(fwd, form, in, out, dt, dims, stream);
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (video)

@@ -48,9 +48,7 @@ constexpr int kTileBlocks = 64; // blocks across a warp tile (256 pixels)
 constexpr int kTileElems = 4096; // elements of a warp tile, on either side
 
 template <typename T> struct WarpTiles {
-    static constexpr int KT = sizeof(T) == 2 ? 4 : 2;  // tiles per CTA, all loaded at once (32 KB)
-    static constexpr int TILE_BYTES = kTileElems * sizeof(T);
-    static constexpr int SMEM = KT * TILE_BYTES + 8 * KT; // buffers + mbarriers
+    static constexpr int KT = sizeof(T) == 2 ? 4 : 2; // tiles per CTA, all loaded at once (32 KB)
 };
 
 struct TileGrid {
@@ -902,12 +900,39 @@ template <bool VIDEO> struct SingleRows {
     static constexpr int RB = VIDEO ? 8 : 16; // block rows of a tile
 };
 
-template <typename T, bool VIDEO, bool FWD>
+// Shared memory of the single-level kernel; ROWS: the row form, as for the two-level kernel
+// (32 staged pixel rows of 128 pixels on the forward, 64 coefficient rows of 64 on the inverse).
+template <typename T, bool FWD, bool ROWS> struct SingleSmem {
+    static constexpr int KT = !ROWS ? WarpTiles<T>::KT : sizeof(T) == 2 ? 2 : 1;
+    static constexpr int NR = FWD ? 32 : 64;
+    static constexpr int ROW = (FWD ? 128 : 64) * (int)sizeof(T) + 16;
+    static constexpr int TILE = ROWS ? NR * ROW : kTileElems * (int)sizeof(T);
+    static constexpr int SMEM = KT * TILE + 8 * KT + (ROWS ? 64 * KT : 0);
+    static_assert(ROW % 16 == 0 && TILE % 16 == 0, "16-byte bulk-copy destinations");
+};
+
+// Four adjacent elements (the two pixels of blocks j and j + 1 in one pixel row) at byte
+// offset o of a 16-byte-aligned staged row, without branches.
+__device__ __forceinline__ void staged_quad(const unsigned char *row, uint32_t o, __nv_bfloat16 *, float *p)
+{
+    const uint32_t *w = reinterpret_cast<const uint32_t *>(row + (o & ~3u));
+    const uint32_t sh = (o & 3u) * 8u;
+    const uint32_t r0 = __funnelshift_r(w[0], w[1], sh), r1 = __funnelshift_r(w[1], w[2], sh);
+    p[0] = bf16_lo(r0), p[1] = bf16_hi(r0), p[2] = bf16_lo(r1), p[3] = bf16_hi(r1);
+}
+__device__ __forceinline__ void staged_quad(const unsigned char *row, uint32_t o, float *, float *p)
+{
+    const float *w = reinterpret_cast<const float *>(row + o); // o is a multiple of 4
+    p[0] = w[0], p[1] = w[1], p[2] = w[2], p[3] = w[3];
+}
+
+template <typename T, bool VIDEO, bool FWD, bool ROWS>
 __global__ void __launch_bounds__(32)
     haar_single_kernel(const __grid_constant__ CUtensorMap xmap2, const __grid_constant__ CUtensorMap xmap1,
-                       const __grid_constant__ CUtensorMap ymap, T *__restrict__ out, const TileGrid tg)
+                       const __grid_constant__ CUtensorMap ymap, const T *__restrict__ src, T *__restrict__ out,
+                       const TileGrid tg)
 {
-    using P = WarpTiles<T>;
+    using P = SingleSmem<T, FWD, ROWS>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RB = SingleRows<VIDEO>::RB;
     constexpr int G = VIDEO ? 8 : 4;
@@ -919,8 +944,8 @@ __global__ void __launch_bounds__(32)
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const int lane = threadIdx.x;
-    T *in_buf = reinterpret_cast<T *>(smem_raw);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * TILE_BYTES);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * P::TILE);
+    unsigned char *row_off = reinterpret_cast<unsigned char *>(bars + KT); // ROWS: [tile][staged row]
 
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &bc) {
         const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
@@ -933,7 +958,73 @@ __global__ void __launch_bounds__(32)
     const uint32_t first = blockIdx.x * (uint32_t)KT;
     const int count = (int)min((uint32_t)KT, tg.ntiles - first);
 
-    if (lane == 0) {
+    if constexpr (ROWS) {
+        if (lane == 0) {
+            for (int s = 0; s < KT; ++s)
+                mbar_init(smem_addr(bars + s), 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        constexpr int VE = 16 / (int)sizeof(T);
+        constexpr int PER = P::NR / 32;
+        const unsigned char *src_b = reinterpret_cast<const unsigned char *>(src);
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t bc;
+            decode(first + s, tx, ty, tq, bc);
+            int64_t start[PER];
+            uint32_t nbulk[PER];
+            bool ok[PER];
+            uint32_t tx_bytes = 0;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                const int r = lane + 32 * k;
+                int64_t off;
+                if constexpr (FWD) {
+                    // Staged row r: frame slot r / (2 RB), pixel row 2 RB ty + r % (2 RB).
+                    const int a = r / (2 * RB);
+                    const int64_t y = (int64_t)2 * RB * ty + r % (2 * RB);
+                    const bool replica = VIDEO && tq == 0;
+                    const int64_t f = !VIDEO || replica ? 0 : 2 * tq - 1 + a;
+                    ok[k] = y < tg.H && !(replica && a != 0); // window 0 reads frame 0 only
+                    off = ((bc * tg.T + f) * tg.H + y) * tg.W + (int64_t)2 * WT * tx;
+                } else {
+                    const int g = r / RB;
+                    const int64_t row = (int64_t)RB * ty + r % RB;
+                    const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                    const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                    ok[k] = row < tg.h;
+                    off = ((b * G + g) * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + (int64_t)WT * tx;
+                }
+                const int mis = (int)(off % VE);
+                start[k] = (off - mis) * (int64_t)sizeof(T);
+                const int64_t avail = tg.n_src * (int64_t)sizeof(T) - start[k];
+                nbulk[k] = !ok[k] ? 0u : avail >= P::ROW ? (uint32_t)P::ROW : (uint32_t)(avail & ~(int64_t)15);
+                // A row that is not loaded is never used for a stored result: offset 0 keeps the
+                // realigned reads inside its staging row.
+                row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T)) : (unsigned char)0;
+                tx_bytes += __reduce_add_sync(0xFFFFFFFFu, nbulk[k]);
+            }
+            const uint32_t bar = smem_addr(bars + s);
+            if (lane == 0)
+                mbar_expect_tx(bar, tx_bytes);
+            __syncwarp();
+            unsigned char *tile = smem_raw + s * P::TILE;
+#pragma unroll
+            for (int k = 0; k < PER; ++k) {
+                if (!ok[k])
+                    continue;
+                unsigned char *dst = tile + (lane + 32 * k) * P::ROW;
+                if (nbulk[k] > 0)
+                    bulk_load(smem_addr(dst), src_b + start[k], nbulk[k], bar);
+                if (nbulk[k] < (uint32_t)P::ROW) { // the tensor's last, partial 16 bytes
+                    const int64_t end = min(tg.n_src * (int64_t)sizeof(T) - start[k], (int64_t)P::ROW);
+                    for (int64_t b = nbulk[k]; b < end; b += (int64_t)sizeof(T))
+                        *reinterpret_cast<T *>(dst + b) = *reinterpret_cast<const T *>(src_b + start[k] + b);
+                }
+            }
+        }
+    } else if (lane == 0) {
         for (int s = 0; s < KT; ++s)
             mbar_init(smem_addr(bars + s), 1);
         fence_barrier_init();
@@ -941,7 +1032,7 @@ __global__ void __launch_bounds__(32)
             int tx, ty, tq;
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
-            const uint32_t dst = smem_addr(in_buf + s * kTileElems), bar = smem_addr(bars + s);
+            const uint32_t dst = smem_addr(smem_raw + s * P::TILE), bar = smem_addr(bars + s);
             if constexpr (FWD) {
                 if (VIDEO && tq > 0) {
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
@@ -967,9 +1058,11 @@ __global__ void __launch_bounds__(32)
         int tx, ty, tq;
         int64_t bc;
         decode(first + s, tx, ty, tq, bc);
-        const T *tin = in_buf + s * kTileElems;
+        const unsigned char *tile = smem_raw + s * P::TILE;
+        const T *tin = reinterpret_cast<const T *>(tile);
         const int64_t j0 = (int64_t)tx * WT + 2 * lane; // this lane's first block column
-        const bool col_ok = j0 < tg.w;                  // w is even: block j0 + 1 exists too
+        const bool col_ok = j0 < tg.w;
+        const bool pair_ok = !ROWS || j0 + 1 < tg.w;    // block j0 + 1 exists (w is even outside the row form)
         const bool replica = VIDEO && tq == 0;
 
 #pragma unroll 2
@@ -981,16 +1074,29 @@ __global__ void __launch_bounds__(32)
                     const int fa = replica ? 0 : a;
 #pragma unroll
                     for (int r = 0; r < 2; ++r) {
-                        const T *src = tin + (fa * 2 * RB + 2 * rb + r) * 2 * WT + 4 * lane;
-                        const float2 p01 = SRow<T>::load_pair(src), p23 = SRow<T>::load_pair(src + 2);
-                        v[a][r][0] = make_float2(p01.x, p23.x); // pixel 0 of blocks j0, j0 + 1
-                        v[a][r][1] = make_float2(p01.y, p23.y); // pixel 1
+                        float q[4]; // pixels 0, 1 of block j0, then of block j0 + 1
+                        if constexpr (ROWS) {
+                            const int sr = fa * 2 * RB + 2 * rb + r;
+                            staged_quad(tile + sr * P::ROW, row_off[s * 64 + sr] + lane * 4 * (uint32_t)sizeof(T),
+                                        (T *)nullptr, q);
+                        } else {
+                            const T *px = tin + (fa * 2 * RB + 2 * rb + r) * 2 * WT + 4 * lane;
+                            const float2 p01 = SRow<T>::load_pair(px), p23 = SRow<T>::load_pair(px + 2);
+                            q[0] = p01.x, q[1] = p01.y, q[2] = p23.x, q[3] = p23.y;
+                        }
+                        v[a][r][0] = make_float2(q[0], q[2]); // pixel 0 of blocks j0, j0 + 1
+                        v[a][r][1] = make_float2(q[1], q[3]); // pixel 1
                     }
                 }
             } else {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float2 p = SRow<T>::load_pair(tin + (g * RB + rb) * WT + 2 * lane);
+                    float2 p;
+                    if constexpr (ROWS)
+                        p = staged_pair(tile + (g * RB + rb) * P::ROW,
+                                        row_off[s * 64 + g * RB + rb] + lane * 2 * (uint32_t)sizeof(T), (T *)nullptr);
+                    else
+                        p = SRow<T>::load_pair(tin + (g * RB + rb) * WT + 2 * lane);
                     if constexpr (VIDEO)
                         v[g >> 2][(g >> 1) & 1][g & 1] = p;
                     else
@@ -1023,16 +1129,40 @@ __global__ void __launch_bounds__(32)
             }
             const float2 scale = make_float2(SCALE, SCALE);
             const int64_t row = (int64_t)ty * RB + rb; // block row
+            bool pairs = true;
+            if constexpr (FWD && ROWS) {
+                // Pair stores when every storing lane's G pairs are aligned and whole (the alignment
+                // alternates with g only when the plane stride is odd), element stores otherwise;
+                // one warp-wide vote, taken before any lane leaves.
+                const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
+                const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
+                const T *yq = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                const uintptr_t amask = 2 * sizeof(T) - 1;
+                pairs = __all_sync(0xFFFFFFFFu, !col_ok || (pair_ok && ((uintptr_t)yq & amask) == 0 &&
+                                                            ((uintptr_t)(yq + tg.C.d * plane) & amask) == 0));
+            }
             if (!col_ok || row >= tg.h)
                 continue;
             if constexpr (FWD) {
                 const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
                 const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
                 T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
+                if (!ROWS || pairs) {
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float2 p = VIDEO ? v[g >> 2][(g >> 1) & 1][g & 1] : v[0][g >> 1][g & 1];
-                    gstore_pair(yp + (int64_t)g * tg.C.d * plane, __fmul2_rn(p, scale));
+                    for (int g = 0; g < G; ++g) {
+                        const float2 p = VIDEO ? v[g >> 2][(g >> 1) & 1][g & 1] : v[0][g >> 1][g & 1];
+                        gstore_pair(yp + (int64_t)g * tg.C.d * plane, __fmul2_rn(p, scale));
+                    }
+                } else {
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float2 q =
+                            __fmul2_rn(VIDEO ? v[g >> 2][(g >> 1) & 1][g & 1] : v[0][g >> 1][g & 1], scale);
+                        T *dst = yp + (int64_t)g * tg.C.d * plane;
+                        dst[0] = to_elem<T>(q.x);
+                        if (pair_ok)
+                            dst[1] = to_elem<T>(q.y);
+                    }
                 }
             } else {
                 T *xb = out + (bc * tg.T) * tg.H * tg.W + (2 * row) * tg.W + 2 * j0;
@@ -1046,7 +1176,8 @@ __global__ void __launch_bounds__(32)
                         const float2 q0 = __fmul2_rn(v[a][r][0], scale), q1 = __fmul2_rn(v[a][r][1], scale);
                         T *dst = xb + f * tg.H * tg.W + r * tg.W;
                         SRow<T>::store_pair(dst, make_float2(q0.x, q1.x));     // block j0: pixels 0, 1
-                        SRow<T>::store_pair(dst + 2, make_float2(q0.y, q1.y)); // block j0 + 1
+                        if (pair_ok)
+                            SRow<T>::store_pair(dst + 2, make_float2(q0.y, q1.y)); // block j0 + 1
                     }
                 }
             }
@@ -1243,10 +1374,10 @@ tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count
 namespace tok {
 namespace {
 
-template <typename T, bool VIDEO, bool FWD>
+template <typename T, bool VIDEO, bool FWD, bool ROWS>
 tok_status launch_single(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    using P = WarpTiles<T>;
+    using P = SingleSmem<T, FWD, ROWS>;
     constexpr int G = VIDEO ? 8 : 4, RB = SingleRows<VIDEO>::RB, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
@@ -1254,7 +1385,9 @@ tok_status launch_single(const void *in, void *out, const HaarDims &d, cudaStrea
     memset(&xm2, 0, sizeof xm2);
     memset(&xm1, 0, sizeof xm1);
     memset(&ym, 0, sizeof ym);
-    if (FWD) {
+    if (ROWS) {
+        // The row form reads the source through its pointer (bulk copies); no tensor map.
+    } else if (FWD) {
         const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
         const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
         const uint32_t box2[3] = {2u * WT, 2u * RB, 2u}, box1[3] = {2u * WT, 2u * RB, 1u};
@@ -1283,50 +1416,62 @@ tok_status launch_single(const void *in, void *out, const HaarDims &d, cudaStrea
     tg.h = d.h;
     tg.w = d.w;
     tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B * d.C);
-    const cudaError_t attr_err = cudaFuncSetAttribute(haar_single_kernel<T, VIDEO, FWD>,
+    tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_single_kernel<T, VIDEO, FWD, ROWS>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_single_kernel<T, VIDEO, FWD><<<grid, 32, P::SMEM, stream>>>(xm2, xm1, ym, (T *)out, tg);
+    haar_single_kernel<T, VIDEO, FWD, ROWS>
+        <<<grid, 32, P::SMEM, stream>>>(xm2, xm1, ym, (const T *)in, (T *)out, tg);
     return launch_status();
+}
+
+template <typename T, bool VIDEO, bool FWD>
+tok_status launch_single_form(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    return rows ? launch_single<T, VIDEO, FWD, true>(in, out, d, stream)
+                : launch_single<T, VIDEO, FWD, false>(in, out, d, stream);
 }
 
 } // namespace
 
-bool haar_single_tma_eligible(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d)
+HaarTmaForm haar_single_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
-    // Only the source goes through TMA (pixels on the forward, coefficients on the inverse);
-    // both directions store element pairs (the forward's at even block columns, w even; the
-    // inverse's at even pixel columns, W even).
     const int64_t es = dt == TOK_F32 ? 4 : 2;
-    if (!aligned(in, 16) || !aligned(out, 2 * es) || ((fwd ? d.W : d.w) * es) % 16 != 0 || d.w % 2 != 0)
-        return false;
     const int64_t ntiles = ((d.w + 63) / 64) * (d.h / 8 + 1) * d.Tq * d.B * d.C;
     if (d.B * d.C * d.T >= (int64_t)1 << 31 || 8 * d.B >= (int64_t)1 << 31 || d.W >= (int64_t)1 << 31 ||
-        d.H >= (int64_t)1 << 31 || ntiles >= (int64_t)1 << 32)
-        return false;
-    return sm_count() > 0;
+        d.H >= (int64_t)1 << 31 || ntiles >= (int64_t)1 << 32 || sm_count() <= 0 || !aligned(in, 16))
+        return HaarTmaForm::none;
+    // Box form: only the source goes through TMA (pixels on the forward, coefficients on the
+    // inverse), so its rows must be whole 16-byte units; both directions store element pairs
+    // (the forward's at even block columns, w even; the inverse's at even pixel columns, W even).
+    if (aligned(out, 2 * es) && ((fwd ? d.W : d.w) * es) % 16 == 0 && d.w % 2 == 0)
+        return HaarTmaForm::boxes;
+    // Row form: any row length; the forward votes between pair and element stores, the inverse
+    // stores pixel pairs (W is even).
+    return aligned(out, fwd ? es : 2 * es) ? HaarTmaForm::rows : HaarTmaForm::none;
 }
 
-tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d,
-                                  cudaStream_t stream)
+tok_status haar_single_tma_launch(bool fwd, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
+                                  const HaarDims &d, cudaStream_t stream)
 {
+    const bool rows = form == HaarTmaForm::rows;
     if (dt == TOK_BF16) {
         using B16 = __nv_bfloat16;
         if (d.video)
-            return fwd ? launch_single<B16, true, true>(in, out, d, stream)
-                       : launch_single<B16, true, false>(in, out, d, stream);
-        return fwd ? launch_single<B16, false, true>(in, out, d, stream)
-                   : launch_single<B16, false, false>(in, out, d, stream);
+            return fwd ? launch_single_form<B16, true, true>(rows, in, out, d, stream)
+                       : launch_single_form<B16, true, false>(rows, in, out, d, stream);
+        return fwd ? launch_single_form<B16, false, true>(rows, in, out, d, stream)
+                   : launch_single_form<B16, false, false>(rows, in, out, d, stream);
     }
     if (d.video)
-        return fwd ? launch_single<float, true, true>(in, out, d, stream)
-                   : launch_single<float, true, false>(in, out, d, stream);
-    return fwd ? launch_single<float, false, true>(in, out, d, stream)
-               : launch_single<float, false, false>(in, out, d, stream);
+        return fwd ? launch_single_form<float, true, true>(rows, in, out, d, stream)
+                   : launch_single_form<float, true, false>(rows, in, out, d, stream);
+    return fwd ? launch_single_form<float, false, true>(rows, in, out, d, stream)
+               : launch_single_form<float, false, false>(rows, in, out, d, stream);
 }
 
 } // namespace tok

@@ -37,9 +37,9 @@ tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in,
 
 // Single-level patcher / unpatcher (patch_size=2): pixels [B, C, T, H, W] <->
 // coefficients [B, G*C, Tq, h, w] with G = 8 (video), 4 (images), Tq = (T + 1) / 2, h = H/2.
-bool haar_single_tma_eligible(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d);
-tok_status haar_single_tma_launch(bool fwd, const void *in, void *out, tok_dtype dt, const HaarDims &d,
-                                  cudaStream_t stream);
+HaarTmaForm haar_single_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d);
+tok_status haar_single_tma_launch(bool fwd, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
+                                  const HaarDims &d, cudaStream_t stream);
 
 // Channels-last two-level patcher: pixels [B, C, T, H, W] -> [B, Tq, h, w, G*C] (1 <= C <= 4).
 bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);

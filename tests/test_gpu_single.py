@@ -40,10 +40,11 @@ CASES = [
     ((1, 2, 5, 36, 160), synth.BF16, "TMA bf16, ragged block rows"),
     ((2, 3, 1, 40, 96), synth.BF16, "TMA image"),
     ((1, 2, 1, 18, 24), synth.F32, "TMA image fp32"),
-    ((1, 2, 5, 12, 24), synth.BF16, "TMA forward (w = 12: coefficient rows not 16-byte units), register inverse"),
-    ((1, 2, 9, 10, 22), synth.BF16, "register bf16"),
-    ((1, 1, 3, 6, 14), synth.F32, "register fp32"),
-    ((2, 2, 1, 6, 10), synth.BF16, "register image"),
+    ((1, 2, 5, 12, 24), synth.BF16, "TMA forward (w = 12: coefficient rows not 16-byte units), row-form inverse"),
+    ((1, 2, 9, 10, 22), synth.BF16, "row form bf16, odd w"),
+    ((1, 1, 3, 6, 14), synth.F32, "row form fp32, odd w"),
+    ((2, 2, 1, 6, 10), synth.BF16, "row form image, odd w"),
+    ((1, 1, 5, 8, 1276), synth.BF16, "row form bf16, long odd rows"),
     ((1, 1, 1, 2, 2), synth.F32, "smallest image"),
     ((1, 1, 3, 2, 2), synth.F32, "smallest video"),
 ]
@@ -96,3 +97,22 @@ def test_single_bad_arguments_raise():
     with pytest.raises(hwp.TokError):
         hwp.tok_haar_fwd_single(torch.zeros(1, 1, 3, 7, 8, device="cuda"),
                                 torch.zeros(1, 8, 2, 3, 4, device="cuda"))  # H odd
+
+
+@pytest.mark.parametrize("shape,dtype", [((1, 2, 9, 10, 22), torch.bfloat16), ((1, 1, 3, 6, 14), torch.float32),
+                                         ((2, 2, 1, 6, 10), torch.bfloat16), ((1, 2, 5, 12, 24), torch.bfloat16)])
+def test_single_rows_form_equals_register_kernels(shape, dtype):
+    """The row form (16-byte-aligned sources whose rows are not 16-byte units) against the register
+    kernels (a view one element past a 16-byte boundary), bit for bit, both directions."""
+    from tests.test_gpu_rows import empty_off, off_view
+    x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
+    y = hwp.haar_fwd_single(x)
+    y_reg = empty_off(y.shape, dtype)
+    hwp.tok_haar_fwd_single(off_view(x), y_reg)
+    hwp.tok_check_device()
+    assert torch.equal(y, y_reg)
+    xr = hwp.haar_inv_single(y, *shape[2:])
+    xr_reg = empty_off(shape, dtype)
+    hwp.tok_haar_inv_single(off_view(y), xr_reg)
+    hwp.tok_check_device()
+    assert torch.equal(xr, xr_reg)
