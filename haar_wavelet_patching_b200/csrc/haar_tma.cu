@@ -719,19 +719,28 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 constexpr int kClPitch = 66; // staged row length in elements (64 blocks + 2 of padding)
 
-template <typename T, int NC> struct ClTiles {
+template <typename T, int NC, bool ROWS = false> struct ClTiles {
     static constexpr int REGION_ELEMS = 64 * kClPitch; // >= kTileElems; a multiple of 128 bytes
     static constexpr int REGION_BYTES = REGION_ELEMS * sizeof(T);
     static constexpr int KT = (32768 / (NC * REGION_BYTES)) > 0 ? 32768 / (NC * REGION_BYTES) : 1;
-    static constexpr int SMEM = KT * NC * REGION_BYTES + 8 * KT;
+    // Row form: a channel's 16 pixel rows staged at ROW bytes each (the row and 16 bytes of
+    // slack) fill no more than its region; one offset byte per staged row after the barriers.
+    static constexpr int ROW = 256 * (int)sizeof(T) + 16;
+    static_assert(16 * ROW <= REGION_BYTES, "staged rows fit a channel's region");
+    static constexpr int SMEM = KT * NC * REGION_BYTES + 8 * KT + (ROWS ? 16 * NC * KT : 0);
 };
 
-template <typename T, bool VIDEO, int NC>
+// ROWS: the pixel rows are not whole 16-byte units (bf16 with W % 8 == 4, so w is odd): each
+// of a tile's 16 pixel rows per channel is staged by one bulk copy from the 16-byte boundary
+// below it and read back realigned (as in the planar kernel's row form).  Staged at ROW-byte
+// pitch, block row rw's pixels end where its results (rows of kClPitch) end or earlier, so the
+// results still overwrite only pixels already read.
+template <typename T, bool VIDEO, int NC, bool ROWS>
 __global__ void __launch_bounds__(32)
     haar_cl_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
-                   T *__restrict__ out, const TileGrid tg)
+                   const T *__restrict__ src, T *__restrict__ out, const TileGrid tg)
 {
-    using P = ClTiles<T, NC>;
+    using P = ClTiles<T, NC, ROWS>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
     constexpr int G = VIDEO ? 64 : 16;
@@ -746,6 +755,7 @@ __global__ void __launch_bounds__(32)
     const int lane = threadIdx.x;
     T *buf = reinterpret_cast<T *>(smem_raw);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + KT * NC * P::REGION_BYTES);
+    unsigned char *row_off = reinterpret_cast<unsigned char *>(bars + KT); // ROWS: [tile][channel][row]
 
     auto decode = [&](uint32_t n, int &tx, int &ty, int &tq, int64_t &b) {
         const uint32_t q1 = tg.ntx.div(n), q2 = tg.nty.div(q1), q3 = tg.nq.div(q2);
@@ -758,7 +768,61 @@ __global__ void __launch_bounds__(32)
     const uint32_t first = blockIdx.x * (uint32_t)KT;
     const int count = (int)min((uint32_t)KT, tg.ntiles - first);
 
-    if (lane == 0) {
+    if constexpr (ROWS) {
+        if (lane == 0) {
+            for (int s = 0; s < KT; ++s)
+                mbar_init(smem_addr(bars + s), 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        constexpr int VE = 16 / (int)sizeof(T);
+        const unsigned char *src_b = reinterpret_cast<const unsigned char *>(src);
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t b;
+            decode(first + s, tx, ty, tq, b);
+            int64_t start[2];
+            uint32_t nbulk[2];
+            bool ok[2];
+            uint32_t tx_bytes = 0;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                // Staged row r: channel r / 16, frame slot (r % 16) / (4 RW), pixel row
+                // 4 RW ty + r % (4 RW); NC * 16 <= 64 rows per tile, two per lane.
+                const int r = lane + 32 * k, c = r / 16, rr16 = r % 16, a = rr16 / (4 * RW);
+                const int64_t y = (int64_t)4 * RW * ty + rr16 % (4 * RW);
+                const bool replica = VIDEO && tq == 0;
+                const int64_t f = !VIDEO || replica ? 0 : 4 * tq - 3 + a;
+                ok[k] = r < 16 * NC && y < tg.H && !(replica && a != 0); // window 0 reads frame 0 only
+                const int64_t off = (((b * NC + c) * tg.T + f) * tg.H + y) * tg.W + (int64_t)4 * WT * tx;
+                const int mis = (int)(off % VE);
+                start[k] = (off - mis) * (int64_t)sizeof(T);
+                const int64_t avail = tg.n_src * (int64_t)sizeof(T) - start[k];
+                nbulk[k] = !ok[k] ? 0u : avail >= P::ROW ? (uint32_t)P::ROW : (uint32_t)(avail & ~(int64_t)15);
+                if (r < 16 * NC) // a row not loaded is never used for a stored result: offset 0
+                    row_off[(s * NC + c) * 16 + rr16] = ok[k] ? (unsigned char)(mis * (int)sizeof(T)) : (unsigned char)0;
+                tx_bytes += __reduce_add_sync(0xFFFFFFFFu, nbulk[k]);
+            }
+            const uint32_t bar = smem_addr(bars + s);
+            if (lane == 0)
+                mbar_expect_tx(bar, tx_bytes);
+            __syncwarp();
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                if (!ok[k])
+                    continue;
+                const int r = lane + 32 * k, c = r / 16, rr16 = r % 16;
+                unsigned char *dst = reinterpret_cast<unsigned char *>(buf + (s * NC + c) * P::REGION_ELEMS) + rr16 * P::ROW;
+                if (nbulk[k] > 0)
+                    bulk_load(smem_addr(dst), src_b + start[k], nbulk[k], bar);
+                if (nbulk[k] < (uint32_t)P::ROW) { // the tensor's last, partial 16 bytes
+                    const int64_t end = min(tg.n_src * (int64_t)sizeof(T) - start[k], (int64_t)P::ROW);
+                    for (int64_t e = nbulk[k]; e < end; e += (int64_t)sizeof(T))
+                        *reinterpret_cast<T *>(dst + e) = *reinterpret_cast<const T *>(src_b + start[k] + e);
+                }
+            }
+        }
+    } else if (lane == 0) {
         for (int s = 0; s < KT; ++s)
             mbar_init(smem_addr(bars + s), 1);
         fence_barrier_init();
@@ -804,8 +868,16 @@ __global__ void __launch_bounds__(32)
                 for (int a = 0; a < NA; ++a) {
                     const int fa = replica ? 0 : a;
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr)
-                        SRow<T>::load(region + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                    for (int rr = 0; rr < 4; ++rr) {
+                        if constexpr (ROWS) {
+                            const int sr = fa * 4 * RW + 4 * rw + rr;
+                            staged_row8(reinterpret_cast<const unsigned char *>(region) + sr * P::ROW,
+                                        row_off[(s * NC + c) * 16 + sr] + lane * 8 * (uint32_t)sizeof(T), (T *)nullptr,
+                                        v[a][rr]);
+                        } else {
+                            SRow<T>::load(region + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
+                        }
+                    }
                 }
 #pragma unroll
                 for (int a = 0; a < NA; ++a)
@@ -835,14 +907,14 @@ __global__ void __launch_bounds__(32)
         }
         __syncwarp(); // every channel is staged
         constexpr int PIECES = G * NC / VEC; // 16-byte pieces of one block's run
-        const int64_t nblk = min((int64_t)WT, tg.w - (int64_t)tx * WT); // even: w is
+        const int64_t nblk = min((int64_t)WT, tg.w - (int64_t)tx * WT); // odd only in a row's last tile
 #pragma unroll 1
         for (int rw = 0; rw < RW; ++rw) {
             const int64_t row = (int64_t)ty * RW + rw;
             if (row >= tg.h)
                 continue;
             T *yrow = out + (((b * tg.Tq + tq) * tg.h + row) * tg.w + (int64_t)tx * WT) * (G * NC);
-            const int total = (int)(nblk / 2) * PIECES; // (block pair, piece) items
+            const int total = (int)((nblk + 1) / 2) * PIECES; // (block pair, piece) items
 #pragma unroll 2
             for (int it = lane; it < total; it += 32) {
                 const int pr = it / PIECES, q = it - pr * PIECES; // block pair, piece
@@ -873,7 +945,8 @@ __global__ void __launch_bounds__(32)
                 }
                 T *dst = yrow + (int64_t)(2 * pr) * (G * NC) + q * VEC;
                 *reinterpret_cast<uint4 *>(dst) = r0;
-                *reinterpret_cast<uint4 *>(dst + G * NC) = r1;
+                if (2 * pr + 1 < nblk) // an odd last block has no partner
+                    *reinterpret_cast<uint4 *>(dst + G * NC) = r1;
             }
         }
     }
@@ -1479,22 +1552,24 @@ tok_status haar_single_tma_launch(bool fwd, HaarTmaForm form, const void *in, vo
 namespace tok {
 namespace {
 
-template <typename T, bool VIDEO, int NC>
+template <typename T, bool VIDEO, int NC, bool ROWS>
 tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    using P = ClTiles<T, NC>;
+    using P = ClTiles<T, NC, ROWS>;
     constexpr int RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
     CUtensorMap xm4, xm1;
     memset(&xm4, 0, sizeof xm4);
     memset(&xm1, 0, sizeof xm1);
-    const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
-    const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
-    const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
-    if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
-        (VIDEO && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
-        return TOK_ERR_SHAPE;
+    if (!ROWS) { // the row form reads the pixels through their pointer (bulk copies)
+        const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
+        const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
+        const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
+        if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
+            (VIDEO && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
+            return TOK_ERR_SHAPE;
+    }
     const int64_t ntx = (d.w + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
     TileGrid tg{};
     tg.ntx = FastDiv((uint32_t)ntx);
@@ -1508,29 +1583,30 @@ tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t 
     tg.h = d.h;
     tg.w = d.w;
     tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B);
-    const cudaError_t attr_err =
-        cudaFuncSetAttribute(haar_cl_kernel<T, VIDEO, NC>, cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
+    tg.n_src = d.B * d.C * d.T * d.H * d.W;
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_cl_kernel<T, VIDEO, NC, ROWS>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_cl_kernel<T, VIDEO, NC><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, (T *)out, tg);
+    haar_cl_kernel<T, VIDEO, NC, ROWS><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, (const T *)in, (T *)out, tg);
     return launch_status();
 }
 
 template <typename T, bool VIDEO>
-tok_status launch_cl_c(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+tok_status launch_cl_c(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     switch (d.C) {
     case 1:
-        return launch_cl<T, VIDEO, 1>(in, out, d, stream);
+        return rows ? launch_cl<T, VIDEO, 1, true>(in, out, d, stream) : launch_cl<T, VIDEO, 1, false>(in, out, d, stream);
     case 2:
-        return launch_cl<T, VIDEO, 2>(in, out, d, stream);
+        return rows ? launch_cl<T, VIDEO, 2, true>(in, out, d, stream) : launch_cl<T, VIDEO, 2, false>(in, out, d, stream);
     case 3:
-        return launch_cl<T, VIDEO, 3>(in, out, d, stream);
+        return rows ? launch_cl<T, VIDEO, 3, true>(in, out, d, stream) : launch_cl<T, VIDEO, 3, false>(in, out, d, stream);
     default:
-        return launch_cl<T, VIDEO, 4>(in, out, d, stream);
+        return rows ? launch_cl<T, VIDEO, 4, true>(in, out, d, stream) : launch_cl<T, VIDEO, 4, false>(in, out, d, stream);
     }
 }
 
@@ -1538,19 +1614,19 @@ tok_status launch_cl_c(const void *in, void *out, const HaarDims &d, cudaStream_
 
 bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d)
 {
-    // The pixel side takes the box form; a block's G*C outputs are whole 16-byte pieces at any w,
-    // and the copy-out works on block pairs (w even).
-    const int64_t es = dt == TOK_F32 ? 4 : 2;
-    return d.C >= 1 && d.C <= 4 && aligned(in, 16) && aligned(out, 16) && (d.W * es) % 16 == 0 && d.w % 2 == 0 &&
-           tma_limits_ok(d) && sm_count() > 0;
+    // Any w: the pixel side takes the box form where its rows are whole 16-byte units and the row
+    // form otherwise (bf16 with odd w); a block's G*C outputs are whole 16-byte pieces at any w.
+    return d.C >= 1 && d.C <= 4 && aligned(in, 16) && aligned(out, 16) && tma_limits_ok(d) && sm_count() > 0;
 }
 
 tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream)
 {
+    const bool rows = (d.W * (dt == TOK_F32 ? 4 : 2)) % 16 != 0;
     if (dt == TOK_BF16)
-        return d.video ? launch_cl_c<__nv_bfloat16, true>(in, out, d, stream)
-                       : launch_cl_c<__nv_bfloat16, false>(in, out, d, stream);
-    return d.video ? launch_cl_c<float, true>(in, out, d, stream) : launch_cl_c<float, false>(in, out, d, stream);
+        return d.video ? launch_cl_c<__nv_bfloat16, true>(rows, in, out, d, stream)
+                       : launch_cl_c<__nv_bfloat16, false>(rows, in, out, d, stream);
+    return d.video ? launch_cl_c<float, true>(rows, in, out, d, stream)
+                   : launch_cl_c<float, false>(rows, in, out, d, stream);
 }
 
 } // namespace tok

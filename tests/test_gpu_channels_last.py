@@ -21,9 +21,15 @@ CASES = [
     ((2, 3, 1, 36, 64), torch.bfloat16, "TMA image, partial block rows"),
     ((1, 3, 9, 16, 72), torch.bfloat16, "TMA, w = 18 (coefficient rows not whole 16-byte units)"),
     ((1, 2, 5, 8, 40), torch.float32, "TMA fp32, w = 10"),
+    ((1, 3, 9, 12, 44), torch.float32, "TMA fp32, odd w = 11"),
+    ((1, 1, 1, 20, 28), torch.float32, "TMA fp32 image, odd w = 7"),
+    ((1, 3, 9, 16, 76), torch.bfloat16, "row form, w = 19"),
+    ((2, 1, 5, 8, 1292), torch.bfloat16, "row form, w = 323 (six tiles, odd last)"),
+    ((1, 4, 13, 12, 300), torch.bfloat16, "row form, C = 4, w = 75"),
+    ((1, 2, 1, 8, 20), torch.bfloat16, "row form image, w = 5"),
+    ((2, 3, 1, 36, 52), torch.bfloat16, "row form image, partial block rows, w = 13"),
     ((1, 5, 9, 16, 64), torch.bfloat16, "register, C = 5"),
-    ((1, 3, 9, 12, 44), torch.float32, "register, ragged row"),
-    ((1, 2, 1, 8, 20), torch.bfloat16, "register image"),
+    ((1, 5, 5, 8, 44), torch.bfloat16, "register, C = 5, odd w"),
 ]
 
 
@@ -35,8 +41,8 @@ def test_channels_last_is_the_planar_result_permuted(shape, dtype, note):
     assert torch.equal(y_cl, hwp.haar_fwd(x).permute(0, 2, 3, 4, 1))
 
 
-def test_channels_last_matches_oracle():
-    shape = (1, 3, 9, 32, 64)
+@pytest.mark.parametrize("shape", [(1, 3, 9, 32, 64), (1, 2, 9, 16, 76)], ids=["box form", "row form, odd w"])
+def test_channels_last_matches_oracle(shape):
     x_np = synth.uniform(shape, seed=17, dtype=synth.BF16)
     x64 = synth.to_f64(x_np, synth.BF16)
     got = to_f64(hwp.haar_fwd_channels_last(to_device(x_np, synth.BF16)))
@@ -44,6 +50,19 @@ def test_channels_last_matches_oracle():
     tol = np.moveaxis(haar_bf16_tolerance(oracle.haar_fwd(x64), expand_to_channels(block_abs_sums(x64), 64), True),
                       1, -1)
     assert got.shape == ref.shape and (np.abs(got - ref) <= tol).all()
+
+
+@pytest.mark.parametrize("shape,dtype", [((1, 3, 9, 16, 76), torch.bfloat16), ((2, 2, 1, 12, 36), torch.bfloat16),
+                                         ((1, 3, 5, 8, 44), torch.float32)])
+def test_channels_last_tile_kernels_equal_register_kernel(shape, dtype):
+    """A source one element past a 16-byte boundary takes the register kernel: same bits."""
+    x = (torch.rand(shape, device="cuda") * 2 - 1).to(dtype)
+    buf = torch.empty(x.numel() + 1, dtype=dtype, device="cuda")
+    xo = buf[1:].view(shape)
+    xo.copy_(x)
+    assert xo.data_ptr() % 16 != 0
+    assert torch.equal(hwp.haar_fwd_channels_last(x), hwp.haar_fwd_channels_last(xo))
+    hwp.tok_check_device()
 
 
 def test_channels_last_bad_arguments_raise():
