@@ -708,14 +708,16 @@ __global__ void __launch_bounds__(32)
 // Channels-last patcher: y [B, Tq, h, w, G*C] (G = 64 on video, 16 on images),
 // channel g*C + c as in the planar layout, so a block's G*C coefficients are
 // contiguous.  A tile is one block row (four on images) of 64 blocks across with
-// all NC input channels: NC TMA loads on one barrier.  Per channel, each lane
+// all NC input channels on one barrier: NC TMA box loads, or 16 NC row copies when
+// the pixel rows are not whole 16-byte units (ROWS, below).  Per channel, each lane
 // transforms its two blocks as in the planar kernel and, once the warp has read
 // that channel's pixels, writes the results back over them as [row][g][block]
 // pairs, rows padded to 66 elements (4-byte shared stores, consecutive across
 // lanes).  The copy-out gives each lane a (block pair, 16-byte piece of the run):
 // consecutive lanes take consecutive pieces, so a warp's store covers about two
 // contiguous runs instead of 32 scattered sectors, and the padding puts the pieces'
-// different (g, c) sources in different banks.
+// different (g, c) sources in different banks.  With odd w the last block of a row
+// of blocks has no partner and is stored alone.
 // ---------------------------------------------------------------------------
 constexpr int kClPitch = 66; // staged row length in elements (64 blocks + 2 of padding)
 
