@@ -91,3 +91,26 @@ def test_threaded_baseline_parts_are_the_whole_oracle_step():
             ref_idx, _, _ = oracle.fsq_encode(lat[g:g + 1], w)
             assert np.array_equal(idx, ref_idx)
             np.testing.assert_array_equal(dec, oracle.fsq_decode(ref_idx, w)[0])
+
+
+def test_recorded_traffic_only_for_the_current_kernel_sources(tmp_path, monkeypatch):
+    """roofline.traffic comes from the profiles row whose digest matches the kernel sources
+    as they are; a row taken on other sources (or a missing file) gives null."""
+    import shutil
+    csrc = tmp_path / "haar_wavelet_patching_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for fn in bench.KERNEL_SOURCES["haar_fwd"]:
+        shutil.copy(os.path.join(ROOT, "haar_wavelet_patching_b200", "csrc", fn), csrc / fn)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("haar_fwd") is None  # no profiles file
+    digest = bench.kernel_source_digest("haar_fwd")
+    (tmp_path / "profiles").mkdir()
+    table = "| kernel | bytes | digest | note |\n|---|---|---|---|\n"
+    (tmp_path / "profiles" / "dram_traffic.md").write_text(table + "| haar_fwd | 123456 | 0000000000000000 | old |\n")
+    assert bench.recorded_traffic("haar_fwd") is None
+    (tmp_path / "profiles" / "dram_traffic.md").write_text(table + f"| haar_fwd | 123456 | {digest} | current |\n")
+    assert bench.recorded_traffic("haar_fwd") == 123456.0
+    assert bench.recorded_traffic("haar_inv") is None  # a row names its kernel
+    with open(csrc / "haar_tma.cu", "a") as f:  # any edit of a source the kernel is built from
+        f.write("\n")
+    assert bench.recorded_traffic("haar_fwd") is None
