@@ -708,8 +708,9 @@ __global__ void __launch_bounds__(32)
 // Channels-last patcher: y [B, Tq, h, w, G*C] (G = 64 on video, 16 on images),
 // channel g*C + c as in the planar layout, so a block's G*C coefficients are
 // contiguous.  A tile is one block row (four on images) of 64 blocks across with
-// all NC input channels on one barrier: NC TMA box loads, or 16 NC row copies when
-// the pixel rows are not whole 16-byte units (ROWS, below).  Per channel, each lane
+// all NC input channels on one barrier: NC TMA box loads; when the pixel rows are
+// not whole 16-byte units, 3 NC pair-row boxes on video (PAIRS) or 16 NC row copies on
+// images (ROWS), both below.  Per channel, each lane
 // transforms its two blocks as in the planar kernel and, once the warp has read
 // that channel's pixels, writes the results back over them as [row][g][block]
 // pairs, rows padded to 66 elements (4-byte shared stores, consecutive across
@@ -737,11 +738,20 @@ template <typename T, int NC, bool ROWS = false> struct ClTiles {
 // below it and read back realigned (as in the planar kernel's row form).  Staged at ROW-byte
 // pitch, block row rw's pixels end where its results (rows of kClPitch) end or earlier, so the
 // results still overwrite only pixels already read.
-template <typename T, bool VIDEO, int NC, bool ROWS>
+//
+// PAIRS (video, bf16, W % 8 == 4): the same rows through tensor boxes.  Two pixel rows taken as
+// one row of 2W elements have a 4W-byte stride, a 16-byte multiple, so the maps view each
+// frame as [H/2][2W]: the even pixel rows of a tile are one box at x = 256 tx, the odd ones a
+// box at x = W + 256 tx - 4 (the 16-byte boundary 4 elements before them: 2W = 8 mod 16
+// bytes) and an 8-element box after it for the last 4 pixels.  Per channel: even rows at byte
+// 0 of its region, odd rows at 4096, the tail boxes at 8192 (2080 bytes per frame in all).
+template <typename T, bool VIDEO, int NC, bool ROWS, bool PAIRS>
 __global__ void __launch_bounds__(32)
     haar_cl_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
+                   const __grid_constant__ CUtensorMap xtail4, const __grid_constant__ CUtensorMap xtail1,
                    const T *__restrict__ src, T *__restrict__ out, const TileGrid tg)
 {
+    static_assert(!PAIRS || (VIDEO && !ROWS && sizeof(T) == 2), "pair rows: bf16 video only");
     using P = ClTiles<T, NC, ROWS>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
@@ -824,6 +834,27 @@ __global__ void __launch_bounds__(32)
                 }
             }
         }
+    } else if (PAIRS && lane == 0) {
+        for (int s = 0; s < KT; ++s)
+            mbar_init(smem_addr(bars + s), 1);
+        fence_barrier_init();
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t b;
+            decode(first + s, tx, ty, tq, b);
+            const uint32_t bar = smem_addr(bars + s);
+            const bool full = tq > 0;
+            mbar_expect_tx(bar, NC * (full ? NA : 1) * 2080u);
+            const int x_even = 4 * WT * tx, x_odd = (int)tg.W + 4 * WT * tx - 4;
+            for (int c = 0; c < NC; ++c) {
+                const uint32_t dst = smem_addr(buf + (s * NC + c) * P::REGION_ELEMS);
+                const int frame0 = (int)((b * NC + c) * tg.T), z = full ? frame0 + 4 * tq - 3 : frame0;
+                const CUtensorMap *mrow = full ? &xmap4 : &xmap1, *mtail = full ? &xtail4 : &xtail1;
+                tma_load_3d(dst, mrow, x_even, 2 * ty, z, bar);
+                tma_load_3d(dst + 4096, mrow, x_odd, 2 * ty, z, bar);
+                tma_load_3d(dst + 8192, mtail, x_odd + 4 * WT, 2 * ty, z, bar);
+            }
+        }
     } else if (lane == 0) {
         for (int s = 0; s < KT; ++s)
             mbar_init(smem_addr(bars + s), 1);
@@ -876,6 +907,23 @@ __global__ void __launch_bounds__(32)
                             staged_row8(reinterpret_cast<const unsigned char *>(region) + sr * P::ROW,
                                         row_off[(s * NC + c) * 16 + sr] + lane * 8 * (uint32_t)sizeof(T), (T *)nullptr,
                                         v[a][rr]);
+                        } else if constexpr (PAIRS) {
+                            // Pixel row rr of frame slot fa: box row fa * 2 + rr / 2 of the even
+                            // (rr even) or odd box; an odd row starts 4 elements into its box row
+                            // and lane 31's last 4 pixels sit in the tail box.
+                            const int br = fa * 2 + rr / 2;
+                            if (rr % 2 == 0) {
+                                SRow<T>::load(region + br * 256 + 8 * lane, v[a][rr]);
+                            } else {
+                                const T *odd = region + 2048 + br * 256 + 4 + 8 * lane;
+                                const uint2 lo = *reinterpret_cast<const uint2 *>(odd);
+                                const uint2 hi =
+                                    *reinterpret_cast<const uint2 *>(lane < 31 ? odd + 4 : region + 4096 + br * 8);
+                                v[a][rr][0] = make_float2(bf16_lo(lo.x), bf16_lo(hi.x));
+                                v[a][rr][1] = make_float2(bf16_hi(lo.x), bf16_hi(hi.x));
+                                v[a][rr][2] = make_float2(bf16_lo(lo.y), bf16_lo(hi.y));
+                                v[a][rr][3] = make_float2(bf16_hi(lo.y), bf16_hi(hi.y));
+                            }
                         } else {
                             SRow<T>::load(region + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
                         }
@@ -1554,17 +1602,29 @@ tok_status haar_single_tma_launch(bool fwd, HaarTmaForm form, const void *in, vo
 namespace tok {
 namespace {
 
-template <typename T, bool VIDEO, int NC, bool ROWS>
+template <typename T, bool VIDEO, int NC, bool ROWS, bool PAIRS>
 tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     using P = ClTiles<T, NC, ROWS>;
     constexpr int RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
-    CUtensorMap xm4, xm1;
+    CUtensorMap xm4, xm1, xt4, xt1;
     memset(&xm4, 0, sizeof xm4);
     memset(&xm1, 0, sizeof xm1);
-    if (!ROWS) { // the row form reads the pixels through their pointer (bulk copies)
+    memset(&xt4, 0, sizeof xt4);
+    memset(&xt1, 0, sizeof xt1);
+    if (PAIRS) { // each frame as [H/2][2W]: rows of two pixel rows, 4W-byte strides
+        const uint64_t xdims[3] = {(uint64_t)(2 * d.W), (uint64_t)(d.H / 2), (uint64_t)(d.B * d.C * d.T)};
+        const uint64_t xstr[2] = {2 * d.W * es, d.H * d.W * es};
+        const uint32_t box4[3] = {4u * WT, 2u, 4u}, box1[3] = {4u * WT, 2u, 1u}, tail4[3] = {8u, 2u, 4u},
+                       tail1[3] = {8u, 2u, 1u};
+        if (!encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4) ||
+            !encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
+            !encode_tensor_map(&xt4, dt, 3, in, xdims, xstr, tail4) ||
+            !encode_tensor_map(&xt1, dt, 3, in, xdims, xstr, tail1))
+            return TOK_ERR_SHAPE;
+    } else if (!ROWS) { // the row form reads the pixels through their pointer (bulk copies)
         const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
         const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
         const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
@@ -1586,15 +1646,29 @@ tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t 
     tg.w = d.w;
     tg.ntiles = (uint32_t)(ntx * nty * d.Tq * d.B);
     tg.n_src = d.B * d.C * d.T * d.H * d.W;
-    const cudaError_t attr_err = cudaFuncSetAttribute(haar_cl_kernel<T, VIDEO, NC, ROWS>,
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_cl_kernel<T, VIDEO, NC, ROWS, PAIRS>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_cl_kernel<T, VIDEO, NC, ROWS><<<grid, 32, P::SMEM, stream>>>(xm4, xm1, (const T *)in, (T *)out, tg);
+    haar_cl_kernel<T, VIDEO, NC, ROWS, PAIRS>
+        <<<grid, 32, P::SMEM, stream>>>(xm4, xm1, xt4, xt1, (const T *)in, (T *)out, tg);
     return launch_status();
+}
+
+// Form per call: tensor boxes (pixel rows of whole 16-byte units), pair-row boxes (bf16 video,
+// W % 8 == 4), or row copies (bf16 images with W % 8 == 4).
+template <typename T, bool VIDEO, int NC>
+tok_status launch_cl_form(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
+{
+    if (!rows)
+        return launch_cl<T, VIDEO, NC, false, false>(in, out, d, stream);
+    if constexpr (VIDEO && sizeof(T) == 2)
+        return launch_cl<T, VIDEO, NC, false, true>(in, out, d, stream);
+    else
+        return launch_cl<T, VIDEO, NC, true, false>(in, out, d, stream);
 }
 
 template <typename T, bool VIDEO>
@@ -1602,13 +1676,13 @@ tok_status launch_cl_c(bool rows, const void *in, void *out, const HaarDims &d, 
 {
     switch (d.C) {
     case 1:
-        return rows ? launch_cl<T, VIDEO, 1, true>(in, out, d, stream) : launch_cl<T, VIDEO, 1, false>(in, out, d, stream);
+        return launch_cl_form<T, VIDEO, 1>(rows, in, out, d, stream);
     case 2:
-        return rows ? launch_cl<T, VIDEO, 2, true>(in, out, d, stream) : launch_cl<T, VIDEO, 2, false>(in, out, d, stream);
+        return launch_cl_form<T, VIDEO, 2>(rows, in, out, d, stream);
     case 3:
-        return rows ? launch_cl<T, VIDEO, 3, true>(in, out, d, stream) : launch_cl<T, VIDEO, 3, false>(in, out, d, stream);
+        return launch_cl_form<T, VIDEO, 3>(rows, in, out, d, stream);
     default:
-        return rows ? launch_cl<T, VIDEO, 4, true>(in, out, d, stream) : launch_cl<T, VIDEO, 4, false>(in, out, d, stream);
+        return launch_cl_form<T, VIDEO, 4>(rows, in, out, d, stream);
     }
 }
 

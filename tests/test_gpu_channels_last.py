@@ -23,9 +23,12 @@ CASES = [
     ((1, 2, 5, 8, 40), torch.float32, "TMA fp32, w = 10"),
     ((1, 3, 9, 12, 44), torch.float32, "TMA fp32, odd w = 11"),
     ((1, 1, 1, 20, 28), torch.float32, "TMA fp32 image, odd w = 7"),
-    ((1, 3, 9, 16, 76), torch.bfloat16, "row form, w = 19"),
-    ((2, 1, 5, 8, 1292), torch.bfloat16, "row form, w = 323 (six tiles, odd last)"),
-    ((1, 4, 13, 12, 300), torch.bfloat16, "row form, C = 4, w = 75"),
+    ((1, 3, 9, 16, 76), torch.bfloat16, "pair rows, w = 19"),
+    ((2, 1, 5, 8, 1292), torch.bfloat16, "pair rows, w = 323 (six tiles, odd last)"),
+    ((1, 4, 13, 12, 300), torch.bfloat16, "pair rows, C = 4, w = 75"),
+    ((1, 1, 5, 4, 4), torch.bfloat16, "pair rows, w = 1"),
+    ((1, 3, 5, 8, 260), torch.bfloat16, "pair rows, w = 65 (a one-block last tile)"),
+    ((2, 2, 9, 8, 516), torch.bfloat16, "pair rows, B = 2, w = 129"),
     ((1, 2, 1, 8, 20), torch.bfloat16, "row form image, w = 5"),
     ((2, 3, 1, 36, 52), torch.bfloat16, "row form image, partial block rows, w = 13"),
     ((1, 5, 9, 16, 64), torch.bfloat16, "register, C = 5"),
@@ -41,7 +44,7 @@ def test_channels_last_is_the_planar_result_permuted(shape, dtype, note):
     assert torch.equal(y_cl, hwp.haar_fwd(x).permute(0, 2, 3, 4, 1))
 
 
-@pytest.mark.parametrize("shape", [(1, 3, 9, 32, 64), (1, 2, 9, 16, 76)], ids=["box form", "row form, odd w"])
+@pytest.mark.parametrize("shape", [(1, 3, 9, 32, 64), (1, 2, 9, 16, 76)], ids=["box form", "pair rows, odd w"])
 def test_channels_last_matches_oracle(shape):
     x_np = synth.uniform(shape, seed=17, dtype=synth.BF16)
     x64 = synth.to_f64(x_np, synth.BF16)
