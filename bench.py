@@ -102,6 +102,26 @@ def recorded_traffic(kernel):
     return None
 
 
+def earlier_traffic(kernel):
+    """The newest recorded row of a kernel taken on other sources than the current ones, as
+    {"bytes", "digest", "current_digest"}, or None: shown beside a null roofline.traffic so
+    that the last capture stays visible, labelled as not describing the current build."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    try:
+        lines = open(path).read().splitlines()
+    except OSError:
+        return None
+    digest = kernel_source_digest(kernel)
+    for ln in lines:
+        parts = [p.strip() for p in ln.strip().strip("|").split("|")]
+        if len(parts) >= 3 and parts[0] == kernel and parts[2] != digest:
+            try:
+                return {"bytes": float(parts[1]), "digest": parts[2], "current_digest": digest}
+            except ValueError:
+                continue
+    return None
+
+
 def max_over_ranks(v: float, device) -> float:
     """Max of a per-rank time over the default process group (any backend); v itself on one rank."""
     import torch
@@ -693,6 +713,10 @@ def run_ours(args, rank, world, local_rank):
                              "bytes": g["bytes"]} for n, g in single.items()},
         "patch_embed": patch_embed_report(embed, peak),
     }
+    if line["roofline"]["traffic"] is None:
+        earlier = earlier_traffic(dom)
+        if earlier is not None:
+            line["roofline"]["traffic_earlier_sources"] = earlier
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
         line["cpu_baseline_threads"] = cpu_baseline_threads()

@@ -114,3 +114,23 @@ def test_recorded_traffic_only_for_the_current_kernel_sources(tmp_path, monkeypa
     with open(csrc / "haar_tma.cu", "a") as f:  # any edit of a source the kernel is built from
         f.write("\n")
     assert bench.recorded_traffic("haar_fwd") is None
+
+
+def test_earlier_traffic_is_labelled_with_both_digests(tmp_path, monkeypatch):
+    """With no row for the current sources, the newest row of the kernel is shown apart from
+    roofline.traffic, with its digest and the current one."""
+    import shutil
+    csrc = tmp_path / "haar_wavelet_patching_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    for fn in bench.KERNEL_SOURCES["haar_fwd"]:
+        shutil.copy(os.path.join(ROOT, "haar_wavelet_patching_b200", "csrc", fn), csrc / fn)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    (tmp_path / "profiles").mkdir()
+    table = "| kernel | bytes | digest | note |\n|---|---|---|---|\n"
+    (tmp_path / "profiles" / "dram_traffic.md").write_text(table + "| haar_fwd | 777 | 00000000aaaaaaaa | old |\n")
+    digest = bench.kernel_source_digest("haar_fwd")
+    assert bench.recorded_traffic("haar_fwd") is None
+    assert bench.earlier_traffic("haar_fwd") == {"bytes": 777.0, "digest": "00000000aaaaaaaa",
+                                                 "current_digest": digest}
+    (tmp_path / "profiles" / "dram_traffic.md").write_text(table + f"| haar_fwd | 888 | {digest} | now |\n")
+    assert bench.earlier_traffic("haar_fwd") is None and bench.recorded_traffic("haar_fwd") == 888.0
