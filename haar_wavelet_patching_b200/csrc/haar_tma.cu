@@ -1659,16 +1659,18 @@ tok_status launch_cl(const void *in, void *out, const HaarDims &d, cudaStream_t 
 }
 
 // Form per call: tensor boxes (pixel rows of whole 16-byte units), pair-row boxes (bf16 video,
-// W % 8 == 4), or row copies (bf16 images with W % 8 == 4).
+// W % 8 == 4; their x coordinates, up to 2W + 508, must fit 32 bits), or row copies (bf16 images
+// with W % 8 == 4, and wider video).
 template <typename T, bool VIDEO, int NC>
 tok_status launch_cl_form(bool rows, const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
     if (!rows)
         return launch_cl<T, VIDEO, NC, false, false>(in, out, d, stream);
-    if constexpr (VIDEO && sizeof(T) == 2)
-        return launch_cl<T, VIDEO, NC, false, true>(in, out, d, stream);
-    else
-        return launch_cl<T, VIDEO, NC, true, false>(in, out, d, stream);
+    if constexpr (VIDEO && sizeof(T) == 2) {
+        if (2 * d.W + 512 < ((int64_t)1 << 31))
+            return launch_cl<T, VIDEO, NC, false, true>(in, out, d, stream);
+    }
+    return launch_cl<T, VIDEO, NC, true, false>(in, out, d, stream);
 }
 
 template <typename T, bool VIDEO>
