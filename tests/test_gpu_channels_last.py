@@ -74,3 +74,10 @@ def test_channels_last_bad_arguments_raise():
                                        torch.zeros(1, 192, 3, 8, 16, device="cuda"))
     with pytest.raises((ValueError, hwp.TokError)):  # T % 4 != 1: the shape helper or the library refuses
         hwp.haar_fwd_channels_last(torch.zeros(1, 3, 8, 32, 64, device="cuda"))
+
+
+@pytest.mark.parametrize("shape", [(0, 3, 9, 32, 64), (1, 2, 5, 0, 76), (2, 1, 1, 8, 0)])
+def test_channels_last_empty_is_noop(shape):
+    y = hwp.haar_fwd_channels_last(torch.empty(shape, device="cuda", dtype=torch.bfloat16))
+    hwp.tok_check_device()
+    assert y.shape == hwp.channels_last_shape(*shape) and y.numel() == 0

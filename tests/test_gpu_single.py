@@ -116,3 +116,13 @@ def test_single_rows_form_equals_register_kernels(shape, dtype):
     hwp.tok_haar_inv_single(off_view(y), xr_reg)
     hwp.tok_check_device()
     assert torch.equal(xr, xr_reg)
+
+
+@pytest.mark.parametrize("shape", [(0, 3, 9, 16, 16), (1, 2, 5, 0, 8), (2, 1, 1, 8, 0)])
+def test_single_empty_is_noop(shape):
+    x = torch.empty(shape, device="cuda", dtype=torch.bfloat16)
+    y = hwp.haar_fwd_single(x)
+    assert y.shape == hwp.single_coeff_shape(*shape)
+    xr = hwp.haar_inv_single(y, *shape[2:])
+    hwp.tok_check_device()
+    assert xr.shape == x.shape
