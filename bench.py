@@ -472,7 +472,9 @@ CONV_CH = (256, 256)  # C_mid, C_out of the factorized convolution after the pat
 def time_patch_embed(torch, hwp, stream, x, dev, iters=10):
     """The patcher's channels-last output feeding the first causal factorized convolution
     (1x3x3 then 3x1x1 causal) on the headline clip, each call timed alone: flops of the two
-    implicit GEMMs, 2 * positions * (C_mid * 9 * C_in + C_out * 3 * C_mid)."""
+    implicit GEMMs, 2 * positions * (C_mid * 9 * C_in + C_out * 3 * C_mid).  patch_embed_fused
+    is the patcher fused into the 1x3x3 convolution (one kernel, pixels in, the spatial layer's
+    output out): the same flops as conv_spatial, the work of haar_fwd_channels_last + conv_spatial."""
     B, C, T, H, W = x.shape
     Cmid, Cout = CONV_CH
     y_cl = torch.empty(hwp.channels_last_shape(B, C, T, H, W), dtype=torch.bfloat16, device=dev)
@@ -481,9 +483,13 @@ def time_patch_embed(torch, hwp, stream, x, dev, iters=10):
     ws = (torch.randn((Cmid, 3, 3, Cin), generator=g, device=dev) * (9 * Cin) ** -0.5).to(torch.bfloat16)
     wt = (torch.randn((Cout, 3, Cmid), generator=g, device=dev) * (3 * Cmid) ** -0.5).to(torch.bfloat16)
     mid = torch.empty((Bq, Tq, h, w, Cmid), dtype=torch.bfloat16, device=dev)
+    mid2 = torch.empty_like(mid)
     out = torch.empty((Bq, Tq, h, w, Cout), dtype=torch.bfloat16, device=dev)
+    wp = hwp.patch_embed_pack_weights(ws)  # once per filter, outside the timed calls
     pos = Bq * Tq * h * w
     calls = {
+        "patch_embed_fused": (lambda: hwp.tok_patch_embed_spatial(x, wp, mid2), 2 * pos * Cmid * 9 * Cin,
+                              (x.numel() + mid2.numel()) * 2, 1),
         "haar_fwd_channels_last": (lambda: hwp.tok_haar_fwd_channels_last(x, y_cl), 0,
                                    (x.numel() + y_cl.numel()) * 2, 1),
         "conv_spatial": (lambda: hwp.tok_conv_spatial(y_cl, ws, mid), 2 * pos * Cmid * 9 * Cin,
@@ -502,7 +508,7 @@ def time_patch_embed(torch, hwp, stream, x, dev, iters=10):
         e1.record(stream)
         torch.cuda.synchronize()
         res[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "flops": flops, "bytes": nbytes}
-    del y_cl, mid, out
+    del y_cl, mid, mid2, out
     return res
 
 
@@ -537,6 +543,103 @@ def time_streaming(torch, hwp, stream, dev, iters=GRAD_ITERS):
         torch.cuda.synchronize()
         out[name] = {"ms": max_over_ranks(e0.elapsed_time(e1) / iters, dev), "bytes": nbytes, "launches": 1}
     return out
+
+
+STRESS_ITERS = 10
+
+
+def _flush_l2(torch, bufs):
+    """Evict L2 between timed kernels: write one buffer larger than L2, then read another, so
+    the next kernel starts with neither its inputs nor dirty lines of the flush in L2."""
+    bufs[0].zero_()
+    bufs[1].sum()
+
+
+def time_sequence(torch, stream, calls, iters, flush=None):
+    """Run the calls back to back on one stream `iters` times after one warm-up pass, an event
+    pair around each call (a flush, if given, runs between calls outside the events); returns
+    the mean ms per call."""
+    for _, call in calls:
+        call()
+    torch.cuda.synchronize()
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in calls]
+           for _ in range(iters)]
+    for k in range(iters):
+        for (_, call), (e0, e1) in zip(calls, evs[k]):
+            if flush is not None:
+                flush()
+            e0.record(stream)
+            call()
+            e1.record(stream)
+    torch.cuda.synchronize()
+    return {name: float(np.mean([evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(iters)]))
+            for i, (name, _) in enumerate(calls)}
+
+
+def stress_inputs(torch, cfg, dev):
+    """Seeded host inputs of a Haar config (pinned, then copied once to the device) and the
+    latent of the matching FSQ config."""
+    import synth
+    shape = synth.HAAR_CONFIGS[cfg]["shape"]
+    x_host = torch.empty(shape, dtype=torch.int16).pin_memory()
+    synth.haar_input(cfg, out=x_host.numpy().view(np.uint16))
+    x = x_host.view(torch.bfloat16).to(dev)
+    del x_host
+    u = torch.from_numpy(synth.fsq_input(cfg)).to(dev)
+    return x, u
+
+
+def time_stress(torch, hwp, stream, w_dev, dev, iters=STRESS_ITERS):
+    """BASELINE configs 5 and 2, outside the headline step.  Config 5: four 121-frame 1088x1920
+    clips [4,3,121,1088,1920] bf16 through the patcher and unpatcher, then FSQ encode + decode of
+    the [4,16,16*68*120] latent, back to back on one stream (its Haar tensors are 6 GB each, so
+    nothing survives in L2 from one call to the next; its 35 MB latent is L2-sized).  Config 2:
+    the image path on [16,3,1024,1024] bf16 (2D Haar) and FSQ on [16,16,64*64]; every tensor
+    but none of the Haar pairs exceeds L2, so L2 is flushed before each call (outside its
+    events).  Per call: mean ms, algorithmic bytes (inputs read once, outputs written once)."""
+    out = {}
+    for cfg in (5, 2):
+        x, u = stress_inputs(torch, cfg, dev)
+        B, C, T, H, W = x.shape
+        y = torch.empty(hwp.haar_coeff_shape(B, C, T, H, W), dtype=x.dtype, device=dev)
+        xr = torch.empty_like(x)
+        idx = torch.empty(u.shape[0], u.shape[2], dtype=torch.int32, device=dev)
+        ur = torch.empty_like(u)
+        hx, hy = haar_bytes(x.shape)
+        fu, fi = fsq_bytes(u.shape)
+        calls = [("haar_fwd", lambda: hwp.tok_haar_fwd(x, y)), ("haar_inv", lambda: hwp.tok_haar_inv(y, xr)),
+                 ("fsq_encode", lambda: hwp.tok_fsq_encode(u, w_dev, idx)),
+                 ("fsq_decode", lambda: hwp.tok_fsq_decode(idx, w_dev, ur))]
+        nbytes = {"haar_fwd": hx + hy, "haar_inv": hx + hy, "fsq_encode": fu + fi, "fsq_decode": fu + fi}
+        flush = None
+        if cfg == 2:
+            fb = [torch.empty(256 << 20, dtype=torch.uint8, device=dev) for _ in range(2)]
+            flush = lambda: _flush_l2(torch, fb)  # noqa: E731
+        ms = time_sequence(torch, stream, calls, iters, flush)
+        out[cfg] = {"clip": list(x.shape), "latent": list(u.shape),
+                    "calls": {n: {"ms": max_over_ranks(ms[n], dev), "bytes": nbytes[n]} for n in ms},
+                    "voxels": B * T * H * W, "tokens": u.shape[0] * u.shape[2]}
+        del x, u, y, xr, idx, ur
+        torch.cuda.empty_cache()
+    return out
+
+
+def stress_report(stress, peak):
+    rep = {}
+    for cfg, d in stress.items():
+        e = {"clip": d["clip"], "latent": d["latent"],
+             "l2": "flushed before each call" if cfg == 2 else "no flush: each Haar tensor is 6 GB, back to back"}
+        for n, g in d["calls"].items():
+            gbs = g["bytes"] / (g["ms"] / 1e3) / 1e9
+            r = {"ms": round(g["ms"], 4), "GB/s": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4),
+                 "bytes": g["bytes"]}
+            if n.startswith("haar"):
+                r["mvoxel_per_s"] = round(d["voxels"] / g["ms"] / 1e3, 1)
+            else:
+                r["mtoken_per_s"] = round(d["tokens"] / g["ms"] / 1e3, 1)
+            e[n] = r
+        rep[f"config{cfg}"] = e
+    return rep
 
 
 def tensor_peak():
@@ -670,6 +773,7 @@ def run_ours(args, rank, world, local_rank):
     streaming = time_streaming(torch, hwp, stream, dev)
     single = time_single(torch, hwp, stream, x, dev)
     embed = time_patch_embed(torch, hwp, stream, x, dev)
+    stress = time_stress(torch, hwp, stream, w_dev, dev) if not args.no_stress else None
     barrier()
 
     if rank != 0:
@@ -713,6 +817,8 @@ def run_ours(args, rank, world, local_rank):
                              "bytes": g["bytes"]} for n, g in single.items()},
         "patch_embed": patch_embed_report(embed, peak),
     }
+    if stress is not None:
+        line["stress"] = stress_report(stress, peak)
     if line["roofline"]["traffic"] is None:
         earlier = earlier_traffic(dom)
         if earlier is not None:
@@ -731,6 +837,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-stress", action="store_true", help="skip the config 5 / config 2 block")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

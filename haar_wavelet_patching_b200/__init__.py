@@ -23,11 +23,12 @@ FSQ_CODEBOOK = 64000
 FSQ_DIM = 6
 
 # Every symbol include/tok.h declares.
-ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device", "tok_haar_fwd",
+ABI_SYMBOLS = ("tok_abi_version", "tok_status_str", "tok_last_cuda_error", "tok_check_device",
+               "tok_selftest_wait_timeout", "tok_haar_fwd",
                "tok_haar_inv", "tok_haar_fwd_adjoint", "tok_haar_inv_adjoint", "tok_haar_fwd_windows",
                "tok_haar_inv_windows", "tok_haar_fwd_single", "tok_haar_inv_single", "tok_haar_fwd_channels_last", "tok_haar_padded_extents", "tok_haar_fwd_padded", "tok_haar_inv_cropped",
                "tok_haar_fwd_chunk", "tok_haar_inv_chunk", "tok_conv_spatial", "tok_conv_temporal_causal",
-               "tok_conv_factorized", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
+               "tok_conv_factorized", "tok_patch_embed_pack_weights", "tok_patch_embed_spatial", "tok_fsq_encode", "tok_fsq_decode", "tok_fsq_backward_workspace_size",
                "tok_fsq_encode_backward", "tok_fsq_encode_backward_noalloc", "tok_fsq_decode_backward")
 
 _lib = None
@@ -59,6 +60,8 @@ def lib():
         L.tok_last_cuda_error.argtypes = []
         L.tok_check_device.restype = i32
         L.tok_check_device.argtypes = [vp]
+        L.tok_selftest_wait_timeout.restype = i32
+        L.tok_selftest_wait_timeout.argtypes = [ctypes.c_uint32, vp]
         for f in (L.tok_haar_fwd, L.tok_haar_inv, L.tok_haar_fwd_adjoint, L.tok_haar_inv_adjoint,
                   L.tok_haar_fwd_single, L.tok_haar_inv_single, L.tok_haar_fwd_channels_last):
             f.restype = i32
@@ -85,6 +88,10 @@ def lib():
         for f in (L.tok_conv_spatial, L.tok_conv_temporal_causal):
             f.restype = i32
             f.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, vp]
+        L.tok_patch_embed_pack_weights.restype = i32
+        L.tok_patch_embed_pack_weights.argtypes = [vp, vp, i64, i64, vp]
+        L.tok_patch_embed_spatial.restype = i32
+        L.tok_patch_embed_spatial.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, vp]
         L.tok_conv_factorized.restype = i32
         L.tok_conv_factorized.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, vp]
         L.tok_fsq_encode.restype = i32
@@ -154,6 +161,14 @@ def tok_check_device(device=None, stream=None):
     if stream is None:
         stream = torch.cuda.current_stream(device)
     _check(lib().tok_check_device(ctypes.c_void_p(stream.cuda_stream)), "tok_check_device")
+
+
+def tok_selftest_wait_timeout(polls: int, device=None, stream=None):
+    """Launch the failure-channel self-test: a kernel whose barrier wait runs out after
+    `polls` polls and counts a timeout (the next tok_check_device raises TOK_ERR_TIMEOUT)."""
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    _check(lib().tok_selftest_wait_timeout(polls, ctypes.c_void_p(stream.cuda_stream)), "tok_selftest_wait_timeout")
 
 
 def tok_haar_fwd(x: torch.Tensor, y: torch.Tensor, stream=None):
@@ -375,6 +390,45 @@ def tok_conv_factorized(x, ws, wt, mid, y, stream=None):
     _check(lib().tok_conv_factorized(_ptr(x), _ptr(ws), _ptr(wt), _ptr(mid), _ptr(y), B, T, h, w, Cin, Cmid, Cout,
                                      k, _stream(x, stream)), "tok_conv_factorized")
     return y
+
+
+def tok_patch_embed_pack_weights(ws: torch.Tensor, wp: torch.Tensor, stream=None):
+    """Reorder the spatial filter ws [Cmid, 3, 3, 64C] for the fused call: wp [Cmid, 9C, 64]."""
+    _cuda(ws, "ws"), _cuda(wp, "wp")
+    Cmid, C = ws.shape[0], ws.shape[3] // 64
+    if (ws.dim() != 4 or tuple(ws.shape[1:3]) != (3, 3) or ws.shape[3] != 64 * C or ws.dtype != torch.bfloat16
+            or tuple(wp.shape) != (Cmid, 9 * C, 64) or wp.dtype != torch.bfloat16):
+        raise ValueError("ws must be bf16 [Cmid, 3, 3, 64C] and wp bf16 [Cmid, 9C, 64]")
+    _check(lib().tok_patch_embed_pack_weights(_ptr(ws), _ptr(wp), C, Cmid, _stream(ws, stream)),
+           "tok_patch_embed_pack_weights")
+    return wp
+
+
+def tok_patch_embed_spatial(x: torch.Tensor, wp: torch.Tensor, y: torch.Tensor, stream=None):
+    """The patcher fused into the 1 x 3 x 3 convolution: x [B,C,T,H,W] bf16 pixels, wp the packed
+    filter [Cmid, 9C, 64] -> y [B, T', H/4, W/4, Cmid] bf16."""
+    _cuda(x, "x"), _cuda(wp, "wp"), _cuda(y, "y")
+    if x.dim() != 5 or x.dtype != torch.bfloat16 or wp.dtype != torch.bfloat16 or y.dtype != torch.bfloat16:
+        raise ValueError("x [B, C, T, H, W], wp and y must be bf16")
+    B, C, T, H, W = x.shape
+    Cmid = wp.shape[0]
+    if tuple(wp.shape) != (Cmid, 9 * C, 64) or tuple(y.shape) != (B, latent_frames(T), H // 4, W // 4, Cmid):
+        raise ValueError("wp must be [Cmid, 9C, 64] and y [B, T', H/4, W/4, Cmid]")
+    _check(lib().tok_patch_embed_spatial(_ptr(x), _ptr(wp), _ptr(y), B, C, T, H, W, Cmid, _stream(x, stream)),
+           "tok_patch_embed_spatial")
+    return y
+
+
+def patch_embed_pack_weights(ws, stream=None):
+    Cmid, C = ws.shape[0], ws.shape[3] // 64
+    wp = torch.empty((Cmid, 9 * C, 64), dtype=torch.bfloat16, device=ws.device)
+    return tok_patch_embed_pack_weights(ws, wp, stream)
+
+
+def patch_embed_spatial(x, wp, stream=None):
+    B, C, T, H, W = x.shape
+    y = torch.empty((B, latent_frames(T), H // 4, W // 4, wp.shape[0]), dtype=torch.bfloat16, device=x.device)
+    return tok_patch_embed_spatial(x, wp, y, stream)
 
 
 def conv_factorized(x, ws, wt, stream=None):

@@ -8,6 +8,7 @@ loads on machines without a GPU (calls then fail with TOK_ERR_CUDA).
 """
 import glob
 import os
+import re
 import subprocess
 import sys
 
@@ -45,19 +46,35 @@ def cutlass_includes():
     raise RuntimeError("CUTLASS headers with the sm100 convolution builders were not found")
 
 
+_INCLUDE_RE = re.compile(r'^\s*#\s*include\s*"([^"]+)"', re.M)
+
+
+def local_headers(path, seen=None):
+    """The repository headers a source includes, directly or through other repository headers."""
+    seen = set() if seen is None else seen
+    with open(path) as f:
+        text = f.read()
+    for name in _INCLUDE_RE.findall(text):
+        for d in (os.path.dirname(path), CSRC, INCLUDE):
+            cand = os.path.join(d, name)
+            if os.path.exists(cand) and cand not in seen:
+                seen.add(cand)
+                local_headers(cand, seen)
+                break
+    return seen
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
-    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) + \
-        glob.glob(os.path.join(INCLUDE, "*.h"))
-    newest_header = max(os.path.getmtime(d) for d in headers)
     os.makedirs(BUILD, exist_ok=True)
     nvcc = _nvcc()
     objs, rebuilt = [], False
     for src in sources:
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
         objs.append(obj)
+        deps = [src, *local_headers(src)]
         if not force and os.path.exists(obj) and \
-                os.path.getmtime(obj) >= max(os.path.getmtime(src), newest_header):
+                os.path.getmtime(obj) >= max(os.path.getmtime(d) for d in deps):
             continue
         cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
         if os.path.basename(src) in CUTLASS_SOURCES:

@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "tma.cuh"
+#include "umma.cuh"
 #include "tok_common.cuh"
 #include "tok_internal.h"
 
@@ -59,6 +60,26 @@ bool encode_tensor_map(CUtensorMap *map, CUtensorMapDataType dtype, int rank, co
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool encode_tensor_map_sw128(CUtensorMap *map, int rank, const void *base, const uint64_t *dims,
+                             const uint64_t *strides_bytes, const uint32_t *box)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 fn = encoder();
+    if (!fn)
+        return false;
+    cuuint64_t gdim[5], gstr[4];
+    cuuint32_t bdim[5], estr[5];
+    for (int i = 0; i < rank; ++i) {
+        gdim[i] = dims[i];
+        bdim[i] = box[i];
+        estr[i] = 1;
+        if (i + 1 < rank)
+            gstr[i] = strides_bytes[i];
+    }
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gdim, gstr, bdim,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count()
 {
     static int counts[64] = {0};
@@ -84,15 +105,17 @@ extern "C" int tok_last_cuda_error(void) { return tok::g_last_cuda_error; }
 
 extern "C" tok_status tok_check_device(cudaStream_t stream)
 {
-    unsigned int nh = 0, nf = 0, nb = 0;
+    unsigned int nh = 0, nf = 0, nb = 0, nc = 0;
     tok_status st = tok::read_and_clear_haar_timeouts(stream, &nh);
     if (st == TOK_OK)
         st = tok::read_and_clear_fsq_timeouts(stream, &nf);
     if (st == TOK_OK)
         st = tok::read_and_clear_fsq_bwd_timeouts(stream, &nb);
+    if (st == TOK_OK)
+        st = tok::read_and_clear_conv_timeouts(stream, &nc);
     if (st != TOK_OK)
         return st;
-    return (nh || nf || nb) ? TOK_ERR_TIMEOUT : TOK_OK;
+    return (nh || nf || nb || nc) ? TOK_ERR_TIMEOUT : TOK_OK;
 }
 
 extern "C" const char *tok_status_str(tok_status status)
@@ -116,7 +139,7 @@ extern "C" const char *tok_status_str(tok_status status)
         return "TOK_ERR_TIMEOUT: a kernel stopped after a barrier wait ran out; its output is incomplete";
     case TOK_ERR_TOO_LARGE:
         return "TOK_ERR_TOO_LARGE: the call needs more than the 3 MB fixed scratch of the allocation-free call "
-               "(at most 8388608 tokens at C = 16)";
+               "(at most 8388608 tokens at C = 16), or runs on a device ordinal above 63";
     }
     return "unknown tok_status";
 }

@@ -132,6 +132,8 @@ tok_status spatial_call(const void *x, const void *ws, void *y, int64_t B, int64
     const tok_status st = check_conv(x, ws, y, B, T, h, w, Cin, Cout, k * k, &ni, &no);
     if (st != TOK_OK || B * T * h * w == 0)
         return st;
+    if (conv_tc_eligible(Cin, Cout))
+        return conv_tc_spatial(x, ws, y, B, T, h, w, Cin, Cout, k, stream);
     const int pad = (int)(k - 1) / 2, kk = (int)k;
     typename Spatial::Problem p(cutlass::conv::Mode::kCrossCorrelation, {(int)(B * T), (int)h, (int)w, (int)Cin},
                                 {(int)Cout, kk, kk, (int)Cin}, {pad, pad}, {pad, pad}, {1, 1}, {1, 1}, 1);
@@ -147,6 +149,8 @@ tok_status temporal_call(const void *x, const void *wt, void *y, int64_t B, int6
     const tok_status st = check_conv(x, wt, y, B, T, h, w, Cin, Cout, k, &ni, &no);
     if (st != TOK_OK || B * T * h * w == 0)
         return st;
+    if (conv_tc_eligible(Cin, Cout))
+        return conv_tc_temporal(x, wt, y, B, T, h, w, Cin, Cout, k, stream);
     typename Temporal::Problem p(cutlass::conv::Mode::kCrossCorrelation,
                                  {(int)B, (int)T, (int)h, (int)w, (int)Cin}, {(int)Cout, (int)k, 1, 1, (int)Cin},
                                  {(int)k - 1, 0, 0}, {0, 0, 0}, {1, 1, 1}, {1, 1, 1}, 1);

@@ -1,0 +1,798 @@
+// The first causal factorized convolution after the patcher, as hand-written
+// implicit GEMMs on the 5th-generation tensor cores.
+//
+// Source: "Cosmos World Foundation Model Platform for Physical AI (Cosmos-Predict1)"
+// notes, model architecture item 1: after the 2-level Haar transform the encoder's
+// convolutions are factorized -- a 1 x k x k spatial convolution, then a k x 1 x 1
+// temporal convolution padded by k - 1 on the past side only.
+//
+// Activations are channels-last bf16 [frames, h, w, C]; fp32 accumulation.  A CTA
+// owns one SM and walks its tiles persistently.  A tile is 128 output positions --
+// 16 rows x 8 columns of one frame -- by up to 256 output channels: the MMA is
+// M = 128, N = 256, and each K step is 64 input channels of one tap.  Warp roles:
+//   warp 0     tensor copies: per K step, the activation box [64 ch, 8 cols,
+//              16 rows] of the tap's frame / shift (zero-filled outside the frame)
+//              and the filter box [64 k, N] into one of kStages stages, both in the
+//              128-byte swizzle the MMA reads;
+//   warp 1     one thread issues tcgen05.mma (4 per K step, K = 16 each) into a
+//              tensor-memory accumulator and commits each stage back to warp 0;
+//   warps 2-5  epilogue: tensor memory -> registers (each thread one position, its
+//              lane of the accumulator), round to bf16, 16-byte stores.
+// Two accumulators in tensor memory (2 x N columns) let a tile's epilogue overlap
+// the next tile's MMAs.  The temporal convolution orders tiles time-fastest, so the
+// k frames a tile reads are read again by the next tiles while they are in L2; the
+// spatial one orders them column-block-fastest for the halo rows.
+//
+// Waits are bounded: a barrier that does not complete in time raises the CTA's
+// abort flag, every role leaves its loop, the copies and MMAs already issued are
+// waited for (bounded), tensor memory is freed and a timeout is counted for
+// tok_check_device().  No load is broadcast to a cluster.
+#include <algorithm>
+#include <cstring>
+
+#include "tok_common.cuh"
+#include "tok_internal.h"
+#include "umma.cuh"
+
+namespace tok {
+
+// Convolution kernels that gave up on a barrier wait since the last check.
+static __device__ unsigned int g_conv_timeouts = 0;
+
+namespace {
+
+constexpr int kTileRows = 16, kTileCols = 8, kBM = kTileRows * kTileCols; // positions per tile
+constexpr int kBK = 64;                                                   // K per stage: one 128-byte row
+constexpr int kStages = 4;
+constexpr int kThreads = 192; // 6 warps
+constexpr uint32_t kABytes = kBM * kBK * 2;
+
+struct ConvGeom {
+    int frames;   // B * T
+    int T;        // frames per clip
+    int h, w;
+    int cin;      // input channels (multiple of 64)
+    int n;        // output channels
+    int bn;       // output channels per tile
+    int n_tiles;  // n / bn
+    int tiles_x, tiles_y;
+    int ntiles;
+    int k;        // taps per axis
+    int temporal; // 1: causal temporal (k x 1 x 1), 0: spatial (1 x k x k, 'same' zeros)
+};
+
+struct TileCoord {
+    int f;   // frame index in [0, B*T)
+    int t;   // frame within its clip
+    int y0, x0, n0;
+    int kb0; // first K step (temporal: taps before the clip's first frame are skipped)
+    int nkb; // K steps of this tile
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const ConvGeom &g, int i)
+{
+    TileCoord c;
+    const int nchunk = g.cin / kBK;
+    int r = i, xb, yb, nb;
+    if (g.temporal) { // time fastest: the k frames a tile reads are read by the next tiles too
+        c.t = r % g.T;
+        r /= g.T;
+        nb = r % g.n_tiles;
+        r /= g.n_tiles;
+        xb = r % g.tiles_x;
+        r /= g.tiles_x;
+        yb = r % g.tiles_y;
+        const int b = r / g.tiles_y;
+        c.f = b * g.T + c.t;
+        const int dt0 = max(0, g.k - 1 - c.t);
+        c.kb0 = dt0 * nchunk;
+        c.nkb = (g.k - dt0) * nchunk;
+    } else { // output-channel tiles fastest (they share the activations), then column blocks
+        nb = r % g.n_tiles;
+        r /= g.n_tiles;
+        xb = r % g.tiles_x;
+        r /= g.tiles_x;
+        yb = r % g.tiles_y;
+        c.f = r / g.tiles_y;
+        c.t = 0;
+        c.kb0 = 0;
+        c.nkb = g.k * g.k * nchunk;
+    }
+    c.y0 = yb * kTileRows;
+    c.x0 = xb * kTileCols;
+    c.n0 = nb * g.bn;
+    return c;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+               __nv_bfloat16 *__restrict__ out, const ConvGeom g)
+{
+    __shared__ __align__(8) uint64_t full[kStages], empty[kStages], accf[2], acce[2], drain;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const uint32_t bbytes = (uint32_t)g.bn * kBK * 2;
+    const uint32_t stage_bytes = kABytes + bbytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ncols = g.bn <= 16 ? 32u : g.bn <= 32 ? 64u : g.bn <= 64 ? 128u : g.bn <= 128 ? 256u : 512u;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_addr(&accf[a]), 1);
+            mbar_init(smem_addr(&acce[a]), 4);
+        }
+        mbar_init(smem_addr(&drain), 1);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(&tmem_base_s), ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    volatile int *abort = &abort_s;
+    const int nchunk = g.cin / kBK;
+
+    if (warp == 0 && lane == 0) {
+        // Tensor copies.
+        uint32_t it = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x) {
+            const TileCoord c = decode_tile(g, i);
+            for (int kb = 0; kb < c.nkb; ++kb, ++it) {
+                const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+                if (!wait_or_abort(smem_addr(&empty[s]), ph ^ 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes, fb = smem_addr(&full[s]);
+                const int kk = c.kb0 + kb, tap = kk / nchunk, ch = (kk - tap * nchunk) * kBK;
+                mbar_expect_tx(fb, stage_bytes);
+                if (g.temporal)
+                    tma_load_4d(sa, &amap, ch, c.x0, c.y0, c.f - (g.k - 1) + tap, fb);
+                else {
+                    const int pad = (g.k - 1) / 2, dy = tap / g.k, dx = tap - dy * g.k;
+                    tma_load_4d(sa, &amap, ch, c.x0 + dx - pad, c.y0 + dy - pad, c.f, fb);
+                }
+                tma_load_2d(sb, &bmap, kk * kBK, c.n0, fb);
+            }
+        }
+        if (!ok) // let the copies already issued land before the CTA exits (each wait bounded)
+            for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+                mbar_wait(smem_addr(&full[j % kStages]), (j / kStages) & 1u);
+    } else if (warp == 1 && lane == 0) {
+        // MMA issue.
+        const uint32_t idesc = idesc_bf16_f32(kBM, g.bn);
+        uint32_t it = 0, tc = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x, ++tc) {
+            const TileCoord c = decode_tile(g, i);
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&acce[acc]), (use & 1u) ^ 1u, abort))
+                break;
+            tc_fence_after();
+            const uint32_t d = tmem + acc * (uint32_t)g.bn;
+            for (int kb = 0; kb < c.nkb; ++kb, ++it) {
+                const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+                if (!wait_or_abort(smem_addr(&full[s]), ph, abort)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes;
+                const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
+#pragma unroll
+                for (int k = 0; k < kBK / 16; ++k)
+                    umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                umma_commit(smem_addr(&empty[s]));
+            }
+            if (ok)
+                umma_commit(smem_addr(&accf[acc]));
+        }
+        // Every MMA issued has completed before tensor memory is freed.
+        umma_commit(smem_addr(&drain));
+        mbar_wait(smem_addr(&drain), 0u);
+    } else if (warp >= 2) {
+        // Epilogue: warp q = warp % 4 reads accumulator lanes 32q .. 32q + 31.
+        const int q = warp & 3, row = 32 * q + lane;
+        const int r = row / kTileCols, jj = row - r * kTileCols;
+        uint32_t tc = 0;
+        for (int i = blockIdx.x; i < g.ntiles; i += gridDim.x, ++tc) {
+            const TileCoord c = decode_tile(g, i);
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&accf[acc]), use & 1u, abort))
+                break;
+            tc_fence_after();
+            const int y = c.y0 + r, x = c.x0 + jj;
+            const bool valid = y < g.h && x < g.w;
+            __nv_bfloat16 *o = out + (((int64_t)c.f * g.h + y) * g.w + x) * g.n + c.n0;
+            for (int cb = 0; cb < g.bn; cb += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * (uint32_t)g.bn + (uint32_t)cb, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        *reinterpret_cast<uint4 *>(o + cb + 8 * s) = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * s + 0]), __uint_as_float(v[8 * s + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 2]), __uint_as_float(v[8 * s + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 4]), __uint_as_float(v[8 * s + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 6]), __uint_as_float(v[8 * s + 7])));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&acce[acc]));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+    if (threadIdx.x == 0 && *abort)
+        atomicAdd(&g_conv_timeouts, 1u);
+}
+
+size_t conv_smem_bytes(int bn) { return (size_t)kStages * (kABytes + (uint32_t)bn * kBK * 2) + 1024; }
+
+bool fits_int(int64_t v) { return v >= 0 && v < ((int64_t)1 << 31); }
+
+// The tensor-core form takes Cin a multiple of 64 and Cout a multiple of 32 up to 256
+// or a multiple of 256; 32-bit extents.
+bool tc_eligible(int64_t Cin, int64_t Cout)
+{
+    return Cin >= 64 && Cin % 64 == 0 && Cout >= 32 && Cout % 32 == 0 && (Cout <= 256 || Cout % 256 == 0);
+}
+
+tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y, int64_t B, int64_t T, int64_t h,
+                          int64_t w, int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream)
+{
+    ConvGeom g{};
+    g.frames = (int)(B * T);
+    g.T = (int)T;
+    g.h = (int)h;
+    g.w = (int)w;
+    g.cin = (int)Cin;
+    g.n = (int)Cout;
+    g.bn = Cout <= 256 ? (int)Cout : 256;
+    g.n_tiles = (int)(Cout / g.bn);
+    g.tiles_x = (int)((w + kTileCols - 1) / kTileCols);
+    g.tiles_y = (int)((h + kTileRows - 1) / kTileRows);
+    const int64_t ntiles = (int64_t)g.frames * g.tiles_x * g.tiles_y * g.n_tiles;
+    if (!fits_int(ntiles))
+        return TOK_ERR_SHAPE;
+    g.ntiles = (int)ntiles;
+    g.k = (int)k;
+    g.temporal = temporal ? 1 : 0;
+
+    CUtensorMap amap, bmap;
+    const uint64_t adims[4] = {(uint64_t)Cin, (uint64_t)w, (uint64_t)h, (uint64_t)g.frames};
+    const uint64_t astr[3] = {(uint64_t)Cin * 2, (uint64_t)w * Cin * 2, (uint64_t)h * w * Cin * 2};
+    const uint32_t abox[4] = {kBK, kTileCols, kTileRows, 1};
+    const int64_t ktot = (temporal ? k : k * k) * Cin;
+    const uint64_t bdims[2] = {(uint64_t)ktot, (uint64_t)Cout};
+    const uint64_t bstr[1] = {(uint64_t)ktot * 2};
+    const uint32_t bbox[2] = {kBK, (uint32_t)g.bn};
+    if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, abox) ||
+        !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox))
+        return TOK_ERR_SHAPE;
+
+    const size_t smem = conv_smem_bytes(g.bn);
+    cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    const int sms = sm_count();
+    if (sms <= 0)
+        return launch_status();
+    const int grid = (int)std::min<int64_t>(ntiles, sms);
+    conv_tc_kernel<<<grid, kThreads, smem, stream>>>(amap, bmap, static_cast<__nv_bfloat16 *>(y), g);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// The patcher fused into the spatial convolution (k = 3).  The A operand of each
+// K step is made in shared memory by four Haar warps from the pixels, so the
+// coefficients never reach HBM.  Its K order is (input channel c, column shift dx,
+// row shift dy, the 64 subbands g of c): plane (c, dx) holds, for the tile's 16 + 2
+// latent rows and 8 columns shifted by dx - 1, the 64 coefficients of colour c as one
+// 128-byte swizzled row per position (row q = r * 8 + j: one tile row is one 1024-byte
+// swizzle atom), and the three K steps dy = 0, 1, 2 are that plane seen from atom dy.
+// The filter is read in the same K order from a packed copy (tok_patch_embed_pack_weights).
+//   warp 0     tensor copies of the packed filter, kFStages stages of [64 k, N];
+//   warp 1     MMA issue (planes and filter stages as they fill);
+//   warps 2-5  epilogue, as in conv_tc_kernel;
+//   warps 6-9  Haar: per colour, one tensor copy of the pixels the tile's 3 x 3
+//              neighbourhood reads ([4 frames][72 rows][48 cols], two buffers, the
+//              next colour's copy issued before this colour's planes are made); per
+//              plane, each of 72 threads transforms two horizontally adjacent blocks
+//              in packed f32x2 pairs -- the butterflies of the planar patcher in its
+//              order (columns, rows, frames; then x 1/8), so the coefficients are the
+//              patcher's bits -- rounds them to bf16 and writes both positions' rows.
+// Latent positions outside the frame read zero pixels (the tensor copy fills zeros),
+// which is exactly the convolution's zero padding of the coefficients.
+// ---------------------------------------------------------------------------
+constexpr int kFStages = 3;                      // filter stages
+constexpr int kPlanes = 3;                       // A planes in flight
+constexpr int kPlaneRows = kTileRows + 2;        // latent rows of a plane
+constexpr uint32_t kPlaneBytes = kPlaneRows * kTileCols * 128; // 18 KB
+constexpr int kPixCols = 48, kPixRows = 4 * kPlaneRows, kPixFrames = 4;
+constexpr uint32_t kPixBytes = kPixCols * kPixRows * kPixFrames * 2; // 27 KB
+constexpr int kEmbedThreads = 320;               // 10 warps
+constexpr int kHaarThreads = 128;
+constexpr int kHaarFirst = 192;                  // first Haar thread
+
+struct EmbedGeom {
+    int B, C, Tq, h, w;   // pixels [B, C, 4*Tq - 3, 4h, 4w]; output [B, Tq, h, w, n]
+    int n, bn, n_tiles;
+    int tiles_x, tiles_y, ntiles;
+};
+
+struct EmbedTile {
+    int b, tq, y0, x0, n0;
+};
+
+__device__ __forceinline__ EmbedTile decode_embed(const EmbedGeom &g, int i)
+{
+    EmbedTile e;
+    const int nb = i % g.n_tiles; // output-channel tiles fastest: they read the same pixels
+    int r = i / g.n_tiles;
+    const int xb = r % g.tiles_x;
+    r /= g.tiles_x;
+    const int yb = r % g.tiles_y;
+    r /= g.tiles_y;
+    e.tq = r % g.Tq;
+    e.b = r / g.Tq;
+    e.y0 = yb * kTileRows;
+    e.x0 = xb * kTileCols;
+    e.n0 = nb * g.bn;
+    return e;
+}
+
+__device__ __forceinline__ float2 f2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 f2sub(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.0f, -1.0f), a); }
+
+// Two levels of the causal full-packet Haar transform along one axis on four pairs,
+// unnormalized, natural order k = 2 * b2 + b1 (the planar patcher's butterflies).
+__device__ __forceinline__ void wht4x2(float2 &a0, float2 &a1, float2 &a2, float2 &a3)
+{
+    const float2 l0 = f2add(a0, a1), h0 = f2sub(a0, a1), l1 = f2add(a2, a3), h1 = f2sub(a2, a3);
+    a0 = f2add(l0, l1);
+    a1 = f2add(h0, h1);
+    a2 = f2sub(l0, l1);
+    a3 = f2sub(h0, h1);
+}
+
+// Per-axis indices of subband g = 8 * s2 + s1, s = 4 * b_t + 2 * b_y + b_x (bit 1: high band).
+__host__ __device__ constexpr int sb_kt(int g) { return 2 * ((g >> 3) >> 2) + ((g & 7) >> 2); }
+__host__ __device__ constexpr int sb_ky(int g) { return 2 * (((g >> 3) >> 1) & 1) + (((g & 7) >> 1) & 1); }
+__host__ __device__ constexpr int sb_kx(int g) { return 2 * ((g >> 3) & 1) + (g & 1); }
+
+__device__ __forceinline__ void issue_pixels(const CUtensorMap *xmap, const EmbedTile &e, int c, uint32_t dst,
+                                             uint32_t bar)
+{
+    mbar_expect_tx(bar, kPixBytes);
+    tma_load_5d(dst, xmap, 4 * e.x0 - 8, 4 * e.y0 - 4, 4 * e.tq - 3, c, e.b, bar);
+}
+
+__global__ void __launch_bounds__(kEmbedThreads, 1)
+patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
+                   __nv_bfloat16 *__restrict__ out, const EmbedGeom g)
+{
+    __shared__ __align__(8) uint64_t ffull[kFStages], fempty[kFStages], pfull[kPlanes], pempty[kPlanes], xfull[2],
+        accf[2], acce[2], drain, hsync;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const uint32_t fbytes = (uint32_t)g.bn * kBK * 2;
+    const uint32_t fbase = base, pbase = fbase + kFStages * fbytes, xbase = pbase + kPlanes * kPlaneBytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ncols = g.bn <= 16 ? 32u : g.bn <= 32 ? 64u : g.bn <= 64 ? 128u : g.bn <= 128 ? 256u : 512u;
+    const int kper = 9 * g.C; // K steps per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kFStages; ++s) {
+            mbar_init(smem_addr(&ffull[s]), 1);
+            mbar_init(smem_addr(&fempty[s]), 1);
+        }
+        for (int p = 0; p < kPlanes; ++p) {
+            mbar_init(smem_addr(&pfull[p]), kHaarThreads);
+            mbar_init(smem_addr(&pempty[p]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_addr(&xfull[a]), 1);
+            mbar_init(smem_addr(&accf[a]), 1);
+            mbar_init(smem_addr(&acce[a]), 4);
+        }
+        mbar_init(smem_addr(&drain), 1);
+        mbar_init(smem_addr(&hsync), kHaarThreads);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_addr(&tmem_base_s), ncols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    volatile int *abort = &abort_s;
+
+    if (warp == 0 && lane == 0) {
+        // Filter copies, in the tile's K order.
+        uint32_t it = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x) {
+            const EmbedTile e = decode_embed(g, i);
+            for (int kb = 0; kb < kper; ++kb, ++it) {
+                const uint32_t s = it % kFStages, ph = (it / kFStages) & 1u;
+                if (!wait_or_abort(smem_addr(&fempty[s]), ph ^ 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t fb = smem_addr(&ffull[s]);
+                mbar_expect_tx(fb, fbytes);
+                tma_load_2d(fbase + s * fbytes, &bmap, kb * kBK, e.n0, fb);
+            }
+        }
+        if (!ok)
+            for (uint32_t j = it > kFStages ? it - kFStages : 0; j < it; ++j)
+                mbar_wait(smem_addr(&ffull[j % kFStages]), (j / kFStages) & 1u);
+    } else if (warp == 1 && lane == 0) {
+        // MMA issue: per plane (c, dx), the three row shifts dy.
+        const uint32_t idesc = idesc_bf16_f32(kBM, g.bn);
+        uint32_t it = 0, pi = 0, tc = 0;
+        bool ok = true;
+        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x, ++tc) {
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&acce[acc]), (use & 1u) ^ 1u, abort))
+                break;
+            tc_fence_after();
+            const uint32_t d = tmem + acc * (uint32_t)g.bn;
+            for (int pl = 0; pl < 3 * g.C && ok; ++pl, ++pi) {
+                const uint32_t slot = pi % kPlanes;
+                if (!wait_or_abort(smem_addr(&pfull[slot]), (pi / kPlanes) & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                for (int dy = 0; dy < 3; ++dy, ++it) {
+                    const uint32_t s = it % kFStages, ph = (it / kFStages) & 1u;
+                    if (!wait_or_abort(smem_addr(&ffull[s]), ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(pbase + slot * kPlaneBytes + (uint32_t)dy * 1024u);
+                    const uint64_t bd = sw128_desc(fbase + s * fbytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
+                    umma_commit(smem_addr(&fempty[s]));
+                }
+                if (ok)
+                    umma_commit(smem_addr(&pempty[slot]));
+            }
+            if (ok)
+                umma_commit(smem_addr(&accf[acc]));
+        }
+        umma_commit(smem_addr(&drain));
+        mbar_wait(smem_addr(&drain), 0u);
+    } else if (warp >= 2 && warp < 6) {
+        // Epilogue.
+        const int q = warp & 3, row = 32 * q + lane;
+        const int r = row / kTileCols, jj = row - r * kTileCols;
+        uint32_t tc = 0;
+        for (int i = blockIdx.x; i < g.ntiles; i += gridDim.x, ++tc) {
+            const EmbedTile e = decode_embed(g, i);
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&accf[acc]), use & 1u, abort))
+                break;
+            tc_fence_after();
+            const int y = e.y0 + r, x = e.x0 + jj;
+            const bool valid = y < g.h && x < g.w;
+            __nv_bfloat16 *o = out + ((((int64_t)e.b * g.Tq + e.tq) * g.h + y) * g.w + x) * g.n + e.n0;
+            for (int cb = 0; cb < g.bn; cb += 32) {
+                uint32_t v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * (uint32_t)g.bn + (uint32_t)cb, v);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        *reinterpret_cast<uint4 *>(o + cb + 8 * s) = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * s + 0]), __uint_as_float(v[8 * s + 1])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 2]), __uint_as_float(v[8 * s + 3])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 4]), __uint_as_float(v[8 * s + 5])),
+                            pack_bf16x2(__uint_as_float(v[8 * s + 6]), __uint_as_float(v[8 * s + 7])));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(smem_addr(&acce[acc]));
+        }
+    } else if (warp >= 6) {
+        // Haar warps.
+        const int ht = threadIdx.x - kHaarFirst;
+        const int pr = ht >> 2, jp = ht & 3; // work item: plane row pr (0..17), columns 2 jp, 2 jp + 1
+        const bool worker = ht < kPlaneRows * 4;
+        uint32_t ci = 0, pi = 0; // colours and planes made so far
+        bool ok = true;
+        int i = blockIdx.x;
+        if (ht == 0 && i < g.ntiles)
+            issue_pixels(&xmap, decode_embed(g, i), 0, xbase, smem_addr(&xfull[0]));
+        for (; i < g.ntiles && ok; i += gridDim.x) {
+            const EmbedTile e = decode_embed(g, i);
+            for (int c = 0; c < g.C && ok; ++c, ++ci) {
+                // Once every Haar thread is done with the buffer of colour ci - 1 (a barrier phase per
+                // colour; its wait is bounded like the others), colour ci + 1 is copied into it.
+                mbar_arrive(smem_addr(&hsync));
+                if (!wait_or_abort(smem_addr(&hsync), ci & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                if (ht == 0) {
+                    const bool last_c = c + 1 == g.C;
+                    const int ni = last_c ? i + (int)gridDim.x : i;
+                    if (ni < g.ntiles) {
+                        fence_proxy_async_smem();
+                        const uint32_t nb = (ci + 1) & 1u;
+                        issue_pixels(&xmap, last_c ? decode_embed(g, ni) : e, last_c ? 0 : c + 1,
+                                     xbase + nb * kPixBytes, smem_addr(&xfull[nb]));
+                    }
+                }
+                const uint32_t xb = ci & 1u;
+                if (!wait_or_abort(smem_addr(&xfull[xb]), (ci >> 1) & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                const unsigned char *pix = smem_raw + (xbase + xb * kPixBytes - smem_addr(smem_raw));
+                for (int dx = 0; dx < 3; ++dx, ++pi) {
+                    const uint32_t slot = pi % kPlanes;
+                    if (!wait_or_abort(smem_addr(&pempty[slot]), ((pi / kPlanes) & 1u) ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (worker) {
+                        // Blocks at latent (y0 - 1 + pr, x0 + 2 jp + dx - 1 + {0, 1}): pixel rows 4 pr ..,
+                        // columns 4 (2 jp + dx + 1) .. of the staged box; window 0 reads frame 0 (box frame 3)
+                        // four times.
+                        float2 v[4][4][4];
+                        const int col = 4 * (2 * jp + dx + 1);
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const int fa = e.tq == 0 ? 3 : a;
+#pragma unroll
+                            for (int rr = 0; rr < 4; ++rr) {
+                                const unsigned char *rowp = pix + ((fa * kPixRows + 4 * pr + rr) * kPixCols + col) * 2;
+                                const uint2 p0 = *reinterpret_cast<const uint2 *>(rowp);
+                                const uint2 p1 = *reinterpret_cast<const uint2 *>(rowp + 8);
+                                v[a][rr][0] = make_float2(bf16_lo(p0.x), bf16_lo(p1.x));
+                                v[a][rr][1] = make_float2(bf16_hi(p0.x), bf16_hi(p1.x));
+                                v[a][rr][2] = make_float2(bf16_lo(p0.y), bf16_lo(p1.y));
+                                v[a][rr][3] = make_float2(bf16_hi(p0.y), bf16_hi(p1.y));
+                            }
+                        }
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+#pragma unroll
+                            for (int rr = 0; rr < 4; ++rr)
+                                wht4x2(v[a][rr][0], v[a][rr][1], v[a][rr][2], v[a][rr][3]);
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                wht4x2(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
+#pragma unroll
+                        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                wht4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
+                        unsigned char *plane = smem_raw + (pbase + slot * kPlaneBytes - smem_addr(smem_raw));
+                        const float2 eighth = make_float2(0.125f, 0.125f);
+#pragma unroll
+                        for (int k8 = 0; k8 < 8; ++k8) {
+                            uint32_t lo[4], hi[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int g0 = 8 * k8 + 2 * u, g1 = g0 + 1;
+                                const float2 a0 = __fmul2_rn(v[sb_kt(g0)][sb_ky(g0)][sb_kx(g0)], eighth);
+                                const float2 a1 = __fmul2_rn(v[sb_kt(g1)][sb_ky(g1)][sb_kx(g1)], eighth);
+                                lo[u] = pack_bf16x2(a0.x, a1.x);
+                                hi[u] = pack_bf16x2(a0.y, a1.y);
+                            }
+                            const int q0 = pr * kTileCols + 2 * jp, q1 = q0 + 1;
+                            *reinterpret_cast<uint4 *>(plane + sw128_offset(q0, 8 * k8)) =
+                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                            *reinterpret_cast<uint4 *>(plane + sw128_offset(q1, 8 * k8)) =
+                                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                        }
+                    }
+                    fence_proxy_async_smem(); // the plane's writes are visible to the tensor cores
+                    mbar_arrive(smem_addr(&pfull[slot]));
+                }
+            }
+        }
+        if (ht == 0 && !ok) // the pixel copies issued and not yet waited for
+            for (uint32_t j = ci; j < ci + 2; ++j)
+                mbar_wait(smem_addr(&xfull[j & 1u]), (j >> 1) & 1u);
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, ncols);
+    }
+    if (threadIdx.x == 0 && *abort)
+        atomicAdd(&g_conv_timeouts, 1u);
+}
+
+size_t embed_smem_bytes(int bn)
+{
+    return (size_t)kFStages * bn * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes + 1024;
+}
+
+// Packed filter: wp[n][(c * 3 + dx) * 3 + dy][g] = ws[n][dy][dx][g * C + c].
+__global__ void pack_embed_weights_kernel(const __nv_bfloat16 *__restrict__ ws, __nv_bfloat16 *__restrict__ wp,
+                                          int C, int64_t total)
+{
+    const int64_t o = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (o >= total)
+        return;
+    const int K = 576 * C;
+    const int64_t n = o / K;
+    const int kk = (int)(o - n * K), kb = kk / 64, gg = kk - kb * 64;
+    const int c = kb / 9, dx = (kb / 3) % 3, dy = kb % 3;
+    wp[o] = ws[((n * 3 + dy) * 3 + dx) * (int64_t)(64 * C) + gg * C + c];
+}
+
+} // namespace
+
+bool conv_tc_eligible(int64_t Cin, int64_t Cout) { return tc_eligible(Cin, Cout); }
+
+tok_status conv_tc_temporal(const void *x, const void *wt, void *y, int64_t B, int64_t T, int64_t h, int64_t w,
+                            int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream)
+{
+    return conv_tc_launch(true, x, wt, y, B, T, h, w, Cin, Cout, k, stream);
+}
+
+tok_status conv_tc_spatial(const void *x, const void *ws, void *y, int64_t B, int64_t T, int64_t h, int64_t w,
+                           int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream)
+{
+    return conv_tc_launch(false, x, ws, y, B, T, h, w, Cin, Cout, k, stream);
+}
+
+bool patch_embed_eligible(int64_t C, int64_t Cmid) { return C >= 1 && C <= 8 && tc_eligible(64 * C, Cmid); }
+
+tok_status patch_embed_pack(const void *ws, void *wp, int64_t C, int64_t Cmid, cudaStream_t stream)
+{
+    const int64_t total = Cmid * 576 * C;
+    if (total == 0)
+        return TOK_OK;
+    const int threads = 256;
+    pack_embed_weights_kernel<<<(unsigned)((total + threads - 1) / threads), threads, 0, stream>>>(
+        static_cast<const __nv_bfloat16 *>(ws), static_cast<__nv_bfloat16 *>(wp), (int)C, total);
+    return launch_status();
+}
+
+tok_status patch_embed_launch(const void *x, const void *wp, void *y, int64_t B, int64_t C, int64_t T, int64_t H,
+                              int64_t W, int64_t Cmid, cudaStream_t stream)
+{
+    EmbedGeom g{};
+    g.B = (int)B;
+    g.C = (int)C;
+    g.Tq = (int)(1 + (T - 1) / 4);
+    g.h = (int)(H / 4);
+    g.w = (int)(W / 4);
+    g.n = (int)Cmid;
+    g.bn = Cmid <= 256 ? (int)Cmid : 256;
+    g.n_tiles = (int)(Cmid / g.bn);
+    g.tiles_x = (g.w + kTileCols - 1) / kTileCols;
+    g.tiles_y = (g.h + kTileRows - 1) / kTileRows;
+    const int64_t ntiles = B * g.Tq * (int64_t)g.tiles_x * g.tiles_y * g.n_tiles;
+    if (!fits_int(ntiles))
+        return TOK_ERR_SHAPE;
+    g.ntiles = (int)ntiles;
+
+    CUtensorMap xmap, bmap;
+    const uint64_t xdims[5] = {(uint64_t)W, (uint64_t)H, (uint64_t)T, (uint64_t)C, (uint64_t)B};
+    const uint64_t xstr[4] = {(uint64_t)W * 2, (uint64_t)H * W * 2, (uint64_t)T * H * W * 2,
+                              (uint64_t)C * T * H * W * 2};
+    const uint32_t xbox[5] = {kPixCols, kPixRows, kPixFrames, 1, 1};
+    const uint64_t bdims[2] = {(uint64_t)(576 * C), (uint64_t)Cmid};
+    const uint64_t bstr[1] = {(uint64_t)(576 * C) * 2};
+    const uint32_t bbox[2] = {kBK, (uint32_t)g.bn};
+    if (!encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, x, xdims, xstr, xbox) ||
+        !encode_tensor_map_sw128(&bmap, 2, wp, bdims, bstr, bbox))
+        return TOK_ERR_SHAPE;
+    const size_t smem = embed_smem_bytes(g.bn);
+    cudaError_t e = cudaFuncSetAttribute(patch_embed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    const int sms = sm_count();
+    if (sms <= 0)
+        return launch_status();
+    const int grid = (int)std::min<int64_t>(ntiles, sms);
+    patch_embed_kernel<<<grid, kEmbedThreads, smem, stream>>>(xmap, bmap, static_cast<__nv_bfloat16 *>(y), g);
+    return launch_status();
+}
+
+tok_status read_and_clear_conv_timeouts(cudaStream_t stream, unsigned int *count)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(count, g_conv_timeouts, sizeof(unsigned int), 0,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e == cudaSuccess && *count)
+        e = cudaMemcpyToSymbolAsync(g_conv_timeouts, &zero, sizeof(unsigned int), 0, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    return TOK_OK;
+}
+
+} // namespace tok
+
+// ---------------------------------------------------------------------------
+// C ABI of the fused patch embedding (declared in tok.h).
+// ---------------------------------------------------------------------------
+extern "C" tok_status tok_patch_embed_pack_weights(const void *ws, void *wp, int64_t C, int64_t Cmid,
+                                                    cudaStream_t stream)
+{
+    using namespace tok;
+    if (!patch_embed_eligible(C, Cmid))
+        return TOK_ERR_SHAPE;
+    if (!ws || !wp)
+        return TOK_ERR_NULL;
+    if (!aligned(ws, 2) || !aligned(wp, 16))
+        return TOK_ERR_ALIGN;
+    const int64_t bytes = Cmid * 576 * C * 2;
+    if (overlaps(ws, bytes, wp, bytes))
+        return TOK_ERR_ALIAS;
+    return patch_embed_pack(ws, wp, C, Cmid, stream);
+}
+
+extern "C" tok_status tok_patch_embed_spatial(const void *x, const void *wp, void *y, int64_t B, int64_t C,
+                                              int64_t T, int64_t H, int64_t W, int64_t Cmid, cudaStream_t stream)
+{
+    using namespace tok;
+    if (B < 0 || T < 5 || T % 4 != 1 || H < 0 || W < 0 || H % 4 || W % 8 || !patch_embed_eligible(C, Cmid))
+        return TOK_ERR_SHAPE;
+    const int64_t Tq = 1 + (T - 1) / 4, h = H / 4, w = W / 4;
+    int64_t nx, ny, pos;
+    if (!prod_ok({B, C, T, H, W, 2}, &nx) || !prod_ok({B, Tq, h, w}, &pos) || !prod_ok({pos, Cmid, 2}, &ny) ||
+        !fits_int(nx / 2) || !fits_int(ny / 2) || !fits_int(B * C) || H > 65536 || W > 65536)
+        return TOK_ERR_SHAPE;
+    if (pos == 0)
+        return TOK_OK;
+    if (!x || !wp || !y)
+        return TOK_ERR_NULL;
+    if (!aligned(x, 16) || !aligned(wp, 16) || !aligned(y, 16))
+        return TOK_ERR_ALIGN;
+    const int64_t nw = Cmid * 576 * C * 2;
+    if (overlaps(x, nx, y, ny) || overlaps(wp, nw, y, ny))
+        return TOK_ERR_ALIAS;
+    return patch_embed_launch(x, wp, y, B, C, T, H, W, Cmid, stream);
+}

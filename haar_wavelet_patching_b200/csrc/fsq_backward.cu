@@ -856,7 +856,9 @@ float *g_noalloc_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up once per
-// device (with that device current) and cached.
+// device (with that device current) and cached for the life of the process; a
+// device reset would invalidate it.  The cache covers device ordinals 0..63;
+// a higher ordinal is refused with TOK_ERR_TOO_LARGE.
 tok_status noalloc_scratch(float **out)
 {
     int dev = 0;
@@ -866,7 +868,7 @@ tok_status noalloc_scratch(float **out)
         return TOK_ERR_CUDA;
     }
     if (dev < 0 || dev >= kMaxDevices)
-        return TOK_ERR_CUDA;
+        return TOK_ERR_TOO_LARGE;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
     if (!g_noalloc_addr[dev]) {
         void *p = nullptr;

@@ -1474,6 +1474,31 @@ tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in,
                : launch_form<float, true, false, false, false>(form, in, out, d, stream);
 }
 
+// Self-test of the failure channel: one single-warp CTA whose barrier phase cannot
+// complete, because lane 0 declares 16 bytes of transaction that no copy ever
+// delivers.  Its wait gives up after `polls` polls, as a TMA kernel's wait does after
+// kWaitPolls, and counts a timeout.  No copy was issued, so nothing can land in this
+// CTA's shared memory after the kernel exits.
+__global__ void __launch_bounds__(32) wait_timeout_selftest_kernel(uint32_t polls)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(b, 16);
+        bool done = false;
+        for (uint32_t i = 0; i < polls && !done; ++i)
+            done = mbar_try_wait(b, 0u);
+        if (!done)
+            atomicAdd(&g_wait_timeouts, 1u);
+    }
+    __syncwarp();
+}
+
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count)
 {
     unsigned int zero = 0;
@@ -1708,3 +1733,11 @@ tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const Haa
 }
 
 } // namespace tok
+
+extern "C" tok_status tok_selftest_wait_timeout(uint32_t polls, cudaStream_t stream)
+{
+    if (polls < 1 || polls > tok::kWaitPolls)
+        return TOK_ERR_SHAPE;
+    tok::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>(polls);
+    return tok::launch_status();
+}

@@ -45,11 +45,20 @@ tok_status haar_single_tma_launch(bool fwd, HaarTmaForm form, const void *in, vo
 bool haar_cl_tma_eligible(const void *in, const void *out, tok_dtype dt, const HaarDims &d);
 tok_status haar_cl_tma_launch(const void *in, void *out, tok_dtype dt, const HaarDims &d, cudaStream_t stream);
 
+// Hand-written tensor-core convolutions (conv_tc.cu): eligible for Cin % 64 == 0 and
+// Cout % 32 == 0 (Cout <= 256, or a multiple of 256); arguments checked by the caller.
+bool conv_tc_eligible(int64_t Cin, int64_t Cout);
+tok_status conv_tc_temporal(const void *x, const void *wt, void *y, int64_t B, int64_t T, int64_t h, int64_t w,
+                            int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream);
+tok_status conv_tc_spatial(const void *x, const void *ws, void *y, int64_t B, int64_t T, int64_t h, int64_t w,
+                           int64_t Cin, int64_t Cout, int64_t k, cudaStream_t stream);
+
 // Synchronize `stream`, return in *count the barrier-wait timeouts of this device's
 // Haar (resp. FSQ, FSQ backward) kernels since the last call, and clear them.
 tok_status read_and_clear_haar_timeouts(cudaStream_t stream, unsigned int *count);
 tok_status read_and_clear_fsq_timeouts(cudaStream_t stream, unsigned int *count);
 tok_status read_and_clear_fsq_bwd_timeouts(cudaStream_t stream, unsigned int *count);
+tok_status read_and_clear_conv_timeouts(cudaStream_t stream, unsigned int *count);
 
 // Remembers a CUDA error for tok_last_cuda_error().
 void record_cuda_error(cudaError_t e);

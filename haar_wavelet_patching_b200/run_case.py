@@ -22,9 +22,11 @@ def main():
                                                      "haar_fwd_padded", "haar_inv_cropped", "haar_fwd_chunk",
                                                      "haar_inv_chunk", "fsq_encode", "fsq_decode",
                                                      "fsq_encode_backward", "fsq_decode_backward",
-                                                     "conv_spatial", "conv_temporal", "conv_factorized"))
+                                                     "conv_spatial", "conv_temporal", "conv_factorized",
+                                                     "patch_embed"))
     ap.add_argument("--shape", required=True,
-                    help="B,C,T,H,W for haar ops; B,C,S for fsq ops; B,T,h,w,Cin,Cmid,Cout for conv ops")
+                    help="B,C,T,H,W for haar ops; B,C,S for fsq ops; B,T,h,w,Cin,Cmid,Cout for conv ops; "
+                         "B,C,T,H,W,Cmid for patch_embed")
     ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--codes", action="store_true", help="fsq_encode: also write the codes")
@@ -37,7 +39,17 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op.startswith("conv"):
+    if a.op == "patch_embed":
+        B, C, T, H, W, Cmid = shape
+        bf = torch.bfloat16
+        x = (torch.rand((B, C, T, H, W), generator=g, device=dev) * 2 - 1).to(bf)
+        ws = (torch.randn((Cmid, 3, 3, 64 * C), generator=g, device=dev) * (9 * 64 * C) ** -0.5).to(bf)
+        wp = hwp.patch_embed_pack_weights(ws)
+        y = torch.empty((B, hwp.latent_frames(T), H // 4, W // 4, Cmid), dtype=bf, device=dev)
+        run = lambda: hwp.tok_patch_embed_spatial(x, wp, y)  # noqa: E731
+        flops = 2 * y.numel() // Cmid * Cmid * 9 * 64 * C
+        nbytes = (x.numel() + y.numel()) * 2
+    elif a.op.startswith("conv"):
         B, T, h, w, Cin, Cmid, Cout = shape
         bf = torch.bfloat16
         x = (torch.randn((B, T, h, w, Cin), generator=g, device=dev) * 0.5).to(bf)
@@ -123,7 +135,7 @@ def main():
     e1.record()
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / a.iters
-    extra = f", {flops / ms / 1e9:.1f} TFLOP/s" if a.op.startswith("conv") else ""
+    extra = f", {flops / ms / 1e9:.1f} TFLOP/s" if a.op.startswith(("conv", "patch")) else ""
     print(f"{a.op} {shape} {a.dtype}: {ms * 1e3:.1f} us per launch, {nbytes / ms / 1e6:.1f} GB/s{extra}")
 
 

@@ -70,7 +70,8 @@ typedef enum {
     TOK_ERR_ALIAS = 5, /* an input buffer overlaps an output buffer */
     TOK_ERR_CUDA = 6,   /* a CUDA call or kernel launch failed; see tok_last_cuda_error() */
     TOK_ERR_TIMEOUT = 7, /* reported by tok_check_device(): a kernel stopped after a bounded wait ran out */
-    TOK_ERR_TOO_LARGE = 8 /* the problem exceeds the fixed scratch of tok_fsq_encode_backward_noalloc */
+    TOK_ERR_TOO_LARGE = 8 /* the problem (or the device ordinal) exceeds the fixed scratch of
+                             tok_fsq_encode_backward_noalloc */
 } tok_status;
 
 typedef enum {
@@ -97,6 +98,21 @@ TOK_API int tok_last_cuda_error(void);
  * asynchronous calls.  Returns TOK_OK, TOK_ERR_TIMEOUT or TOK_ERR_CUDA.
  */
 TOK_API tok_status tok_check_device(cudaStream_t stream);
+
+/*
+ * tok_selftest_wait_timeout -- exercise the failure channel that
+ * tok_check_device reads.  Launches on `stream` one single-warp kernel whose
+ * shared-memory barrier waits for 16 bytes of copy that nothing ever issues;
+ * the wait gives up after `polls` polls (1 <= polls <= 2^22, the TMA kernels'
+ * own limit; a few thousand end within milliseconds), counts a timeout as the
+ * TMA kernels do when a wait runs out, and the kernel returns.  No copy is in
+ * flight at any time, so the device stays usable.  The next
+ * tok_check_device(stream) returns TOK_ERR_TIMEOUT and clears the count; the
+ * one after it returns TOK_OK.  Not part of the pages' method: a test hook for
+ * the error channel.  Returns TOK_ERR_SHAPE for `polls` out of range,
+ * TOK_ERR_CUDA if the launch fails.
+ */
+TOK_API tok_status tok_selftest_wait_timeout(uint32_t polls, cudaStream_t stream);
 
 /*
  * tok_haar_fwd -- two-level causal full-packet Haar patcher.
@@ -293,6 +309,37 @@ TOK_API tok_status tok_conv_factorized(const void *x, const void *ws, const void
                                        int64_t k, cudaStream_t stream);
 
 /*
+ * The patcher fused into the spatial convolution after it (k = 3), one kernel:
+ * [notes] model architecture item 1 (the 1 x k x k convolution right after the
+ * 2-level Haar transform) on the coefficients of [guide] 7.1 (Patcher3D, two
+ * levels, channel (8*s2 + s1)*C + c).  The coefficients are made in shared
+ * memory as the tensor cores' operand (the patcher's own bf16 values) and never
+ * reach HBM.
+ *
+ * tok_patch_embed_pack_weights -- reorder the spatial filter for the fused call:
+ *   ws : [Cmid, 3, 3, 64C] bf16, the layout of tok_conv_spatial (input)
+ *   wp : [Cmid, 9C, 64] bf16, wp[n][(c*3 + dx)*3 + dy][g] = ws[n][dy][dx][g*C + c]
+ *        (output, caller-owned, 1152*C*Cmid bytes; 16-byte aligned)
+ *   Run once per filter; the fused call reads wp.  Shape rule as below.
+ *
+ * tok_patch_embed_spatial -- y = tok_conv_spatial(channels-last patcher(x), ws)
+ *   with k = 3 ('same' zero padding in space):
+ *   x  : [B, C, T, H, W] bf16 pixels, video (T = 1 + 4k, T >= 5), H % 4 == 0,
+ *        W % 8 == 0 (input)
+ *   wp : the packed filter above (input)
+ *   y  : [B, T', H/4, W/4, Cmid] bf16, T' = 1 + (T-1)/4 (output)
+ *   Shape rule: 1 <= C <= 8; Cmid a multiple of 32, at most 256 or a multiple
+ *   of 256; 32-bit element counts.  Pointers 16-byte aligned (TOK_ERR_ALIGN);
+ *   y must not overlap x or wp (TOK_ERR_ALIAS).  fp32 accumulation, one bf16
+ *   rounding.  Not on the pages' API: the layer the pages name, with weights
+ *   the caller provides.
+ */
+TOK_API tok_status tok_patch_embed_pack_weights(const void *ws, void *wp, int64_t C, int64_t Cmid,
+                                                cudaStream_t stream);
+TOK_API tok_status tok_patch_embed_spatial(const void *x, const void *wp, void *y, int64_t B, int64_t C, int64_t T,
+                                           int64_t H, int64_t W, int64_t Cmid, cudaStream_t stream);
+
+/*
  * tok_fsq_encode -- fused 1x1 projection + FSQ quantization + index pack.
  * [guide] 7.2 (bound with tanh, rounding, levels [8,8,8,5,5,5], implicit
  * codebook of 64000, mixed-radix codes_to_indices), [guide] 6.2 (indices
@@ -378,8 +425,11 @@ TOK_API tok_status tok_fsq_encode_backward(const float *u, const float *w, const
  *     (concurrent streams, other host threads) race and must be serialized by
  *     the caller; a call overwrites whatever an earlier call left there;
  *   - the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) and caches it; make that first call before any
- *     stream capture.
+ *     (cudaGetSymbolAddress) and caches it for the life of the process; make
+ *     that first call before any stream capture, and do not reset the device
+ *     (cudaDeviceReset) between calls: a reset invalidates the cached address;
+ *   - the cache covers device ordinals 0 to 63: a call on a higher ordinal
+ *     returns TOK_ERR_TOO_LARGE before anything runs.
  * It allocates nothing.  Arguments, outputs and results are those of
  * tok_fsq_encode_backward.
  */

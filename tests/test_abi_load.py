@@ -57,6 +57,12 @@ def fwd(lib, x, y, dt, B, C, T, H, W):
     return lib.tok_haar_fwd(x, y, dt, B, C, T, H, W, NULL)
 
 
+def test_selftest_poll_range(lib):
+    # out-of-range poll counts are rejected before any launch
+    assert lib.tok_selftest_wait_timeout(0, NULL) == hwp.TOK_ERR_SHAPE
+    assert lib.tok_selftest_wait_timeout((1 << 22) + 1, NULL) == hwp.TOK_ERR_SHAPE
+
+
 def test_haar_shape_rules(lib):
     assert fwd(lib, A, Bp, 0, 1, 3, 3, 64, 64) == hwp.TOK_ERR_SHAPE    # T % 4 != 1
     assert fwd(lib, A, Bp, 0, 1, 3, 5, 62, 64) == hwp.TOK_ERR_SHAPE    # H % 4
@@ -218,3 +224,23 @@ def test_conv_rules(lib):
     assert sp(X, Wg, X, 1, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_ERR_ALIAS
     assert fz(X, Wg, Wg, M, X, 1, 2, 8, 8, 16, 16, 16, 3, NULL) == hwp.TOK_ERR_ALIAS
     assert sp(NULL, NULL, NULL, 0, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_OK     # empty
+
+
+def test_patch_embed_rules(lib):
+    pe, pk = lib.tok_patch_embed_spatial, lib.tok_patch_embed_pack_weights
+    X, Wp, Y = F(0x100000), F(0x800000), F(0x1000000)
+    assert pe(X, Wp, Y, 1, 3, 7, 64, 64, 256, NULL) == hwp.TOK_ERR_SHAPE    # T % 4 != 1
+    assert pe(X, Wp, Y, 1, 3, 1, 64, 64, 256, NULL) == hwp.TOK_ERR_SHAPE    # images: video only
+    assert pe(X, Wp, Y, 1, 3, 9, 64, 60, 256, NULL) == hwp.TOK_ERR_SHAPE    # W % 8 != 0
+    assert pe(X, Wp, Y, 1, 3, 9, 62, 64, 256, NULL) == hwp.TOK_ERR_SHAPE    # H % 4 != 0
+    assert pe(X, Wp, Y, 1, 3, 9, 64, 64, 48, NULL) == hwp.TOK_ERR_SHAPE     # Cmid not a multiple of 32
+    assert pe(X, Wp, Y, 1, 3, 9, 64, 64, 288, NULL) == hwp.TOK_ERR_SHAPE    # above 256, not a multiple of 256
+    assert pe(X, Wp, Y, 1, 9, 9, 64, 64, 256, NULL) == hwp.TOK_ERR_SHAPE    # C > 8
+    assert pe(NULL, Wp, Y, 1, 3, 9, 64, 64, 256, NULL) == hwp.TOK_ERR_NULL
+    assert pe(F(0x100008), Wp, Y, 1, 3, 9, 64, 64, 256, NULL) == hwp.TOK_ERR_ALIGN
+    assert pe(X, Wp, X, 1, 3, 9, 64, 64, 256, NULL) == hwp.TOK_ERR_ALIAS
+    assert pe(NULL, NULL, NULL, 0, 3, 9, 64, 64, 256, NULL) == hwp.TOK_OK      # empty
+    assert pk(X, Wp, 3, 48, NULL) == hwp.TOK_ERR_SHAPE
+    assert pk(NULL, Wp, 3, 256, NULL) == hwp.TOK_ERR_NULL
+    assert pk(X, F(0x800008), 3, 256, NULL) == hwp.TOK_ERR_ALIGN
+    assert pk(X, X, 3, 256, NULL) == hwp.TOK_ERR_ALIAS

@@ -13,7 +13,6 @@ Tolerances, from the arithmetic of the kernels:
   FSQ decode backward: grad_codes is a C-term fp32 chain: <= 20 * 2^-24 * sum_c |w_ic| |g_c|;
     grad_w: <= 1e-5 * sum_tokens |g_c| (|zhat| <= 1).
 """
-import math
 
 import numpy as np
 import pytest
@@ -22,7 +21,7 @@ import torch
 import haar_wavelet_patching_b200 as hwp
 import oracle
 import synth
-from tests.helpers import U, expand_blocks_to_pixels, expand_to_channels, ulp_bf16
+from tests.helpers import U, check_bf16, expand_blocks_to_pixels, expand_to_channels
 
 pytestmark = pytest.mark.gpu
 
@@ -59,8 +58,7 @@ def test_haar_adjoints_match_oracle(shape, dtype):
     else:
         # coefficient-block sums |gy| per block, for the pixel-side result
         a = np.abs(gy64).reshape(B, 64, C, *gy64.shape[2:]).sum(axis=1)
-        bound_x = ulp_bf16(ref_x) + 36 * U * expand_blocks_to_pixels(a, T) / 8 * 1.01
-        assert (np.abs(got_x - ref_x) <= bound_x).all()
+        check_bf16(got_x, ref_x, 36 * U * expand_blocks_to_pixels(a, T) / 8 * 1.01, "patcher adjoint")
         # pixel-block sums |gx| per block, for the coefficient-side result (window 0 reads one frame)
         ax = np.abs(gx64)
         sp = ax.reshape(B, C, T, H // 4, 4, W // 4, 4).sum(axis=(4, 6))
@@ -68,8 +66,7 @@ def test_haar_adjoints_match_oracle(shape, dtype):
         blk = np.empty((B, C, Tq) + sp.shape[3:])
         blk[:, :, 0] = sp[:, :, 0]
         blk[:, :, 1:] = sp[:, :, 1:].reshape(B, C, Tq - 1, 4, *sp.shape[3:]).sum(axis=3)
-        bound_y = ulp_bf16(ref_y) + 6 * U * expand_to_channels(blk, 64) / 8 * 1.01
-        assert (np.abs(got_y - ref_y) <= bound_y).all()
+        check_bf16(got_y, ref_y, 6 * U * expand_to_channels(blk, 64) / 8 * 1.01, "unpatcher adjoint")
 
 
 def test_haar_adjoint_dot_product_on_gpu():

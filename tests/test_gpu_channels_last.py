@@ -9,7 +9,7 @@ import torch
 import haar_wavelet_patching_b200 as hwp
 import oracle
 import synth
-from tests.helpers import block_abs_sums, expand_to_channels, haar_bf16_tolerance, to_device, to_f64
+from tests.helpers import block_abs_sums, check_bf16, expand_to_channels, haar_fp32_bound, to_device, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -50,9 +50,9 @@ def test_channels_last_matches_oracle(shape):
     x64 = synth.to_f64(x_np, synth.BF16)
     got = to_f64(hwp.haar_fwd_channels_last(to_device(x_np, synth.BF16)))
     ref = oracle.haar_fwd_channels_last(x64)
-    tol = np.moveaxis(haar_bf16_tolerance(oracle.haar_fwd(x64), expand_to_channels(block_abs_sums(x64), 64), True),
-                      1, -1)
-    assert got.shape == ref.shape and (np.abs(got - ref) <= tol).all()
+    E = np.moveaxis(haar_fp32_bound(expand_to_channels(block_abs_sums(x64), 64), True), 1, -1)
+    assert got.shape == ref.shape
+    check_bf16(got, ref, E, "channels-last")
 
 
 @pytest.mark.parametrize("shape,dtype", [((1, 3, 9, 16, 76), torch.bfloat16), ((2, 2, 1, 12, 36), torch.bfloat16),

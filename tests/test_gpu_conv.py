@@ -14,7 +14,7 @@ import haar_wavelet_patching_b200 as hwp
 import oracle
 import synth
 from oracle import conv as oconv
-from tests.helpers import U, to_device, ulp_bf16
+from tests.helpers import U, check_bf16, to_device, ulp_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -37,9 +37,7 @@ def test_spatial_matches_oracle(shape, Cout):
     hwp.tok_conv_spatial(to_device(x, synth.BF16), to_device(ws, synth.BF16), y)
     hwp.tok_check_device()
     ref = oconv.spatial_conv(x64, ws64)
-    tol = ulp_bf16(ref) + 2 * 9 * Cin * U * oconv.spatial_conv(np.abs(x64), np.abs(ws64))
-    err = np.abs(as_f64(y) - ref)
-    assert (err <= tol).all(), f"{(err > tol).sum()} outputs beyond tolerance, worst {(err / tol).max():.3g}"
+    check_bf16(as_f64(y), ref, 2 * 9 * Cin * U * oconv.spatial_conv(np.abs(x64), np.abs(ws64)), "spatial")
 
 
 @pytest.mark.parametrize("shape,Cout", [((2, 7, 6, 10, 64), 128), ((1, 4, 16, 16, 256), 256), ((1, 1, 4, 4, 64), 64)])
@@ -51,19 +49,20 @@ def test_temporal_causal_matches_oracle(shape, Cout):
     hwp.tok_conv_temporal_causal(to_device(x, synth.BF16), to_device(wt, synth.BF16), y)
     hwp.tok_check_device()
     ref = oconv.temporal_causal_conv(x64, wt64)
-    tol = ulp_bf16(ref) + 2 * 3 * Cin * U * oconv.temporal_causal_conv(np.abs(x64), np.abs(wt64))
-    err = np.abs(as_f64(y) - ref)
-    assert (err <= tol).all(), f"{(err > tol).sum()} outputs beyond tolerance"
+    check_bf16(as_f64(y), ref, 2 * 3 * Cin * U * oconv.temporal_causal_conv(np.abs(x64), np.abs(wt64)), "temporal")
 
 
 def factorized_tolerance(x64, ws64, wt64):
+    """The oracle chain and the fp32 error of the kernels' value before the final bf16 rounding:
+    the temporal layer's accumulation plus the intermediate's own error (its bf16 rounding and
+    accumulation bound) carried through the temporal weights."""
     Cin, Cmid = x64.shape[-1], ws64.shape[0]
     s = oconv.spatial_conv(x64, ws64)
     s_err = ulp_bf16(s) + 2 * 9 * Cin * U * oconv.spatial_conv(np.abs(x64), np.abs(ws64))
     ref = oconv.temporal_causal_conv(oconv.round_bf16(s), wt64)
-    tol = (ulp_bf16(ref) + 2 * 3 * Cmid * U * oconv.temporal_causal_conv(np.abs(s), np.abs(wt64))
-           + oconv.temporal_causal_conv(s_err, np.abs(wt64)))
-    return ref, tol
+    E = (2 * 3 * Cmid * U * oconv.temporal_causal_conv(np.abs(s), np.abs(wt64))
+         + oconv.temporal_causal_conv(s_err, np.abs(wt64)))
+    return ref, E
 
 
 def test_factorized_matches_oracle():
@@ -73,9 +72,8 @@ def test_factorized_matches_oracle():
     wt, wt64 = bf16_input((Cout, 3, Cmid), seed=131, std=(3 * Cmid) ** -0.5)
     y = hwp.conv_factorized(to_device(x, synth.BF16), to_device(ws, synth.BF16), to_device(wt, synth.BF16))
     hwp.tok_check_device()
-    ref, tol = factorized_tolerance(x64, ws64, wt64)
-    err = np.abs(as_f64(y) - ref)
-    assert (err <= tol).all(), f"{(err > tol).sum()} outputs beyond tolerance"
+    ref, E = factorized_tolerance(x64, ws64, wt64)
+    check_bf16(as_f64(y), ref, E, "factorized")
 
 
 def test_patcher_then_convolution():
@@ -99,8 +97,89 @@ def test_patcher_then_convolution():
     bs[:, :, 0] = 4 * blocks[:, :, 0]
     bs[:, :, 1:] = blocks[:, :, 1:].reshape(B, C, Tq - 1, 4, H // 4, W // 4).sum(axis=3)
     c_err = 2 * ulp_bf16(coeff) + 6 * U * np.moveaxis(np.concatenate([bs] * 64, axis=1), 1, -1) / 8 * 1.01
-    ref, tol = factorized_tolerance(coeff, ws64, wt64)
+    ref, E = factorized_tolerance(coeff, ws64, wt64)
     carried = oconv.temporal_causal_conv(oconv.spatial_conv(c_err, np.abs(ws64)), np.abs(wt64))
-    tol = tol + carried
-    err = np.abs(as_f64(out) - ref)
-    assert (err <= tol).all(), f"{(err > tol).sum()} outputs beyond tolerance"
+    check_bf16(as_f64(out), ref, E + carried, "patcher -> factorized")
+
+
+# ---------------------------------------------------------------------------
+# The hand-written tensor-core kernels: more tile shapes, several output-channel tiles, k = 5.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("shape,Cout,k", [((1, 3, 20, 24, 128), 512, 3), ((2, 2, 17, 9, 64), 96, 3),
+                                          ((1, 2, 12, 16, 64), 32, 5)],
+                         ids=["two channel tiles", "ragged tiles", "k=5"])
+def test_spatial_tile_shapes(shape, Cout, k):
+    B, T, h, w, Cin = shape
+    x, x64 = bf16_input(shape, seed=151)
+    ws, ws64 = bf16_input((Cout, k, k, Cin), seed=157, std=(k * k * Cin) ** -0.5)
+    y = torch.empty((B, T, h, w, Cout), dtype=torch.bfloat16, device="cuda")
+    hwp.tok_conv_spatial(to_device(x, synth.BF16), to_device(ws, synth.BF16), y)
+    hwp.tok_check_device()
+    ref = oconv.spatial_conv(x64, ws64)
+    check_bf16(as_f64(y), ref, 2 * k * k * Cin * U * oconv.spatial_conv(np.abs(x64), np.abs(ws64)), "spatial")
+
+
+@pytest.mark.parametrize("shape,Cout,k", [((2, 5, 17, 9, 64), 96, 3), ((1, 6, 8, 8, 128), 512, 3),
+                                          ((2, 7, 4, 12, 64), 64, 5)],
+                         ids=["ragged tiles, two clips", "two channel tiles", "k=5"])
+def test_temporal_tile_shapes(shape, Cout, k):
+    B, T, h, w, Cin = shape
+    x, x64 = bf16_input(shape, seed=163)
+    wt, wt64 = bf16_input((Cout, k, Cin), seed=167, std=(k * Cin) ** -0.5)
+    y = torch.empty((B, T, h, w, Cout), dtype=torch.bfloat16, device="cuda")
+    hwp.tok_conv_temporal_causal(to_device(x, synth.BF16), to_device(wt, synth.BF16), y)
+    hwp.tok_check_device()
+    ref = oconv.temporal_causal_conv(x64, wt64)
+    check_bf16(as_f64(y), ref, 2 * k * Cin * U * oconv.temporal_causal_conv(np.abs(x64), np.abs(wt64)), "temporal")
+
+
+# ---------------------------------------------------------------------------
+# The patcher fused into the spatial convolution.
+# ---------------------------------------------------------------------------
+def patcher_coeff_error(xp64, coeff):
+    """Per coefficient: how far the kernel's bf16 coefficient may be from the oracle's coefficient
+    rounded to bf16 -- two bf16 ulps plus the 6-stage butterfly bound of its block's 64 pixels."""
+    B, C, T, H, W = xp64.shape
+    blocks = np.abs(xp64).reshape(B, C, T, H // 4, 4, W // 4, 4).sum(axis=(4, 6))
+    Tq = 1 + (T - 1) // 4
+    bs = np.empty((B, C, Tq, H // 4, W // 4))
+    bs[:, :, 0] = 4 * blocks[:, :, 0]
+    bs[:, :, 1:] = blocks[:, :, 1:].reshape(B, C, Tq - 1, 4, H // 4, W // 4).sum(axis=3)
+    return 2 * ulp_bf16(coeff) + 6 * U * np.moveaxis(np.concatenate([bs] * 64, axis=1), 1, -1) / 8 * 1.01
+
+
+EMBED = [((1, 3, 9, 64, 64), 256, "three colours, whole tiles"),
+         ((2, 2, 13, 36, 72), 64, "ragged tiles, two clips"),
+         ((1, 1, 5, 16, 32), 512, "two channel tiles"),
+         ((1, 4, 5, 68, 40), 128, "four colours, ragged rows")]
+
+
+@pytest.mark.parametrize("shape,Cmid,note", EMBED, ids=[e[2] for e in EMBED])
+def test_patch_embed_matches_oracle_chain(shape, Cmid, note):
+    """Pixels -> fused patcher + 1x3x3 convolution, against the oracle patcher (rounded to bf16, as the
+    kernel rounds its coefficients) and the oracle convolution.  The kernel's coefficients may differ
+    from the oracle's rounded ones by patcher_coeff_error, carried through the filter."""
+    B, C, T, H, W = shape
+    xp = synth.uniform(shape, seed=173 + C, dtype=synth.BF16)
+    xp64 = synth.to_f64(xp, synth.BF16)
+    Cin = 64 * C
+    ws, ws64 = bf16_input((Cmid, 3, 3, Cin), seed=179, std=(9 * Cin) ** -0.5)
+    wp = hwp.patch_embed_pack_weights(to_device(ws, synth.BF16))
+    y = hwp.patch_embed_spatial(to_device(xp, synth.BF16), wp)
+    hwp.tok_check_device()
+    coeff = oconv.round_bf16(oracle.haar_fwd_channels_last(xp64))
+    ref = oconv.spatial_conv(coeff, ws64)
+    E = (2 * 9 * Cin * U * oconv.spatial_conv(np.abs(coeff), np.abs(ws64))
+         + oconv.spatial_conv(patcher_coeff_error(xp64, coeff), np.abs(ws64)))
+    strict = check_bf16(as_f64(y), ref, E, note)
+    print(f"{note}: {strict} of {y.numel()} outputs beyond a plain 1 bf16 ulp")
+
+
+def test_packed_filter_layout():
+    """wp[n][(c*3 + dx)*3 + dy][g] = ws[n][dy][dx][g*C + c], bit for bit."""
+    C, Cmid = 3, 64
+    ws = torch.randn((Cmid, 3, 3, 64 * C), device="cuda").to(torch.bfloat16)
+    wp = hwp.patch_embed_pack_weights(ws)
+    torch.cuda.synchronize()
+    ref = ws.view(Cmid, 3, 3, 64, C).permute(0, 4, 2, 1, 3).reshape(Cmid, 9 * C, 64)
+    assert torch.equal(wp, ref)

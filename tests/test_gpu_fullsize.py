@@ -14,7 +14,7 @@ import haar_wavelet_patching_b200 as hwp
 import oracle
 import synth
 from oracle import conv as oconv
-from tests.helpers import U, haar_bf16_tolerance, to_device, ulp_bf16
+from tests.helpers import U, check_bf16, haar_fp32_bound, to_device, ulp_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -92,9 +92,53 @@ def test_conv_chain_full_size_sampled(clip):
             ref += wt64[:, dt, :] @ sb[f - a]
             t_abs += np.abs(wt64[:, dt, :]) @ np.abs(sb[f - a])
             carried += np.abs(wt64[:, dt, :]) @ s_err[f - a]
-        tol = ulp_bf16(ref) + 2 * 3 * Cmid * U * t_abs + carried
         got = out[0, t, i, j].double().cpu().numpy()
-        assert (np.abs(got - ref) <= tol).all(), f"sample {(t, i, j)}: {(np.abs(got - ref) > tol).sum()} channels"
+        check_bf16(got, ref, 2 * 3 * Cmid * U * t_abs + carried, f"sample {(t, i, j)}")
+
+
+def test_patch_embed_full_size(clip):
+    """Headline clip through the fused patcher + 1x3x3 convolution (bench.py patch_embed_fused):
+    every output against the two-call chain (channels-last patcher, then tok_conv_spatial) -- the
+    same bf16 coefficients summed in another order, so each pair differs by at most two fp32
+    accumulation bounds plus the bf16 rounding -- and sampled outputs against the oracle chain."""
+    import torch.nn.functional as F
+    x, xd = clip
+    Cin, Cmid = 192, 256
+    ws = synth.normal((Cmid, 3, 3, Cin), seed=211, std=(9 * Cin) ** -0.5, dtype=synth.BF16)
+    ws64 = synth.to_f64(ws, synth.BF16)
+    wsd = to_device(ws, synth.BF16)
+    y = hwp.patch_embed_spatial(xd, hwp.patch_embed_pack_weights(wsd))
+    y_cl = hwp.haar_fwd_channels_last(xd)
+    mid = torch.empty_like(y)
+    hwp.tok_conv_spatial(y_cl, wsd, mid)
+    hwp.tok_check_device()
+    _, Tq, h, w, _ = y_cl.shape
+    with torch.backends.cudnn.flags(enabled=True, allow_tf32=False):
+        a = y_cl[0].float().abs().permute(0, 3, 1, 2)                        # [Tq, Cin, h, w]
+        S = F.conv2d(a, wsd.float().abs().permute(0, 3, 1, 2), padding=1)     # sum |c| |w| per output
+    E = (2 * 2 * 9 * Cin * U * 1.01) * S.permute(0, 2, 3, 1).double()
+    m = mid[0].double()
+    tol = torch.maximum(torch.ldexp(torch.ones_like(m), torch.frexp((m.abs() + E).clamp(min=2.0 ** -126))[1] - 8),
+                        torch.zeros_like(m)) + E
+    bad = int(((y[0].double() - m).abs() > tol).sum())
+    assert bad == 0, f"{bad} fused outputs differ from the two-call chain beyond the accumulation bounds"
+    del a, S, E, m, tol
+    for (t, i, j) in SAMPLES:
+        i0, i1, j0, j1 = max(0, i - 1), min(h, i + 2), max(0, j - 1), min(w, j + 2)
+        if t == 0:
+            crop = pixels(x, 0, 1, 4 * i0, 4 * i1, 4 * j0, 4 * j1)
+            cf = oracle.haar_fwd_chunk(crop, first=True)
+        else:
+            crop = pixels(x, 4 * t - 3, 4 * t + 1, 4 * i0, 4 * i1, 4 * j0, 4 * j1)
+            cf = oracle.haar_fwd_chunk(crop, first=False)
+        cb = oconv.round_bf16(np.moveaxis(cf, 1, -1))                      # [1, 1, nh, nw, 192]
+        blk = np.abs(crop).reshape(1, 3, crop.shape[2], i1 - i0, 4, j1 - j0, 4).sum(axis=(4, 6))
+        bs = 4 * blk if t == 0 else blk.reshape(1, 3, 1, 4, i1 - i0, j1 - j0).sum(axis=3)
+        c_err = 2 * ulp_bf16(cb) + 6 * U * np.moveaxis(np.concatenate([bs] * 64, axis=1), 1, -1) / 8 * 1.01
+        ref = oconv.spatial_conv(cb, ws64)[0, 0, i - i0, j - j0]
+        E = (2 * 9 * Cin * U * oconv.spatial_conv(np.abs(cb), np.abs(ws64))[0, 0, i - i0, j - j0]
+             + oconv.spatial_conv(c_err, np.abs(ws64))[0, 0, i - i0, j - j0])
+        check_bf16(y[0, t, i, j].double().cpu().numpy(), ref, E, f"fused sample {(t, i, j)}")
 
 
 def test_padded_and_chunk_full_size_sampled():
@@ -114,12 +158,12 @@ def test_padded_and_chunk_full_size_sampled():
         bsum = np.abs(pixels(x, 0, 1, 4 * i, 4 * i + 4, 4 * j, 4 * j + 4)).sum() * 4 if tq == 0 else \
             sum(np.abs(pixels(x, f, f + 1, 4 * i, 4 * i + 4, 4 * j, 4 * j + 4)).sum()
                 for f in (frames or range(4 * tq - 3, 4 * tq + 1)))
-        assert (np.abs(got - ref) <= haar_bf16_tolerance(ref, bsum, True)).all(), f"padded window {(tq, i, j)}"
+        check_bf16(got, ref, haar_fp32_bound(bsum, True), f"padded window {(tq, i, j)}")
         if tq < 30:  # continuation window q reads frames 4q .. 4q + 3
             refc = window_coeffs(x, 0, i, j, list(range(4 * tq, 4 * tq + 4)))[0]
             gotc = yc[0, :, tq, i, j].double().cpu().numpy()
             bs = sum(np.abs(pixels(x, f, f + 1, 4 * i, 4 * i + 4, 4 * j, 4 * j + 4)).sum() for f in range(4 * tq, 4 * tq + 4))
-            assert (np.abs(gotc - refc) <= haar_bf16_tolerance(refc, bs, True)).all(), f"chunk window {(tq, i, j)}"
+            check_bf16(gotc, refc, haar_fp32_bound(bs, True), f"chunk window {(tq, i, j)}")
     # the cropped inverse: the last window rebuilds frames 117..119 (its fourth sample is cropped)
     xr = hwp.haar_inv_cropped(yp, 120, 720, 1280, 16, 8)
     hwp.tok_check_device()
@@ -128,8 +172,7 @@ def test_padded_and_chunk_full_size_sampled():
         ref = oracle.haar_inv_chunk(coef, 4, 4, 4, first=False)[0, :, :3]
         got = xr[0, :, 117:120, 4 * i:4 * i + 4, 4 * j:4 * j + 4].double().cpu().numpy()
         per_c = np.abs(coef).reshape(64, 3).sum(axis=0)[:, None, None, None]  # channel c's 64 coefficients
-        tol = haar_bf16_tolerance(ref, per_c, True)
-        assert (np.abs(got - ref) <= tol).all(), f"cropped inverse block {(i, j)}"
+        check_bf16(got, ref, haar_fp32_bound(per_c, True), f"cropped inverse block {(i, j)}")
 
 
 def test_single_level_full_size_sampled(clip):
@@ -143,8 +186,7 @@ def test_single_level_full_size_sampled(clip):
         ref = oracle.haar_level_fwd(crop)[:, 0 if tq == 0 else 1, 0, 0]
         got = y1[0, :, tq, i, j].double().cpu().numpy()
         s = np.abs(crop[:, [0, 0]] if tq == 0 else crop[:, 1:]).sum(axis=(1, 2, 3))
-        tol = ulp_bf16(ref) + 5 * U * np.tile(s, 8) * 2 ** -1.5 * 1.01
-        assert (np.abs(got - ref) <= tol).all(), f"single-level window {(tq, i, j)}"
+        check_bf16(got, ref, 5 * U * np.tile(s, 8) * 2 ** -1.5 * 1.01, f"single-level window {(tq, i, j)}")
 
 
 def test_adjoints_full_size_sampled():
@@ -167,8 +209,8 @@ def test_adjoints_full_size_sampled():
             ref = oracle.haar_inv_chunk(cw, 4, 4, 4, first=False)[0]
             got = gx[0, :, 4 * tq - 3:4 * tq + 1, 4 * i:4 * i + 4, 4 * j:4 * j + 4].double().cpu().numpy()
             d = 6
-        tol = ulp_bf16(ref) + d * U * np.abs(cw).reshape(64, 3).sum(axis=0)[:, None, None, None] / 8 * 1.01
-        assert (np.abs(got - ref) <= tol).all(), f"patcher adjoint window {(tq, i, j)}"
+        check_bf16(got, ref, d * U * np.abs(cw).reshape(64, 3).sum(axis=0)[:, None, None, None] / 8 * 1.01,
+                   f"patcher adjoint window {(tq, i, j)}")
         # the unpatcher's adjoint: window tq >= 1 is the forward transform of its 4 frames; window 0 sees
         # (0, 0, 0, frame 0)
         px = g2[:, :, max(0, 4 * tq - 3):4 * tq + 1, 4 * i:4 * i + 4, 4 * j:4 * j + 4].double().cpu().numpy()
@@ -181,7 +223,7 @@ def test_adjoints_full_size_sampled():
             ref = oracle.haar_fwd_chunk(px, first=False)[0, :, 0, 0, 0]
             s = np.tile(np.abs(px[0]).sum(axis=(1, 2, 3)), 64)
         got = gyy[0, :, tq, i, j].double().cpu().numpy()
-        assert (np.abs(got - ref) <= ulp_bf16(ref) + 6 * U * s / 8 * 1.01).all(), f"unpatcher adjoint {(tq, i, j)}"
+        check_bf16(got, ref, 6 * U * s / 8 * 1.01, f"unpatcher adjoint {(tq, i, j)}")
 
 
 def test_fsq_backward_full_latent():
@@ -226,7 +268,7 @@ def test_image_beyond_the_tile_kernels_limits():
     blocks = np.stack([x[0, 0, 0, 4 * i:4 * i + 4, 4 * j:4 * j + 4].double().cpu().numpy() for i, j in pos])
     ref = oracle.haar_fwd(blocks[:, None, None])  # [n, 16, 1, 1, 1]
     got = np.stack([y[0, :, 0, i, j].double().cpu().numpy() for i, j in pos])
-    tol = haar_bf16_tolerance(ref[:, :, 0, 0, 0], np.abs(blocks).sum(axis=(1, 2))[:, None], False)
-    assert (np.abs(got - ref[:, :, 0, 0, 0]) <= tol).all()
+    check_bf16(got, ref[:, :, 0, 0, 0], haar_fp32_bound(np.abs(blocks).sum(axis=(1, 2))[:, None], False),
+               "32768x32768 image")
     del x, y, xr
     torch.cuda.empty_cache()
