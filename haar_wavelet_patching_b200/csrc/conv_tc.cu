@@ -6,27 +6,33 @@
 // convolutions are factorized -- a 1 x k x k spatial convolution, then a k x 1 x 1
 // temporal convolution padded by k - 1 on the past side only.
 //
-// Activations are channels-last bf16 [frames, h, w, C]; fp32 accumulation.  A CTA
-// owns one SM and walks its tiles persistently.  A tile is 128 output positions --
-// 16 rows x 8 columns of one frame -- by up to 256 output channels: the MMA is
-// M = 128, N = 256, and each K step is 64 input channels of one tap.  Warp roles:
+// Activations are channels-last bf16 [frames, h, w, C]; fp32 accumulation.  The
+// MMA is the 2-SM form: a CTA pair (a 2 x 1 x 1 cluster, one CTA per SM) computes
+// 256 output positions -- two tiles of 16 rows x 8 columns of one frame, one per
+// CTA -- by up to 256 output channels, M = 256 and N = 256, each CTA loading its own
+// tile's activations and half of the filter, so the filter crosses L2 half as often
+// per flop as with one-CTA 128 x 256 tiles.  Each K step is 64 input channels of one
+// tap.  The pair walks its tiles persistently.  Warp roles in each CTA:
 //   warp 0     tensor copies: per K step, the activation box [64 ch, 8 cols,
 //              16 rows] of the tap's frame / shift (zero-filled outside the frame)
-//              and the filter box [64 k, N] into one of kStages stages, both in the
-//              128-byte swizzle the MMA reads;
-//   warp 1     one thread issues tcgen05.mma (4 per K step, K = 16 each) into a
-//              tensor-memory accumulator and commits each stage back to warp 0;
+//              and its half of the filter box [64 k, N / 2], into one of kStages
+//              stages in the 128-byte swizzle the MMA reads; completion is counted
+//              on the leader CTA's barrier;
+//   warp 1     (leader only) one thread issues tcgen05.mma (4 per K step, K = 16
+//              each) into the pair's tensor-memory accumulator and commits each stage
+//              back to both CTAs' copy warps;
 //   warps 2-5  epilogue: tensor memory -> registers (each thread one position, its
-//              lane of the accumulator), round to bf16, 16-byte stores.
+//              lane of this CTA's accumulator half), round to bf16, 16-byte stores.
 // Two accumulators in tensor memory (2 x N columns) let a tile's epilogue overlap
 // the next tile's MMAs.  The temporal convolution orders tiles time-fastest, so the
 // k frames a tile reads are read again by the next tiles while they are in L2; the
-// spatial one orders them column-block-fastest for the halo rows.
+// spatial one orders them column-block-fastest for the halo rows.  No load is
+// broadcast to the pair: every copy fills only its own CTA's shared memory.
 //
 // Waits are bounded: a barrier that does not complete in time raises the CTA's
 // abort flag, every role leaves its loop, the copies and MMAs already issued are
 // waited for (bounded), tensor memory is freed and a timeout is counted for
-// tok_check_device().  No load is broadcast to a cluster.
+// tok_check_device().
 #include <algorithm>
 #include <cstring>
 
@@ -41,11 +47,12 @@ static __device__ unsigned int g_conv_timeouts = 0;
 
 namespace {
 
-constexpr int kTileRows = 16, kTileCols = 8, kBM = kTileRows * kTileCols; // positions per tile
+constexpr int kTileRows = 16, kTileCols = 8, kBM = kTileRows * kTileCols; // positions per CTA tile
 constexpr int kBK = 64;                                                   // K per stage: one 128-byte row
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kThreads = 192; // 6 warps
 constexpr uint32_t kABytes = kBM * kBK * 2;
+constexpr uint16_t kPairMask = 0x3; // both CTAs of the pair
 
 struct ConvGeom {
     int frames;   // B * T
@@ -53,10 +60,11 @@ struct ConvGeom {
     int h, w;
     int cin;      // input channels (multiple of 64)
     int n;        // output channels
-    int bn;       // output channels per tile
+    int bn;       // output channels per pair tile (each CTA loads bn / 2 filter rows)
     int n_tiles;  // n / bn
-    int tiles_x, tiles_y;
-    int ntiles;
+    int tiles_xp; // column-block pairs
+    int tiles_y;
+    int npairs;   // pair tiles
     int k;        // taps per axis
     int temporal; // 1: causal temporal (k x 1 x 1), 0: spatial (1 x k x k, 'same' zeros)
 };
@@ -69,18 +77,19 @@ struct TileCoord {
     int nkb; // K steps of this tile
 };
 
-__device__ __forceinline__ TileCoord decode_tile(const ConvGeom &g, int i)
+// Pair tile i, this CTA's half (rank): column block 2 * xp + rank.
+__device__ __forceinline__ TileCoord decode_tile(const ConvGeom &g, int i, uint32_t rank)
 {
     TileCoord c;
     const int nchunk = g.cin / kBK;
-    int r = i, xb, yb, nb;
+    int r = i, xp, yb, nb;
     if (g.temporal) { // time fastest: the k frames a tile reads are read by the next tiles too
         c.t = r % g.T;
         r /= g.T;
         nb = r % g.n_tiles;
         r /= g.n_tiles;
-        xb = r % g.tiles_x;
-        r /= g.tiles_x;
+        xp = r % g.tiles_xp;
+        r /= g.tiles_xp;
         yb = r % g.tiles_y;
         const int b = r / g.tiles_y;
         c.f = b * g.T + c.t;
@@ -90,8 +99,8 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvGeom &g, int i)
     } else { // output-channel tiles fastest (they share the activations), then column blocks
         nb = r % g.n_tiles;
         r /= g.n_tiles;
-        xb = r % g.tiles_x;
-        r /= g.tiles_x;
+        xp = r % g.tiles_xp;
+        r /= g.tiles_xp;
         yb = r % g.tiles_y;
         c.f = r / g.tiles_y;
         c.t = 0;
@@ -99,24 +108,86 @@ __device__ __forceinline__ TileCoord decode_tile(const ConvGeom &g, int i)
         c.nkb = g.k * g.k * nchunk;
     }
     c.y0 = yb * kTileRows;
-    c.x0 = xb * kTileCols;
+    c.x0 = (2 * xp + (int)rank) * kTileCols;
     c.n0 = nb * g.bn;
     return c;
 }
 
+__device__ __forceinline__ uint32_t tmem_cols(int bn)
+{
+    return bn <= 16 ? 32u : bn <= 32 ? 64u : bn <= 64 ? 128u : bn <= 128 ? 256u : 512u;
+}
+
+constexpr uint32_t kEpiBytes = 4 * 2 * 4096; // per CTA: 4 epilogue warps x 2 staging buffers of 4 KB
+
+// Epilogue of one CTA's tile; warp q = warp % 4 holds accumulator lanes 32q .. 32q + 31,
+// the tile's rows 4q .. 4q + 3.  Per 64 output channels: tensor memory -> registers ->
+// bf16 rows of a 128-byte-swizzled staging buffer of the warp (two, alternating) -> one
+// tensor store of the box [64 ch, 8 cols, 4 rows] at (n0 + cb, x0, y0 + 4q, f); the store
+// clips positions outside the frame and writes whole lines.  A last group of 32 channels
+// (bn % 64 == 32) is stored from registers, positions outside the frame skipped.
+__device__ __forceinline__ void store_tile(uint32_t tmem_acc, int q, int lane, const CUtensorMap *omap, int f, int y0,
+                                           int x0, int n0, uint32_t stage, unsigned char *stage_ptr, uint32_t &sbuf,
+                                           __nv_bfloat16 *o, bool valid, int bn)
+{
+    const uint32_t t0 = tmem_acc + ((uint32_t)(32 * q) << 16);
+    int cb = 0;
+    for (; cb + 64 <= bn; cb += 64) {
+        uint32_t v[64];
+        tmem_ld64(t0 + (uint32_t)cb, v);
+        tmem_wait_ld();
+        const uint32_t b = sbuf & 1u;
+        if (lane == 0)
+            bulk_wait_read<1>(); // the store that used this buffer two chunks ago has read it
+        __syncwarp();
+        unsigned char *buf = stage_ptr + b * 4096u;
+#pragma unroll
+        for (int s8 = 0; s8 < 8; ++s8)
+            *reinterpret_cast<uint4 *>(buf + sw128_offset((uint32_t)lane, 8u * s8)) =
+                make_uint4(pack_bf16x2(__uint_as_float(v[8 * s8 + 0]), __uint_as_float(v[8 * s8 + 1])),
+                           pack_bf16x2(__uint_as_float(v[8 * s8 + 2]), __uint_as_float(v[8 * s8 + 3])),
+                           pack_bf16x2(__uint_as_float(v[8 * s8 + 4]), __uint_as_float(v[8 * s8 + 5])),
+                           pack_bf16x2(__uint_as_float(v[8 * s8 + 6]), __uint_as_float(v[8 * s8 + 7])));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+            tma_store_4d(omap, n0 + cb, x0, y0 + 4 * q, f, stage + b * 4096u);
+            bulk_commit();
+        }
+        ++sbuf;
+    }
+    if (cb < bn) {
+        uint32_t v[32];
+        tmem_ld32(t0 + (uint32_t)cb, v);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                *reinterpret_cast<uint4 *>(o + cb + 8 * s) =
+                    make_uint4(pack_bf16x2(__uint_as_float(v[8 * s + 0]), __uint_as_float(v[8 * s + 1])),
+                               pack_bf16x2(__uint_as_float(v[8 * s + 2]), __uint_as_float(v[8 * s + 3])),
+                               pack_bf16x2(__uint_as_float(v[8 * s + 4]), __uint_as_float(v[8 * s + 5])),
+                               pack_bf16x2(__uint_as_float(v[8 * s + 6]), __uint_as_float(v[8 * s + 7])));
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-               __nv_bfloat16 *__restrict__ out, const ConvGeom g)
+               const __grid_constant__ CUtensorMap omap, __nv_bfloat16 *__restrict__ out, const ConvGeom g)
 {
     __shared__ __align__(8) uint64_t full[kStages], empty[kStages], accf[2], acce[2], drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-    const uint32_t bbytes = (uint32_t)g.bn * kBK * 2;
+    const uint32_t bbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of the filter tile
     const uint32_t stage_bytes = kABytes + bbytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t ncols = g.bn <= 16 ? 32u : g.bn <= 32 ? 64u : g.bn <= 64 ? 128u : g.bn <= 128 ? 256u : 512u;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const uint32_t ncols = tmem_cols(g.bn);
+    const int pair = blockIdx.x >> 1, npair_ctas = gridDim.x >> 1;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -125,57 +196,59 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_addr(&accf[a]), 1);
-            mbar_init(smem_addr(&acce[a]), 4);
+            mbar_init(smem_addr(&acce[a]), 8); // 4 epilogue warps in each CTA
         }
         mbar_init(smem_addr(&drain), 1);
         abort_s = 0;
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_addr(&tmem_base_s), ncols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_addr(&tmem_base_s), ncols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync(); // both CTAs' barriers exist before any copy or arrive reaches them
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
     volatile int *abort = &abort_s;
     const int nchunk = g.cin / kBK;
 
     if (warp == 0 && lane == 0) {
-        // Tensor copies.
+        // Tensor copies of this CTA's operands; completion counted on the leader's barrier.
         uint32_t it = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x) {
-            const TileCoord c = decode_tile(g, i);
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
+            const TileCoord c = decode_tile(g, i, rank);
             for (int kb = 0; kb < c.nkb; ++kb, ++it) {
                 const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
                 if (!wait_or_abort(smem_addr(&empty[s]), ph ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes, fb = smem_addr(&full[s]);
+                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes;
+                const uint32_t fb = mapa_shared(smem_addr(&full[s]), 0);
                 const int kk = c.kb0 + kb, tap = kk / nchunk, ch = (kk - tap * nchunk) * kBK;
-                mbar_expect_tx(fb, stage_bytes);
+                if (leader)
+                    mbar_expect_tx(smem_addr(&full[s]), 2 * stage_bytes);
                 if (g.temporal)
-                    tma_load_4d(sa, &amap, ch, c.x0, c.y0, c.f - (g.k - 1) + tap, fb);
+                    tma_load_4d_pair(sa, &amap, ch, c.x0, c.y0, c.f - (g.k - 1) + tap, fb);
                 else {
                     const int pad = (g.k - 1) / 2, dy = tap / g.k, dx = tap - dy * g.k;
-                    tma_load_4d(sa, &amap, ch, c.x0 + dx - pad, c.y0 + dy - pad, c.f, fb);
+                    tma_load_4d_pair(sa, &amap, ch, c.x0 + dx - pad, c.y0 + dy - pad, c.f, fb);
                 }
-                tma_load_2d(sb, &bmap, kk * kBK, c.n0, fb);
+                tma_load_2d_pair(sb, &bmap, kk * kBK, c.n0 + (int)rank * (g.bn / 2), fb);
             }
         }
-        if (!ok) // let the copies already issued land before the CTA exits (each wait bounded)
+        if (!ok && leader) // let the copies already issued land before the CTA exits (each wait bounded)
             for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
                 mbar_wait(smem_addr(&full[j % kStages]), (j / kStages) & 1u);
-    } else if (warp == 1 && lane == 0) {
-        // MMA issue.
-        const uint32_t idesc = idesc_bf16_f32(kBM, g.bn);
+    } else if (warp == 1 && lane == 0 && leader) {
+        // MMA issue for the pair.
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
         uint32_t it = 0, tc = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x, ++tc) {
-            const TileCoord c = decode_tile(g, i);
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
+            const TileCoord c = decode_tile(g, i, 0);
             const uint32_t acc = tc & 1u, use = tc >> 1;
             if (!wait_or_abort(smem_addr(&acce[acc]), (use & 1u) ^ 1u, abort))
                 break;
@@ -192,61 +265,57 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
 #pragma unroll
                 for (int k = 0; k < kBK / 16; ++k)
-                    umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
-                umma_commit(smem_addr(&empty[s]));
+                    umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                umma_commit_pair(smem_addr(&empty[s]), kPairMask);
             }
             if (ok)
-                umma_commit(smem_addr(&accf[acc]));
+                umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
         }
         // Every MMA issued has completed before tensor memory is freed.
-        umma_commit(smem_addr(&drain));
+        umma_commit_pair(smem_addr(&drain), 0x1);
         mbar_wait(smem_addr(&drain), 0u);
     } else if (warp >= 2) {
-        // Epilogue: warp q = warp % 4 reads accumulator lanes 32q .. 32q + 31.
+        // Epilogue of this CTA's tile; each warp then frees the accumulator on the leader.
         const int q = warp & 3, row = 32 * q + lane;
         const int r = row / kTileCols, jj = row - r * kTileCols;
-        uint32_t tc = 0;
-        for (int i = blockIdx.x; i < g.ntiles; i += gridDim.x, ++tc) {
-            const TileCoord c = decode_tile(g, i);
+        const uint32_t acce0 = mapa_shared(smem_addr(&acce[0]), 0), acce1 = mapa_shared(smem_addr(&acce[1]), 0);
+        const uint32_t stage = base + kStages * stage_bytes + (uint32_t)q * 8192u;
+        unsigned char *stage_ptr = smem_raw + (stage - smem_addr(smem_raw));
+        uint32_t tc = 0, sbuf = 0;
+        for (int i = pair; i < g.npairs; i += npair_ctas, ++tc) {
+            const TileCoord c = decode_tile(g, i, rank);
             const uint32_t acc = tc & 1u, use = tc >> 1;
             if (!wait_or_abort(smem_addr(&accf[acc]), use & 1u, abort))
                 break;
             tc_fence_after();
             const int y = c.y0 + r, x = c.x0 + jj;
-            const bool valid = y < g.h && x < g.w;
             __nv_bfloat16 *o = out + (((int64_t)c.f * g.h + y) * g.w + x) * g.n + c.n0;
-            for (int cb = 0; cb < g.bn; cb += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * (uint32_t)g.bn + (uint32_t)cb, v);
-                tmem_wait_ld();
-                if (valid) {
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        *reinterpret_cast<uint4 *>(o + cb + 8 * s) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * s + 0]), __uint_as_float(v[8 * s + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 2]), __uint_as_float(v[8 * s + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 4]), __uint_as_float(v[8 * s + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 6]), __uint_as_float(v[8 * s + 7])));
-                }
-            }
+            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage, stage_ptr, sbuf, o,
+                       y < g.h && x < g.w, g.bn);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(smem_addr(&acce[acc]));
+                mbar_arrive_cluster(acc ? acce1 : acce0);
         }
+        if (lane == 0)
+            bulk_wait_all(); // the tile stores have completed before the CTA exits
     }
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync(); // neither CTA frees the pair's tensor memory while the other still uses it
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, ncols);
+        tmem_dealloc_pair(tmem, ncols);
     }
     if (threadIdx.x == 0 && *abort)
         atomicAdd(&g_conv_timeouts, 1u);
 }
 
-size_t conv_smem_bytes(int bn) { return (size_t)kStages * (kABytes + (uint32_t)bn * kBK * 2) + 1024; }
+size_t conv_smem_bytes(int bn)
+{
+    return (size_t)kStages * (kABytes + (uint32_t)(bn / 2) * kBK * 2) + kEpiBytes + 1024;
+}
 
 bool fits_int(int64_t v) { return v >= 0 && v < ((int64_t)1 << 31); }
 
@@ -255,6 +324,48 @@ bool fits_int(int64_t v) { return v >= 0 && v < ((int64_t)1 << 31); }
 bool tc_eligible(int64_t Cin, int64_t Cout)
 {
     return Cin >= 64 && Cin % 64 == 0 && Cout >= 32 && Cout % 32 == 0 && (Cout <= 256 || Cout % 256 == 0);
+}
+
+// Launch a pair kernel: as many pairs as can be resident at once (each CTA needs a whole
+// SM), at most one per pair tile.
+template <typename K, typename G>
+tok_status launch_pairs(K kernel, int64_t npairs, size_t smem, int threads, cudaStream_t stream,
+                        const CUtensorMap &m0, const CUtensorMap &m1, const CUtensorMap &m2, __nv_bfloat16 *out,
+                        const G &g)
+{
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    const int sms = sm_count();
+    if (sms <= 0)
+        return launch_status();
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(npairs, sms / 2)), 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int resident = 0;
+    e = cudaOccupancyMaxActiveClusters(&resident, kernel, &cfg);
+    if (e != cudaSuccess || resident <= 0) {
+        record_cuda_error(e != cudaSuccess ? e : cudaErrorInvalidConfiguration);
+        return TOK_ERR_CUDA;
+    }
+    cfg.gridDim = dim3((unsigned)(2 * std::min<int64_t>(npairs, resident)), 1, 1);
+    e = cudaLaunchKernelEx(&cfg, kernel, m0, m1, m2, out, g);
+    if (e != cudaSuccess) {
+        record_cuda_error(e);
+        return TOK_ERR_CUDA;
+    }
+    return launch_status();
 }
 
 tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y, int64_t B, int64_t T, int64_t h,
@@ -269,12 +380,13 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
     g.n = (int)Cout;
     g.bn = Cout <= 256 ? (int)Cout : 256;
     g.n_tiles = (int)(Cout / g.bn);
-    g.tiles_x = (int)((w + kTileCols - 1) / kTileCols);
+    const int64_t tiles_x = (w + kTileCols - 1) / kTileCols;
+    g.tiles_xp = (int)((tiles_x + 1) / 2);
     g.tiles_y = (int)((h + kTileRows - 1) / kTileRows);
-    const int64_t ntiles = (int64_t)g.frames * g.tiles_x * g.tiles_y * g.n_tiles;
-    if (!fits_int(ntiles))
+    const int64_t npairs = (int64_t)g.frames * g.tiles_xp * g.tiles_y * g.n_tiles;
+    if (!fits_int(npairs))
         return TOK_ERR_SHAPE;
-    g.ntiles = (int)ntiles;
+    g.npairs = (int)npairs;
     g.k = (int)k;
     g.temporal = temporal ? 1 : 0;
 
@@ -285,23 +397,17 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
     const int64_t ktot = (temporal ? k : k * k) * Cin;
     const uint64_t bdims[2] = {(uint64_t)ktot, (uint64_t)Cout};
     const uint64_t bstr[1] = {(uint64_t)ktot * 2};
-    const uint32_t bbox[2] = {kBK, (uint32_t)g.bn};
+    const uint32_t bbox[2] = {kBK, (uint32_t)(g.bn / 2)};
+    CUtensorMap omap;
+    const uint64_t odims[4] = {(uint64_t)Cout, (uint64_t)w, (uint64_t)h, (uint64_t)g.frames};
+    const uint64_t ostr[3] = {(uint64_t)Cout * 2, (uint64_t)w * Cout * 2, (uint64_t)h * w * Cout * 2};
+    const uint32_t obox[4] = {(uint32_t)std::min<int64_t>(64, Cout), kTileCols, 4, 1};
     if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, abox) ||
-        !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox))
+        !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox) ||
+        !encode_tensor_map_sw128(&omap, 4, y, odims, ostr, obox))
         return TOK_ERR_SHAPE;
-
-    const size_t smem = conv_smem_bytes(g.bn);
-    cudaError_t e = cudaFuncSetAttribute(conv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-        record_cuda_error(e);
-        return TOK_ERR_CUDA;
-    }
-    const int sms = sm_count();
-    if (sms <= 0)
-        return launch_status();
-    const int grid = (int)std::min<int64_t>(ntiles, sms);
-    conv_tc_kernel<<<grid, kThreads, smem, stream>>>(amap, bmap, static_cast<__nv_bfloat16 *>(y), g);
-    return launch_status();
+    return launch_pairs(conv_tc_kernel, npairs, conv_smem_bytes(g.bn), kThreads, stream, amap, bmap, omap,
+                        static_cast<__nv_bfloat16 *>(y), g);
 }
 
 // ---------------------------------------------------------------------------
@@ -327,7 +433,7 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
 // which is exactly the convolution's zero padding of the coefficients.
 // ---------------------------------------------------------------------------
 constexpr int kFStages = 3;                      // filter stages
-constexpr int kPlanes = 3;                       // A planes in flight
+constexpr int kPlanes = 5;                       // A planes in flight (a ring)
 constexpr int kPlaneRows = kTileRows + 2;        // latent rows of a plane
 constexpr uint32_t kPlaneBytes = kPlaneRows * kTileCols * 128; // 18 KB
 constexpr int kPixCols = 48, kPixRows = 4 * kPlaneRows, kPixFrames = 4;
@@ -339,26 +445,27 @@ constexpr int kHaarFirst = 192;                  // first Haar thread
 struct EmbedGeom {
     int B, C, Tq, h, w;   // pixels [B, C, 4*Tq - 3, 4h, 4w]; output [B, Tq, h, w, n]
     int n, bn, n_tiles;
-    int tiles_x, tiles_y, ntiles;
+    int tiles_xp, tiles_y, npairs;
 };
 
 struct EmbedTile {
     int b, tq, y0, x0, n0;
 };
 
-__device__ __forceinline__ EmbedTile decode_embed(const EmbedGeom &g, int i)
+// Pair tile i, this CTA's half (rank): column block 2 * xp + rank.
+__device__ __forceinline__ EmbedTile decode_embed(const EmbedGeom &g, int i, uint32_t rank)
 {
     EmbedTile e;
     const int nb = i % g.n_tiles; // output-channel tiles fastest: they read the same pixels
     int r = i / g.n_tiles;
-    const int xb = r % g.tiles_x;
-    r /= g.tiles_x;
+    const int xp = r % g.tiles_xp;
+    r /= g.tiles_xp;
     const int yb = r % g.tiles_y;
     r /= g.tiles_y;
     e.tq = r % g.Tq;
     e.b = r / g.Tq;
     e.y0 = yb * kTileRows;
-    e.x0 = xb * kTileCols;
+    e.x0 = (2 * xp + (int)rank) * kTileCols;
     e.n0 = nb * g.bn;
     return e;
 }
@@ -391,7 +498,7 @@ __device__ __forceinline__ void issue_pixels(const CUtensorMap *xmap, const Embe
 
 __global__ void __launch_bounds__(kEmbedThreads, 1)
 patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
-                   __nv_bfloat16 *__restrict__ out, const EmbedGeom g)
+                   const __grid_constant__ CUtensorMap omap, __nv_bfloat16 *__restrict__ out, const EmbedGeom g)
 {
     __shared__ __align__(8) uint64_t ffull[kFStages], fempty[kFStages], pfull[kPlanes], pempty[kPlanes], xfull[2],
         accf[2], acce[2], drain, hsync;
@@ -399,10 +506,14 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-    const uint32_t fbytes = (uint32_t)g.bn * kBK * 2;
+    const uint32_t fbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of a filter stage
     const uint32_t fbase = base, pbase = fbase + kFStages * fbytes, xbase = pbase + kPlanes * kPlaneBytes;
+    const uint32_t ebase = xbase + 2 * kPixBytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t ncols = g.bn <= 16 ? 32u : g.bn <= 32 ? 64u : g.bn <= 64 ? 128u : g.bn <= 128 ? 256u : 512u;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const uint32_t ncols = tmem_cols(g.bn);
+    const int pair = blockIdx.x >> 1, npair_ctas = gridDim.x >> 1;
     const int kper = 9 * g.C; // K steps per tile
 
     if (threadIdx.x == 0) {
@@ -411,13 +522,13 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
             mbar_init(smem_addr(&fempty[s]), 1);
         }
         for (int p = 0; p < kPlanes; ++p) {
-            mbar_init(smem_addr(&pfull[p]), kHaarThreads);
+            mbar_init(smem_addr(&pfull[p]), 8); // 4 Haar warps in each CTA
             mbar_init(smem_addr(&pempty[p]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_addr(&xfull[a]), 1);
             mbar_init(smem_addr(&accf[a]), 1);
-            mbar_init(smem_addr(&acce[a]), 4);
+            mbar_init(smem_addr(&acce[a]), 8);
         }
         mbar_init(smem_addr(&drain), 1);
         mbar_init(smem_addr(&hsync), kHaarThreads);
@@ -425,41 +536,42 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
         fence_barrier_init();
     }
     if (warp == 0) {
-        tmem_alloc(smem_addr(&tmem_base_s), ncols);
-        tmem_relinquish();
+        tmem_alloc_pair(smem_addr(&tmem_base_s), ncols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = tmem_base_s;
     volatile int *abort = &abort_s;
 
     if (warp == 0 && lane == 0) {
-        // Filter copies, in the tile's K order.
+        // This CTA's half of the filter, in the tile's K order; counted on the leader's barrier.
         uint32_t it = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x) {
-            const EmbedTile e = decode_embed(g, i);
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
+            const EmbedTile e = decode_embed(g, i, rank);
             for (int kb = 0; kb < kper; ++kb, ++it) {
                 const uint32_t s = it % kFStages, ph = (it / kFStages) & 1u;
                 if (!wait_or_abort(smem_addr(&fempty[s]), ph ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
-                const uint32_t fb = smem_addr(&ffull[s]);
-                mbar_expect_tx(fb, fbytes);
-                tma_load_2d(fbase + s * fbytes, &bmap, kb * kBK, e.n0, fb);
+                if (leader)
+                    mbar_expect_tx(smem_addr(&ffull[s]), 2 * fbytes);
+                tma_load_2d_pair(fbase + s * fbytes, &bmap, kb * kBK, e.n0 + (int)rank * (g.bn / 2),
+                                 mapa_shared(smem_addr(&ffull[s]), 0));
             }
         }
-        if (!ok)
+        if (!ok && leader)
             for (uint32_t j = it > kFStages ? it - kFStages : 0; j < it; ++j)
                 mbar_wait(smem_addr(&ffull[j % kFStages]), (j / kFStages) & 1u);
-    } else if (warp == 1 && lane == 0) {
-        // MMA issue: per plane (c, dx), the three row shifts dy.
-        const uint32_t idesc = idesc_bf16_f32(kBM, g.bn);
+    } else if (warp == 1 && lane == 0 && leader) {
+        // MMA issue for the pair: per plane (c, dx), the three row shifts dy.
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
         uint32_t it = 0, pi = 0, tc = 0;
         bool ok = true;
-        for (int i = blockIdx.x; i < g.ntiles && ok; i += gridDim.x, ++tc) {
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
             const uint32_t acc = tc & 1u, use = tc >> 1;
             if (!wait_or_abort(smem_addr(&acce[acc]), (use & 1u) ^ 1u, abort))
                 break;
@@ -482,63 +594,58 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                     const uint64_t bd = sw128_desc(fbase + s * fbytes);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
-                    umma_commit(smem_addr(&fempty[s]));
+                        umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
+                    umma_commit_pair(smem_addr(&fempty[s]), kPairMask);
                 }
                 if (ok)
-                    umma_commit(smem_addr(&pempty[slot]));
+                    umma_commit_pair(smem_addr(&pempty[slot]), kPairMask);
             }
             if (ok)
-                umma_commit(smem_addr(&accf[acc]));
+                umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
         }
-        umma_commit(smem_addr(&drain));
+        umma_commit_pair(smem_addr(&drain), 0x1);
         mbar_wait(smem_addr(&drain), 0u);
     } else if (warp >= 2 && warp < 6) {
-        // Epilogue.
+        // Epilogue of this CTA's tile.
         const int q = warp & 3, row = 32 * q + lane;
         const int r = row / kTileCols, jj = row - r * kTileCols;
-        uint32_t tc = 0;
-        for (int i = blockIdx.x; i < g.ntiles; i += gridDim.x, ++tc) {
-            const EmbedTile e = decode_embed(g, i);
+        const uint32_t acce0 = mapa_shared(smem_addr(&acce[0]), 0), acce1 = mapa_shared(smem_addr(&acce[1]), 0);
+        const uint32_t stage = ebase + (uint32_t)q * 8192u;
+        unsigned char *stage_ptr = smem_raw + (stage - smem_addr(smem_raw));
+        uint32_t tc = 0, sbuf = 0;
+        for (int i = pair; i < g.npairs; i += npair_ctas, ++tc) {
+            const EmbedTile e = decode_embed(g, i, rank);
             const uint32_t acc = tc & 1u, use = tc >> 1;
             if (!wait_or_abort(smem_addr(&accf[acc]), use & 1u, abort))
                 break;
             tc_fence_after();
-            const int y = e.y0 + r, x = e.x0 + jj;
-            const bool valid = y < g.h && x < g.w;
-            __nv_bfloat16 *o = out + ((((int64_t)e.b * g.Tq + e.tq) * g.h + y) * g.w + x) * g.n + e.n0;
-            for (int cb = 0; cb < g.bn; cb += 32) {
-                uint32_t v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + acc * (uint32_t)g.bn + (uint32_t)cb, v);
-                tmem_wait_ld();
-                if (valid) {
-#pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        *reinterpret_cast<uint4 *>(o + cb + 8 * s) = make_uint4(
-                            pack_bf16x2(__uint_as_float(v[8 * s + 0]), __uint_as_float(v[8 * s + 1])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 2]), __uint_as_float(v[8 * s + 3])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 4]), __uint_as_float(v[8 * s + 5])),
-                            pack_bf16x2(__uint_as_float(v[8 * s + 6]), __uint_as_float(v[8 * s + 7])));
-                }
-            }
+            const int y = e.y0 + r, x = e.x0 + jj, f = e.b * g.Tq + e.tq;
+            __nv_bfloat16 *o = out + (((int64_t)f * g.h + y) * g.w + x) * g.n + e.n0;
+            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, f, e.y0, e.x0, e.n0, stage, stage_ptr, sbuf, o,
+                       y < g.h && x < g.w, g.bn);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(smem_addr(&acce[acc]));
+                mbar_arrive_cluster(acc ? acce1 : acce0);
         }
+        if (lane == 0)
+            bulk_wait_all();
     } else if (warp >= 6) {
-        // Haar warps.
+        // Haar warps of this CTA's tile.  Per colour, each of 90 threads transforms two adjacent
+        // latent columns u0 = 2 up - 1, u0 + 1 (up = 0..4; u = -1 .. 8 relative to x0) of plane row
+        // pr and writes each position into every plane dx whose window holds it (plane column
+        // j = u + 1 - dx): the colour's three planes are made in one pass.
         const int ht = threadIdx.x - kHaarFirst;
-        const int pr = ht >> 2, jp = ht & 3; // work item: plane row pr (0..17), columns 2 jp, 2 jp + 1
-        const bool worker = ht < kPlaneRows * 4;
+        const int pr = ht / 5, up = ht - 5 * pr, u0 = 2 * up - 1;
+        const bool worker = ht < kPlaneRows * 5;
         uint32_t ci = 0, pi = 0; // colours and planes made so far
         bool ok = true;
-        int i = blockIdx.x;
-        if (ht == 0 && i < g.ntiles)
-            issue_pixels(&xmap, decode_embed(g, i), 0, xbase, smem_addr(&xfull[0]));
-        for (; i < g.ntiles && ok; i += gridDim.x) {
-            const EmbedTile e = decode_embed(g, i);
-            for (int c = 0; c < g.C && ok; ++c, ++ci) {
+        int i = pair;
+        if (ht == 0 && i < g.npairs)
+            issue_pixels(&xmap, decode_embed(g, i, rank), 0, xbase, smem_addr(&xfull[0]));
+        for (; i < g.npairs && ok; i += npair_ctas) {
+            const EmbedTile e = decode_embed(g, i, rank);
+            for (int c = 0; c < g.C && ok; ++c, ++ci, pi += 3) {
                 // Once every Haar thread is done with the buffer of colour ci - 1 (a barrier phase per
                 // colour; its wait is bounded like the others), colour ci + 1 is copied into it.
                 mbar_arrive(smem_addr(&hsync));
@@ -548,11 +655,11 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                 }
                 if (ht == 0) {
                     const bool last_c = c + 1 == g.C;
-                    const int ni = last_c ? i + (int)gridDim.x : i;
-                    if (ni < g.ntiles) {
+                    const int ni = last_c ? i + npair_ctas : i;
+                    if (ni < g.npairs) {
                         fence_proxy_async_smem();
                         const uint32_t nb = (ci + 1) & 1u;
-                        issue_pixels(&xmap, last_c ? decode_embed(g, ni) : e, last_c ? 0 : c + 1,
+                        issue_pixels(&xmap, last_c ? decode_embed(g, ni, rank) : e, last_c ? 0 : c + 1,
                                      xbase + nb * kPixBytes, smem_addr(&xfull[nb]));
                     }
                 }
@@ -561,71 +668,79 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                     ok = false;
                     break;
                 }
-                const unsigned char *pix = smem_raw + (xbase + xb * kPixBytes - smem_addr(smem_raw));
-                for (int dx = 0; dx < 3; ++dx, ++pi) {
-                    const uint32_t slot = pi % kPlanes;
-                    if (!wait_or_abort(smem_addr(&pempty[slot]), ((pi / kPlanes) & 1u) ^ 1u, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    if (worker) {
-                        // Blocks at latent (y0 - 1 + pr, x0 + 2 jp + dx - 1 + {0, 1}): pixel rows 4 pr ..,
-                        // columns 4 (2 jp + dx + 1) .. of the staged box; window 0 reads frame 0 (box frame 3)
-                        // four times.
-                        float2 v[4][4][4];
-                        const int col = 4 * (2 * jp + dx + 1);
+                uint32_t slot[3];
+                for (int dx = 0; dx < 3 && ok; ++dx) {
+                    slot[dx] = (pi + dx) % kPlanes;
+                    ok = wait_or_abort(smem_addr(&pempty[slot[dx]]), (((pi + dx) / kPlanes) & 1u) ^ 1u, abort);
+                }
+                if (!ok)
+                    break;
+                if (worker) {
+                    // Staged pixel columns of latent u: 4 (u + 2) .. + 3 (the box starts two blocks left of
+                    // x0); rows 4 pr ..; window 0 reads frame 0 (box frame 3) four times.
+                    const unsigned char *pix = smem_raw + (xbase + xb * kPixBytes - smem_addr(smem_raw));
+                    float2 v[4][4][4];
+                    const int col = 4 * (u0 + 2);
 #pragma unroll
-                        for (int a = 0; a < 4; ++a) {
-                            const int fa = e.tq == 0 ? 3 : a;
+                    for (int a = 0; a < 4; ++a) {
+                        const int fa = e.tq == 0 ? 3 : a;
 #pragma unroll
-                            for (int rr = 0; rr < 4; ++rr) {
-                                const unsigned char *rowp = pix + ((fa * kPixRows + 4 * pr + rr) * kPixCols + col) * 2;
-                                const uint2 p0 = *reinterpret_cast<const uint2 *>(rowp);
-                                const uint2 p1 = *reinterpret_cast<const uint2 *>(rowp + 8);
-                                v[a][rr][0] = make_float2(bf16_lo(p0.x), bf16_lo(p1.x));
-                                v[a][rr][1] = make_float2(bf16_hi(p0.x), bf16_hi(p1.x));
-                                v[a][rr][2] = make_float2(bf16_lo(p0.y), bf16_lo(p1.y));
-                                v[a][rr][3] = make_float2(bf16_hi(p0.y), bf16_hi(p1.y));
-                            }
+                        for (int rr = 0; rr < 4; ++rr) {
+                            const unsigned char *rowp = pix + ((fa * kPixRows + 4 * pr + rr) * kPixCols + col) * 2;
+                            const uint2 p0 = *reinterpret_cast<const uint2 *>(rowp);
+                            const uint2 p1 = *reinterpret_cast<const uint2 *>(rowp + 8);
+                            v[a][rr][0] = make_float2(bf16_lo(p0.x), bf16_lo(p1.x));
+                            v[a][rr][1] = make_float2(bf16_hi(p0.x), bf16_hi(p1.x));
+                            v[a][rr][2] = make_float2(bf16_lo(p0.y), bf16_lo(p1.y));
+                            v[a][rr][3] = make_float2(bf16_hi(p0.y), bf16_hi(p1.y));
                         }
+                    }
 #pragma unroll
-                        for (int a = 0; a < 4; ++a)
-#pragma unroll
-                            for (int rr = 0; rr < 4; ++rr)
-                                wht4x2(v[a][rr][0], v[a][rr][1], v[a][rr][2], v[a][rr][3]);
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-#pragma unroll
-                            for (int d = 0; d < 4; ++d)
-                                wht4x2(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
+                    for (int a = 0; a < 4; ++a)
 #pragma unroll
                         for (int rr = 0; rr < 4; ++rr)
+                            wht4x2(v[a][rr][0], v[a][rr][1], v[a][rr][2], v[a][rr][3]);
 #pragma unroll
-                            for (int d = 0; d < 4; ++d)
-                                wht4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
-                        unsigned char *plane = smem_raw + (pbase + slot * kPlaneBytes - smem_addr(smem_raw));
-                        const float2 eighth = make_float2(0.125f, 0.125f);
+                    for (int a = 0; a < 4; ++a)
 #pragma unroll
-                        for (int k8 = 0; k8 < 8; ++k8) {
-                            uint32_t lo[4], hi[4];
+                        for (int d = 0; d < 4; ++d)
+                            wht4x2(v[a][0][d], v[a][1][d], v[a][2][d], v[a][3][d]);
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int g0 = 8 * k8 + 2 * u, g1 = g0 + 1;
-                                const float2 a0 = __fmul2_rn(v[sb_kt(g0)][sb_ky(g0)][sb_kx(g0)], eighth);
-                                const float2 a1 = __fmul2_rn(v[sb_kt(g1)][sb_ky(g1)][sb_kx(g1)], eighth);
-                                lo[u] = pack_bf16x2(a0.x, a1.x);
-                                hi[u] = pack_bf16x2(a0.y, a1.y);
-                            }
-                            const int q0 = pr * kTileCols + 2 * jp, q1 = q0 + 1;
-                            *reinterpret_cast<uint4 *>(plane + sw128_offset(q0, 8 * k8)) =
-                                make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                            *reinterpret_cast<uint4 *>(plane + sw128_offset(q1, 8 * k8)) =
-                                make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                        for (int d = 0; d < 4; ++d)
+                            wht4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
+                    unsigned char *planes = smem_raw + (pbase - smem_addr(smem_raw));
+                    const float2 eighth = make_float2(0.125f, 0.125f);
+#pragma unroll
+                    for (int k8 = 0; k8 < 8; ++k8) {
+                        uint32_t lo[4], hi[4];
+#pragma unroll
+                        for (int uu = 0; uu < 4; ++uu) {
+                            const int g0 = 8 * k8 + 2 * uu, g1 = g0 + 1;
+                            const float2 a0 = __fmul2_rn(v[sb_kt(g0)][sb_ky(g0)][sb_kx(g0)], eighth);
+                            const float2 a1 = __fmul2_rn(v[sb_kt(g1)][sb_ky(g1)][sb_kx(g1)], eighth);
+                            lo[uu] = pack_bf16x2(a0.x, a1.x);
+                            hi[uu] = pack_bf16x2(a0.y, a1.y);
+                        }
+                        const uint4 vlo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        const uint4 vhi = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+#pragma unroll
+                        for (int dx = 0; dx < 3; ++dx) {
+                            unsigned char *plane = planes + slot[dx] * kPlaneBytes;
+                            const int j0 = u0 + 1 - dx, j1 = j0 + 1;
+                            if (j0 >= 0 && j0 < kTileCols)
+                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j0, 8 * k8)) = vlo;
+                            if (j1 >= 0 && j1 < kTileCols)
+                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j1, 8 * k8)) = vhi;
                         }
                     }
-                    fence_proxy_async_smem(); // the plane's writes are visible to the tensor cores
-                    mbar_arrive(smem_addr(&pfull[slot]));
                 }
+                fence_proxy_async_smem(); // the planes' writes are visible to the tensor cores
+                __syncwarp();
+                if (lane == 0)
+                    for (int dx = 0; dx < 3; ++dx)
+                        mbar_arrive_cluster(mapa_shared(smem_addr(&pfull[slot[dx]]), 0));
             }
         }
         if (ht == 0 && !ok) // the pixel copies issued and not yet waited for
@@ -635,9 +750,10 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, ncols);
+        tmem_dealloc_pair(tmem, ncols);
     }
     if (threadIdx.x == 0 && *abort)
         atomicAdd(&g_conv_timeouts, 1u);
@@ -645,7 +761,8 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
 
 size_t embed_smem_bytes(int bn)
 {
-    return (size_t)kFStages * bn * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes + 1024;
+    return (size_t)kFStages * (bn / 2) * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes + kEpiBytes +
+           1024;
 }
 
 // Packed filter: wp[n][(c * 3 + dx) * 3 + dy][g] = ws[n][dy][dx][g * C + c].
@@ -703,12 +820,12 @@ tok_status patch_embed_launch(const void *x, const void *wp, void *y, int64_t B,
     g.n = (int)Cmid;
     g.bn = Cmid <= 256 ? (int)Cmid : 256;
     g.n_tiles = (int)(Cmid / g.bn);
-    g.tiles_x = (g.w + kTileCols - 1) / kTileCols;
+    g.tiles_xp = ((g.w + kTileCols - 1) / kTileCols + 1) / 2;
     g.tiles_y = (g.h + kTileRows - 1) / kTileRows;
-    const int64_t ntiles = B * g.Tq * (int64_t)g.tiles_x * g.tiles_y * g.n_tiles;
-    if (!fits_int(ntiles))
+    const int64_t npairs = B * g.Tq * (int64_t)g.tiles_xp * g.tiles_y * g.n_tiles;
+    if (!fits_int(npairs))
         return TOK_ERR_SHAPE;
-    g.ntiles = (int)ntiles;
+    g.npairs = (int)npairs;
 
     CUtensorMap xmap, bmap;
     const uint64_t xdims[5] = {(uint64_t)W, (uint64_t)H, (uint64_t)T, (uint64_t)C, (uint64_t)B};
@@ -717,22 +834,17 @@ tok_status patch_embed_launch(const void *x, const void *wp, void *y, int64_t B,
     const uint32_t xbox[5] = {kPixCols, kPixRows, kPixFrames, 1, 1};
     const uint64_t bdims[2] = {(uint64_t)(576 * C), (uint64_t)Cmid};
     const uint64_t bstr[1] = {(uint64_t)(576 * C) * 2};
-    const uint32_t bbox[2] = {kBK, (uint32_t)g.bn};
+    const uint32_t bbox[2] = {kBK, (uint32_t)(g.bn / 2)};
+    CUtensorMap omap;
+    const uint64_t odims[4] = {(uint64_t)Cmid, (uint64_t)g.w, (uint64_t)g.h, (uint64_t)(B * g.Tq)};
+    const uint64_t ostr[3] = {(uint64_t)Cmid * 2, (uint64_t)g.w * Cmid * 2, (uint64_t)g.h * g.w * Cmid * 2};
+    const uint32_t obox[4] = {(uint32_t)std::min<int64_t>(64, Cmid), kTileCols, 4, 1};
     if (!encode_tensor_map(&xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, x, xdims, xstr, xbox) ||
-        !encode_tensor_map_sw128(&bmap, 2, wp, bdims, bstr, bbox))
+        !encode_tensor_map_sw128(&bmap, 2, wp, bdims, bstr, bbox) ||
+        !encode_tensor_map_sw128(&omap, 4, y, odims, ostr, obox))
         return TOK_ERR_SHAPE;
-    const size_t smem = embed_smem_bytes(g.bn);
-    cudaError_t e = cudaFuncSetAttribute(patch_embed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) {
-        record_cuda_error(e);
-        return TOK_ERR_CUDA;
-    }
-    const int sms = sm_count();
-    if (sms <= 0)
-        return launch_status();
-    const int grid = (int)std::min<int64_t>(ntiles, sms);
-    patch_embed_kernel<<<grid, kEmbedThreads, smem, stream>>>(xmap, bmap, static_cast<__nv_bfloat16 *>(y), g);
-    return launch_status();
+    return launch_pairs(patch_embed_kernel, npairs, embed_smem_bytes(g.bn), kEmbedThreads, stream, xmap, bmap, omap,
+                        static_cast<__nv_bfloat16 *>(y), g);
 }
 
 tok_status read_and_clear_conv_timeouts(cudaStream_t stream, unsigned int *count)
