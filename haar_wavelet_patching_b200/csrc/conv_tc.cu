@@ -312,6 +312,180 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         atomicAdd(&g_conv_timeouts, 1u);
 }
 
+// The spatial convolution with its activation tiles read once per column shift: for
+// each 64-channel chunk c and column shift dx, one tensor copy brings the plane of
+// 16 + k - 1 rows x 8 columns (rows y0 - pad .., columns x0 + dx - pad ..) in the
+// 128-byte swizzle, and the k row shifts dy are that plane seen from row-atom dy (one
+// tile row of 8 positions is one 1024-byte swizzle atom).  K order (c, dx, dy); the
+// filter stages follow it.  Planes and filter stages are separate rings.
+constexpr int kPStages = 6;  // filter stages of the plane kernel
+constexpr int kPPlanes = 4;  // activation planes in flight
+constexpr int kMaxPlaneK = 7;
+
+__global__ void __launch_bounds__(kThreads, 1)
+conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                   const __grid_constant__ CUtensorMap omap, __nv_bfloat16 *__restrict__ out, const ConvGeom g)
+{
+    __shared__ __align__(8) uint64_t bfull[kPStages], bempty[kPStages], pfull[kPPlanes], pempty[kPPlanes], accf[2],
+        acce[2], drain;
+    __shared__ uint32_t tmem_base_s;
+    __shared__ int abort_s;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const uint32_t bbytes = (uint32_t)(g.bn / 2) * kBK * 2;
+    const uint32_t plane_bytes = (uint32_t)(kTileRows + g.k - 1) * kTileCols * 128;
+    const uint32_t bbase = base, pbase = bbase + kPStages * bbytes, ebase = pbase + kPPlanes * plane_bytes;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const uint32_t ncols = tmem_cols(g.bn);
+    const int pair = blockIdx.x >> 1, npair_ctas = gridDim.x >> 1;
+    const int nchunk = g.cin / kBK, pad = (g.k - 1) / 2;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPStages; ++s) {
+            mbar_init(smem_addr(&bfull[s]), 1);
+            mbar_init(smem_addr(&bempty[s]), 1);
+        }
+        for (int p = 0; p < kPPlanes; ++p) {
+            mbar_init(smem_addr(&pfull[p]), 1);
+            mbar_init(smem_addr(&pempty[p]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_addr(&accf[a]), 1);
+            mbar_init(smem_addr(&acce[a]), 8);
+        }
+        mbar_init(smem_addr(&drain), 1);
+        abort_s = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc_pair(smem_addr(&tmem_base_s), ncols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = tmem_base_s;
+    volatile int *abort = &abort_s;
+
+    if (warp == 0 && lane == 0) {
+        // Planes and filter stages of this CTA, counted on the leader's barriers.
+        uint32_t it = 0, pi = 0;
+        bool ok = true;
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
+            const TileCoord c = decode_tile(g, i, rank);
+            for (int ch = 0; ch < nchunk && ok; ++ch)
+                for (int dx = 0; dx < g.k && ok; ++dx, ++pi) {
+                    const uint32_t slot = pi % kPPlanes;
+                    if (!wait_or_abort(smem_addr(&pempty[slot]), ((pi / kPPlanes) & 1u) ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (leader)
+                        mbar_expect_tx(smem_addr(&pfull[slot]), 2 * plane_bytes);
+                    tma_load_4d_pair(pbase + slot * plane_bytes, &amap, ch * kBK, c.x0 + dx - pad, c.y0 - pad, c.f,
+                                     mapa_shared(smem_addr(&pfull[slot]), 0));
+                    for (int dy = 0; dy < g.k; ++dy, ++it) {
+                        const uint32_t s = it % kPStages, ph = (it / kPStages) & 1u;
+                        if (!wait_or_abort(smem_addr(&bempty[s]), ph ^ 1u, abort)) {
+                            ok = false;
+                            break;
+                        }
+                        if (leader)
+                            mbar_expect_tx(smem_addr(&bfull[s]), 2 * bbytes);
+                        tma_load_2d_pair(bbase + s * bbytes, &bmap, (dy * g.k + dx) * g.cin + ch * kBK,
+                                         c.n0 + (int)rank * (g.bn / 2), mapa_shared(smem_addr(&bfull[s]), 0));
+                    }
+                }
+        }
+        if (!ok && leader) {
+            for (uint32_t j = it > kPStages ? it - kPStages : 0; j < it; ++j)
+                mbar_wait(smem_addr(&bfull[j % kPStages]), (j / kPStages) & 1u);
+            for (uint32_t j = pi > kPPlanes ? pi - kPPlanes : 0; j < pi; ++j)
+                mbar_wait(smem_addr(&pfull[j % kPPlanes]), (j / kPPlanes) & 1u);
+        }
+    } else if (warp == 1 && lane == 0 && leader) {
+        const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
+        uint32_t it = 0, pi = 0, tc = 0;
+        bool ok = true;
+        for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&acce[acc]), (use & 1u) ^ 1u, abort))
+                break;
+            tc_fence_after();
+            const uint32_t d = tmem + acc * (uint32_t)g.bn;
+            for (int pl = 0; pl < nchunk * g.k && ok; ++pl, ++pi) {
+                const uint32_t slot = pi % kPPlanes;
+                if (!wait_or_abort(smem_addr(&pfull[slot]), (pi / kPPlanes) & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                for (int dy = 0; dy < g.k; ++dy, ++it) {
+                    const uint32_t s = it % kPStages, ph = (it / kPStages) & 1u;
+                    if (!wait_or_abort(smem_addr(&bfull[s]), ph, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = sw128_desc(pbase + slot * plane_bytes + (uint32_t)dy * 1024u);
+                    const uint64_t bd = sw128_desc(bbase + s * bbytes);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k)
+                        umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
+                    umma_commit_pair(smem_addr(&bempty[s]), kPairMask);
+                }
+                if (ok)
+                    umma_commit_pair(smem_addr(&pempty[slot]), kPairMask);
+            }
+            if (ok)
+                umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
+        }
+        umma_commit_pair(smem_addr(&drain), 0x1);
+        mbar_wait(smem_addr(&drain), 0u);
+    } else if (warp >= 2) {
+        const int q = warp & 3, row = 32 * q + lane;
+        const int r = row / kTileCols, jj = row - r * kTileCols;
+        const uint32_t acce0 = mapa_shared(smem_addr(&acce[0]), 0), acce1 = mapa_shared(smem_addr(&acce[1]), 0);
+        const uint32_t stage = ebase + (uint32_t)q * 8192u;
+        unsigned char *stage_ptr = smem_raw + (stage - smem_addr(smem_raw));
+        uint32_t tc = 0, sbuf = 0;
+        for (int i = pair; i < g.npairs; i += npair_ctas, ++tc) {
+            const TileCoord c = decode_tile(g, i, rank);
+            const uint32_t acc = tc & 1u, use = tc >> 1;
+            if (!wait_or_abort(smem_addr(&accf[acc]), use & 1u, abort))
+                break;
+            tc_fence_after();
+            const int y = c.y0 + r, x = c.x0 + jj;
+            __nv_bfloat16 *o = out + (((int64_t)c.f * g.h + y) * g.w + x) * g.n + c.n0;
+            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage, stage_ptr, sbuf, o,
+                       y < g.h && x < g.w, g.bn);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_cluster(acc ? acce1 : acce0);
+        }
+        if (lane == 0)
+            bulk_wait_all();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, ncols);
+    }
+    if (threadIdx.x == 0 && *abort)
+        atomicAdd(&g_conv_timeouts, 1u);
+}
+
+size_t planes_smem_bytes(int bn, int k)
+{
+    return (size_t)kPStages * (bn / 2) * kBK * 2 + (size_t)kPPlanes * (kTileRows + k - 1) * kTileCols * 128 +
+           kEpiBytes + 1024;
+}
+
 size_t conv_smem_bytes(int bn)
 {
     return (size_t)kStages * (kABytes + (uint32_t)(bn / 2) * kBK * 2) + kEpiBytes + 1024;
@@ -402,6 +576,16 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
     const uint64_t odims[4] = {(uint64_t)Cout, (uint64_t)w, (uint64_t)h, (uint64_t)g.frames};
     const uint64_t ostr[3] = {(uint64_t)Cout * 2, (uint64_t)w * Cout * 2, (uint64_t)h * w * Cout * 2};
     const uint32_t obox[4] = {(uint32_t)std::min<int64_t>(64, Cout), kTileCols, 4, 1};
+    const bool planes = !temporal && k <= kMaxPlaneK;
+    if (planes) {
+        const uint32_t pbox[4] = {kBK, kTileCols, (uint32_t)(kTileRows + k - 1), 1};
+        if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, pbox) ||
+            !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox) ||
+            !encode_tensor_map_sw128(&omap, 4, y, odims, ostr, obox))
+            return TOK_ERR_SHAPE;
+        return launch_pairs(conv_planes_kernel, npairs, planes_smem_bytes(g.bn, (int)k), kThreads, stream, amap, bmap,
+                            omap, static_cast<__nv_bfloat16 *>(y), g);
+    }
     if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, abox) ||
         !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox) ||
         !encode_tensor_map_sw128(&omap, 4, y, odims, ostr, obox))

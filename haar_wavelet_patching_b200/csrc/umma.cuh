@@ -149,11 +149,26 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar)
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-// Wait for phase `parity` of the barrier.  Gives up (false) after kWaitPolls polls,
-// raising the CTA's abort flag, or as soon as another role has raised it; every role
-// then leaves its loop, so no thread of the CTA waits for work that will not come.
+// Non-blocking test of phase `parity` (no suspension when the phase is still open).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of the barrier: a non-blocking test first (a stage that is
+// already full costs no suspension), then polls that may suspend.  Gives up (false)
+// after kWaitPolls polls, raising the CTA's abort flag, or as soon as another role has
+// raised it; every role then leaves its loop, so no thread of the CTA waits for work
+// that will not come.
 __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity, volatile int *abort)
 {
+    if (mbar_test_wait(bar, parity))
+        return true;
     for (uint32_t i = 0; i < kWaitPolls; ++i) {
         if (mbar_try_wait(bar, parity))
             return true;
