@@ -49,7 +49,8 @@ namespace {
 
 constexpr int kTileRows = 16, kTileCols = 8, kBM = kTileRows * kTileCols; // positions per CTA tile
 constexpr int kBK = 64;                                                   // K per stage: one 128-byte row
-constexpr int kStages = 6;
+constexpr int kStages = 3; // stages of kStageK K blocks
+constexpr int kStageK = 2; // (the MMA loop below is written for two)
 constexpr int kThreads = 192; // 6 warps
 constexpr uint32_t kABytes = kBM * kBK * 2;
 constexpr uint16_t kPairMask = 0x3; // both CTAs of the pair
@@ -67,6 +68,7 @@ struct ConvGeom {
     int npairs;   // pair tiles
     int k;        // taps per axis
     int temporal; // 1: causal temporal (k x 1 x 1), 0: spatial (1 x k x k, 'same' zeros)
+    int nstages;  // ring size of the plane kernel
 };
 
 struct TileCoord {
@@ -118,14 +120,16 @@ __device__ __forceinline__ uint32_t tmem_cols(int bn)
     return bn <= 16 ? 32u : bn <= 32 ? 64u : bn <= 64 ? 128u : bn <= 128 ? 256u : 512u;
 }
 
-constexpr uint32_t kEpiBytes = 4 * 2 * 4096; // per CTA: 4 epilogue warps x 2 staging buffers of 4 KB
+// Epilogue staging per CTA: 4 epilogue warps x NBUF buffers of 4 KB.
+constexpr uint32_t epi_bytes(int nbuf) { return 4u * (uint32_t)nbuf * 4096u; }
 
 // Epilogue of one CTA's tile; warp q = warp % 4 holds accumulator lanes 32q .. 32q + 31,
 // the tile's rows 4q .. 4q + 3.  Per 64 output channels: tensor memory -> registers ->
-// bf16 rows of a 128-byte-swizzled staging buffer of the warp (two, alternating) -> one
+// bf16 rows of a 128-byte-swizzled staging buffer of the warp (NBUF, in turn) -> one
 // tensor store of the box [64 ch, 8 cols, 4 rows] at (n0 + cb, x0, y0 + 4q, f); the store
 // clips positions outside the frame and writes whole lines.  A last group of 32 channels
 // (bn % 64 == 32) is stored from registers, positions outside the frame skipped.
+template <int NBUF>
 __device__ __forceinline__ void store_tile(uint32_t tmem_acc, int q, int lane, const CUtensorMap *omap, int f, int y0,
                                            int x0, int n0, uint32_t stage, unsigned char *stage_ptr, uint32_t &sbuf,
                                            __nv_bfloat16 *o, bool valid, int bn)
@@ -136,9 +140,9 @@ __device__ __forceinline__ void store_tile(uint32_t tmem_acc, int q, int lane, c
         uint32_t v[64];
         tmem_ld64(t0 + (uint32_t)cb, v);
         tmem_wait_ld();
-        const uint32_t b = sbuf & 1u;
+        const uint32_t b = sbuf % NBUF;
         if (lane == 0)
-            bulk_wait_read<1>(); // the store that used this buffer two chunks ago has read it
+            bulk_wait_read<NBUF - 1>(); // the store that last used this buffer has read it
         __syncwarp();
         unsigned char *buf = stage_ptr + b * 4096u;
 #pragma unroll
@@ -181,8 +185,9 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-    const uint32_t bbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of the filter tile
-    const uint32_t stage_bytes = kABytes + bbytes;
+    const uint32_t bbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of a filter K block
+    // A stage holds kStageK K blocks: their activation boxes, then their filter halves.
+    const uint32_t stage_bytes = kStageK * (kABytes + bbytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
@@ -219,33 +224,38 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
             const TileCoord c = decode_tile(g, i, rank);
-            for (int kb = 0; kb < c.nkb; ++kb, ++it) {
+            for (int kb = 0; kb < c.nkb; kb += kStageK, ++it) {
+                const int nk = min(kStageK, c.nkb - kb);
                 const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
                 if (!wait_or_abort(smem_addr(&empty[s]), ph ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
-                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes;
+                const uint32_t sa = base + s * stage_bytes, sb = sa + kStageK * kABytes;
                 const uint32_t fb = mapa_shared(smem_addr(&full[s]), 0);
-                const int kk = c.kb0 + kb, tap = kk / nchunk, ch = (kk - tap * nchunk) * kBK;
                 if (leader)
-                    mbar_expect_tx(smem_addr(&full[s]), 2 * stage_bytes);
-                if (g.temporal)
-                    tma_load_4d_pair(sa, &amap, ch, c.x0, c.y0, c.f - (g.k - 1) + tap, fb);
-                else {
-                    const int pad = (g.k - 1) / 2, dy = tap / g.k, dx = tap - dy * g.k;
-                    tma_load_4d_pair(sa, &amap, ch, c.x0 + dx - pad, c.y0 + dy - pad, c.f, fb);
+                    mbar_expect_tx(smem_addr(&full[s]), 2 * (uint32_t)nk * (kABytes + bbytes));
+                for (int j = 0; j < nk; ++j) {
+                    const int kk = c.kb0 + kb + j, tap = kk / nchunk, ch = (kk - tap * nchunk) * kBK;
+                    if (g.temporal)
+                        tma_load_4d_pair(sa + j * kABytes, &amap, ch, c.x0, c.y0, c.f - (g.k - 1) + tap, fb);
+                    else {
+                        const int pad = (g.k - 1) / 2, dy = tap / g.k, dx = tap - dy * g.k;
+                        tma_load_4d_pair(sa + j * kABytes, &amap, ch, c.x0 + dx - pad, c.y0 + dy - pad, c.f, fb);
+                    }
+                    tma_load_2d_pair(sb + j * bbytes, &bmap, kk * kBK, c.n0 + (int)rank * (g.bn / 2), fb);
                 }
-                tma_load_2d_pair(sb, &bmap, kk * kBK, c.n0 + (int)rank * (g.bn / 2), fb);
             }
         }
         if (!ok && leader) // let the copies already issued land before the CTA exits (each wait bounded)
             for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
                 mbar_wait(smem_addr(&full[j % kStages]), (j / kStages) & 1u);
     } else if (warp == 1 && lane == 0 && leader) {
-        // MMA issue for the pair.
+        // MMA issue for the pair: one wait and one commit per stage of kStageK K blocks, ring
+        // positions and descriptors kept as running values (this thread is the narrowest point).
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
-        uint32_t it = 0, tc = 0;
+        const uint64_t adesc0 = sw128_desc(base), bdesc0 = sw128_desc(base + kStageK * kABytes);
+        uint32_t s = 0, ph = 0, tc = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
             const TileCoord c = decode_tile(g, i, 0);
@@ -254,19 +264,28 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
                 break;
             tc_fence_after();
             const uint32_t d = tmem + acc * (uint32_t)g.bn;
-            for (int kb = 0; kb < c.nkb; ++kb, ++it) {
-                const uint32_t s = it % kStages, ph = (it / kStages) & 1u;
+            for (int kb = 0; kb < c.nkb; kb += kStageK) {
                 if (!wait_or_abort(smem_addr(&full[s]), ph, abort)) {
                     ok = false;
                     break;
                 }
-                tc_fence_after();
-                const uint32_t sa = base + s * stage_bytes, sb = sa + kABytes;
-                const uint64_t ad = sw128_desc(sa), bd = sw128_desc(sb);
-#pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                const uint64_t a0 = adesc0 + ((s * stage_bytes) >> 4), b0 = bdesc0 + ((s * stage_bytes) >> 4);
+                umma_bf16_pair(d, a0, b0, idesc, kb != 0);
+                umma_bf16_pair(d, a0 + 2, b0 + 2, idesc, 1u);
+                umma_bf16_pair(d, a0 + 4, b0 + 4, idesc, 1u);
+                umma_bf16_pair(d, a0 + 6, b0 + 6, idesc, 1u);
+                if (kb + 1 < c.nkb) {
+                    const uint64_t a1 = a0 + (kABytes >> 4), b1 = b0 + (bbytes >> 4);
+                    umma_bf16_pair(d, a1, b1, idesc, 1u);
+                    umma_bf16_pair(d, a1 + 2, b1 + 2, idesc, 1u);
+                    umma_bf16_pair(d, a1 + 4, b1 + 4, idesc, 1u);
+                    umma_bf16_pair(d, a1 + 6, b1 + 6, idesc, 1u);
+                }
                 umma_commit_pair(smem_addr(&empty[s]), kPairMask);
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
             if (ok)
                 umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
@@ -290,8 +309,8 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
             tc_fence_after();
             const int y = c.y0 + r, x = c.x0 + jj;
             __nv_bfloat16 *o = out + (((int64_t)c.f * g.h + y) * g.w + x) * g.n + c.n0;
-            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage, stage_ptr, sbuf, o,
-                       y < g.h && x < g.w, g.bn);
+            store_tile<2>(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage, stage_ptr, sbuf, o,
+                          y < g.h && x < g.w, g.bn);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -316,25 +335,34 @@ conv_tc_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__
 // each 64-channel chunk c and column shift dx, one tensor copy brings the plane of
 // 16 + k - 1 rows x 8 columns (rows y0 - pad .., columns x0 + dx - pad ..) in the
 // 128-byte swizzle, and the k row shifts dy are that plane seen from row-atom dy (one
-// tile row of 8 positions is one 1024-byte swizzle atom).  K order (c, dx, dy); the
-// filter stages follow it.  Planes and filter stages are separate rings.
-constexpr int kPStages = 6;  // filter stages of the plane kernel
-constexpr int kPPlanes = 4;  // activation planes in flight
-constexpr int kMaxPlaneK = 7;
+// tile row of 8 positions is one 1024-byte swizzle atom).  K order (c, dx, dy).  A
+// stage holds one plane and the k filter K blocks it meets, so the MMA thread waits and
+// commits once per 4k MMAs: a single issuing thread pays for each barrier operation
+// (a wait or a commit costs it about as long as one or two MMAs), and at one wait and
+// one commit per K block it could not keep the 2-SM tensor core busy.
+constexpr int kMaxPStages = 3;
+constexpr int kMaxPlaneK = 5;
+constexpr int kPlaneEpiBuf = 1; // one staging buffer per epilogue warp (shared memory goes to the stages)
+
+__host__ __device__ constexpr uint32_t plane_stage_bytes(int bn, int k)
+{
+    return (uint32_t)(kTileRows + k - 1) * kTileCols * 128 + (uint32_t)k * (uint32_t)(bn / 2) * kBK * 2;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
                    const __grid_constant__ CUtensorMap omap, __nv_bfloat16 *__restrict__ out, const ConvGeom g)
 {
-    __shared__ __align__(8) uint64_t bfull[kPStages], bempty[kPStages], pfull[kPPlanes], pempty[kPPlanes], accf[2],
-        acce[2], drain;
+    __shared__ __align__(8) uint64_t full[kMaxPStages], empty[kMaxPStages], accf[2], acce[2], drain;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
+    const int nst = g.nstages;
     const uint32_t bbytes = (uint32_t)(g.bn / 2) * kBK * 2;
     const uint32_t plane_bytes = (uint32_t)(kTileRows + g.k - 1) * kTileCols * 128;
-    const uint32_t bbase = base, pbase = bbase + kPStages * bbytes, ebase = pbase + kPPlanes * plane_bytes;
+    const uint32_t stage_bytes = plane_stage_bytes(g.bn, g.k);
+    const uint32_t ebase = base + (uint32_t)nst * stage_bytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
@@ -343,13 +371,9 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
     const int nchunk = g.cin / kBK, pad = (g.k - 1) / 2;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kPStages; ++s) {
-            mbar_init(smem_addr(&bfull[s]), 1);
-            mbar_init(smem_addr(&bempty[s]), 1);
-        }
-        for (int p = 0; p < kPPlanes; ++p) {
-            mbar_init(smem_addr(&pfull[p]), 1);
-            mbar_init(smem_addr(&pempty[p]), 1);
+        for (int s = 0; s < nst; ++s) {
+            mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_addr(&accf[a]), 1);
@@ -370,44 +394,34 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
     volatile int *abort = &abort_s;
 
     if (warp == 0 && lane == 0) {
-        // Planes and filter stages of this CTA, counted on the leader's barriers.
-        uint32_t it = 0, pi = 0;
+        // Per stage: the plane and its k filter halves of this CTA, counted on the leader's barrier.
+        uint32_t it = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
             const TileCoord c = decode_tile(g, i, rank);
             for (int ch = 0; ch < nchunk && ok; ++ch)
-                for (int dx = 0; dx < g.k && ok; ++dx, ++pi) {
-                    const uint32_t slot = pi % kPPlanes;
-                    if (!wait_or_abort(smem_addr(&pempty[slot]), ((pi / kPPlanes) & 1u) ^ 1u, abort)) {
+                for (int dx = 0; dx < g.k; ++dx, ++it) {
+                    const uint32_t s = it % nst, ph = (it / nst) & 1u;
+                    if (!wait_or_abort(smem_addr(&empty[s]), ph ^ 1u, abort)) {
                         ok = false;
                         break;
                     }
+                    const uint32_t sa = base + s * stage_bytes, sb = sa + plane_bytes;
+                    const uint32_t fb = mapa_shared(smem_addr(&full[s]), 0);
                     if (leader)
-                        mbar_expect_tx(smem_addr(&pfull[slot]), 2 * plane_bytes);
-                    tma_load_4d_pair(pbase + slot * plane_bytes, &amap, ch * kBK, c.x0 + dx - pad, c.y0 - pad, c.f,
-                                     mapa_shared(smem_addr(&pfull[slot]), 0));
-                    for (int dy = 0; dy < g.k; ++dy, ++it) {
-                        const uint32_t s = it % kPStages, ph = (it / kPStages) & 1u;
-                        if (!wait_or_abort(smem_addr(&bempty[s]), ph ^ 1u, abort)) {
-                            ok = false;
-                            break;
-                        }
-                        if (leader)
-                            mbar_expect_tx(smem_addr(&bfull[s]), 2 * bbytes);
-                        tma_load_2d_pair(bbase + s * bbytes, &bmap, (dy * g.k + dx) * g.cin + ch * kBK,
-                                         c.n0 + (int)rank * (g.bn / 2), mapa_shared(smem_addr(&bfull[s]), 0));
-                    }
+                        mbar_expect_tx(smem_addr(&full[s]), 2 * stage_bytes);
+                    tma_load_4d_pair(sa, &amap, ch * kBK, c.x0 + dx - pad, c.y0 - pad, c.f, fb);
+                    for (int dy = 0; dy < g.k; ++dy)
+                        tma_load_2d_pair(sb + dy * bbytes, &bmap, (dy * g.k + dx) * g.cin + ch * kBK,
+                                         c.n0 + (int)rank * (g.bn / 2), fb);
                 }
         }
-        if (!ok && leader) {
-            for (uint32_t j = it > kPStages ? it - kPStages : 0; j < it; ++j)
-                mbar_wait(smem_addr(&bfull[j % kPStages]), (j / kPStages) & 1u);
-            for (uint32_t j = pi > kPPlanes ? pi - kPPlanes : 0; j < pi; ++j)
-                mbar_wait(smem_addr(&pfull[j % kPPlanes]), (j / kPPlanes) & 1u);
-        }
+        if (!ok && leader)
+            for (uint32_t j = it > (uint32_t)nst ? it - nst : 0; j < it; ++j)
+                mbar_wait(smem_addr(&full[j % nst]), (j / nst) & 1u);
     } else if (warp == 1 && lane == 0 && leader) {
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
-        uint32_t it = 0, pi = 0, tc = 0;
+        uint32_t it = 0, tc = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
             const uint32_t acc = tc & 1u, use = tc >> 1;
@@ -415,28 +429,20 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
                 break;
             tc_fence_after();
             const uint32_t d = tmem + acc * (uint32_t)g.bn;
-            for (int pl = 0; pl < nchunk * g.k && ok; ++pl, ++pi) {
-                const uint32_t slot = pi % kPPlanes;
-                if (!wait_or_abort(smem_addr(&pfull[slot]), (pi / kPPlanes) & 1u, abort)) {
+            for (int pl = 0; pl < nchunk * g.k; ++pl, ++it) {
+                const uint32_t s = it % nst, ph = (it / nst) & 1u;
+                if (!wait_or_abort(smem_addr(&full[s]), ph, abort)) {
                     ok = false;
                     break;
                 }
-                for (int dy = 0; dy < g.k; ++dy, ++it) {
-                    const uint32_t s = it % kPStages, ph = (it / kPStages) & 1u;
-                    if (!wait_or_abort(smem_addr(&bfull[s]), ph, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t ad = sw128_desc(pbase + slot * plane_bytes + (uint32_t)dy * 1024u);
-                    const uint64_t bd = sw128_desc(bbase + s * bbytes);
+                const uint32_t sa = base + s * stage_bytes, sb = sa + plane_bytes;
+                for (int dy = 0; dy < g.k; ++dy) {
+                    const uint64_t ad = sw128_desc(sa + (uint32_t)dy * 1024u), bd = sw128_desc(sb + dy * bbytes);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k)
                         umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
-                    umma_commit_pair(smem_addr(&bempty[s]), kPairMask);
                 }
-                if (ok)
-                    umma_commit_pair(smem_addr(&pempty[slot]), kPairMask);
+                umma_commit_pair(smem_addr(&empty[s]), kPairMask);
             }
             if (ok)
                 umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
@@ -447,7 +453,7 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
         const int q = warp & 3, row = 32 * q + lane;
         const int r = row / kTileCols, jj = row - r * kTileCols;
         const uint32_t acce0 = mapa_shared(smem_addr(&acce[0]), 0), acce1 = mapa_shared(smem_addr(&acce[1]), 0);
-        const uint32_t stage = ebase + (uint32_t)q * 8192u;
+        const uint32_t stage = ebase + (uint32_t)q * (kPlaneEpiBuf * 4096u);
         unsigned char *stage_ptr = smem_raw + (stage - smem_addr(smem_raw));
         uint32_t tc = 0, sbuf = 0;
         for (int i = pair; i < g.npairs; i += npair_ctas, ++tc) {
@@ -458,8 +464,8 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
             tc_fence_after();
             const int y = c.y0 + r, x = c.x0 + jj;
             __nv_bfloat16 *o = out + (((int64_t)c.f * g.h + y) * g.w + x) * g.n + c.n0;
-            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage, stage_ptr, sbuf, o,
-                       y < g.h && x < g.w, g.bn);
+            store_tile<kPlaneEpiBuf>(tmem + acc * (uint32_t)g.bn, q, lane, &omap, c.f, c.y0, c.x0, c.n0, stage,
+                                     stage_ptr, sbuf, o, y < g.h && x < g.w, g.bn);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -480,15 +486,23 @@ conv_planes_kernel(const __grid_constant__ CUtensorMap amap, const __grid_consta
         atomicAdd(&g_conv_timeouts, 1u);
 }
 
-size_t planes_smem_bytes(int bn, int k)
+// Stages of the plane kernel that fit (with the epilogue staging and the alignment slack) in
+// the 227 KB of shared memory a CTA may have; 0 if fewer than two fit.
+int plane_stages(int bn, int k)
 {
-    return (size_t)kPStages * (bn / 2) * kBK * 2 + (size_t)kPPlanes * (kTileRows + k - 1) * kTileCols * 128 +
-           kEpiBytes + 1024;
+    const int64_t room = 232448 - 1024 - 1024 - (int64_t)epi_bytes(kPlaneEpiBuf); // static barriers and slack
+    const int n = (int)std::min<int64_t>(kMaxPStages, room / plane_stage_bytes(bn, k));
+    return n >= 2 ? n : 0;
+}
+
+size_t planes_smem_bytes(int bn, int k, int nst)
+{
+    return (size_t)nst * plane_stage_bytes(bn, k) + epi_bytes(kPlaneEpiBuf) + 1024;
 }
 
 size_t conv_smem_bytes(int bn)
 {
-    return (size_t)kStages * (kABytes + (uint32_t)(bn / 2) * kBK * 2) + kEpiBytes + 1024;
+    return (size_t)kStages * kStageK * (kABytes + (uint32_t)(bn / 2) * kBK * 2) + epi_bytes(2) + 1024;
 }
 
 bool fits_int(int64_t v) { return v >= 0 && v < ((int64_t)1 << 31); }
@@ -576,15 +590,15 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
     const uint64_t odims[4] = {(uint64_t)Cout, (uint64_t)w, (uint64_t)h, (uint64_t)g.frames};
     const uint64_t ostr[3] = {(uint64_t)Cout * 2, (uint64_t)w * Cout * 2, (uint64_t)h * w * Cout * 2};
     const uint32_t obox[4] = {(uint32_t)std::min<int64_t>(64, Cout), kTileCols, 4, 1};
-    const bool planes = !temporal && k <= kMaxPlaneK;
-    if (planes) {
+    g.nstages = temporal || k > kMaxPlaneK ? 0 : plane_stages(g.bn, (int)k);
+    if (g.nstages) {
         const uint32_t pbox[4] = {kBK, kTileCols, (uint32_t)(kTileRows + k - 1), 1};
         if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, pbox) ||
             !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox) ||
             !encode_tensor_map_sw128(&omap, 4, y, odims, ostr, obox))
             return TOK_ERR_SHAPE;
-        return launch_pairs(conv_planes_kernel, npairs, planes_smem_bytes(g.bn, (int)k), kThreads, stream, amap, bmap,
-                            omap, static_cast<__nv_bfloat16 *>(y), g);
+        return launch_pairs(conv_planes_kernel, npairs, planes_smem_bytes(g.bn, (int)k, g.nstages), kThreads, stream,
+                            amap, bmap, omap, static_cast<__nv_bfloat16 *>(y), g);
     }
     if (!encode_tensor_map_sw128(&amap, 4, x, adims, astr, abox) ||
         !encode_tensor_map_sw128(&bmap, 2, wts, bdims, bstr, bbox) ||
@@ -603,7 +617,7 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
 // 128-byte swizzled row per position (row q = r * 8 + j: one tile row is one 1024-byte
 // swizzle atom), and the three K steps dy = 0, 1, 2 are that plane seen from atom dy.
 // The filter is read in the same K order from a packed copy (tok_patch_embed_pack_weights).
-//   warp 0     tensor copies of the packed filter, kFStages stages of [64 k, N];
+//   warp 0     tensor copies of the packed filter, kFStages stages of [64 k, N / 2];
 //   warp 1     MMA issue (planes and filter stages as they fill);
 //   warps 2-5  epilogue, as in conv_tc_kernel;
 //   warps 6-9  Haar: per colour, one tensor copy of the pixels the tile's 3 x 3
@@ -616,7 +630,8 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
 // Latent positions outside the frame read zero pixels (the tensor copy fills zeros),
 // which is exactly the convolution's zero padding of the coefficients.
 // ---------------------------------------------------------------------------
-constexpr int kFStages = 3;                      // filter stages
+constexpr int kFStages = 3;                      // filter stages of one K block
+constexpr int kEmbedEpiBuf = 2;                  // staging buffers per epilogue warp
 constexpr int kPlanes = 5;                       // A planes in flight (a ring)
 constexpr int kPlaneRows = kTileRows + 2;        // latent rows of a plane
 constexpr uint32_t kPlaneBytes = kPlaneRows * kTileCols * 128; // 18 KB
@@ -690,7 +705,7 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
-    const uint32_t fbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of a filter stage
+    const uint32_t fbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of a filter K block
     const uint32_t fbase = base, pbase = fbase + kFStages * fbytes, xbase = pbase + kPlanes * kPlaneBytes;
     const uint32_t ebase = xbase + 2 * kPixBytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -730,13 +745,13 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
     volatile int *abort = &abort_s;
 
     if (warp == 0 && lane == 0) {
-        // This CTA's half of the filter, in the tile's K order; counted on the leader's barrier.
-        uint32_t it = 0;
+        // This CTA's half of the filter, one K block per stage in the tile's K order; counted on
+        // the leader's barrier.
+        uint32_t s = 0, ph = 0, issued = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
             const EmbedTile e = decode_embed(g, i, rank);
-            for (int kb = 0; kb < kper; ++kb, ++it) {
-                const uint32_t s = it % kFStages, ph = (it / kFStages) & 1u;
+            for (int kb = 0; kb < kper; ++kb) {
                 if (!wait_or_abort(smem_addr(&fempty[s]), ph ^ 1u, abort)) {
                     ok = false;
                     break;
@@ -745,15 +760,24 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                     mbar_expect_tx(smem_addr(&ffull[s]), 2 * fbytes);
                 tma_load_2d_pair(fbase + s * fbytes, &bmap, kb * kBK, e.n0 + (int)rank * (g.bn / 2),
                                  mapa_shared(smem_addr(&ffull[s]), 0));
+                ++issued;
+                if (++s == kFStages) {
+                    s = 0;
+                    ph ^= 1u;
+                }
             }
         }
         if (!ok && leader)
-            for (uint32_t j = it > kFStages ? it - kFStages : 0; j < it; ++j)
+            for (uint32_t j = issued > kFStages ? issued - kFStages : 0; j < issued; ++j)
                 mbar_wait(smem_addr(&ffull[j % kFStages]), (j / kFStages) & 1u);
     } else if (warp == 1 && lane == 0 && leader) {
-        // MMA issue for the pair: per plane (c, dx), the three row shifts dy.
+        // MMA issue for the pair.  This single thread is the pipeline's narrowest point (each
+        // barrier test or commit costs it about as long as an MMA), so the loop keeps its ring
+        // positions and descriptors as running values: per plane (c, dx) one wait and one commit,
+        // per row shift dy one filter stage.
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
-        uint32_t it = 0, pi = 0, tc = 0;
+        const uint64_t adesc0 = sw128_desc(pbase), bdesc0 = sw128_desc(fbase);
+        uint32_t fs = 0, fph = 0, ps = 0, pph = 0, tc = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas, ++tc) {
             const uint32_t acc = tc & 1u, use = tc >> 1;
@@ -761,28 +785,36 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                 break;
             tc_fence_after();
             const uint32_t d = tmem + acc * (uint32_t)g.bn;
-            for (int pl = 0; pl < 3 * g.C && ok; ++pl, ++pi) {
-                const uint32_t slot = pi % kPlanes;
-                if (!wait_or_abort(smem_addr(&pfull[slot]), (pi / kPlanes) & 1u, abort)) {
+            for (int pl = 0; pl < 3 * g.C && ok; ++pl) {
+                if (!wait_or_abort(smem_addr(&pfull[ps]), pph, abort)) {
                     ok = false;
                     break;
                 }
-                for (int dy = 0; dy < 3; ++dy, ++it) {
-                    const uint32_t s = it % kFStages, ph = (it / kFStages) & 1u;
-                    if (!wait_or_abort(smem_addr(&ffull[s]), ph, abort)) {
+                const uint64_t ad = adesc0 + ((ps * kPlaneBytes) >> 4);
+#pragma unroll
+                for (int dy = 0; dy < 3; ++dy) {
+                    if (!wait_or_abort(smem_addr(&ffull[fs]), fph, abort)) {
                         ok = false;
                         break;
                     }
-                    tc_fence_after();
-                    const uint64_t ad = sw128_desc(pbase + slot * kPlaneBytes + (uint32_t)dy * 1024u);
-                    const uint64_t bd = sw128_desc(fbase + s * fbytes);
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (pl | dy | k) != 0);
-                    umma_commit_pair(smem_addr(&fempty[s]), kPairMask);
+                    const uint64_t a = ad + (uint64_t)(dy * 64), b = bdesc0 + ((fs * fbytes) >> 4);
+                    umma_bf16_pair(d, a, b, idesc, (pl | dy) != 0);
+                    umma_bf16_pair(d, a + 2, b + 2, idesc, 1u);
+                    umma_bf16_pair(d, a + 4, b + 4, idesc, 1u);
+                    umma_bf16_pair(d, a + 6, b + 6, idesc, 1u);
+                    umma_commit_pair(smem_addr(&fempty[fs]), kPairMask);
+                    if (++fs == kFStages) {
+                        fs = 0;
+                        fph ^= 1u;
+                    }
                 }
-                if (ok)
-                    umma_commit_pair(smem_addr(&pempty[slot]), kPairMask);
+                if (!ok)
+                    break;
+                umma_commit_pair(smem_addr(&pempty[ps]), kPairMask);
+                if (++ps == kPlanes) {
+                    ps = 0;
+                    pph ^= 1u;
+                }
             }
             if (ok)
                 umma_commit_pair(smem_addr(&accf[acc]), kPairMask);
@@ -794,7 +826,7 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
         const int q = warp & 3, row = 32 * q + lane;
         const int r = row / kTileCols, jj = row - r * kTileCols;
         const uint32_t acce0 = mapa_shared(smem_addr(&acce[0]), 0), acce1 = mapa_shared(smem_addr(&acce[1]), 0);
-        const uint32_t stage = ebase + (uint32_t)q * 8192u;
+        const uint32_t stage = ebase + (uint32_t)q * (kEmbedEpiBuf * 4096u);
         unsigned char *stage_ptr = smem_raw + (stage - smem_addr(smem_raw));
         uint32_t tc = 0, sbuf = 0;
         for (int i = pair; i < g.npairs; i += npair_ctas, ++tc) {
@@ -805,8 +837,8 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
             tc_fence_after();
             const int y = e.y0 + r, x = e.x0 + jj, f = e.b * g.Tq + e.tq;
             __nv_bfloat16 *o = out + (((int64_t)f * g.h + y) * g.w + x) * g.n + e.n0;
-            store_tile(tmem + acc * (uint32_t)g.bn, q, lane, &omap, f, e.y0, e.x0, e.n0, stage, stage_ptr, sbuf, o,
-                       y < g.h && x < g.w, g.bn);
+            store_tile<kEmbedEpiBuf>(tmem + acc * (uint32_t)g.bn, q, lane, &omap, f, e.y0, e.x0, e.n0, stage,
+                                     stage_ptr, sbuf, o, y < g.h && x < g.w, g.bn);
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -945,8 +977,8 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
 
 size_t embed_smem_bytes(int bn)
 {
-    return (size_t)kFStages * (bn / 2) * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes + kEpiBytes +
-           1024;
+    return (size_t)kFStages * (bn / 2) * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes +
+           epi_bytes(kEmbedEpiBuf) + 1024;
 }
 
 // Packed filter: wp[n][(c * 3 + dx) * 3 + dy][g] = ws[n][dy][dx][g * C + c].
