@@ -30,22 +30,6 @@ def _nvcc():
     return "nvcc"
 
 
-# Files whose kernels come from CUTLASS's sm100 templates (header-only, vendored in the image).
-CUTLASS_SOURCES = ("conv.cu",)
-
-
-def cutlass_includes():
-    """Include directories of the CUTLASS tree vendored with flashinfer in this image."""
-    import importlib.util
-    spec = importlib.util.find_spec("flashinfer")
-    roots = [os.path.join(os.path.dirname(spec.origin), "data", "cutlass")] if spec and spec.origin else []
-    for root in roots:
-        inc, util = os.path.join(root, "include"), os.path.join(root, "tools", "util", "include")
-        if os.path.exists(os.path.join(inc, "cutlass", "conv", "collective", "builders", "sm100_umma_builder.inl")):
-            return [inc, util]
-    raise RuntimeError("CUTLASS headers with the sm100 convolution builders were not found")
-
-
 _INCLUDE_RE = re.compile(r'^\s*#\s*include\s*"([^"]+)"', re.M)
 
 
@@ -77,10 +61,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
                 os.path.getmtime(obj) >= max(os.path.getmtime(d) for d in deps):
             continue
         cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
-        if os.path.basename(src) in CUTLASS_SOURCES:
-            for inc in cutlass_includes():
-                cmd += ["-I", inc]
-            cmd += ["-diag-suppress", "20012"]  # CUTLASS's defaulted host-device constructors
         if verbose:
             cmd.insert(1, "-Xptxas=-v")
         subprocess.run(cmd, check=True)

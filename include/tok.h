@@ -285,8 +285,10 @@ TOK_API tok_status tok_haar_inv_chunk(const void *y, void *x, tok_dtype dt, int6
  * architecture item 1: a 1 x k x k spatial convolution, then a k x 1 x 1 temporal
  * convolution padded by k - 1 on the past side only), on the tensor cores:
  * channels-last bf16 activations, bf16 weights, fp32 accumulation, bf16 results.
- * Cross-correlation (no kernel flip), no bias.  Channel counts are multiples of 8
- * (at least 8); all pointers are 16-byte aligned device memory.  Errors:
+ * Cross-correlation (no kernel flip), no bias.  Cin (and Cmid, the temporal
+ * convolution's input) is a positive multiple of 64; Cout (and Cmid, the spatial
+ * convolution's output) is a multiple of 32, at most 256 or a multiple of 256;
+ * k <= 15; all pointers are 16-byte aligned device memory.  Errors:
  * TOK_ERR_SHAPE (channels, k, or 32-bit extents), TOK_ERR_NULL, TOK_ERR_ALIGN,
  * TOK_ERR_ALIAS (an input overlaps the output), TOK_ERR_CUDA.  Not on the pages'
  * API: the layer the pages name, with weights the caller provides.

@@ -216,14 +216,17 @@ def test_channels_last_rules(lib):
 def test_conv_rules(lib):
     sp, tp, fz = lib.tok_conv_spatial, lib.tok_conv_temporal_causal, lib.tok_conv_factorized
     X, Wg, Y, M = F(0x100000), F(0x200000), F(0x300000), F(0x400000)
-    assert sp(X, Wg, Y, 1, 2, 8, 8, 12, 16, 3, NULL) == hwp.TOK_ERR_SHAPE    # Cin not a multiple of 8
-    assert sp(X, Wg, Y, 1, 2, 8, 8, 16, 16, 2, NULL) == hwp.TOK_ERR_SHAPE    # even spatial k
-    assert tp(X, Wg, Y, 1, 2, 8, 8, 16, 16, 0, NULL) == hwp.TOK_ERR_SHAPE
-    assert sp(NULL, Wg, Y, 1, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_ERR_NULL
-    assert sp(F(0x100008), Wg, Y, 1, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_ERR_ALIGN
-    assert sp(X, Wg, X, 1, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_ERR_ALIAS
-    assert fz(X, Wg, Wg, M, X, 1, 2, 8, 8, 16, 16, 16, 3, NULL) == hwp.TOK_ERR_ALIAS
-    assert sp(NULL, NULL, NULL, 0, 2, 8, 8, 16, 16, 3, NULL) == hwp.TOK_OK     # empty
+    assert sp(X, Wg, Y, 1, 2, 8, 8, 32, 64, 3, NULL) == hwp.TOK_ERR_SHAPE    # Cin not a multiple of 64
+    assert sp(X, Wg, Y, 1, 2, 8, 8, 64, 48, 3, NULL) == hwp.TOK_ERR_SHAPE    # Cout not a multiple of 32
+    assert tp(X, Wg, Y, 1, 2, 8, 8, 64, 288, 3, NULL) == hwp.TOK_ERR_SHAPE   # above 256, not a multiple of 256
+    assert sp(X, Wg, Y, 1, 2, 8, 8, 64, 64, 2, NULL) == hwp.TOK_ERR_SHAPE    # even spatial k
+    assert tp(X, Wg, Y, 1, 2, 8, 8, 64, 64, 0, NULL) == hwp.TOK_ERR_SHAPE
+    assert fz(X, Wg, Wg, M, Y, 1, 2, 8, 8, 64, 96, 64, 3, NULL) == hwp.TOK_ERR_SHAPE  # Cmid feeds a Cin
+    assert sp(NULL, Wg, Y, 1, 2, 8, 8, 64, 64, 3, NULL) == hwp.TOK_ERR_NULL
+    assert sp(F(0x100008), Wg, Y, 1, 2, 8, 8, 64, 64, 3, NULL) == hwp.TOK_ERR_ALIGN
+    assert sp(X, Wg, X, 1, 2, 8, 8, 64, 64, 3, NULL) == hwp.TOK_ERR_ALIAS
+    assert fz(X, Wg, Wg, M, X, 1, 2, 8, 8, 64, 64, 64, 3, NULL) == hwp.TOK_ERR_ALIAS
+    assert sp(NULL, NULL, NULL, 0, 2, 8, 8, 64, 64, 3, NULL) == hwp.TOK_OK     # empty
 
 
 def test_patch_embed_rules(lib):
