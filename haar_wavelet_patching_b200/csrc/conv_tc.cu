@@ -11,18 +11,22 @@
 // 256 output positions -- two tiles of 16 rows x 8 columns of one frame, one per
 // CTA -- by up to 256 output channels, M = 256 and N = 256, each CTA loading its own
 // tile's activations and half of the filter, so the filter crosses L2 half as often
-// per flop as with one-CTA 128 x 256 tiles.  Each K step is 64 input channels of one
-// tap.  The pair walks its tiles persistently.  Warp roles in each CTA:
-//   warp 0     tensor copies: per K step, the activation box [64 ch, 8 cols,
+// per flop as with one-CTA 128 x 256 tiles.  Each K block is 64 input channels of one
+// tap, and a stage holds kStageK of them.  The pair walks its tiles persistently.
+// Warp roles in each CTA:
+//   warp 0     tensor copies: per K block, the activation box [64 ch, 8 cols,
 //              16 rows] of the tap's frame / shift (zero-filled outside the frame)
 //              and its half of the filter box [64 k, N / 2], into one of kStages
 //              stages in the 128-byte swizzle the MMA reads; completion is counted
 //              on the leader CTA's barrier;
-//   warp 1     (leader only) one thread issues tcgen05.mma (4 per K step, K = 16
-//              each) into the pair's tensor-memory accumulator and commits each stage
-//              back to both CTAs' copy warps;
+//   warp 1     (leader only) one thread issues tcgen05.mma (4 per K block, K = 16
+//              each) into the pair's tensor-memory accumulator, waiting and
+//              committing once per stage (each barrier operation costs this thread
+//              about as long as one or two MMAs), the commit releasing the stage to
+//              both CTAs' copy warps;
 //   warps 2-5  epilogue: tensor memory -> registers (each thread one position, its
-//              lane of this CTA's accumulator half), round to bf16, 16-byte stores.
+//              lane of this CTA's accumulator half), round to bf16, through a
+//              128-byte-swizzled staging buffer to tensor stores of whole lines.
 // Two accumulators in tensor memory (2 x N columns) let a tile's epilogue overlap
 // the next tile's MMAs.  The temporal convolution orders tiles time-fastest, so the
 // k frames a tile reads are read again by the next tiles while they are in L2; the

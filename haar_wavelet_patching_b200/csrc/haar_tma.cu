@@ -32,6 +32,7 @@
 // tok_check_device() reports.  Every load fills only this CTA's own shared memory.
 #include <cstring>
 #include <numeric>
+#include <type_traits>
 
 #include "tma.cuh"
 #include "tok_common.cuh"
@@ -45,6 +46,7 @@ static __device__ unsigned int g_wait_timeouts = 0;
 namespace {
 
 constexpr int kTileBlocks = 64; // blocks across a warp tile (256 pixels)
+constexpr int kGroupSalign = 16; // grouped rows: largest tile shift unit (16 bf16 = one 32-byte sector)
 constexpr int kTileElems = 4096; // elements of a warp tile, on either side
 
 template <typename T> struct WarpTiles {
@@ -71,6 +73,9 @@ struct TileGrid {
     // Inverse, row form: the plane stride is a multiple of 16 bytes, so the staged rows of one
     // block row (one per group) all sit at the same offset in their staged copies.
     int planes_share_offset;
+    // Inverse with run-time store widths: the widest store (bytes, up to 16) that every pixel
+    // row of the call allows (the destination's alignment and W elements' bytes).
+    int sw;
 };
 
 // Source frame of frame f of a T-frame clip mirrored about its last frame (period 2(T-1)).
@@ -180,17 +185,18 @@ __device__ __forceinline__ void gstore_row(float *p, const float2 *v)
 // (the issuing lane copies a last partial 16 bytes element by element).  Stores pick
 // their width from the destination address at run time.
 // ---------------------------------------------------------------------------
-template <typename T, bool FWD, bool ROWS> struct TileSmem {
+template <typename T, bool FWD, bool ROWS, int GR = 0> struct TileSmem {
     // The row form spends more instructions per tile (row offsets, realigned reads, stores of
     // run-time width), so it trades tiles per CTA for resident warps: ~17 KB per CTA.
     static constexpr int KT = !ROWS ? WarpTiles<T>::KT : sizeof(T) == 2 ? 2 : 1;
     static constexpr int NR = FWD ? 16 : 64;                              // staged rows of a tile
     static constexpr int ROW = (FWD ? 256 : 64) * (int)sizeof(T) + 16;     // a source row and its slack
-    static constexpr int TILE = ROWS ? NR * ROW : kTileElems * (int)sizeof(T);
+    // Grouped rows (GR > 0): the 16 pixel rows' 256-element boxes, then 128 bytes of tail slots
+    // per part (16 bytes per pixel row, in the order of the part's box rows).
+    static constexpr int TILE = ROWS ? NR * ROW : kTileElems * (int)sizeof(T) + GR * 128;
     static constexpr int SMEM = KT * TILE + 8 * KT + (ROWS ? 64 * KT : 0); // tiles, barriers, row offsets
     static_assert(ROW % 16 == 0 && TILE % 16 == 0, "16-byte bulk-copy destinations");
 };
-constexpr unsigned char kRowSkipped = 0xFF; // a staged row that was not loaded (past the tensor edge)
 
 // Realigned reads from a 16-byte-aligned staged row, without branches, so the rows of a
 // tile are scheduled together: aligned 8- or 4-byte loads from at or below the offset,
@@ -242,6 +248,35 @@ __device__ __forceinline__ float2 staged_pair(const unsigned char *row, uint32_t
 {
     const float *w = reinterpret_cast<const float *>(row + o); // o is a multiple of 4
     return make_float2(w[0], w[1]);
+}
+
+// ---------------------------------------------------------------------------
+// Grouped-row form (bf16 video forward, W % 8 == 4, odd w).  A pixel row of W elements is
+// not a whole number of 16-byte units, but GR = 2 of them are, so the tensor maps view each
+// frame as [H / 2][2 W]: row y of the clip is part p = y % 2 of group row y / 2.  A tile
+// takes one tensor box per part, [frames][its two rows of that part][256 elements], from the
+// 16-byte boundary at or below the part's first pixel, and, for the part that does not start
+// on the boundary (2 W = 8 mod 16 bytes: exactly one of the two), a tail box of the 8
+// elements that follow it (16 bytes per pixel row).  A window that runs past the clip takes
+// its frames one by one and its tails by one 16-byte bulk copy per pixel row.  The odd w is
+// what makes this form pay: tiles may then start one block left of a pair boundary
+// (TileGrid::salign), which keeps every coefficient-pair store aligned, where the row form
+// falls back to element stores on every other block row.  (With an even w the row form,
+// which keeps twice as many warps resident, measured faster.)
+// ---------------------------------------------------------------------------
+
+// Eight elements (blocks j, j+1 of one pixel row) at byte offset o (a multiple of 8) of a
+// 512-byte box row m whose next 16 bytes are in the tail slot t -> four pairs, as SRow::load.
+// Only lane 31 reaches the tail.
+__device__ __forceinline__ void grouped_row8(const unsigned char *m, const unsigned char *t, uint32_t o, float2 *v)
+{
+    const uint2 lo = *reinterpret_cast<const uint2 *>(m + o);
+    const uint32_t o2 = o + 8;
+    const uint2 hi = *reinterpret_cast<const uint2 *>(o2 < 512 ? m + o2 : t + (o2 - 512));
+    v[0] = make_float2(bf16_lo(lo.x), bf16_lo(hi.x));
+    v[1] = make_float2(bf16_hi(lo.x), bf16_hi(hi.x));
+    v[2] = make_float2(bf16_lo(lo.y), bf16_lo(hi.y));
+    v[3] = make_float2(bf16_hi(lo.y), bf16_hi(hi.y));
 }
 
 // A pixel-row store whose alignment is known only at run time (the destination's rows are
@@ -307,6 +342,48 @@ template <bool ROWS, typename T> __device__ __forceinline__ void store_pixel_row
     }
 }
 
+// One pixel row of blocks j, j+1 in stores of SW bytes, SW a width every row of the call allows
+// (TileGrid::sw): no test of the address.
+template <int SW> __device__ __forceinline__ void store_row_width(__nv_bfloat16 *p, const float2 *v)
+{
+    const uint32_t w[4] = {pack_bf16x2(v[0].x, v[1].x), pack_bf16x2(v[2].x, v[3].x), pack_bf16x2(v[0].y, v[1].y),
+                           pack_bf16x2(v[2].y, v[3].y)};
+    if constexpr (SW >= 16) {
+        *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    } else if constexpr (SW == 8) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(w[0], w[1]);
+        *reinterpret_cast<uint2 *>(p + 4) = make_uint2(w[2], w[3]);
+    } else if constexpr (SW == 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            reinterpret_cast<uint32_t *>(p)[k] = w[k];
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            reinterpret_cast<unsigned short *>(p)[2 * k] = (unsigned short)(w[k] & 0xFFFFu);
+            reinterpret_cast<unsigned short *>(p)[2 * k + 1] = (unsigned short)(w[k] >> 16);
+        }
+    }
+}
+template <int SW> __device__ __forceinline__ void store_row_width(float *p, const float2 *v)
+{
+    if constexpr (SW >= 16) {
+        gstore_row(p, v);
+    } else if constexpr (SW == 8) {
+#pragma unroll
+        for (int k = 0; k < 4; k += 2) {
+            *reinterpret_cast<float2 *>(p + k) = make_float2(v[k].x, v[k + 1].x);
+            *reinterpret_cast<float2 *>(p + 4 + k) = make_float2(v[k].y, v[k + 1].y);
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            p[k] = v[k].x;
+            p[4 + k] = v[k].y;
+        }
+    }
+}
+
 // Video: one block row (tile rows = 1); images: four block rows, done one after another.
 template <bool VIDEO> struct TileRows {
     static constexpr int RW = VIDEO ? 1 : 4;
@@ -321,16 +398,20 @@ template <bool VIDEO> struct TileRows {
 // stores of any alignment, w may be odd); it reads the source through `src` (tg.n_src
 // elements) instead of the tensor maps.  ANYST (inverse, box form): the source takes the box
 // form but the pixel rows are not whole 16-byte units, so their stores take the row form's
-// run-time widths.
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false>
+// run-time widths.  GR = 2 (bf16 video forward): the grouped-row form above; its tiles may start one
+// block left of a pair boundary (TileGrid::salign with an odd w), so a lane's pair can
+// straddle column 0 or the last column, and such a lane stores its one block alone.
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false, int GR = 0>
 __global__ void __launch_bounds__(32)
     haar_tma_kernel(const __grid_constant__ CUtensorMap xmap4, const __grid_constant__ CUtensorMap xmap1,
-                    const __grid_constant__ CUtensorMap ymap, const T *__restrict__ src, T *__restrict__ out,
+                    const __grid_constant__ CUtensorMap ymap, const __grid_constant__ CUtensorMap xtail4,
+                    const __grid_constant__ CUtensorMap xtail1, const T *__restrict__ src, T *__restrict__ out,
                     const TileGrid tg)
 {
     static_assert(!(EXT && ADJ), "the adjoints take the plain form");
     static_assert(!(ANYST && (FWD || ROWS)), "ANYST: the inverse's box form only");
-    using P = TileSmem<T, FWD, ROWS>;
+    static_assert(GR == 0 || (GR == 2 && VIDEO && FWD && !ROWS && sizeof(T) == 2), "grouped rows: bf16 video forward");
+    using P = TileSmem<T, FWD, ROWS, GR>;
     constexpr int KT = P::KT, WT = kTileBlocks;
     constexpr int RW = TileRows<VIDEO>::RW;
     constexpr int G = VIDEO ? 64 : 16;  // channel groups
@@ -383,7 +464,7 @@ __global__ void __launch_bounds__(32)
             const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0);
             int64_t start[PER]; // byte offset of each staged row in the source (16-byte aligned)
             uint32_t nbulk[PER];
-            bool ok[PER];
+            bool ok[PER], zero[PER]; // zero: a row past the clip's last row that the transform reads
             uint32_t tx_bytes = 0;
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
@@ -400,6 +481,7 @@ __global__ void __launch_bounds__(32)
                     else if (VIDEO)
                         f = EXT ? mirror_frame(4 * tq + tg.fbase + a, tg.T) : 4 * tq - 3 + a;
                     ok[k] = loaded;
+                    zero[k] = EXT && r < P::NR && y >= tg.H && !(VIDEO && replica && a != 0);
                     off = ((bc * tg.T + f) * tg.H + y) * tg.W + (int64_t)4 * WT * tx;
                 } else {
                     // Staged row r: group r / RW, block row RW ty + r % RW.
@@ -408,6 +490,7 @@ __global__ void __launch_bounds__(32)
                     const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
                     const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
                     ok[k] = row < tg.h;
+                    zero[k] = false;
                     off = ((b * G + g) * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + (int64_t)WT * tx;
                 }
                 const int mis = (int)(off % VE);
@@ -416,12 +499,11 @@ __global__ void __launch_bounds__(32)
                 // before the tensor's end (a valid row starts before the end).
                 const int64_t avail = tg.n_src * (int64_t)sizeof(T) - start[k];
                 nbulk[k] = !ok[k] ? 0u : avail >= P::ROW ? (uint32_t)P::ROW : (uint32_t)(avail & ~(int64_t)15);
-                // A row that is not loaded reads as zeros where its values are used (rows past the
-                // clip's last row on the padded forward); elsewhere its results are never stored
-                // and it is read at offset 0 of its (stale) staging row.
+                // A row that is not loaded is staged as zeros where its values are used (rows past
+                // the clip's last row on the padded forward); elsewhere its results are never
+                // stored and it is read at offset 0 of its (stale) staging row.
                 if (r < P::NR)
-                    row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T))
-                                                : FWD && EXT ? kRowSkipped : (unsigned char)0;
+                    row_off[s * 64 + r] = ok[k] ? (unsigned char)(mis * (int)sizeof(T)) : (unsigned char)0;
                 tx_bytes += __reduce_add_sync(0xFFFFFFFFu, nbulk[k]);
             }
             const uint32_t bar = smem_addr(bars + s);
@@ -432,9 +514,13 @@ __global__ void __launch_bounds__(32)
             const unsigned char *src_b = reinterpret_cast<const unsigned char *>(src);
 #pragma unroll
             for (int k = 0; k < PER; ++k) {
-                if (!ok[k])
-                    continue;
                 unsigned char *dst = tile + (lane + 32 * k) * P::ROW;
+                if (!ok[k]) {
+                    if (zero[k])
+                        for (int b = 0; b < P::ROW; b += 16)
+                            *reinterpret_cast<uint4 *>(dst + b) = make_uint4(0u, 0u, 0u, 0u);
+                    continue;
+                }
                 if (nbulk[k] > 0)
                     bulk_load(smem_addr(dst), src_b + start[k], nbulk[k], bar);
                 if (nbulk[k] < (uint32_t)P::ROW) {
@@ -442,6 +528,86 @@ __global__ void __launch_bounds__(32)
                     const int64_t end = min(tg.n_src * (int64_t)sizeof(T) - start[k], (int64_t)P::ROW);
                     for (int64_t b = nbulk[k]; b < end; b += (int64_t)sizeof(T))
                         *reinterpret_cast<T *>(dst + b) = *reinterpret_cast<const T *>(src_b + start[k] + b);
+                }
+            }
+        }
+    } else if constexpr (GR != 0) {
+        if (lane == 0) {
+            for (int s = 0; s < KT; ++s)
+                mbar_init(smem_addr(bars + s), 1);
+            fence_barrier_init();
+        }
+        __syncwarp();
+        constexpr int R = 4 * RW / GR;                                  // rows of a part in one frame slice
+        constexpr uint32_t PART = (uint32_t)kTileElems * sizeof(T) / GR; // bytes of one part's box
+        constexpr uint32_t TAILS = (uint32_t)kTileElems * sizeof(T);     // the tail slots: 128 bytes per part
+        for (int s = 0; s < count; ++s) {
+            int tx, ty, tq;
+            int64_t bc;
+            decode(first + s, tx, ty, tq, bc);
+            const int x0 = 4 * col0(tx, ty, tq); // first pixel column (may be negative: TMA fills zeros)
+            const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0);
+            const bool mirrored = VIDEO && EXT && !replica && 4 * tq + tg.fbase + 3 >= tg.T;
+            const uint32_t bar = smem_addr(bars + s);
+            unsigned char *tile = smem_raw + s * P::TILE;
+            const int z0 = (int)(bc * tg.T), gy = R * ty; // frame of the clip, group row of the tile
+            if (!mirrored) {
+                // One box per part and one tail box per part that does not start on a 16-byte
+                // boundary, from one window of frames: all issued by lane 0.
+                if (lane == 0) {
+                    const int nf = VIDEO && !replica ? NA : 1;
+                    const int z = !VIDEO || replica ? z0 : EXT ? z0 + 4 * tq + tg.fbase : z0 + 4 * tq - 3;
+                    const CUtensorMap *mrow = nf == 1 ? &xmap1 : &xmap4, *mtail = nf == 1 ? &xtail1 : &xtail4;
+                    uint32_t nmis = 0;
+#pragma unroll
+                    for (int pt = 0; pt < GR; ++pt)
+                        nmis += ((x0 + pt * (int)tg.W) & 7) != 0;
+                    mbar_expect_tx(bar, (uint32_t)nf * (FRAME_BYTES + nmis * R * 16u));
+#pragma unroll
+                    for (int pt = 0; pt < GR; ++pt) {
+                        const int xq = x0 + pt * (int)tg.W, xb = xq - (xq & 7);
+                        tma_load_3d(smem_addr(tile + pt * PART), mrow, xb, gy, z, bar);
+                        if (xq & 7)
+                            tma_load_3d(smem_addr(tile + TAILS + pt * 128), mtail, xb + 4 * WT, gy, z, bar);
+                    }
+                }
+            } else {
+                // A window that runs past the clip: frame by frame, mirrored about the last frame;
+                // lanes 0 .. 15 copy the tails of staged row `lane` (frame slot a, pixel row yi).
+                const unsigned char *src_b = reinterpret_cast<const unsigned char *>(src);
+                const int a = lane / (4 * RW), yi = lane % (4 * RW), part = yi % GR;
+                const int64_t y = (int64_t)4 * RW * ty + yi;
+                const int f = mirror_frame(4 * tq + tg.fbase + a, tg.T);
+                const int xp = x0 + part * (int)tg.W;
+                const int mis = xp & 7; // elements from the 16-byte boundary below the row's first pixel
+                const int64_t tstart = (((bc * tg.T + f) * tg.H + (y - part)) * tg.W + (xp - mis) + 4 * WT) *
+                                       (int64_t)sizeof(T); // the 16 bytes after the part's box
+                const bool want = lane < 16 && y < tg.H && mis != 0;
+                const int64_t avail = tg.n_src * (int64_t)sizeof(T) - tstart;
+                const uint32_t nbulk = want && avail >= 16 ? 16u : 0u;
+                const uint32_t tail_bytes = __reduce_add_sync(0xFFFFFFFFu, nbulk);
+                unsigned char *tslot = tile + TAILS + part * 128 + (a * R + yi / GR) * 16;
+                if (lane == 0)
+                    mbar_expect_tx(bar, (uint32_t)NA * FRAME_BYTES + tail_bytes);
+                __syncwarp();
+                if (lane == 0) {
+#pragma unroll
+                    for (int pt = 0; pt < GR; ++pt) {
+                        const int xq = x0 + pt * (int)tg.W, xb = xq - (xq & 7);
+                        for (int fa = 0; fa < NA; ++fa)
+                            tma_load_3d(smem_addr(tile + pt * PART + fa * R * 512), &xmap1, xb, gy,
+                                        z0 + mirror_frame(4 * tq + tg.fbase + fa, tg.T), bar);
+                    }
+                }
+                if (nbulk) {
+                    bulk_load(smem_addr(tslot), src_b + tstart, 16u, bar);
+                } else if (lane < 16) {
+                    // No copy: zeros (rows past the clip read as zeros), or the tensor's last,
+                    // partial 16 bytes element by element.
+                    *reinterpret_cast<uint4 *>(tslot) = make_uint4(0u, 0u, 0u, 0u);
+                    if (want)
+                        for (int64_t e = 0; e < avail; e += (int64_t)sizeof(T))
+                            *reinterpret_cast<T *>(tslot + e) = *reinterpret_cast<const T *>(src_b + tstart + e);
                 }
             }
         }
@@ -497,7 +663,10 @@ __global__ void __launch_bounds__(32)
         const unsigned char *tile = smem_raw + s * P::TILE;
         const T *tin = reinterpret_cast<const T *>(tile);
         const int64_t j0 = (int64_t)col0(tx, ty, tq) + 2 * lane; // this lane's first block column
-        const bool col_ok = j0 >= 0 && j0 < tg.w;
+        // Some block of this lane's pair is in the tensor (the grouped form's shifted tiles can
+        // put block j0 = -1 left of column 0); both are (a pair store may be used).
+        const bool col_ok = (GR ? j0 >= -1 : j0 >= 0) && j0 < tg.w;
+        const bool interior = j0 >= 0 && j0 + 1 < tg.w;
         const bool pair_ok = !ROWS || j0 + 1 < tg.w;    // block j0 + 1 exists (w is even outside the row form)
         const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0); // window 0 of a video
 
@@ -515,33 +684,44 @@ __global__ void __launch_bounds__(32)
                             for (int d = 0; d < 4; ++d)
                                 v[a][rr][d] = make_float2(0.0f, 0.0f);
                         } else if constexpr (ROWS) {
+                            // Rows past the clip's last row were staged as zeros.
                             const int r = fa * 4 * RW + 4 * rw + rr;
-                            const unsigned mb = row_off[s * 64 + r];
-                            if (EXT && mb == kRowSkipped) { // a row past the clip's last row: zeros
-#pragma unroll
-                                for (int d = 0; d < 4; ++d)
-                                    v[a][rr][d] = make_float2(0.0f, 0.0f);
-                            } else {
-                                staged_row8(tile + r * P::ROW, mb + lane * 8 * (uint32_t)sizeof(T), (T *)nullptr,
-                                            v[a][rr]);
-                                if (EXT) {
-                                    // Columns past the clip's last column read as zeros (the staged
-                                    // row runs on into the next one).
-                                    const int64_t c0 = (int64_t)4 * WT * tx + 8 * lane;
-                                    if (c0 + 8 > tg.W) {
-#pragma unroll
-                                        for (int d = 0; d < 4; ++d) {
-                                            if (c0 + d >= tg.W)
-                                                v[a][rr][d].x = 0.0f;
-                                            if (c0 + 4 + d >= tg.W)
-                                                v[a][rr][d].y = 0.0f;
-                                        }
-                                    }
-                                }
-                            }
+                            staged_row8(tile + r * P::ROW, row_off[s * 64 + r] + lane * 8 * (uint32_t)sizeof(T),
+                                        (T *)nullptr, v[a][rr]);
+                        } else if constexpr (GR != 0) {
+                            // Pixel row yi of frame slot fa: row fa * R + yi / GR of part yi % GR's
+                            // box and of its tail slots.
+                            constexpr int R = 4 * RW / GR;
+                            constexpr uint32_t PART = (uint32_t)kTileElems * sizeof(T) / GR;
+                            const int yi = 4 * rw + rr, pt = yi % GR;
+                            const int x0 = 4 * col0(tx, ty, tq);
+                            const uint32_t o = (uint32_t)((x0 + pt * (int)tg.W) & 7) * (uint32_t)sizeof(T) +
+                                               16u * (uint32_t)lane;
+                            grouped_row8(tile + pt * PART + (fa * R + yi / GR) * 512,
+                                             tile + kTileElems * sizeof(T) + pt * 128 + (fa * R + yi / GR) * 16, o,
+                                             v[a][rr]);
                         } else {
                             SRow<T>::load(tin + (fa * 4 * RW + 4 * rw + rr) * 4 * WT + 8 * lane, v[a][rr]);
                         }
+                    }
+                }
+                if constexpr (EXT && (ROWS || GR != 0)) {
+                    // Columns past the clip's last column read as zeros (a staged row or a part's
+                    // box runs on into the next pixel row): one test per tile row, after all its
+                    // reads, so that no branch separates them.
+                    const int64_t c0 = (GR ? (int64_t)4 * col0(tx, ty, tq) : (int64_t)4 * WT * tx) + 8 * lane;
+                    if (c0 + 8 > tg.W) {
+#pragma unroll
+                        for (int a = 0; a < NA; ++a)
+#pragma unroll
+                            for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+                                for (int d = 0; d < 4; ++d) {
+                                    if (c0 + d >= tg.W)
+                                        v[a][rr][d].x = 0.0f;
+                                    if (c0 + 4 + d >= tg.W)
+                                        v[a][rr][d].y = 0.0f;
+                                }
                     }
                 }
             } else {
@@ -600,17 +780,18 @@ __global__ void __launch_bounds__(32)
 
             const int64_t row = (int64_t)ty * RW + rw; // block row
             bool pairs = true;
-            if constexpr (FWD && ROWS) {
+            if constexpr (FWD && (ROWS || GR != 0)) {
                 // A pair store is aligned iff its element offset is even, which alternates with g
                 // only when the plane stride is odd.  One warp-wide choice per tile row (taken before
-                // any lane leaves; addresses only): pair stores when every storing lane's 64 pairs
-                // are aligned and whole, element stores otherwise.
+                // any lane leaves; addresses only): pair stores when every lane with a whole pair
+                // has its 64 pairs aligned, element stores otherwise.  A lane whose pair is cut by
+                // the tensor's edge stores its one block alone either way.
                 const int64_t b = tg.C.div((uint32_t)bc), c = bc - b * tg.C.d;
                 const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
                 const T *yq = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
                 const uintptr_t amask = 2 * sizeof(T) - 1;
-                pairs = __all_sync(0xFFFFFFFFu, !col_ok || (pair_ok && ((uintptr_t)yq & amask) == 0 &&
-                                                            ((uintptr_t)(yq + tg.C.d * plane) & amask) == 0));
+                pairs = __all_sync(0xFFFFFFFFu, !interior || (((uintptr_t)yq & amask) == 0 &&
+                                                              ((uintptr_t)(yq + tg.C.d * plane) & amask) == 0));
             }
             if (!col_ok || row >= tg.h)
                 continue;
@@ -621,21 +802,23 @@ __global__ void __launch_bounds__(32)
                 const int64_t plane = (int64_t)tg.Tq * tg.h * tg.w;
                 const uint32_t cstride = (uint32_t)(tg.C.d * plane);
                 T *yp = out + (b * G * tg.C.d + c) * plane + ((int64_t)tq * tg.h + row) * tg.w + j0;
-                if constexpr (ROWS) {
-                    if (pairs) {
+                if constexpr (ROWS || GR != 0) {
+                    if (pairs && interior) {
 #pragma unroll
                         for (int g = 0; g < G; ++g) {
                             const float2 p = VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)];
                             gstore_pair(yp + (uint64_t)((uint32_t)g * cstride), __fmul2_rn(p, scale));
                         }
                     } else {
+                        const bool first_ok = j0 >= 0, second_ok = j0 + 1 < tg.w;
 #pragma unroll
                         for (int g = 0; g < G; ++g) {
                             const float2 q = __fmul2_rn(
                                 VIDEO ? v[kt_of(g)][ky_of(g)][kx_of(g)] : v[0][ky2_of(g)][kx2_of(g)], scale);
                             T *dst = yp + (uint64_t)((uint32_t)g * cstride);
-                            dst[0] = to_elem<T>(q.x);
-                            if (pair_ok)
+                            if (first_ok)
+                                dst[0] = to_elem<T>(q.x);
+                            if (second_ok)
                                 dst[1] = to_elem<T>(q.y);
                         }
                     }
@@ -662,31 +845,66 @@ __global__ void __launch_bounds__(32)
                     }
                     continue;
                 }
+                // Run-time store widths, both blocks' pixels inside the crop: every row stored at the
+                // call's one width, with no test per row.  (Not in the row form's extended calls:
+                // there the second copy of the store code cost more than the tests it saves.)
+                const bool uniform = ((ROWS && !EXT) || ANYST) && pair_ok &&
+                                     (!EXT || (4 * row + 3 < tg.H && 4 * j0 + 8 <= tg.W));
+                if (uniform) {
+                    auto put_all = [&](auto width) {
+                        constexpr int SW = decltype(width)::value;
 #pragma unroll
-                for (int a = 0; a < NA; ++a) {
-                    if (replica && a != 3)
-                        continue;
-                    const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
-                    if (EXT && f >= tg.T) // cropped frames
-                        continue;
+                        for (int a = 0; a < NA; ++a) {
+                            if (replica && a != 3)
+                                continue;
+                            const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
+                            if (EXT && f >= tg.T) // cropped frames
+                                continue;
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
-                        float2 o[4];
+                            for (int rr = 0; rr < 4; ++rr) {
+                                float2 o[4];
 #pragma unroll
-                        for (int d = 0; d < 4; ++d)
-                            o[d] = __fmul2_rn(v[a][rr][d], scale);
-                        T *dst = xb + f * tg.H * tg.W + rr * tg.W;
-                        if (!EXT) {
-                            store_pixel_row<ROWS || ANYST>(dst, o, pair_ok);
-                        } else if (4 * row + rr < tg.H) { // cropped rows and columns
-                            const int64_t col = 4 * j0;
-                            if (col + 8 <= tg.W) {
-                                store_pixel_row<ROWS || ANYST>(dst, o, true);
-                            } else {
+                                for (int d = 0; d < 4; ++d)
+                                    o[d] = __fmul2_rn(v[a][rr][d], scale);
+                                store_row_width<SW>(xb + f * tg.H * tg.W + rr * tg.W, o);
+                            }
+                        }
+                    };
+                    if (tg.sw >= 16)
+                        put_all(std::integral_constant<int, 16>());
+                    else if (tg.sw == 8)
+                        put_all(std::integral_constant<int, 8>());
+                    else if (tg.sw == 4)
+                        put_all(std::integral_constant<int, 4>());
+                    else
+                        put_all(std::integral_constant<int, 2>());
+                } else {
 #pragma unroll
-                                for (int d = 0; d < 8; ++d)
-                                    if (col + d < tg.W)
-                                        dst[d] = to_elem<T>(d < 4 ? o[d].x : o[d - 4].y);
+                    for (int a = 0; a < NA; ++a) {
+                        if (replica && a != 3)
+                            continue;
+                        const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
+                        if (EXT && f >= tg.T) // cropped frames
+                            continue;
+#pragma unroll
+                        for (int rr = 0; rr < 4; ++rr) {
+                            float2 o[4];
+#pragma unroll
+                            for (int d = 0; d < 4; ++d)
+                                o[d] = __fmul2_rn(v[a][rr][d], scale);
+                            T *dst = xb + f * tg.H * tg.W + rr * tg.W;
+                            if (!EXT) {
+                                store_pixel_row<ROWS || ANYST>(dst, o, pair_ok);
+                            } else if (4 * row + rr < tg.H) { // cropped rows and columns
+                                const int64_t col = 4 * j0;
+                                if (col + 8 <= tg.W) {
+                                    store_pixel_row<ROWS || ANYST>(dst, o, true);
+                                } else {
+#pragma unroll
+                                    for (int d = 0; d < 8; ++d)
+                                        if (col + d < tg.W)
+                                            dst[d] = to_elem<T>(d < 4 ? o[d].x : o[d - 4].y);
+                                }
                             }
                         }
                     }
@@ -1318,29 +1536,41 @@ __global__ void __launch_bounds__(32)
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false>
+template <typename T, bool VIDEO, bool FWD, bool ADJ, bool EXT, bool ROWS, bool ANYST = false, int GR = 0>
 tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t stream)
 {
-    using P = TileSmem<T, FWD, ROWS>;
+    using P = TileSmem<T, FWD, ROWS, GR>;
     constexpr int G = VIDEO ? 64 : 16, RW = TileRows<VIDEO>::RW, WT = kTileBlocks;
     const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const uint64_t es = sizeof(T);
     // Only the input side goes through TMA: pixels on the forward, coefficients on the inverse.
-    CUtensorMap xm4, xm1, ym;
+    CUtensorMap xm4, xm1, ym, xt4, xt1;
     memset(&xm4, 0, sizeof xm4);
     memset(&xm1, 0, sizeof xm1);
     memset(&ym, 0, sizeof ym);
+    memset(&xt4, 0, sizeof xt4);
+    memset(&xt1, 0, sizeof xt1);
     if (ROWS) {
         // The row form reads the source through its pointer (bulk copies); no tensor map.
     } else if (FWD) {
-        const uint64_t xdims[3] = {(uint64_t)d.W, (uint64_t)d.H, (uint64_t)(d.B * d.C * d.T)};
-        const uint64_t xstr[2] = {d.W * es, d.H * d.W * es};
-        const uint32_t box4[3] = {4u * WT, 4u * RW, 4u}, box1[3] = {4u * WT, 4u * RW, 1u};
+        // Grouped rows: each frame as [H / GR][GR W], GR pixel rows per row of the map (a
+        // 16-byte multiple), and a box of the tile's rows of one part.
+        const uint64_t g = GR ? (uint64_t)GR : 1u;
+        const uint64_t xdims[3] = {g * d.W, d.H / g, (uint64_t)(d.B * d.C * d.T)};
+        const uint64_t xstr[2] = {g * d.W * es, d.H * d.W * es};
+        const uint32_t rows = 4u * RW / (uint32_t)g;
+        const uint32_t box4[3] = {4u * WT, rows, 4u}, box1[3] = {4u * WT, rows, 1u};
         // The 4-frame box serves windows with four frames of the clip, so a frame axis
         // shorter than 4 never uses it and it is not encoded.
         if (!encode_tensor_map(&xm1, dt, 3, in, xdims, xstr, box1) ||
             (VIDEO && xdims[2] >= 4 && !encode_tensor_map(&xm4, dt, 3, in, xdims, xstr, box4)))
             return TOK_ERR_SHAPE;
+        if (GR) { // the 8 elements after a part's box
+            const uint32_t tail4[3] = {8u, rows, 4u}, tail1[3] = {8u, rows, 1u};
+            if (!encode_tensor_map(&xt1, dt, 3, in, xdims, xstr, tail1) ||
+                (VIDEO && xdims[2] >= 4 && !encode_tensor_map(&xt4, dt, 3, in, xdims, xstr, tail4)))
+                return TOK_ERR_SHAPE;
+        }
     } else {
         const uint64_t ydims[5] = {(uint64_t)d.w, (uint64_t)d.h, (uint64_t)d.Tq, (uint64_t)d.C, (uint64_t)(G * d.B)};
         const uint64_t plane = d.Tq * d.h * d.w * es;
@@ -1353,10 +1583,17 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     // Sector-aligned plane stores (TileGrid::salign): the shifts k w mod salign are multiples of
     // gcd(w, salign), so a row needs at most ceil((w + salign - gcd) / 64) tiles.
     int salign = 0;
-    if (FWD && VIDEO && !ROWS) {
+    if (FWD && VIDEO && !ROWS && !GR) {
         const int64_t sa = 32 / (int64_t)es, plane = d.Tq * d.h * d.w;
         if ((d.w * (int64_t)es) % 32 != 0 && (plane * (int64_t)es) % 32 == 0 && aligned(out, 32))
             salign = (int)sa;
+    } else if (FWD && VIDEO && GR) {
+        // Grouped rows (w may be odd): the largest power of two up to kGroupSalign that divides
+        // a plane, so the shifted tiles' pair stores are aligned (sector-aligned at 16).
+        const int64_t plane = d.Tq * d.h * d.w;
+        for (int64_t sa = kGroupSalign; sa >= 2 && !salign; sa /= 2)
+            if (plane % sa == 0 && aligned(out, (size_t)(sa * (int64_t)es)))
+                salign = (int)sa;
     }
     const int64_t smax = salign ? salign - std::gcd(d.w, (int64_t)salign) : 0;
     const int64_t ntx = (d.w + smax + WT - 1) / WT, nty = (d.h + RW - 1) / RW;
@@ -1378,17 +1615,21 @@ tok_status launch(const void *in, void *out, const HaarDims &d, cudaStream_t str
     tg.n_src = FWD ? d.B * d.C * d.T * d.H * d.W : d.B * G * d.C * d.Tq * d.h * d.w;
     tg.salign = salign;
     tg.planes_share_offset = ((int64_t)d.C * d.Tq * d.h * d.w * (int64_t)es) % 16 == 0;
+    {
+        const uint64_t bits = (uint64_t)(d.W * (int64_t)es) | (uint64_t)(uintptr_t)out | 16u;
+        tg.sw = (int)(bits & (~bits + 1)); // the lowest set bit: 2, 4, 8 or 16
+    }
 
     // Per call: the attribute belongs to the current device.
-    const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST>,
+    const cudaError_t attr_err = cudaFuncSetAttribute(haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST, GR>,
                                                       cudaFuncAttributeMaxDynamicSharedMemorySize, P::SMEM);
     if (attr_err != cudaSuccess) {
         record_cuda_error(attr_err);
         return TOK_ERR_CUDA;
     }
     const unsigned grid = (unsigned)((tg.ntiles + P::KT - 1) / P::KT);
-    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST>
-        <<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, (const T *)in, (T *)out, tg);
+    haar_tma_kernel<T, VIDEO, FWD, ADJ, EXT, ROWS, ANYST, GR>
+        <<<grid, 32, P::SMEM, stream>>>(xm4, xm1, ym, xt4, xt1, (const T *)in, (T *)out, tg);
     return launch_status();
 }
 
@@ -1400,6 +1641,10 @@ tok_status launch_form(HaarTmaForm form, const void *in, void *out, const HaarDi
     if constexpr (!FWD) {
         if (form == HaarTmaForm::boxes_any_store)
             return launch<T, VIDEO, FWD, ADJ, EXT, false, true>(in, out, d, stream);
+    }
+    if constexpr (VIDEO && FWD && sizeof(T) == 2) {
+        if (form == HaarTmaForm::groups)
+            return launch<T, VIDEO, FWD, ADJ, EXT, false, false, 2>(in, out, d, stream);
     }
     return launch<T, VIDEO, FWD, ADJ, EXT, false>(in, out, d, stream);
 }
@@ -1430,6 +1675,12 @@ HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype d
     // odd widths, a destination off a 16-byte boundary): box loads, stores of run-time width.
     if (!fwd && aligned(in, 16) && (d.w * es) % 16 == 0)
         return HaarTmaForm::boxes_any_store;
+    // bf16 video forward whose pixel rows are 8-byte units (two of them are 16-byte units), with
+    // an odd number of coefficient columns: grouped rows (whole pairs of rows of the clip,
+    // coordinates below 2^31).
+    if (fwd && es == 2 && d.video && aligned(in, 16) && d.W % 8 == 4 && d.w % 2 == 1 && d.H % 2 == 0 &&
+        2 * d.W + 1024 < ((int64_t)1 << 31))
+        return HaarTmaForm::groups;
     // Row form: any 16-byte-aligned source.
     return aligned(in, 16) ? HaarTmaForm::rows : HaarTmaForm::none;
 }

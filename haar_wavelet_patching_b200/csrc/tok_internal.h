@@ -26,10 +26,11 @@ struct HaarDims {
 
 // Which form of the TMA kernel takes a planar call in direction fwd: boxes (the source's
 // rows are whole 16-byte units, and so are the destination's where it stores 16-byte rows),
-// boxes_any_store (inverse: box loads, pixel-row stores of run-time width), rows (any
-// 16-byte-aligned source, any row length, any element-aligned destination) or none
-// (register kernels).
-enum class HaarTmaForm { none, boxes, boxes_any_store, rows };
+// boxes_any_store (inverse: box loads, pixel-row stores of run-time width), groups (bf16
+// video forward with W % 8 == 4 and an odd w: tensor boxes over pairs of pixel rows, tiles
+// shifted so that coefficient pairs are stored aligned), rows (any 16-byte-aligned source,
+// any row length, any element-aligned destination) or none (register kernels).
+enum class HaarTmaForm { none, boxes, boxes_any_store, groups, rows };
 HaarTmaForm haar_tma_form(bool fwd, const void *in, const void *out, tok_dtype dt, const HaarDims &d);
 // fwd: pixels -> coefficients; adj: the adjoint variant (video only; images are orthogonal).
 tok_status haar_tma_launch(bool fwd, bool adj, HaarTmaForm form, const void *in, void *out, tok_dtype dt,
