@@ -590,13 +590,13 @@ def stress_inputs(torch, cfg, dev):
 
 
 def time_stress(torch, hwp, stream, w_dev, dev, iters=STRESS_ITERS):
-    """BASELINE configs 5 and 2, outside the headline step.  Config 5: four 121-frame 1088x1920
-    clips [4,3,121,1088,1920] bf16 through the patcher and unpatcher, then FSQ encode + decode of
-    the [4,16,16*68*120] latent, back to back on one stream (its Haar tensors are 6 GB each, so
-    nothing survives in L2 from one call to the next; its 35 MB latent is L2-sized).  Config 2:
-    the image path on [16,3,1024,1024] bf16 (2D Haar) and FSQ on [16,16,64*64]; every tensor
-    but none of the Haar pairs exceeds L2, so L2 is flushed before each call (outside its
-    events).  Per call: mean ms, algorithmic bytes (inputs read once, outputs written once)."""
+    """The throughput-stress clip and the image batch, outside the headline step.  Stress: four
+    121-frame 1088x1920 clips [4,3,121,1088,1920] bf16 through the patcher and unpatcher, then
+    FSQ encode + decode of the [4,16,16*68*120] latent, back to back on one stream (its Haar
+    tensors are 6 GB each, so nothing survives in L2 from one call to the next; its 35 MB latent
+    is L2-sized).  Image batch: the image path on [16,3,1024,1024] bf16 (2D Haar) and FSQ on
+    [16,16,64*64]; none of its tensors exceeds L2, so L2 is flushed before each call (outside
+    its events).  Per call: mean ms, algorithmic bytes (inputs read once, outputs written once)."""
     out = {}
     for cfg in (5, 2):
         x, u = stress_inputs(torch, cfg, dev)
@@ -638,7 +638,7 @@ def stress_report(stress, peak):
             else:
                 r["mtoken_per_s"] = round(d["tokens"] / g["ms"] / 1e3, 1)
             e[n] = r
-        rep[f"config{cfg}"] = e
+        rep["stress_clip" if cfg == 5 else "image_batch"] = e
     return rep
 
 
@@ -837,7 +837,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-stress", action="store_true", help="skip the config 5 / config 2 block")
+    ap.add_argument("--no-stress", action="store_true", help="skip the throughput-stress clip / image batch block")
     args = ap.parse_args()
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -15,7 +15,7 @@ they are conventions shared with the CUDA path):
   - k = 3; the spatial convolution is padded by (k - 1)/2 zeros on every side ("same");
   - no bias, no activation between the two convolutions (one factorized 3D layer);
   - channels: C_in = 64 C (the patcher's output), C_mid = C_out = 256 at the measured
-    size, any multiples of 8 in general; weights layout [C_mid][k][k][C_in] (spatial)
+    size (the oracle takes any counts); weights layout [C_mid][k][k][C_in] (spatial)
     and [C_out][k][C_mid] (temporal), tap dt multiplying frame t - (k - 1) + dt;
   - activations are channels-last [B, T', h, w, C] (the patcher's channels-last output);
   - the network stores activations in bf16: the spatial result is rounded to bf16

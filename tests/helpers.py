@@ -2,7 +2,7 @@
 
 Tolerances (derived from the arithmetic of the kernels):
   fp32 Haar      max |gpu - oracle| <= 1e-5.
-  bf16 outputs   one bf16 ulp of the oracle value (the benchmark spec's figure), read as
+  bf16 outputs   one bf16 ulp of the oracle value (the path's stated figure), read as
                  follows.  The kernel computes an fp32 value v within E of the exact
                  result r (E bounds its fp32 accumulation error) and rounds it once to
                  bf16 (nearest even), so |gpu - r| <= E + ulp(|r| + E) / 2.  The test

@@ -71,7 +71,7 @@ SMALL = [
     # (shape, dtype, note).  TMA box form: the source's rows are whole 16-byte units (forward:
     # W * elem, with w even; inverse: w * elem and W * elem); other 16-byte-aligned sources take
     # the TMA row form.  The register kernels take misaligned views (tests below).
-    ((1, 3, 9, 64, 64), synth.F32, "config 1"),
+    ((1, 3, 9, 64, 64), synth.F32, "clip [1,3,9,64,64] fp32"),
     ((2, 3, 13, 40, 96), synth.BF16, "TMA bf16, partial tiles in x and y"),
     ((1, 2, 9, 36, 80), synth.F32, "TMA fp32, partial tiles"),
     ((2, 2, 17, 64, 544), synth.BF16, "TMA bf16, several tiles per row, ragged last"),
@@ -247,9 +247,12 @@ def _slab_oracle(x_bits, y_host, T, H, W):
     return oracle.haar_fwd(x64), oracle.haar_inv(y_host, T, H, W)
 
 
-@pytest.mark.parametrize("cfg", [3, 5])
+FULL_WORKLOADS = {3: "clip [1,3,121,704,1280]", 5: "clips [4,3,121,1088,1920]"}  # synth workload keys
+
+
+@pytest.mark.parametrize("cfg", [3, 5], ids=["headline_clip", "stress_clips"])
 def test_full_workload_elementwise(cfg):
-    """The 121-frame 704x1280 clip (config 3) and the four 121-frame 1088x1920 clips (config 5)
+    """The 121-frame 704x1280 clip and the four 121-frame 1088x1920 throughput-stress clips
     in full: every coefficient of the forward and every pixel of the inverse compared with the
     oracle, one (b, c) slab at a time (the oracle on host threads, the comparison on the device).
     The inverse is compared with the oracle inverse of the same bf16 coefficients.  Also the
@@ -283,7 +286,7 @@ def test_full_workload_elementwise(cfg):
             ref_y, ref_x = futs.pop(k).result()
             if k + 3 < len(slabs):
                 submit(k + 3)
-            label = f"config {cfg} (b={b}, c={cc})"
+            label = f"{FULL_WORKLOADS[cfg]} (b={b}, c={cc})"
             xs = xd[b, cc].double()
             E = haar_fp32_bound(_window_sums(xs.abs(), T), True)           # [Tq, h, w]
             ys = y[b, cc::C]
@@ -296,15 +299,15 @@ def test_full_workload_elementwise(cfg):
             rt_max = max(rt_max, float((xr[b, cc].double() - xs).abs().max()))
             del ref_y, ref_x, E, Ei, a
     n_y, n_x = y.numel(), xr.numel()
-    print(f"config {cfg}: forward {strict_f} of {n_y} coefficients and inverse {strict_i} of {n_x} pixels "
+    print(f"{FULL_WORKLOADS[cfg]}: forward {strict_f} of {n_y} coefficients and inverse {strict_i} of {n_x} pixels "
           f"beyond a plain 1 bf16 ulp (all in the cancellation regime); round trip max |err| {rt_max:.3g}")
     assert abs(e_out / e_in - 1.0) < 2e-3       # bf16 rounding of the coefficients only
     assert rt_max < 0.05                        # bf16 coefficients: a few bf16 ulps of the block's range
     del y, xr, xd
 
 
-def test_config2_images_full():
+def test_image_batch_full():
     """Image batch [16,3,1024,1024] bf16 compared element by element with the oracle."""
     x = synth.haar_input(2)
-    y, _ = check_fwd(x, synth.BF16, "config 2")
-    check_inv(y, 1, 1024, 1024, "config 2 inverse")
+    y, _ = check_fwd(x, synth.BF16, "image batch [16,3,1024,1024]")
+    check_inv(y, 1, 1024, 1024, "image batch inverse")
