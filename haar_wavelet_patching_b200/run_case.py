@@ -23,10 +23,12 @@ def main():
                                                      "haar_inv_chunk", "fsq_encode", "fsq_decode",
                                                      "fsq_encode_backward", "fsq_decode_backward",
                                                      "conv_spatial", "conv_temporal", "conv_factorized",
-                                                     "patch_embed"))
+                                                     "patch_embed", "step"))
     ap.add_argument("--shape", required=True,
-                    help="B,C,T,H,W for haar ops; B,C,S for fsq ops; B,T,h,w,Cin,Cmid,Cout for conv ops; "
+                    help="B,C,T,H,W for haar ops and step; B,C,S for fsq ops; B,T,h,w,Cin,Cmid,Cout for conv ops; "
                          "B,C,T,H,W,Cmid for patch_embed")
+    ap.add_argument("--latent", default="64,16,56320",
+                    help="step: B,C,S of the FSQ latent (the step is Haar fwd, Haar inv, FSQ encode, FSQ decode)")
     ap.add_argument("--dtype", default="bf16", choices=("bf16", "f32"))
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--codes", action="store_true", help="fsq_encode: also write the codes")
@@ -39,7 +41,23 @@ def main():
     g = torch.Generator(device=dev).manual_seed(0)
     dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
 
-    if a.op == "patch_embed":
+    if a.op == "step":
+        x = (torch.rand(shape, generator=g, device=dev) * 2 - 1).to(dt)
+        y = torch.empty(hwp.haar_coeff_shape(*shape), dtype=dt, device=dev)
+        xr = torch.empty_like(x)
+        L = tuple(int(v) for v in a.latent.split(","))
+        u = torch.randn(L, generator=g, device=dev)
+        w = torch.randn(6, L[1], generator=g, device=dev) / L[1] ** 0.5
+        idx = torch.empty(L[0], L[2], dtype=torch.int32, device=dev)
+        ur = torch.empty_like(u)
+
+        def run():
+            hwp.tok_haar_fwd(x, y)
+            hwp.tok_haar_inv(y, xr)
+            hwp.tok_fsq_encode(u, w, idx)
+            hwp.tok_fsq_decode(idx, w, ur)
+        nbytes = 2 * (x.numel() + y.numel()) * x.element_size() + 2 * (u.numel() + idx.numel()) * 4
+    elif a.op == "patch_embed":
         B, C, T, H, W, Cmid = shape
         bf = torch.bfloat16
         x = (torch.rand((B, C, T, H, W), generator=g, device=dev) * 2 - 1).to(bf)
