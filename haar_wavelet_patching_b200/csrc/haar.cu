@@ -624,7 +624,9 @@ tok_status haar_ext_call(bool fwd, const void *in, void *out, tok_dtype dt, int6
     dims.fbase = fbase;
     dims.rep = rep;
     dims.video = video;
-    dims.ext = true;
+    // The extended form only where frames, rows or columns are padded or cropped: a chunk, or a
+    // clip that needs no padding, takes the plain forms with its window rule (fbase, rep).
+    dims.ext = Tp != T || Hp != H || Wp != W;
     const HaarTmaForm form = haar_tma_form(fwd, in, out, dt, dims);
     if (form != HaarTmaForm::none)
         return haar_tma_launch(fwd, false, form, in, out, dt, dims, stream);

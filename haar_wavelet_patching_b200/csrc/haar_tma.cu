@@ -58,11 +58,12 @@ struct TileGrid {
     int T, Tq, tq0;          // frames, latent frames of the tensor, first latent frame processed
     int64_t H, W, h, w;
     uint32_t ntiles;
-    // Extended form (padding, cropping, streaming chunks): a window tq that is not the
-    // frame-0 replica window reads frames 4*tq + fbase .. + 3 of the T-frame pixel tensor,
-    // mirrored about frame T - 1 past its end; window 0 is the replica window iff rep.
-    // The pixel tensor [T][H][W] may be smaller than the 4h x 4w blocks: the forward
-    // reads zeros there (TMA fill), the inverse does not write there.
+    // A window tq that is not the frame-0 replica window reads frames 4*tq + fbase .. + 3 of
+    // the T-frame pixel tensor; window 0 is the replica window iff rep (fbase = -3, rep = 1
+    // for the whole-video transform; fbase = 0, rep = 0 for a continuation chunk).  Extended
+    // form (padding, cropping): frames past T - 1 are mirrored about it, and the pixel tensor
+    // [T][H][W] may be smaller than the 4h x 4w blocks: the forward reads zeros there (TMA
+    // fill), the inverse does not write there.
     int fbase, rep;
     int64_t n_src; // elements of the source tensor (the row form stops its copies at its end)
     // Video forward, box form: when a coefficient row is not a whole number of 32-byte sectors
@@ -461,7 +462,7 @@ __global__ void __launch_bounds__(32)
             int tx, ty, tq;
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
-            const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0);
+            const bool replica = VIDEO && tg.rep && tq == 0;
             int64_t start[PER]; // byte offset of each staged row in the source (16-byte aligned)
             uint32_t nbulk[PER];
             bool ok[PER], zero[PER]; // zero: a row past the clip's last row that the transform reads
@@ -479,7 +480,7 @@ __global__ void __launch_bounds__(32)
                     if (VIDEO && replica)
                         loaded = loaded && a == 0; // window 0 reads frame 0 only
                     else if (VIDEO)
-                        f = EXT ? mirror_frame(4 * tq + tg.fbase + a, tg.T) : 4 * tq - 3 + a;
+                        f = EXT ? mirror_frame(4 * tq + tg.fbase + a, tg.T) : 4 * tq + tg.fbase + a;
                     ok[k] = loaded;
                     zero[k] = EXT && r < P::NR && y >= tg.H && !(VIDEO && replica && a != 0);
                     off = ((bc * tg.T + f) * tg.H + y) * tg.W + (int64_t)4 * WT * tx;
@@ -546,7 +547,7 @@ __global__ void __launch_bounds__(32)
             int64_t bc;
             decode(first + s, tx, ty, tq, bc);
             const int x0 = 4 * col0(tx, ty, tq); // first pixel column (may be negative: TMA fills zeros)
-            const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0);
+            const bool replica = VIDEO && tg.rep && tq == 0;
             const bool mirrored = VIDEO && EXT && !replica && 4 * tq + tg.fbase + 3 >= tg.T;
             const uint32_t bar = smem_addr(bars + s);
             unsigned char *tile = smem_raw + s * P::TILE;
@@ -556,7 +557,7 @@ __global__ void __launch_bounds__(32)
                 // boundary, from one window of frames: all issued by lane 0.
                 if (lane == 0) {
                     const int nf = VIDEO && !replica ? NA : 1;
-                    const int z = !VIDEO || replica ? z0 : EXT ? z0 + 4 * tq + tg.fbase : z0 + 4 * tq - 3;
+                    const int z = !VIDEO || replica ? z0 : z0 + 4 * tq + tg.fbase;
                     const CUtensorMap *mrow = nf == 1 ? &xmap1 : &xmap4, *mtail = nf == 1 ? &xtail1 : &xtail4;
                     uint32_t nmis = 0;
 #pragma unroll
@@ -636,9 +637,9 @@ __global__ void __launch_bounds__(32)
                                     (int)(bc * tg.T + mirror_frame(4 * tq + tg.fbase + a, tg.T)), bar);
                 }
             } else if constexpr (FWD) {
-                if (VIDEO && tq > 0) {
+                if (VIDEO && !(tg.rep && tq == 0)) {
                     mbar_expect_tx(bar, NA * FRAME_BYTES);
-                    tma_load_3d(dst, &xmap4, x0, 4 * RW * ty, (int)(bc * tg.T + 4 * tq - 3), bar);
+                    tma_load_3d(dst, &xmap4, x0, 4 * RW * ty, (int)(bc * tg.T + 4 * tq + tg.fbase), bar);
                 } else {
                     mbar_expect_tx(bar, FRAME_BYTES);
                     tma_load_3d(dst, &xmap1, x0, 4 * RW * ty, (int)(bc * tg.T), bar);
@@ -668,7 +669,7 @@ __global__ void __launch_bounds__(32)
         const bool col_ok = (GR ? j0 >= -1 : j0 >= 0) && j0 < tg.w;
         const bool interior = j0 >= 0 && j0 + 1 < tg.w;
         const bool pair_ok = !ROWS || j0 + 1 < tg.w;    // block j0 + 1 exists (w is even outside the row form)
-        const bool replica = VIDEO && (EXT ? (tg.rep && tq == 0) : tq == 0); // window 0 of a video
+        const bool replica = VIDEO && tg.rep && tq == 0; // window 0 of a video
 
 #pragma unroll
         for (int rw = 0; rw < RW; ++rw) {
@@ -857,7 +858,7 @@ __global__ void __launch_bounds__(32)
                         for (int a = 0; a < NA; ++a) {
                             if (replica && a != 3)
                                 continue;
-                            const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
+                            const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + tg.fbase + a;
                             if (EXT && f >= tg.T) // cropped frames
                                 continue;
 #pragma unroll
@@ -883,7 +884,7 @@ __global__ void __launch_bounds__(32)
                     for (int a = 0; a < NA; ++a) {
                         if (replica && a != 3)
                             continue;
-                        const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + (EXT ? tg.fbase : -3) + a;
+                        const int64_t f = !VIDEO ? 0 : replica ? 0 : 4 * tq + tg.fbase + a;
                         if (EXT && f >= tg.T) // cropped frames
                             continue;
 #pragma unroll
