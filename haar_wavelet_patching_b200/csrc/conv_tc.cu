@@ -621,22 +621,27 @@ tok_status conv_tc_launch(bool temporal, const void *x, const void *wts, void *y
 // 128-byte swizzled row per position (row q = r * 8 + j: one tile row is one 1024-byte
 // swizzle atom), and the three K steps dy = 0, 1, 2 are that plane seen from atom dy.
 // The filter is read in the same K order from a packed copy (tok_patch_embed_pack_weights).
-//   warp 0     tensor copies of the packed filter, kFStages stages of [64 k, N / 2];
+//   warp 0     tensor copies of the packed filter: a stage holds the three row-shift K blocks
+//              [64 k, N / 2] that one plane meets, so the MMA thread waits and commits once
+//              per plane and filter stage (12 MMAs) -- with a stage per K block its barrier
+//              operations, not the tensor cores, set the pace;
 //   warp 1     MMA issue (planes and filter stages as they fill);
-//   warps 2-5  epilogue, as in conv_tc_kernel;
+//   warps 2-5  epilogue, as in conv_tc_kernel (one staging buffer per warp);
 //   warps 6-9  Haar: per colour, one tensor copy of the pixels the tile's 3 x 3
-//              neighbourhood reads ([4 frames][72 rows][48 cols], two buffers, the
-//              next colour's copy issued before this colour's planes are made); per
-//              plane, each of 72 threads transforms two horizontally adjacent blocks
-//              in packed f32x2 pairs -- the butterflies of the planar patcher in its
-//              order (columns, rows, frames; then x 1/8), so the coefficients are the
-//              patcher's bits -- rounds them to bf16 and writes both positions' rows.
+//              neighbourhood reads ([4 frames][72 rows][48 cols]) into the one pixel
+//              buffer, which the next colour's copy refills as soon as every Haar thread
+//              holds its pixels in registers; each of 90 threads transforms two
+//              horizontally adjacent blocks in packed f32x2 pairs -- the butterflies of the
+//              planar patcher in its order (columns, rows, frames; then x 1/8), so the
+//              coefficients are the patcher's bits -- rounds them to bf16 and writes them
+//              into the colour's three planes, each as soon as a plane slot is free.
 // Latent positions outside the frame read zero pixels (the tensor copy fills zeros),
 // which is exactly the convolution's zero padding of the coefficients.
 // ---------------------------------------------------------------------------
-constexpr int kFStages = 3;                      // filter stages of one K block
-constexpr int kEmbedEpiBuf = 2;                  // staging buffers per epilogue warp
-constexpr int kPlanes = 5;                       // A planes in flight (a ring)
+constexpr int kFGroup = 3;                       // filter K blocks per stage (the row shifts of a plane)
+constexpr int kFStages = 2;                      // filter stages
+constexpr int kEmbedEpiBuf = 1;                  // staging buffers per epilogue warp
+constexpr int kPlanes = 4;                       // A planes in flight (a ring)
 constexpr int kPlaneRows = kTileRows + 2;        // latent rows of a plane
 constexpr uint32_t kPlaneBytes = kPlaneRows * kTileCols * 128; // 18 KB
 constexpr int kPixCols = 48, kPixRows = 4 * kPlaneRows, kPixFrames = 4;
@@ -703,21 +708,22 @@ __global__ void __launch_bounds__(kEmbedThreads, 1)
 patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap bmap,
                    const __grid_constant__ CUtensorMap omap, __nv_bfloat16 *__restrict__ out, const EmbedGeom g)
 {
-    __shared__ __align__(8) uint64_t ffull[kFStages], fempty[kFStages], pfull[kPlanes], pempty[kPlanes], xfull[2],
+    __shared__ __align__(8) uint64_t ffull[kFStages], fempty[kFStages], pfull[kPlanes], pempty[kPlanes], xfull,
         accf[2], acce[2], drain, hsync;
     __shared__ uint32_t tmem_base_s;
     __shared__ int abort_s;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t base = (smem_addr(smem_raw) + 1023u) & ~1023u;
     const uint32_t fbytes = (uint32_t)(g.bn / 2) * kBK * 2; // this CTA's half of a filter K block
-    const uint32_t fbase = base, pbase = fbase + kFStages * fbytes, xbase = pbase + kPlanes * kPlaneBytes;
-    const uint32_t ebase = xbase + 2 * kPixBytes;
+    const uint32_t fstage = kFGroup * fbytes;               // one filter stage
+    const uint32_t fbase = base, pbase = fbase + kFStages * fstage, xbase = pbase + kPlanes * kPlaneBytes;
+    const uint32_t ebase = xbase + kPixBytes;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
     const uint32_t ncols = tmem_cols(g.bn);
     const int pair = blockIdx.x >> 1, npair_ctas = gridDim.x >> 1;
-    const int kper = 9 * g.C; // K steps per tile
+    const int nplanes = 3 * g.C; // planes (and filter stages) per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFStages; ++s) {
@@ -729,10 +735,10 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
             mbar_init(smem_addr(&pempty[p]), 1);
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(smem_addr(&xfull[a]), 1);
             mbar_init(smem_addr(&accf[a]), 1);
             mbar_init(smem_addr(&acce[a]), 8);
         }
+        mbar_init(smem_addr(&xfull), 1);
         mbar_init(smem_addr(&drain), 1);
         mbar_init(smem_addr(&hsync), kHaarThreads);
         abort_s = 0;
@@ -749,21 +755,23 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
     volatile int *abort = &abort_s;
 
     if (warp == 0 && lane == 0) {
-        // This CTA's half of the filter, one K block per stage in the tile's K order; counted on
-        // the leader's barrier.
+        // This CTA's half of the filter, the three K blocks of one plane per stage in the tile's K
+        // order; counted on the leader's barrier.
         uint32_t s = 0, ph = 0, issued = 0;
         bool ok = true;
         for (int i = pair; i < g.npairs && ok; i += npair_ctas) {
             const EmbedTile e = decode_embed(g, i, rank);
-            for (int kb = 0; kb < kper; ++kb) {
+            for (int pl = 0; pl < nplanes; ++pl) {
                 if (!wait_or_abort(smem_addr(&fempty[s]), ph ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
+                const uint32_t fb = mapa_shared(smem_addr(&ffull[s]), 0);
                 if (leader)
-                    mbar_expect_tx(smem_addr(&ffull[s]), 2 * fbytes);
-                tma_load_2d_pair(fbase + s * fbytes, &bmap, kb * kBK, e.n0 + (int)rank * (g.bn / 2),
-                                 mapa_shared(smem_addr(&ffull[s]), 0));
+                    mbar_expect_tx(smem_addr(&ffull[s]), 2 * fstage);
+                for (int dy = 0; dy < kFGroup; ++dy)
+                    tma_load_2d_pair(fbase + s * fstage + dy * fbytes, &bmap, (pl * kFGroup + dy) * kBK,
+                                     e.n0 + (int)rank * (g.bn / 2), fb);
                 ++issued;
                 if (++s == kFStages) {
                     s = 0;
@@ -777,8 +785,8 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
     } else if (warp == 1 && lane == 0 && leader) {
         // MMA issue for the pair.  This single thread is the pipeline's narrowest point (each
         // barrier test or commit costs it about as long as an MMA), so the loop keeps its ring
-        // positions and descriptors as running values: per plane (c, dx) one wait and one commit,
-        // per row shift dy one filter stage.
+        // positions and descriptors as running values: per plane (c, dx) one wait and one commit
+        // on the plane ring and one on the filter ring, around its 12 MMAs.
         const uint32_t idesc = idesc_bf16_f32(2 * kBM, g.bn);
         const uint64_t adesc0 = sw128_desc(pbase), bdesc0 = sw128_desc(fbase);
         uint32_t fs = 0, fph = 0, ps = 0, pph = 0, tc = 0;
@@ -789,31 +797,26 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                 break;
             tc_fence_after();
             const uint32_t d = tmem + acc * (uint32_t)g.bn;
-            for (int pl = 0; pl < 3 * g.C && ok; ++pl) {
-                if (!wait_or_abort(smem_addr(&pfull[ps]), pph, abort)) {
+            for (int pl = 0; pl < nplanes && ok; ++pl) {
+                if (!wait_or_abort(smem_addr(&pfull[ps]), pph, abort) ||
+                    !wait_or_abort(smem_addr(&ffull[fs]), fph, abort)) {
                     ok = false;
                     break;
                 }
-                const uint64_t ad = adesc0 + ((ps * kPlaneBytes) >> 4);
+                const uint64_t ad = adesc0 + ((ps * kPlaneBytes) >> 4), bd = bdesc0 + ((fs * fstage) >> 4);
 #pragma unroll
-                for (int dy = 0; dy < 3; ++dy) {
-                    if (!wait_or_abort(smem_addr(&ffull[fs]), fph, abort)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint64_t a = ad + (uint64_t)(dy * 64), b = bdesc0 + ((fs * fbytes) >> 4);
+                for (int dy = 0; dy < kFGroup; ++dy) {
+                    const uint64_t a = ad + (uint64_t)(dy * 64), b = bd + (uint64_t)((dy * fbytes) >> 4);
                     umma_bf16_pair(d, a, b, idesc, (pl | dy) != 0);
                     umma_bf16_pair(d, a + 2, b + 2, idesc, 1u);
                     umma_bf16_pair(d, a + 4, b + 4, idesc, 1u);
                     umma_bf16_pair(d, a + 6, b + 6, idesc, 1u);
-                    umma_commit_pair(smem_addr(&fempty[fs]), kPairMask);
-                    if (++fs == kFStages) {
-                        fs = 0;
-                        fph ^= 1u;
-                    }
                 }
-                if (!ok)
-                    break;
+                umma_commit_pair(smem_addr(&fempty[fs]), kPairMask);
+                if (++fs == kFStages) {
+                    fs = 0;
+                    fph ^= 1u;
+                }
                 umma_commit_pair(smem_addr(&pempty[ps]), kPairMask);
                 if (++ps == kPlanes) {
                     ps = 0;
@@ -854,52 +857,29 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
         // Haar warps of this CTA's tile.  Per colour, each of 90 threads transforms two adjacent
         // latent columns u0 = 2 up - 1, u0 + 1 (up = 0..4; u = -1 .. 8 relative to x0) of plane row
         // pr and writes each position into every plane dx whose window holds it (plane column
-        // j = u + 1 - dx): the colour's three planes are made in one pass.
+        // j = u + 1 - dx), plane by plane as slots free up.
         const int ht = threadIdx.x - kHaarFirst;
         const int pr = ht / 5, up = ht - 5 * pr, u0 = 2 * up - 1;
         const bool worker = ht < kPlaneRows * 5;
-        uint32_t ci = 0, pi = 0; // colours and planes made so far
+        uint32_t ci = 0, pi = 0, px_issued = 0; // colours started, planes made, pixel copies issued
         bool ok = true;
         int i = pair;
-        if (ht == 0 && i < g.npairs)
-            issue_pixels(&xmap, decode_embed(g, i, rank), 0, xbase, smem_addr(&xfull[0]));
+        if (ht == 0 && i < g.npairs) {
+            issue_pixels(&xmap, decode_embed(g, i, rank), 0, xbase, smem_addr(&xfull));
+            ++px_issued;
+        }
+        const unsigned char *pix = smem_raw + (xbase - smem_addr(smem_raw));
         for (; i < g.npairs && ok; i += npair_ctas) {
             const EmbedTile e = decode_embed(g, i, rank);
-            for (int c = 0; c < g.C && ok; ++c, ++ci, pi += 3) {
-                // Once every Haar thread is done with the buffer of colour ci - 1 (a barrier phase per
-                // colour; its wait is bounded like the others), colour ci + 1 is copied into it.
-                mbar_arrive(smem_addr(&hsync));
-                if (!wait_or_abort(smem_addr(&hsync), ci & 1u, abort)) {
+            for (int c = 0; c < g.C && ok; ++c, ++ci) {
+                if (!wait_or_abort(smem_addr(&xfull), ci & 1u, abort)) {
                     ok = false;
                     break;
                 }
-                if (ht == 0) {
-                    const bool last_c = c + 1 == g.C;
-                    const int ni = last_c ? i + npair_ctas : i;
-                    if (ni < g.npairs) {
-                        fence_proxy_async_smem();
-                        const uint32_t nb = (ci + 1) & 1u;
-                        issue_pixels(&xmap, last_c ? decode_embed(g, ni, rank) : e, last_c ? 0 : c + 1,
-                                     xbase + nb * kPixBytes, smem_addr(&xfull[nb]));
-                    }
-                }
-                const uint32_t xb = ci & 1u;
-                if (!wait_or_abort(smem_addr(&xfull[xb]), (ci >> 1) & 1u, abort)) {
-                    ok = false;
-                    break;
-                }
-                uint32_t slot[3];
-                for (int dx = 0; dx < 3 && ok; ++dx) {
-                    slot[dx] = (pi + dx) % kPlanes;
-                    ok = wait_or_abort(smem_addr(&pempty[slot[dx]]), (((pi + dx) / kPlanes) & 1u) ^ 1u, abort);
-                }
-                if (!ok)
-                    break;
+                // Staged pixel columns of latent u: 4 (u + 2) .. + 3 (the box starts two blocks left of
+                // x0); rows 4 pr ..; window 0 reads frame 0 (box frame 3) four times.
+                float2 v[4][4][4];
                 if (worker) {
-                    // Staged pixel columns of latent u: 4 (u + 2) .. + 3 (the box starts two blocks left of
-                    // x0); rows 4 pr ..; window 0 reads frame 0 (box frame 3) four times.
-                    const unsigned char *pix = smem_raw + (xbase + xb * kPixBytes - smem_addr(smem_raw));
-                    float2 v[4][4][4];
                     const int col = 4 * (u0 + 2);
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
@@ -930,7 +910,10 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
 #pragma unroll
                         for (int d = 0; d < 4; ++d)
                             wht4x2(v[0][rr][d], v[1][rr][d], v[2][rr][d], v[3][rr][d]);
-                    unsigned char *planes = smem_raw + (pbase - smem_addr(smem_raw));
+                }
+                // The 64 coefficients of both blocks as bf16 rows: k8 = 8 subbands (16 bytes) per word group.
+                uint4 vlo[8], vhi[8];
+                if (worker) {
                     const float2 eighth = make_float2(0.125f, 0.125f);
 #pragma unroll
                     for (int k8 = 0; k8 < 8; ++k8) {
@@ -943,29 +926,61 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
                             lo[uu] = pack_bf16x2(a0.x, a1.x);
                             hi[uu] = pack_bf16x2(a0.y, a1.y);
                         }
-                        const uint4 vlo = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                        const uint4 vhi = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-#pragma unroll
-                        for (int dx = 0; dx < 3; ++dx) {
-                            unsigned char *plane = planes + slot[dx] * kPlaneBytes;
-                            const int j0 = u0 + 1 - dx, j1 = j0 + 1;
-                            if (j0 >= 0 && j0 < kTileCols)
-                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j0, 8 * k8)) = vlo;
-                            if (j1 >= 0 && j1 < kTileCols)
-                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j1, 8 * k8)) = vhi;
-                        }
+                        vlo[k8] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                        vhi[k8] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                     }
                 }
-                fence_proxy_async_smem(); // the planes' writes are visible to the tensor cores
-                __syncwarp();
-                if (lane == 0)
-                    for (int dx = 0; dx < 3; ++dx)
-                        mbar_arrive_cluster(mapa_shared(smem_addr(&pfull[slot[dx]]), 0));
+                // The coefficients are in registers: once every Haar thread is here (a barrier phase
+                // per colour, its wait bounded like the others) the next colour's copy refills the
+                // pixel buffer while the planes are written.
+                mbar_arrive(smem_addr(&hsync));
+                if (!wait_or_abort(smem_addr(&hsync), ci & 1u, abort)) {
+                    ok = false;
+                    break;
+                }
+                if (ht == 0) {
+                    const bool last_c = c + 1 == g.C;
+                    const int ni = last_c ? i + npair_ctas : i;
+                    if (ni < g.npairs) {
+                        fence_proxy_async_smem();
+                        issue_pixels(&xmap, last_c ? decode_embed(g, ni, rank) : e, last_c ? 0 : c + 1, xbase,
+                                     smem_addr(&xfull));
+                        ++px_issued;
+                    }
+                }
+                unsigned char *planes = smem_raw + (pbase - smem_addr(smem_raw));
+                for (int dx = 0; dx < 3; ++dx, ++pi) {
+                    const uint32_t slot = pi % kPlanes;
+                    if (!wait_or_abort(smem_addr(&pempty[slot]), ((pi / kPlanes) & 1u) ^ 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    if (worker) {
+                        unsigned char *plane = planes + slot * kPlaneBytes;
+                        const int j0 = u0 + 1 - dx, j1 = j0 + 1;
+                        if (j0 >= 0 && j0 < kTileCols) {
+#pragma unroll
+                            for (int k8 = 0; k8 < 8; ++k8)
+                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j0, 8 * k8)) =
+                                    vlo[k8];
+                        }
+                        if (j1 >= 0 && j1 < kTileCols) {
+#pragma unroll
+                            for (int k8 = 0; k8 < 8; ++k8)
+                                *reinterpret_cast<uint4 *>(plane + sw128_offset(pr * kTileCols + j1, 8 * k8)) =
+                                    vhi[k8];
+                        }
+                    }
+                    fence_proxy_async_smem(); // the plane's writes are visible to the tensor cores
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive_cluster(mapa_shared(smem_addr(&pfull[slot]), 0));
+                }
             }
         }
-        if (ht == 0 && !ok) // the pixel copies issued and not yet waited for
-            for (uint32_t j = ci; j < ci + 2; ++j)
-                mbar_wait(smem_addr(&xfull[j & 1u]), (j >> 1) & 1u);
+        if (ht == 0 && !ok) // a pixel copy issued and not yet waited for
+            for (uint32_t j = ci; j < px_issued; ++j)
+                mbar_wait(smem_addr(&xfull), j & 1u);
     }
 
     tc_fence_before();
@@ -981,7 +996,7 @@ patch_embed_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_consta
 
 size_t embed_smem_bytes(int bn)
 {
-    return (size_t)kFStages * (bn / 2) * kBK * 2 + (size_t)kPlanes * kPlaneBytes + 2 * (size_t)kPixBytes +
+    return (size_t)kFStages * kFGroup * (bn / 2) * kBK * 2 + (size_t)kPlanes * kPlaneBytes + (size_t)kPixBytes +
            epi_bytes(kEmbedEpiBuf) + 1024;
 }
 
