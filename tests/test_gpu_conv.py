@@ -151,7 +151,8 @@ def patcher_coeff_error(xp64, coeff):
 EMBED = [((1, 3, 9, 64, 64), 256, "three colours, whole tiles"),
          ((2, 2, 13, 36, 72), 64, "ragged tiles, two clips"),
          ((1, 1, 5, 16, 32), 512, "two channel tiles"),
-         ((1, 4, 5, 68, 40), 128, "four colours, ragged rows")]
+         ((1, 4, 5, 68, 40), 128, "four colours, ragged rows"),
+         ((1, 8, 9, 16, 24), 32, "eight colours, the smallest channel tile")]
 
 
 @pytest.mark.parametrize("shape,Cmid,note", EMBED, ids=[e[2] for e in EMBED])
