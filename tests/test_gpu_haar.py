@@ -155,6 +155,7 @@ def test_tma_and_register_paths_agree_bitwise(shape, dtype):
     ((2, 2, 29, 40, 72), torch.bfloat16, [(0, 3), (3, 8)]),                      # row-form inverse (W % 32 != 0)
     ((1, 2, 21, 32, 64), torch.float32, [(0, 2), (2, 2), (2, 6)]),               # fp32, an empty chunk
     ((2, 3, 1, 32, 64), torch.bfloat16, [(0, 1)]),                               # image: one window
+    ((1, 2, 25, 64, 1300), torch.bfloat16, [(0, 2), (2, 5), (5, 7)]),            # grouped rows, shifted tiles
 ])
 def test_windows_compose_to_the_full_call(shape, dtype, chunks):
     """Chunks of latent frames, processed separately, give exactly the full result; each chunk
