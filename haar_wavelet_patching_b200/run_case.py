@@ -35,6 +35,10 @@ def main():
     ap.add_argument("--ms", type=int, default=4, help="padded ops: spatial multiple")
     ap.add_argument("--mt", type=int, default=4, help="padded ops: temporal multiple")
     ap.add_argument("--first", action="store_true", help="chunk ops: the first chunk (1 + 4k frames)")
+    ap.add_argument("--flush", action="store_true",
+                    help="flush L2 before each call (a 256 MB write and a 256 MB read, queued ahead of the call so "
+                         "that no host time falls between the events) and time each call alone: for workloads that "
+                         "fit in L2, and launches shorter than a call's host-side cost")
     a = ap.parse_args()
     shape = tuple(int(v) for v in a.shape.split(","))
     dev = torch.device("cuda", 0)
@@ -147,12 +151,24 @@ def main():
     run()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(a.iters):
-        run()
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / a.iters
+    if a.flush:
+        bufs = [torch.empty(256 << 20, dtype=torch.uint8, device=dev) for _ in range(2)]
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(a.iters)]
+        for b0, b1 in evs:
+            bufs[0].zero_()
+            bufs[1].sum()
+            b0.record()
+            run()
+            b1.record()
+        torch.cuda.synchronize()
+        ms = sum(b0.elapsed_time(b1) for b0, b1 in evs) / a.iters
+    else:
+        e0.record()
+        for _ in range(a.iters):
+            run()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / a.iters
     extra = f", {flops / ms / 1e9:.1f} TFLOP/s" if a.op.startswith(("conv", "patch")) else ""
     print(f"{a.op} {shape} {a.dtype}: {ms * 1e3:.1f} us per launch, {nbytes / ms / 1e6:.1f} GB/s{extra}")
 
