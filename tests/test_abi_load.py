@@ -247,3 +247,14 @@ def test_patch_embed_rules(lib):
     assert pk(NULL, Wp, 3, 256, NULL) == hwp.TOK_ERR_NULL
     assert pk(X, F(0x800008), 3, 256, NULL) == hwp.TOK_ERR_ALIGN
     assert pk(X, X, 3, 256, NULL) == hwp.TOK_ERR_ALIAS
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """Without the built library every call raises: there is no CPU fallback to land on."""
+    import torch
+    monkeypatch.setattr(hwp, "LIB_PATH", str(tmp_path / "libtok.so"))
+    monkeypatch.setattr(hwp, "_lib", None)
+    with pytest.raises(ImportError, match="no CPU fallback"):
+        hwp.lib()
+    with pytest.raises((ImportError, ValueError)):
+        hwp.tok_fsq_encode(torch.zeros(1, 16, 4), torch.zeros(6, 16), torch.zeros(1, 4, dtype=torch.int32))
