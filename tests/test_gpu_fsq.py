@@ -67,13 +67,17 @@ def check_decode(idx_np, w_np, label):
     return got
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 4, 5])
-def test_encode_decode_configs(cfg):
+LATENTS = {1: "latent [1,16,4096]", 2: "latent [16,16,4096] (image batch)", 4: "latent [64,16,56320]",
+           5: "latent [4,16,130560] (stress clips)"}  # synth workload keys
+
+
+@pytest.mark.parametrize("cfg", list(LATENTS), ids=[LATENTS[k] for k in LATENTS])
+def test_encode_decode_latents(cfg):
     u = synth.fsq_input(cfg)
     w = synth.fsq_weight(u.shape[1])
-    idx, n_near, n_mism = check_encode(u, w, f"config {cfg}")
-    print(f"config {cfg}: {idx.size} tokens, {n_near} near a boundary, {n_mism} mismatches")
-    check_decode(idx, w, f"config {cfg}")
+    idx, n_near, n_mism = check_encode(u, w, LATENTS[cfg])
+    print(f"{LATENTS[cfg]}: {idx.size} tokens, {n_near} near a boundary, {n_mism} mismatches")
+    check_decode(idx, w, LATENTS[cfg])
 
 
 @pytest.mark.parametrize("B,C,S", [(3, 16, 4100), (2, 16, 132), (1, 16, 128), (3, 16, 4097), (2, 16, 1), (1, 3, 1000),
